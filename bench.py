@@ -1,0 +1,490 @@
+"""Benchmark: causal kernelized linear attention on B200.
+
+One step = one pass of the hot path over one batch of synthetic input:
+``la_prefill`` over the headline workload (``plain_bf16``: B=4, H=8, N=4096,
+d=dv=64, bf16 inputs, plain causal prefill with normaliser).  The metric is
+prefill tokens/s (tokens = B*N per step; each token carries H heads).
+
+Timing: W untimed warm-up steps, then K timed steps.  Inputs stay resident in
+HBM; L2 is flushed (a 256 MiB write, outside the timed events) before every
+timed step because the headline inputs (~50 MB) fit in L2.  Each step is
+timed with CUDA events on the stream the kernels run on; for N GPUs every
+rank processes its own full batch (independent problems: weak scaling, no
+data-path collective) and the time is the max over ranks.
+
+Printed: one JSON line (rank 0).  ``--impl reference`` times the float64 CPU
+oracle (the only reference this method has) on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from causal_kernelized_linear_la_b200 import inputs  # noqa: E402
+
+HEADLINE = "plain_bf16"
+METRIC = "prefill tokens/s and decode state-updates/s on 1 B200; % of roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------
+# work accounting (algorithmic bytes / flops per step)
+
+def prefill_units(p) -> dict:
+    """Tokens, token-heads and the method's own bytes/flops for one prefill."""
+    eb = 2 if p.dtype == "bf16" else 4
+    th = p.B * p.H * p.N
+    chains = p.B * p.H
+    byts = th * (2 * p.d + 2 * p.dv) * eb + chains * p.d * p.dv * 4
+    if p.mode == "gated_delta":
+        byts += th * 8  # alpha, g fp32
+        flops = th * 6 * p.d * p.dv
+    else:
+        byts += chains * p.d * 4
+        flops = th * (4 * p.d * p.dv + 4 * p.d)
+    return {"tokens": p.B * p.N, "token_heads": th, "bytes": byts, "flops": flops}
+
+
+def decode_units(Bs, Hh, d, dv, eb=2) -> dict:
+    states = Bs * Hh
+    byts = states * (2 * d * dv * 4 + 2 * d * 4 + (2 * d + 2 * dv) * eb)
+    return {"state_updates": states, "tokens": Bs, "bytes": byts, "flops": states * 4 * d * dv}
+
+
+def workload_desc(name: str) -> str:
+    w = inputs.WORKLOADS[name]
+    if w["kind"] == "decode":
+        return f"{name}: decode step, {w['S']} sequences x {w['H']} heads, d=dv={w['d']}, fp32 state, bf16 tokens"
+    what = {"plain": "plain causal prefill with normaliser", "decay": "per-head decay prefill with decayed normaliser",
+            "gated_delta": "gated delta rule prefill"}[w.get("mode", "gated_delta")]
+    return (f"{name}: B={w['B']} H={w['H']} N={w['N']} d=dv={w['d']} {w['dtype']} inputs, {what}")
+
+
+# ----------------------------------------------------------------------------
+# clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, path: str | None):
+        self.idx = device_index
+        self.path = path
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = open(self.path, "w") if self.path else subprocess.PIPE
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.text = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            if self.path:
+                self.out.close()
+                self.text = open(self.path).read()
+            else:
+                self.text = out or ""
+
+    def summary(self) -> dict:
+        rows = []
+        for line in self.text.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                rows.append({"sm": float(f[1]), "max": float(f[2]), "util": float(f[4]),
+                             "hw": f[6], "hwt": f[7], "swt": f[8], "pcap": f[9]})
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        busy = [r for r in rows if r["util"] > 0] or rows
+        reasons = set()
+        for r in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(busy)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (weak scaling: each rank owns an independent batch)
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Rank r processes an independent batch drawn with seed base + 1000 r."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: units processed by all ranks / slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+
+def _measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def _to_dev(x, torch):
+    if x is None:
+        return None
+    if x.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _prefill_device_args(p, torch):
+    if p.dtype == "bf16":
+        q, k, v = _to_dev(p.q_bits, torch), _to_dev(p.k_bits, torch), _to_dev(p.v_bits, torch)
+    else:
+        q, k, v = _to_dev(p.q, torch), _to_dev(p.k, torch), _to_dev(p.v, torch)
+    kw = {}
+    if p.mode == "decay":
+        kw["gamma"] = _to_dev(p.gamma, torch)
+    if p.mode == "gated_delta":
+        kw["alpha"], kw["g"] = _to_dev(p.alpha, torch), _to_dev(p.g, torch)
+    return q, k, v, kw
+
+
+def time_prefill(p, steps, warmup, torch, la, flush):
+    """Device time per step (ms) of la_prefill on resident inputs, L2 flushed
+    before every timed step; returns (list of ms, launches per step, buffers)."""
+    q, k, v, kw = _prefill_device_args(p, torch)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    out = torch.empty((B, H, N, dv), device="cuda", dtype=q.dtype)
+    S_out = torch.empty((B, H, d, dv), device="cuda", dtype=torch.float32)
+    z_out = None if p.mode == "gated_delta" else torch.empty((B, H, d), device="cuda", dtype=torch.float32)
+    ws_bytes = la.la_prefill_workspace_bytes(B, H, N, d, dv, p.dtype, p.mode)
+    ws = torch.empty(max(ws_bytes, 16), device="cuda", dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        la.la_prefill(q, k, v, mode=p.mode, eps=p.eps, out=out, S_out=S_out, z_out=z_out, workspace=ws, **kw)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(1)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    la.la_prefill_check(ws)
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def time_prefill_e2e(p, steps, warmup, torch, la):
+    """End to end through the public API with host buffers: pinned host inputs
+    copied in, la_prefill, output copied back, every step inside the events."""
+    pin = lambda x: None if x is None else torch.from_numpy(
+        np.ascontiguousarray(x).view(np.int16) if x.dtype == np.uint16 else np.ascontiguousarray(x)).pin_memory()
+    if p.dtype == "bf16":
+        hq, hk, hv = pin(p.q_bits), pin(p.k_bits), pin(p.v_bits)
+        tdt = torch.bfloat16
+    else:
+        hq, hk, hv = pin(p.q), pin(p.k), pin(p.v)
+        tdt = torch.float32
+    hextra = {}
+    if p.mode == "decay":
+        hextra["gamma"] = pin(p.gamma)
+    if p.mode == "gated_delta":
+        hextra["alpha"], hextra["g"] = pin(p.alpha), pin(p.g)
+    dq = torch.empty(hq.shape, dtype=hq.dtype, device="cuda")
+    dk = torch.empty_like(dq)
+    dvv = torch.empty(hv.shape, dtype=hv.dtype, device="cuda")
+    dextra = {n: torch.empty_like(t, device="cuda") for n, t in hextra.items()}
+    B, H, N, d = p.q.shape
+    dv = p.v.shape[-1]
+    h_out = torch.empty((B, H, N, dv), dtype=tdt).pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = sum(t.numel() * t.element_size() for t in [hq, hk, hv] + list(hextra.values()))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dvv.copy_(hv, non_blocking=True)
+        for n in hextra:
+            dextra[n].copy_(hextra[n], non_blocking=True)
+        o, _, _ = la.la_prefill(dq.view(tdt), dk.view(tdt), dvv.view(tdt), mode=p.mode, eps=p.eps, **dextra)
+        h_out.copy_(o, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps, h2d, d2h
+
+
+def time_decode(steps, warmup, torch, la, seed, Bs=256, Hh=32, d=128, dv=128, pool=8):
+    """Device time per decode step (ms) over `steps` chained steps; tokens come
+    from a pool of `pool` pre-generated steps (identical cost per step)."""
+    st = inputs.make_decode_state(Bs, Hh, d, dv, seed=seed)
+    S = torch.from_numpy(st.S).cuda()
+    z = torch.from_numpy(st.z).cuda()
+    toks = []
+    for s in range(pool):
+        t = inputs.make_decode_token(s, Bs, Hh, d, dv, seed=seed)
+        toks.append(tuple(_to_dev(x, torch) for x in (t.q_bits, t.k_bits, t.v_bits)))
+    out = torch.empty((Bs, Hh, dv), device="cuda", dtype=torch.bfloat16)
+    for i in range(warmup):
+        la.la_decode_step(*toks[i % pool], S, z, out=out)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        la.la_decode_step(*toks[i % pool], S, z, out=out)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+    import causal_kernelized_linear_la_b200 as la
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    hbm_peak, tc_peak, peak_kind = _measured_peaks()
+    spec = inputs.WORKLOADS[args.workload]
+    p = inputs.make_workload(args.workload, seed=rank_seed(spec["seed"], rank))
+    u = prefill_units(p)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+
+    clocks_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if os.path.isdir(
+        os.path.join(ROOT, "gpurun_out")) else None
+    with ClockSampler(local, clocks_path) as clk:
+        barrier()
+        ms = time_prefill(p, args.steps, args.warmup, torch, la, flush)
+        barrier()
+        # keep the device busy a little longer so the clock sampler sees load
+        extra = {}
+        if not args.no_extra:
+            extra = run_extra(args, torch, la, rank, flush)
+    local_total_ms = sum(ms)
+    total_ms = max_over_ranks(local_total_ms, world, device="cuda")
+    ms_per_step = total_ms / args.steps
+    value = aggregate_throughput(u["tokens"] * args.steps, world, total_ms / 1e3)
+    e2e_ms, h2d, d2h = time_prefill_e2e(p, max(3, min(args.steps, 20)), 2, torch, la)
+    e2e_ms = max_over_ranks(e2e_ms, world, device="cuda")
+    e2e_value = aggregate_throughput(u["tokens"], world, e2e_ms / 1e3)
+    clk_sum = clk.summary()
+
+    avg_launch_ms = local_total_ms / args.steps
+    achieved_gbs = u["bytes"] / (avg_launch_ms / 1e3) / 1e9
+    launches_per_step = la_launches_per_step(p)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": path_dtype(p),
+        "data": "synthetic (seeded numpy normal draws; see DESIGN.md input recipe)",
+        "config": {"workload": workload_desc(args.workload), "global_batch": p.B * world, "seq_len": p.N,
+                   "heads": p.H, "d": p.d, "dv": p.dv, "parallelism": f"replicas x{world} (independent batches)",
+                   "l2": "flushed before every timed step (256 MiB write outside the timed events)"},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm_peak, "traffic": None,
+                     "kernel": "la_prefill (whole call)", "peak_kind": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": u["bytes"]},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk_sum,
+    }
+    if extra:
+        line["other_workloads"] = extra
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def path_dtype(p) -> str:
+    return "f32" if p.dtype == "f32" else "bf16"
+
+
+def la_launches_per_step(p) -> int:
+    """Kernels one la_prefill call launches for this workload (our kernels only)."""
+    import causal_kernelized_linear_la_b200 as la
+    fn = getattr(la, "la_prefill_launches", None)
+    return int(fn(p.B, p.H, p.N, p.d, p.dv, p.dtype, p.mode)) if fn else 1
+
+
+def run_extra(args, torch, la, rank, flush):
+    """Device-timed numbers for the other workloads (not the headline line)."""
+    res = {}
+    hbm_peak, _, _ = _measured_peaks()
+    for name in ("decay_bf16", "gdelta_bf16", "plain_f32"):
+        spec = inputs.WORKLOADS[name]
+        p = inputs.make_workload(name, seed=rank_seed(spec["seed"], rank))
+        u = prefill_units(p)
+        steps = 5 if name != "plain_f32" else 50
+        ms = statistics.median(time_prefill(p, steps, 3, torch, la, flush))
+        res[name] = {"tokens_per_s": u["tokens"] / (ms / 1e3), "ms": ms,
+                     "hbm_frac": u["bytes"] / (ms / 1e3) / 1e9 / hbm_peak, "dtype": path_dtype(p)}
+        del p
+    dspec = inputs.WORKLOADS["decode"]
+    dms = time_decode(1000, 20, torch, la, rank_seed(dspec["seed"], rank))
+    du = decode_units(dspec["S"], dspec["H"], dspec["d"], dspec["dv"])
+    res["decode"] = {"state_updates_per_s": du["state_updates"] / (dms / 1e3),
+                     "tokens_per_s": du["tokens"] / (dms / 1e3), "ms_per_step": dms, "chained_steps": 1000,
+                     "hbm_frac": du["bytes"] / (dms / 1e3) / 1e9 / hbm_peak}
+    return res
+
+
+# ----------------------------------------------------------------------------
+# CPU arm: the float64 oracle
+
+def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
+    """Time the oracle as it stands on a bounded sample of the workload: whole
+    chains (all N tokens of one (b,h)), as many as fit the budget."""
+    import oracle
+    spec = inputs.WORKLOADS[workload]
+    p = inputs.make_workload(workload, B=1, H=min(spec["H"], 8))
+    chains = 0
+    t0 = time.perf_counter()
+    elapsed = 0.0
+    threads = oracle.threads()
+    per_call = max(1, min(p.H, threads))
+    while elapsed < budget_s:
+        hs = slice(0, per_call)
+        if p.mode == "gated_delta":
+            oracle.gated_delta(p.q[:, hs], p.k[:, hs], p.v[:, hs], p.alpha[:, hs], p.g[:, hs])
+        else:
+            oracle.kernelized(p.q[:, hs], p.k[:, hs], p.v[:, hs],
+                              None if p.gamma is None else p.gamma[hs], eps=p.eps)
+        chains += per_call
+        elapsed = time.perf_counter() - t0
+    token_heads = chains * p.N
+    value = token_heads / spec["H"] / elapsed  # tokens/s (a token carries H heads)
+    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{chains} whole chains of N={p.N} tokens ({token_heads} token-heads) of {workload}, "
+                      f"{elapsed:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    spec = inputs.WORKLOADS[args.workload]
+    per_step = []
+    for _ in range(args.warmup):
+        cpu_baseline(args.workload, budget_s=args.cpu_seconds / max(1, args.steps + args.warmup))
+    samples = []
+    for _ in range(args.steps):
+        cb = cpu_baseline(args.workload, budget_s=args.cpu_seconds / max(1, args.steps))
+        samples.append(cb)
+        per_step.append(spec["B"] * spec["N"] / cb["value"] * 1e3)
+    value = statistics.median(s["value"] for s in samples)
+    cb = dict(samples[0])
+    cb["value"] = value
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": statistics.median(per_step), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(args.workload)}, "impl": "reference",
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=HEADLINE, choices=[k for k, v in inputs.WORKLOADS.items()
+                                                              if v["kind"] != "decode"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    args.steps = max(1, args.steps)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_gpu(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+// C ABI entry points: argument validation and dispatch to the kernels.
+// Nothing here computes; every step of the path runs in the kernels.
+#include <stdint.h>
+
+#include "la_internal.cuh"
+
+namespace la {
+namespace {
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_ok(int x) { return x == 64 || x == 128; }
+
+la_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+// Final state for an empty sequence: the start state, or zero.
+la_status write_start_state(const PrefillArgs& a)
+{
+    const size_t chains = (size_t)a.B * a.H;
+    const size_t sbytes = chains * a.d * a.dv * sizeof(float);
+    const size_t zbytes = chains * a.d * sizeof(float);
+    cudaError_t e = cudaSuccess;
+    if (a.S0) e = cudaMemcpyAsync(a.S_out, a.S0, sbytes, cudaMemcpyDeviceToDevice, a.stream);
+    else e = cudaMemsetAsync(a.S_out, 0, sbytes, a.stream);
+    if (e == cudaSuccess && a.z_out) {
+        if (a.z0) e = cudaMemcpyAsync(a.z_out, a.z0, zbytes, cudaMemcpyDeviceToDevice, a.stream);
+        else e = cudaMemsetAsync(a.z_out, 0, zbytes, a.stream);
+    }
+    return from_cuda(e);
+}
+
+}  // namespace
+}  // namespace la
+
+using la::PrefillArgs;
+using la::DecodeArgs;
+
+extern "C" {
+
+const char* la_version(void) { return "0.1.0"; }
+
+const char* la_status_string(la_status s)
+{
+    switch (s) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID: return "LA_ERR_INVALID: invalid argument";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: head size or dtype/mode not supported";
+        case LA_ERR_ALIGN: return "LA_ERR_ALIGN: pointer not 16-byte aligned";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA call or kernel launch failed";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT: a bounded device-side wait gave up";
+        case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "unknown la_status";
+}
+
+size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_config* cfg)
+{
+    (void)B; (void)H; (void)N; (void)d; (void)dv; (void)cfg;
+    return 0;
+}
+
+la_status la_prefill(const void* q, const void* k, const void* v,
+                     const float* gamma_or_alpha, const float* g,
+                     void* out, float* S_out, float* z_out,
+                     int B, int H, int N, int d, int dv, const la_config* cfg)
+{
+    if (!cfg) return LA_ERR_INVALID;
+    if (B < 0 || H < 0 || N < 0) return LA_ERR_INVALID;
+    if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
+    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA) return LA_ERR_INVALID;
+    if (!la::head_ok(d) || !la::head_ok(dv)) return LA_ERR_UNSUPPORTED;
+    const bool delta = cfg->mode == LA_GATED_DELTA;
+    const bool work = (long long)B * H > 0;
+    if (work) {
+        if (!S_out) return LA_ERR_INVALID;
+        if (!delta && !z_out) return LA_ERR_INVALID;
+        if (delta && z_out) return LA_ERR_INVALID;
+        if (N > 0 && (!q || !k || !v || !out)) return LA_ERR_INVALID;
+        if (cfg->mode == LA_PLAIN && (gamma_or_alpha || g)) return LA_ERR_INVALID;
+        if (cfg->mode == LA_DECAY && (!gamma_or_alpha || g)) return LA_ERR_INVALID;
+        if (delta && N > 0 && (!gamma_or_alpha || !g)) return LA_ERR_INVALID;
+    }
+    if (!(cfg->eps >= 0.f)) return LA_ERR_INVALID;
+    if (work && ((cfg->S0 && cfg->S0 == S_out) || (cfg->z0 && cfg->z0 == z_out))) return LA_ERR_INVALID;
+    const void* ptrs[] = {q, k, v, gamma_or_alpha, g, out, S_out, z_out, cfg->S0, cfg->z0, cfg->workspace};
+    for (const void* p : ptrs)
+        if (!la::aligned16(p)) return LA_ERR_ALIGN;
+    if (cfg->workspace_bytes < la_prefill_workspace_bytes(B, H, N, d, dv, cfg)) return LA_ERR_WORKSPACE;
+    if (!work) return LA_OK;
+
+    PrefillArgs a{};
+    a.q = q; a.k = k; a.v = v;
+    a.gamma = cfg->mode == LA_DECAY ? gamma_or_alpha : nullptr;
+    a.alpha = delta ? gamma_or_alpha : nullptr;
+    a.g = delta ? g : nullptr;
+    a.out = out; a.S_out = S_out; a.z_out = delta ? nullptr : z_out;
+    a.S0 = cfg->S0; a.z0 = delta ? nullptr : cfg->z0;
+    a.B = B; a.H = H; a.N = N; a.d = d; a.dv = dv;
+    a.eps = cfg->eps; a.dtype = cfg->dtype; a.mode = cfg->mode;
+    a.stream = static_cast<cudaStream_t>(cfg->stream);
+    a.workspace = cfg->workspace; a.workspace_bytes = cfg->workspace_bytes;
+
+    if (N == 0) return la::write_start_state(a);
+    if (delta) return la::from_cuda(la::launch_prefill_simt_gated_delta(a));
+    return la::from_cuda(la::launch_prefill_simt_kernelized(a));
+}
+
+static la_status decode_common_checks(const void* q, const void* k, const void* v, float* S, void* out,
+                                      int B, int H, int d, int dv, const la_config* cfg)
+{
+    if (!cfg) return LA_ERR_INVALID;
+    if (B < 0 || H < 0) return LA_ERR_INVALID;
+    if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
+    if (!la::head_ok(d) || !la::head_ok(dv)) return LA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0 && (!q || !k || !v || !S || !out)) return LA_ERR_INVALID;
+    if ((long long)B * H > 0x7fffffffLL) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
+la_status la_decode_step(const void* q, const void* k, const void* v,
+                         float* S, float* z, void* out,
+                         int B, int H, int d, int dv, const la_config* cfg)
+{
+    la_status st = decode_common_checks(q, k, v, S, out, B, H, d, dv, cfg);
+    if (st != LA_OK) return st;
+    if (cfg->mode != LA_PLAIN) return LA_ERR_INVALID;
+    if ((long long)B * H > 0 && !z) return LA_ERR_INVALID;
+    if (!(cfg->eps >= 0.f)) return LA_ERR_INVALID;
+    const void* ptrs[] = {q, k, v, S, z, out};
+    for (const void* p : ptrs)
+        if (!la::aligned16(p)) return LA_ERR_ALIGN;
+    if ((long long)B * H == 0) return LA_OK;
+    DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v; a.S = S; a.z = z; a.out = out;
+    a.B = B; a.H = H; a.d = d; a.dv = dv; a.eps = cfg->eps; a.dtype = cfg->dtype;
+    a.stream = static_cast<cudaStream_t>(cfg->stream);
+    return la::from_cuda(la::launch_decode_kernelized(a));
+}
+
+la_status la_gated_delta_decode_step(const void* q, const void* k, const void* v,
+                                     const float* alpha, const float* g,
+                                     float* S, void* out,
+                                     int B, int H, int d, int dv, const la_config* cfg)
+{
+    la_status st = decode_common_checks(q, k, v, S, out, B, H, d, dv, cfg);
+    if (st != LA_OK) return st;
+    if (cfg->mode != LA_GATED_DELTA) return LA_ERR_INVALID;
+    if ((long long)B * H > 0 && (!alpha || !g)) return LA_ERR_INVALID;
+    const void* ptrs[] = {q, k, v, alpha, g, S, out};
+    for (const void* p : ptrs)
+        if (!la::aligned16(p)) return LA_ERR_ALIGN;
+    if ((long long)B * H == 0) return LA_OK;
+    DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.g = g; a.S = S; a.out = out;
+    a.B = B; a.H = H; a.d = d; a.dv = dv; a.dtype = cfg->dtype;
+    a.stream = static_cast<cudaStream_t>(cfg->stream);
+    return la::from_cuda(la::launch_decode_gated_delta(a));
+}
+
+la_status la_prefill_check(const void* workspace, void* stream)
+{
+    (void)workspace;
+    return la::from_cuda(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

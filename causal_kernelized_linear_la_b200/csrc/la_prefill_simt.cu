@@ -1,0 +1,271 @@
+// SIMT (CUDA-core, fp32 arithmetic) prefill kernels.
+//
+// These kernels carry the fp32-input path, where bf16 tensor-core operands
+// could not meet a 1e-4 relative error, and they accept bf16 inputs as well.
+//
+// kernelized (LA_PLAIN / LA_DECAY): chunkwise form ("Efficient attention
+// variants" §8).  For a chunk of C tokens with start state (S0, z0), local
+// positions i, j = 0..C-1 and lambda = log gamma:
+//   P_ij  = [j <= i] exp((i-j) lambda) phi(q_i).phi(k_j)     (multiplicative
+//           causal + decay mask, "Transformers Are RNNs" notes)
+//   num_i = sum_j P_ij v_j + exp((i+1) lambda) phi(q_i)^T S0
+//   den_i = sum_j P_ij     + exp((i+1) lambda) phi(q_i)^T z0
+//   o_i   = num_i / (den_i + eps)
+//   S    <- exp(n lambda) S0 + sum_j exp((n-1-j) lambda) phi(k_j) v_j^T
+//   z    <- exp(n lambda) z0 + sum_j exp((n-1-j) lambda) phi(k_j)
+// with n the number of valid tokens in the chunk.  This is the unrolled
+// recurrence S_t = gamma S_{t-1} + phi(k_t) v_t^T of "What Is Linear
+// Attention?" §4/§5.1 regrouped by chunk; it is exact up to rounding order.
+//
+// gated delta (LA_GATED_DELTA): the token recurrence itself, one thread per
+// state column.  Columns of S evolve independently under the delta rule
+// (S^T k is a per-column dot product), so each thread keeps its column of S
+// in registers: vhat_j = S_j.k_t;  S_j <- alpha S_j + g k_t (v_tj - alpha vhat_j);
+// o_tj = S_j.q_t   ("Efficient attention variants" §7.4).
+#include "la_internal.cuh"
+
+namespace la {
+namespace {
+
+constexpr int kChunk = 32;   // tokens per chunk
+constexpr int kThreads = 256;
+
+template <int D, int DVT>
+struct KernelizedSmem {
+    float fq[kChunk][D + 1];
+    float fk[kChunk][D + 1];
+    float vv[kChunk][DVT];
+    float P[kChunk][kChunk + 1];
+    float S[D][DVT];
+    float z[D];
+    float den[kChunk];
+    float wk[kChunk];  // exp((n-1-j) lambda)
+};
+
+template <typename T, int D, int DVT>
+__global__ void __launch_bounds__(kThreads)
+kernelized_chunk_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                      const float* __restrict__ gamma, const float* __restrict__ S0,
+                      const float* __restrict__ z0, T* __restrict__ out, float* __restrict__ S_out,
+                      float* __restrict__ z_out, int H, int N, int dv, float eps)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto& sm = *reinterpret_cast<KernelizedSmem<D, DVT>*>(smem_raw);
+    const int tid = threadIdx.x;
+    const int j0 = blockIdx.y * DVT;       // first value column of this tile
+    const long long chain = blockIdx.x;    // b*H + h
+    const int h = (int)(chain % H);
+    const float lam = gamma ? logf(gamma[h]) : 0.f;
+
+    const T* qc = q + chain * (long long)N * D;
+    const T* kc = k + chain * (long long)N * D;
+    const T* vc = v + chain * (long long)N * dv;
+    T* oc = out + chain * (long long)N * dv;
+
+    for (int e = tid; e < D * DVT; e += kThreads) {
+        const int f = e / DVT, j = e % DVT;
+        sm.S[f][j] = S0 ? S0[chain * (long long)D * dv + (long long)f * dv + j0 + j] : 0.f;
+    }
+    for (int f = tid; f < D; f += kThreads) sm.z[f] = z0 ? z0[chain * D + f] : 0.f;
+
+    for (int c0 = 0; c0 < N; c0 += kChunk) {
+        const int n = min(kChunk, N - c0);
+        __syncthreads();  // previous chunk finished with every buffer
+        for (int e = tid; e < kChunk * D; e += kThreads) {
+            const int t = e / D, f = e % D;
+            const bool ok = t < n;
+            const long long off = (long long)(c0 + t) * D + f;
+            sm.fq[t][f] = ok ? phi(to_f32(qc[off])) : 0.f;
+            sm.fk[t][f] = ok ? phi(to_f32(kc[off])) : 0.f;
+        }
+        for (int e = tid; e < kChunk * DVT; e += kThreads) {
+            const int t = e / DVT, j = e % DVT;
+            sm.vv[t][j] = t < n ? to_f32(vc[(long long)(c0 + t) * dv + j0 + j]) : 0.f;
+        }
+        if (tid < kChunk) sm.wk[tid] = tid < n ? expf((float)(n - 1 - tid) * lam) : 0.f;
+        __syncthreads();
+
+        // P = (phi(Q) phi(K)^T) * mask * decay
+        for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+            const int i = e / kChunk, j = e % kChunk;
+            float s = 0.f;
+            if (j <= i) {
+#pragma unroll 8
+                for (int f = 0; f < D; ++f) s = fmaf(sm.fq[i][f], sm.fk[j][f], s);
+                s *= expf((float)(i - j) * lam);
+            }
+            sm.P[i][j] = s;
+        }
+        __syncthreads();
+
+        // denominators: row sums of P plus the start-state term
+        if (tid < kChunk) {
+            const int i = tid;
+            float r = 0.f;
+            for (int j = 0; j <= i; ++j) r += sm.P[i][j];
+            float qz = 0.f;
+            for (int f = 0; f < D; ++f) qz = fmaf(sm.fq[i][f], sm.z[f], qz);
+            sm.den[i] = r + expf((float)(i + 1) * lam) * qz + eps;
+        }
+        __syncthreads();
+
+        // numerators and outputs
+        for (int e = tid; e < kChunk * DVT; e += kThreads) {
+            const int i = e / DVT, j = e % DVT;
+            if (i >= n) continue;
+            float intra = 0.f;
+            for (int l = 0; l <= i; ++l) intra = fmaf(sm.P[i][l], sm.vv[l][j], intra);
+            float inter = 0.f;
+#pragma unroll 8
+            for (int f = 0; f < D; ++f) inter = fmaf(sm.fq[i][f], sm.S[f][j], inter);
+            const float num = intra + expf((float)(i + 1) * lam) * inter;
+            oc[(long long)(c0 + i) * dv + j0 + j] = from_f32<T>(num / sm.den[i]);
+        }
+        __syncthreads();
+
+        // state carry
+        const float cdec = expf((float)n * lam);
+        for (int e = tid; e < D * DVT; e += kThreads) {
+            const int f = e / DVT, j = e % DVT;
+            float s = 0.f;
+            for (int l = 0; l < n; ++l) s = fmaf(sm.wk[l] * sm.fk[l][f], sm.vv[l][j], s);
+            sm.S[f][j] = fmaf(cdec, sm.S[f][j], s);
+        }
+        for (int f = tid; f < D; f += kThreads) {
+            float s = 0.f;
+            for (int l = 0; l < n; ++l) s = fmaf(sm.wk[l], sm.fk[l][f], s);
+            sm.z[f] = fmaf(cdec, sm.z[f], s);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < D * DVT; e += kThreads) {
+        const int f = e / DVT, j = e % DVT;
+        S_out[chain * (long long)D * dv + (long long)f * dv + j0 + j] = sm.S[f][j];
+    }
+    if (blockIdx.y == 0)
+        for (int f = tid; f < D; f += kThreads) z_out[chain * D + f] = sm.z[f];
+}
+
+template <typename T, int D, int DVT>
+cudaError_t launch_kernelized_t(const PrefillArgs& a)
+{
+    auto kern = kernelized_chunk_simt<T, D, DVT>;
+    const size_t smem = sizeof(KernelizedSmem<D, DVT>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.B * a.H, a.dv / DVT);
+    kern<<<grid, kThreads, smem, a.stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.gamma, a.S0, a.z0,
+                                             (T*)a.out, a.S_out, a.z_out, a.H, a.N, a.dv, a.eps);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// gated delta, token recurrence, one thread per column of S.
+
+constexpr int kDeltaTile = 32;  // tokens staged in shared memory at a time
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128)
+gated_delta_token_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                       const float* __restrict__ alpha, const float* __restrict__ g,
+                       const float* __restrict__ S0, T* __restrict__ out, float* __restrict__ S_out,
+                       int N, int dv)
+{
+    __shared__ __align__(16) float kq[2][kDeltaTile][D];
+    __shared__ float ag[2][kDeltaTile];
+    const int j = blockIdx.y * blockDim.x + threadIdx.x;  // state column
+    const long long chain = blockIdx.x;
+    const bool active = j < dv;
+    const T* qc = q + chain * (long long)N * D;
+    const T* kc = k + chain * (long long)N * D;
+    const T* vc = v + chain * (long long)N * dv;
+    const float* al = alpha + chain * (long long)N;
+    const float* gl = g + chain * (long long)N;
+    T* oc = out + chain * (long long)N * dv;
+
+    float s[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i)
+        s[i] = (S0 && active) ? S0[chain * (long long)D * dv + (long long)i * dv + j] : 0.f;
+
+    for (int t0 = 0; t0 < N; t0 += kDeltaTile) {
+        const int n = min(kDeltaTile, N - t0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < kDeltaTile * D; e += blockDim.x) {
+            const int t = e / D, f = e % D;
+            const long long off = (long long)(t0 + t) * D + f;
+            kq[0][t][f] = t < n ? to_f32(kc[off]) : 0.f;
+            kq[1][t][f] = t < n ? to_f32(qc[off]) : 0.f;
+        }
+        for (int t = threadIdx.x; t < kDeltaTile; t += blockDim.x) {
+            ag[0][t] = t < n ? al[t0 + t] : 1.f;
+            ag[1][t] = t < n ? gl[t0 + t] : 0.f;
+        }
+        __syncthreads();
+        for (int t = 0; t < n; ++t) {
+            const float vt = active ? to_f32(vc[(long long)(t0 + t) * dv + j]) : 0.f;
+            const float at = ag[0][t], gt = ag[1][t];
+            float h0 = 0.f, h1 = 0.f, h2 = 0.f, h3 = 0.f;
+#pragma unroll
+            for (int i = 0; i < D; i += 4) {
+                h0 = fmaf(s[i + 0], kq[0][t][i + 0], h0);
+                h1 = fmaf(s[i + 1], kq[0][t][i + 1], h1);
+                h2 = fmaf(s[i + 2], kq[0][t][i + 2], h2);
+                h3 = fmaf(s[i + 3], kq[0][t][i + 3], h3);
+            }
+            const float vhat = (h0 + h1) + (h2 + h3);        // S_{t-1}^T k_t
+            const float err = gt * (vt - at * vhat);          // g (v - alpha vhat)
+            float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+#pragma unroll
+            for (int i = 0; i < D; i += 4) {
+                s[i + 0] = fmaf(at, s[i + 0], kq[0][t][i + 0] * err);
+                s[i + 1] = fmaf(at, s[i + 1], kq[0][t][i + 1] * err);
+                s[i + 2] = fmaf(at, s[i + 2], kq[0][t][i + 2] * err);
+                s[i + 3] = fmaf(at, s[i + 3], kq[0][t][i + 3] * err);
+                o0 = fmaf(s[i + 0], kq[1][t][i + 0], o0);
+                o1 = fmaf(s[i + 1], kq[1][t][i + 1], o1);
+                o2 = fmaf(s[i + 2], kq[1][t][i + 2], o2);
+                o3 = fmaf(s[i + 3], kq[1][t][i + 3], o3);
+            }
+            if (active) oc[(long long)(t0 + t) * dv + j] = from_f32<T>((o0 + o1) + (o2 + o3));
+        }
+    }
+    if (active) {
+#pragma unroll
+        for (int i = 0; i < D; ++i) S_out[chain * (long long)D * dv + (long long)i * dv + j] = s[i];
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_gdelta_t(const PrefillArgs& a)
+{
+    const int threads = 64;
+    dim3 grid(a.B * a.H, (a.dv + threads - 1) / threads);
+    gated_delta_token_simt<T, D><<<grid, threads, 0, a.stream>>>(
+        (const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.g, a.S0, (T*)a.out, a.S_out, a.N, a.dv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_simt_kernelized(const PrefillArgs& a)
+{
+    if (a.dtype == LA_F32) {
+        if (a.d == 64) return launch_kernelized_t<float, 64, 32>(a);
+        return launch_kernelized_t<float, 128, 32>(a);
+    }
+    if (a.d == 64) return launch_kernelized_t<__nv_bfloat16, 64, 32>(a);
+    return launch_kernelized_t<__nv_bfloat16, 128, 32>(a);
+}
+
+cudaError_t launch_prefill_simt_gated_delta(const PrefillArgs& a)
+{
+    if (a.dtype == LA_F32) {
+        if (a.d == 64) return launch_gdelta_t<float, 64>(a);
+        return launch_gdelta_t<float, 128>(a);
+    }
+    if (a.d == 64) return launch_gdelta_t<__nv_bfloat16, 64>(a);
+    return launch_gdelta_t<__nv_bfloat16, 128>(a);
+}
+
+}  // namespace la

@@ -1,0 +1,171 @@
+/*
+ * la.h -- C ABI of the B200 (sm_100a) causal kernelized linear attention library.
+ *
+ * The library computes, per (batch b, head h) chain of N tokens,
+ *
+ *   kernelized modes (LA_PLAIN, LA_DECAY)
+ *     S_t = gamma_h S_{t-1} + phi(k_t) v_t^T          S: d x dv, fp32
+ *     z_t = gamma_h z_{t-1} + phi(k_t)                z: d,      fp32
+ *     o_t = phi(q_t)^T S_t / (phi(q_t)^T z_t + eps)   (write, then read)
+ *     phi(x) = elu(x) + 1 = (x > 0 ? x + 1 : exp(x)),  gamma_h = 1 in LA_PLAIN
+ *   ("What Is Linear Attention?" §4 and §5.1; "Efficient attention variants"
+ *    §4, §5 and §7.1; eps in the denominator: "Transformers Are RNNs" notes)
+ *
+ *   gated delta mode (LA_GATED_DELTA)
+ *     S_t = alpha_t S_{t-1} + g_t k_t (v_t - alpha_t S_{t-1}^T k_t)^T
+ *     o_t = S_t^T q_t            (no feature map, no normaliser)
+ *   ("Efficient attention variants" §7.4; "What Is Linear Attention?" §5.2-5.3)
+ *
+ * Prefill runs chunkwise: parallel inside a chunk, state carried between
+ * chunks ("Efficient attention variants" §8).  Decode applies the recurrence
+ * to one token per (sequence, head) against a resident state.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - Layouts are row-major and contiguous:
+ *     q, k  [B,H,N,d]     v, out  [B,H,N,dv]      (prefill)
+ *     q, k  [B,H,d]       v, out  [B,H,dv]        (decode)
+ *     S     [B,H,d,dv] fp32, rows = key feature, columns = value
+ *     z     [B,H,d]    fp32
+ *     gamma [H] fp32;  alpha, g [B,H,N] fp32 (prefill) or [B,H] (decode)
+ * - q, k, v and out share the element type cfg->dtype (fp32 or bf16).  All
+ *   arithmetic accumulates in fp32; states are always fp32.
+ * - Every pointer is a DEVICE pointer owned by the caller; the library keeps
+ *   no pointer after a call returns and allocates no device memory.
+ * - Every pointer must be 16-byte aligned (LA_ERR_ALIGN otherwise).
+ * - Calls are asynchronous on cfg->stream (a cudaStream_t; NULL = the legacy
+ *   default stream).  Argument errors are detected before anything is
+ *   launched and returned synchronously; launch failures are reported as
+ *   LA_ERR_CUDA.  Outputs must not alias inputs unless stated.
+ * - Supported head sizes: d, dv in {64, 128}; anything else returns
+ *   LA_ERR_UNSUPPORTED.  B, H, N >= 0 (zero sizes are valid and launch only
+ *   what is needed to write the final state).
+ */
+#ifndef LA_H
+#define LA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID = 1,      /* null pointer where one is required, negative size, bad enum */
+    LA_ERR_UNSUPPORTED = 2,  /* head size or dtype/mode combination not implemented */
+    LA_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned */
+    LA_ERR_CUDA = 4,         /* a CUDA runtime/driver call or kernel launch failed */
+    LA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (reported by la_prefill_check) */
+    LA_ERR_WORKSPACE = 6     /* workspace missing or smaller than la_prefill_workspace_bytes() */
+} la_status;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+typedef enum { LA_PLAIN = 0, LA_DECAY = 1, LA_GATED_DELTA = 2 } la_mode;
+
+typedef struct {
+    la_dtype dtype;          /* element type of q, k, v, out */
+    la_mode mode;            /* which recurrence */
+    float eps;               /* denominator epsilon (kernelized modes); 1e-6 is the usual value */
+    void* stream;            /* cudaStream_t the work is enqueued on */
+    const float* S0;         /* prefill start state [B,H,d,dv] or NULL (zero state) */
+    const float* z0;         /* prefill start normaliser [B,H,d] or NULL (zero); ignored in LA_GATED_DELTA */
+    void* workspace;         /* device scratch for prefill; may be NULL when la_prefill_workspace_bytes() == 0 */
+    size_t workspace_bytes;  /* size of workspace in bytes */
+} la_config;
+
+/*
+ * la_prefill -- causal prefill of B*H chains of N tokens.
+ *
+ * Defined by the recurrences above ("What Is Linear Attention?" §4, §5.1;
+ * "Efficient attention variants" §5, §7.1, §7.4), evaluated chunkwise
+ * ("Efficient attention variants" §8).
+ *
+ *   q, k, v          inputs, layouts above, element type cfg->dtype.
+ *   gamma_or_alpha   LA_PLAIN: must be NULL.  LA_DECAY: gamma [H], each in (0,1].
+ *                    LA_GATED_DELTA: alpha [B,H,N], each in (0,1].
+ *   g                LA_GATED_DELTA: write strength g [B,H,N]; otherwise NULL.
+ *   out              o [B,H,N,dv], element type cfg->dtype.
+ *   S_out            final state S_N [B,H,d,dv] fp32 (required).
+ *   z_out            final normaliser z_N [B,H,d] fp32 (kernelized modes, required);
+ *                    must be NULL in LA_GATED_DELTA.
+ *   cfg              dtype, mode, eps, stream, optional start state and workspace.
+ *
+ * In LA_GATED_DELTA no feature map is applied; k is expected to be
+ * L2-normalised by the caller (the rule is stable for ||k|| = 1, 0 < g <= 1).
+ * S_out and z_out must not overlap cfg->S0 and cfg->z0 (blocks of one call
+ * read the start state while others write the final state); continue a
+ * sequence by alternating two state buffers.  LA_ERR_INVALID if they alias.
+ * Returns LA_OK once the work is enqueued.
+ */
+LA_API la_status la_prefill(const void* q, const void* k, const void* v,
+                     const float* gamma_or_alpha, const float* g,
+                     void* out, float* S_out, float* z_out,
+                     int B, int H, int N, int d, int dv, const la_config* cfg);
+
+/*
+ * la_prefill_workspace_bytes -- device scratch la_prefill needs for these
+ * sizes and this cfg (dtype, mode).  0 means no workspace is needed.  The
+ * workspace carries per-segment state summaries between the kernels of one
+ * call; its content need not be initialised and is dead after the call's
+ * work completes.  Two calls in flight at once need two workspaces.
+ */
+LA_API size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_config* cfg);
+
+/*
+ * la_decode_step -- one decode step for B sequences x H heads, kernelized
+ * recurrence with gamma = 1 (the state cache of "What Is Linear Attention?"
+ * §6; update order of §4: write, then read):
+ *     S += phi(k) v^T;  z += phi(k);  out = phi(q)^T S / (phi(q)^T z + eps)
+ *
+ *   q, k   [B,H,d], v [B,H,dv], element type cfg->dtype.
+ *   S      [B,H,d,dv] fp32, read and updated in place.
+ *   z      [B,H,d] fp32, read and updated in place.
+ *   out    [B,H,dv], element type cfg->dtype.
+ *   cfg    dtype, eps, stream; mode must be LA_PLAIN; S0/z0/workspace unused.
+ */
+LA_API la_status la_decode_step(const void* q, const void* k, const void* v,
+                         float* S, float* z, void* out,
+                         int B, int H, int d, int dv, const la_config* cfg);
+
+/*
+ * la_gated_delta_decode_step -- one decode step of the gated delta rule for
+ * B sequences x H heads ("Efficient attention variants" §7.4):
+ *     S = alpha S + g k (v - alpha S^T k)^T;  out = S^T q
+ *
+ *   q, k   [B,H,d], v [B,H,dv], element type cfg->dtype (k L2-normalised).
+ *   alpha, g  [B,H] fp32.
+ *   S      [B,H,d,dv] fp32, read and updated in place.
+ *   out    [B,H,dv], element type cfg->dtype.
+ *   cfg    dtype, stream; mode must be LA_GATED_DELTA.
+ */
+LA_API la_status la_gated_delta_decode_step(const void* q, const void* k, const void* v,
+                                     const float* alpha, const float* g,
+                                     float* S, void* out,
+                                     int B, int H, int d, int dv, const la_config* cfg);
+
+/*
+ * la_prefill_check -- wait for the work enqueued on `stream` and report any
+ * device-side error recorded in `workspace` by the last la_prefill that used
+ * it (LA_ERR_TIMEOUT if a bounded wait between cooperating blocks gave up).
+ * Synchronises the stream.  A NULL workspace only synchronises.
+ */
+LA_API la_status la_prefill_check(const void* workspace, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+LA_API const char* la_status_string(la_status s);
+
+/* Library version as "major.minor.patch" (static storage). */
+LA_API const char* la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LA_H */

@@ -1,0 +1,91 @@
+"""The C-ABI library loads, exports every symbol include/la.h declares, and
+rejects bad arguments before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import causal_kernelized_linear_la_b200 as la
+from causal_kernelized_linear_la_b200 import LaConfig
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "la.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    return set(re.findall(r"LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(", src))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared() == set(la.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = la.lib()
+    for name in sorted(declared()):
+        assert hasattr(L, name), name
+    assert L.la_version().decode().count(".") == 2
+
+
+def test_status_strings():
+    for code in range(7):
+        assert la.la_status_string(code).startswith("LA_")
+
+
+def _cfg(dtype=la.LA_BF16, mode=0, eps=1e-6, S0=None, z0=None, ws=None, wsb=0):
+    return LaConfig(dtype, mode, eps, None, S0, z0, ws, wsb)
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def _prefill(cfg, B=1, H=1, N=8, d=64, dv=64, q=FAKE, k=FAKE, v=FAKE, ga=None, g=None, out=FAKE, S=FAKE, z=FAKE):
+    c = ctypes.c_void_p
+    return la.lib().la_prefill(c(q), c(k), c(v), c(ga), c(g), c(out), c(S), c(z), B, H, N, d, dv,
+                               None if cfg is None else ctypes.byref(cfg))
+
+
+def test_prefill_validation():
+    assert _prefill(None) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(), B=-1) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(), d=96) == la.LA_ERR_UNSUPPORTED
+    assert _prefill(_cfg(), dv=32) == la.LA_ERR_UNSUPPORTED
+    assert _prefill(_cfg(dtype=7)) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(mode=9)) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(), q=FAKE + 8) == la.LA_ERR_ALIGN
+    assert _prefill(_cfg(), S=0) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(), z=0) == la.LA_ERR_INVALID                  # kernelized needs z_out
+    assert _prefill(_cfg(mode=2), ga=FAKE, g=FAKE) == la.LA_ERR_INVALID  # delta must not get z_out
+    assert _prefill(_cfg(mode=1)) == la.LA_ERR_INVALID                  # decay needs gamma
+    assert _prefill(_cfg(mode=0), ga=FAKE) == la.LA_ERR_INVALID         # plain takes no gamma
+    assert _prefill(_cfg(eps=-1.0)) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(S0=FAKE), S=FAKE) == la.LA_ERR_INVALID          # output aliases start state
+    # nothing to do: valid and launches nothing
+    assert _prefill(_cfg(), B=0) == la.LA_OK
+    assert _prefill(_cfg(), H=0, q=0, k=0, v=0, out=0, S=0, z=0) == la.LA_OK
+
+
+def test_decode_validation():
+    c = ctypes.c_void_p
+    L = la.lib()
+    cfg = _cfg()
+    assert L.la_decode_step(c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), 1, 1, 64, 48, ctypes.byref(cfg)) == la.LA_ERR_UNSUPPORTED
+    assert L.la_decode_step(c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(0), c(FAKE), 1, 1, 64, 64, ctypes.byref(cfg)) == la.LA_ERR_INVALID
+    assert L.la_decode_step(c(FAKE + 4), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), 1, 1, 64, 64, ctypes.byref(cfg)) == la.LA_ERR_ALIGN
+    dcfg = _cfg(mode=2)
+    assert L.la_decode_step(c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), 1, 1, 64, 64, ctypes.byref(dcfg)) == la.LA_ERR_INVALID
+    assert L.la_gated_delta_decode_step(c(FAKE), c(FAKE), c(FAKE), c(0), c(FAKE), c(FAKE), c(FAKE), 1, 1, 64, 64, ctypes.byref(dcfg)) == la.LA_ERR_INVALID
+    assert L.la_gated_delta_decode_step(c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), c(FAKE), 0, 4, 64, 64, ctypes.byref(dcfg)) == la.LA_OK
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 8, 64)
+    with pytest.raises(ValueError):
+        la.la_prefill(q, q, q)
+
+
+def test_workspace_query_is_host_only():
+    n = la.la_prefill_workspace_bytes(2, 16, 32768, 128, 128, "bf16", "decay")
+    assert n >= 0

@@ -1,0 +1,249 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs.
+
+Tolerances (fixed by the workloads' stated bounds):
+  outputs      max|o - o_ref| / max|o_ref| <= 1e-4 (fp32 inputs), 2e-2 (bf16 inputs)
+  final state  ||S - S_ref||_F / ||S_ref||_F <= 1e-2, same for z
+Small cases compare every element of every chain; full-size workloads run in
+the launch configuration the benchmark uses and compare sampled chains (all
+their tokens and their final state) against the oracle.
+"""
+import numpy as np
+import pytest
+
+from causal_kernelized_linear_la_b200 import inputs
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+def _all_chains(p):
+    return [(b, h) for b in range(p.B) for h in range(p.H)]
+
+
+def _check(p, chains=None):
+    chains = _all_chains(p) if chains is None else chains
+    got = H.run_library(p)
+    ref = H.run_oracle(p, chains)
+    H.assert_close(p, got, ref, chains)
+    return got
+
+
+# --- small cases: several chunks, ragged tails, every element ---------------
+
+@pytest.mark.parametrize("N", [1, 7, 31, 32, 33, 64, 100, 256])
+def test_plain_f32_small(N):
+    _check(inputs.make_kernelized(2, 3, N, 64, 64, dtype="f32", mode="plain", seed=100 + N))
+
+
+@pytest.mark.parametrize("d,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+def test_decay_f32_heads(d, dv):
+    _check(inputs.make_kernelized(1, 4, 150, d, dv, dtype="f32", mode="decay", seed=200 + d + dv))
+
+
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 127, 128, 129, 300, 1000, 4133])
+def test_plain_bf16_small(N):
+    _check(inputs.make_kernelized(2, 2, N, 64, 64, dtype="bf16", mode="plain", seed=300 + N))
+
+
+@pytest.mark.parametrize("d,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("N", [77, 1500])
+def test_decay_bf16_heads(d, dv, N):
+    _check(inputs.make_kernelized(1, 16, N, d, dv, dtype="bf16", mode="decay", seed=400 + d + dv + N))
+
+
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 129, 700, 2100])
+def test_gated_delta_bf16_small(N):
+    _check(inputs.make_gated_delta(1, 3, N, 128, 128, dtype="bf16", seed=500 + N))
+
+
+@pytest.mark.parametrize("d,dv", [(64, 64), (64, 128), (128, 64)])
+def test_gated_delta_bf16_heads(d, dv):
+    _check(inputs.make_gated_delta(2, 2, 333, d, dv, dtype="bf16", seed=600 + d + dv))
+
+
+def test_gated_delta_f32_small():
+    _check(inputs.make_gated_delta(1, 2, 190, 64, 64, dtype="f32", seed=700))
+
+
+# --- edge cases ---------------------------------------------------------------
+
+def test_empty_sequence_returns_start_state():
+    import torch
+    import causal_kernelized_linear_la_b200 as la
+    q = torch.empty((2, 3, 0, 64), device="cuda", dtype=torch.bfloat16)
+    S0 = torch.randn(2, 3, 64, 64, device="cuda")
+    z0 = torch.rand(2, 3, 64, device="cuda") + 1
+    o, S, z = la.la_prefill(q, q, q, S0=S0, z0=z0)
+    assert o.numel() == 0
+    assert torch.equal(S, S0) and torch.equal(z, z0)
+    o, S, z = la.la_prefill(q, q, q)
+    assert torch.count_nonzero(S) == 0 and torch.count_nonzero(z) == 0
+
+
+@pytest.mark.parametrize("mode,dtype", [("plain", "bf16"), ("decay", "bf16"), ("plain", "f32"), ("gated_delta", "bf16")])
+def test_continuation_from_start_state(mode, dtype):
+    """prefill(N) == prefill(N1) then prefill(N - N1) from the returned state
+    (start-state support; the state is the whole cache)."""
+    N, N1 = 777, 300
+    if mode == "gated_delta":
+        p = inputs.make_gated_delta(1, 4, N, 128, 128, dtype=dtype, seed=800)
+    else:
+        p = inputs.make_kernelized(1, 4, N, 128, 128, dtype=dtype, mode=mode, seed=801)
+    import copy
+    head = copy.copy(p)
+    tail = copy.copy(p)
+    cut = lambda x, a, b: None if x is None else x[:, :, a:b]
+    for part, (a, b) in ((head, (0, N1)), (tail, (N1, N))):
+        part.N = b - a
+        part.q, part.k, part.v = cut(p.q, a, b), cut(p.k, a, b), cut(p.v, a, b)
+        if dtype == "bf16":
+            part.q_bits, part.k_bits, part.v_bits = cut(p.q_bits, a, b), cut(p.k_bits, a, b), cut(p.v_bits, a, b)
+        part.alpha, part.g = cut(p.alpha, a, b), cut(p.g, a, b)
+    o1, S1, z1 = H.run_library(head)
+    o2, S2, z2 = H.run_library(tail, S0=S1.astype(np.float32), z0=None if z1 is None else z1.astype(np.float32))
+    chains = _all_chains(p)
+    ref = H.run_oracle(p, chains)
+    got = (np.concatenate([o1, o2], axis=2), S2, z2)
+    H.assert_close(p, got, ref, chains)
+
+
+@pytest.mark.parametrize("mode", ["plain", "decay", "gated_delta"])
+def test_no_future_leakage_bit_exact(mode):
+    """'Efficient attention variants' §10/§11: change only future k, v
+    (k += 5, v -= 7 from token t0 on); earlier outputs must be bit-identical."""
+    import copy
+    t0 = 200
+    if mode == "gated_delta":
+        p = inputs.make_gated_delta(1, 2, 700, 128, 128, seed=900)
+    else:
+        p = inputs.make_kernelized(1, 2, 700, 128, 128, mode=mode, seed=901)
+    p2 = copy.copy(p)
+    k2 = p.k.copy(); v2 = p.v.copy()
+    k2[:, :, t0:] += 5.0
+    v2[:, :, t0:] -= 7.0
+    p2.k_bits, p2.k = inputs.bf16_round(k2)
+    p2.v_bits, p2.v = inputs.bf16_round(v2)
+    o1, _, _ = H.run_library(p)
+    o2, _, _ = H.run_library(p2)
+    np.testing.assert_array_equal(o1[:, :, :t0], o2[:, :, :t0])
+    assert not np.array_equal(o1[:, :, t0:], o2[:, :, t0:])
+
+
+def test_misaligned_pointer_is_rejected():
+    import torch
+    import causal_kernelized_linear_la_b200 as la
+    buf = torch.zeros(1 * 1 * 64 * 64 + 1, device="cuda", dtype=torch.bfloat16)
+    q = buf[1:].view(1, 1, 64, 64)
+    with pytest.raises(la.LaError) as ei:
+        la.la_prefill(q, q, q)
+    assert ei.value.code == la.LA_ERR_ALIGN
+
+
+# --- the five workloads at full size -----------------------------------------
+
+def test_workload_plain_f32_full():
+    p = inputs.make_workload("plain_f32")
+    _check(p)
+
+
+def test_workload_plain_bf16_full():
+    p = inputs.make_workload("plain_bf16")
+    _check(p, [(0, 0), (1, 5), (3, 7)])
+
+
+def test_workload_decay_bf16_full():
+    p = inputs.make_workload("decay_bf16")
+    _check(p, [(0, 0), (1, 15)])
+
+
+def test_workload_gdelta_bf16_full():
+    p = inputs.make_workload("gdelta_bf16")
+    _check(p, [(0, 3), (0, 31)])
+
+
+# --- decode -------------------------------------------------------------------
+
+def _decode_chain(Bs, H_, steps, sample):
+    import torch
+    import oracle
+    import causal_kernelized_linear_la_b200 as la
+    st = inputs.make_decode_state(Bs, H_)
+    S = torch.from_numpy(st.S).cuda()
+    z = torch.from_numpy(st.z).cuda()
+    S_ref = st.S[sample[:, 0], sample[:, 1]][:, None].astype(np.float64)
+    z_ref = st.z[sample[:, 0], sample[:, 1]][:, None].astype(np.float64)
+    first = last = None
+    for s in range(steps):
+        t = inputs.make_decode_token(s, Bs, H_)
+        o = la.la_decode_step(H.dev(t.q_bits, torch), H.dev(t.k_bits, torch), H.dev(t.v_bits, torch), S, z)
+        pick = lambda x: x[sample[:, 0], sample[:, 1]][:, None]
+        o_ref, S_ref, z_ref = oracle.decode_step(pick(t.q), pick(t.k), pick(t.v), S_ref, z_ref)
+        if s == 0:
+            first = (o.float().cpu().numpy()[sample[:, 0], sample[:, 1]], o_ref[:, 0])
+        if s == steps - 1:
+            last = (o.float().cpu().numpy()[sample[:, 0], sample[:, 1]], o_ref[:, 0])
+    torch.cuda.synchronize()
+    Sg = S.cpu().numpy()[sample[:, 0], sample[:, 1]]
+    zg = z.cpu().numpy()[sample[:, 0], sample[:, 1]]
+    for got, ref in (first, last):
+        assert H.rel_max(got, ref) <= H.TOL_O["bf16"]
+    assert H.rel_fro(Sg, S_ref[:, 0]) <= H.TOL_STATE
+    assert H.rel_fro(zg, z_ref[:, 0]) <= H.TOL_STATE
+
+
+def test_decode_1000_chained_steps():
+    """1000 chained steps on 8 sequences x 32 heads; o at steps 1 and 1000 and
+    S, z after 1000 steps, all states checked."""
+    Bs, H_ = 8, 32
+    sample = np.array([(b, h) for b in range(Bs) for h in range(H_)])
+    _decode_chain(Bs, H_, 1000, sample)
+
+
+def test_decode_full_size_state():
+    """The full 256 x 32 state in the benchmark's launch configuration, a few
+    chained steps, 24 sampled states."""
+    rng = np.random.default_rng(0)
+    sample = np.stack([rng.integers(0, 256, 24), rng.integers(0, 32, 24)], axis=1)
+    _decode_chain(256, 32, 5, sample)
+
+
+@pytest.mark.parametrize("d,dv", [(128, 128), (64, 64), (64, 128)])
+def test_decode_f32_tokens(d, dv):
+    import torch
+    import oracle
+    import causal_kernelized_linear_la_b200 as la
+    rng = np.random.default_rng(d + dv)
+    Bs, H_ = 5, 3
+    S0 = (0.1 * rng.standard_normal((Bs, H_, d, dv))).astype(np.float32)
+    z0 = (np.abs(rng.standard_normal((Bs, H_, d))) + 1).astype(np.float32)
+    q, k = (rng.standard_normal((2, Bs, H_, d)) / np.sqrt(d)).astype(np.float32)
+    v = (rng.standard_normal((Bs, H_, dv)) / np.sqrt(d)).astype(np.float32)
+    S, z = torch.from_numpy(S0).cuda(), torch.from_numpy(z0).cuda()
+    o = la.la_decode_step(torch.from_numpy(q).cuda(), torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(), S, z)
+    o_ref, S_ref, z_ref = oracle.decode_step(q, k, v, S0, z0)
+    assert H.rel_max(o.cpu().numpy(), o_ref) <= H.TOL_O["f32"]
+    assert H.rel_max(S.cpu().numpy(), S_ref) <= 1e-5
+    assert H.rel_max(z.cpu().numpy(), z_ref) <= 1e-6
+
+
+@pytest.mark.parametrize("d,dv", [(128, 128), (64, 64)])
+def test_gated_delta_decode_steps(d, dv):
+    import torch
+    import oracle
+    import causal_kernelized_linear_la_b200 as la
+    p = inputs.make_gated_delta(4, 8, 20, d, dv, seed=1000 + d)
+    rng = np.random.default_rng(1)
+    S0 = (0.1 * rng.standard_normal((4, 8, d, dv))).astype(np.float32)
+    S = torch.from_numpy(S0).cuda()
+    S_ref = S0.astype(np.float64)
+    for t in range(p.N):
+        o = la.la_gated_delta_decode_step(H.dev(np.ascontiguousarray(p.q_bits[:, :, t]), torch),
+                                          H.dev(np.ascontiguousarray(p.k_bits[:, :, t]), torch),
+                                          H.dev(np.ascontiguousarray(p.v_bits[:, :, t]), torch),
+                                          H.dev(np.ascontiguousarray(p.alpha[:, :, t]), torch),
+                                          H.dev(np.ascontiguousarray(p.g[:, :, t]), torch), S)
+        o_ref, S_ref = oracle.gated_delta_step(p.q[:, :, t], p.k[:, :, t], p.v[:, :, t], p.alpha[:, :, t],
+                                               p.g[:, :, t], S_ref)
+        assert H.rel_max(o.float().cpu().numpy(), o_ref) <= H.TOL_O["bf16"]
+    assert H.rel_fro(S.cpu().numpy(), S_ref) <= H.TOL_STATE
