@@ -3,6 +3,7 @@
 #include <stdint.h>
 
 #include "la_internal.cuh"
+#include "la_prefill_tc.cuh"
 
 namespace la {
 namespace {
@@ -11,6 +12,14 @@ bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr
 bool head_ok(int x) { return x == 64 || x == 128; }
 
 la_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+}  // namespace
+
+// bf16 kernelized prefill runs on the tensor cores; fp32 inputs stay on the
+// fp32 SIMT kernels (bf16 operands could not meet a 1e-4 error bound).
+bool uses_tc_kernelized(la_dtype dt, la_mode m) { return dt == LA_BF16 && (m == LA_PLAIN || m == LA_DECAY); }
+
+namespace {
 
 // Final state for an empty sequence: the start state, or zero.
 la_status write_start_state(const PrefillArgs& a)
@@ -54,7 +63,8 @@ const char* la_status_string(la_status s)
 
 size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_config* cfg)
 {
-    (void)B; (void)H; (void)N; (void)d; (void)dv; (void)cfg;
+    if (!cfg || B <= 0 || H <= 0 || N <= 0 || !la::head_ok(d) || !la::head_ok(dv)) return 0;
+    if (la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return la::tc_workspace_bytes(B, H, N, d, dv);
     return 0;
 }
 
@@ -101,6 +111,7 @@ la_status la_prefill(const void* q, const void* k, const void* v,
 
     if (N == 0) return la::write_start_state(a);
     if (delta) return la::from_cuda(la::launch_prefill_simt_gated_delta(a));
+    if (la::uses_tc_kernelized(a.dtype, a.mode)) return la::from_cuda(la::launch_prefill_tc_kernelized(a));
     return la::from_cuda(la::launch_prefill_simt_kernelized(a));
 }
 
@@ -159,7 +170,10 @@ la_status la_gated_delta_decode_step(const void* q, const void* k, const void* v
 la_status la_prefill_check(const void* workspace, void* stream)
 {
     (void)workspace;
-    return la::from_cuda(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LA_ERR_CUDA;
+    if (la::read_and_clear_device_error(s) != 0) return LA_ERR_TIMEOUT;
+    return LA_OK;
 }
 
 }  // extern "C"

@@ -46,6 +46,8 @@ struct DecodeArgs {
     cudaStream_t stream;
 };
 
+bool uses_tc_kernelized(la_dtype dt, la_mode m);
+
 // SIMT prefill kernels (fp32 arithmetic; fp32 or bf16 inputs).
 cudaError_t launch_prefill_simt_kernelized(const PrefillArgs& a);
 cudaError_t launch_prefill_simt_gated_delta(const PrefillArgs& a);

@@ -1,0 +1,23 @@
+// Host-side interface of the tensor-core prefill kernels.
+#pragma once
+
+#include "la_internal.cuh"
+
+namespace la {
+
+// Sequence split of the tensor-core prefill: segments of L tokens (a multiple
+// of the 64-token chunk), G segments per (batch, head) chain.
+struct TcSegments {
+    int L = 0;
+    int G = 0;
+};
+
+TcSegments tc_segments(int B, int H, int N, int d, int dv);
+size_t tc_workspace_bytes(int B, int H, int N, int d, int dv);
+cudaError_t launch_prefill_tc_kernelized(const PrefillArgs& a);
+
+// Read (and clear) the device error word the tensor-core kernels set when a
+// bounded wait gives up.  Synchronises `stream`.
+unsigned int read_and_clear_device_error(cudaStream_t stream);
+
+}  // namespace la

@@ -14,9 +14,10 @@
 namespace la {
 namespace sm100 {
 
-// Device error word shared by all tensor-core kernels of the library (read
-// and cleared by la_prefill_check).  Non-zero: which wait gave up.
-extern __device__ unsigned int g_device_error;
+// Device error word of the tensor-core kernels of one translation unit (each
+// such unit exports a host function that reads and clears its copy for
+// la_prefill_check).  Non-zero: which wait gave up first.
+static __device__ unsigned int g_device_error = 0;
 
 // Each try_wait can suspend the thread for a while; this bounds a wait to
 // well under a second on B200 while never tripping on legitimate latency.
