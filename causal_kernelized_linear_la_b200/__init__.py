@@ -29,7 +29,7 @@ LA_F32, LA_BF16 = 0, 1
 MODES = {"plain": 0, "decay": 1, "gated_delta": 2}
 
 # Symbols the library exports; the header include/la.h declares exactly these.
-EXPORTS = ("la_prefill", "la_prefill_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
+EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
            "la_prefill_check", "la_status_string", "la_version")
 
 
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         vp, i, cfgp = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(LaConfig)
         L.la_prefill.argtypes = [vp] * 8 + [i] * 5 + [cfgp]
         L.la_prefill.restype = i
+        L.la_prefill_noalloc.argtypes = [vp] * 8 + [i] * 5 + [cfgp]
+        L.la_prefill_noalloc.restype = i
         L.la_prefill_workspace_bytes.argtypes = [i] * 5 + [cfgp]
         L.la_prefill_workspace_bytes.restype = ctypes.c_size_t
         L.la_decode_step.argtypes = [vp] * 6 + [i] * 4 + [cfgp]

@@ -115,6 +115,44 @@ la_status la_prefill(const void* q, const void* k, const void* v,
     return la::from_cuda(la::launch_prefill_simt_kernelized(a));
 }
 
+la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
+                             const float* gamma_or_alpha, const float* g,
+                             void* out, float* S_out, float* z_out,
+                             int B, int H, int N, int d, int dv, const la_config* cfg)
+{
+    if (!cfg) return LA_ERR_INVALID;
+    if (B < 0 || H < 0 || N < 0) return LA_ERR_INVALID;
+    if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
+    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA) return LA_ERR_INVALID;
+    if (!la::head_ok(d) || !la::head_ok(dv)) return LA_ERR_UNSUPPORTED;
+    if (!la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return LA_ERR_UNSUPPORTED;
+    const bool work = (long long)B * H > 0;
+    if (work) {
+        if (!S_out || !z_out) return LA_ERR_INVALID;
+        if (N > 0 && (!q || !k || !v || !out)) return LA_ERR_INVALID;
+        if (cfg->mode == LA_PLAIN && (gamma_or_alpha || g)) return LA_ERR_INVALID;
+        if (cfg->mode == LA_DECAY && (!gamma_or_alpha || g)) return LA_ERR_INVALID;
+    }
+    if (!(cfg->eps >= 0.f)) return LA_ERR_INVALID;
+    if (work && ((cfg->S0 && cfg->S0 == S_out) || (cfg->z0 && cfg->z0 == z_out))) return LA_ERR_INVALID;
+    const void* ptrs[] = {q, k, v, gamma_or_alpha, out, S_out, z_out, cfg->S0, cfg->z0};
+    for (const void* p : ptrs)
+        if (!la::aligned16(p)) return LA_ERR_ALIGN;
+    if (!work) return LA_OK;
+    if (N > 0 && la::tc_segments_noalloc(B, H, N, d, dv).G == 0) return LA_ERR_WORKSPACE;
+
+    PrefillArgs a{};
+    a.q = q; a.k = k; a.v = v;
+    a.gamma = cfg->mode == LA_DECAY ? gamma_or_alpha : nullptr;
+    a.out = out; a.S_out = S_out; a.z_out = z_out;
+    a.S0 = cfg->S0; a.z0 = cfg->z0;
+    a.B = B; a.H = H; a.N = N; a.d = d; a.dv = dv;
+    a.eps = cfg->eps; a.dtype = cfg->dtype; a.mode = cfg->mode;
+    a.stream = static_cast<cudaStream_t>(cfg->stream);
+    if (N == 0) return la::write_start_state(a);
+    return la::from_cuda(la::launch_prefill_tc_kernelized_noalloc(a));
+}
+
 static la_status decode_common_checks(const void* q, const void* k, const void* v, float* S, void* out,
                                       int B, int H, int d, int dv, const la_config* cfg)
 {

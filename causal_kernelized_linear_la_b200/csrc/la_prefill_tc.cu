@@ -28,6 +28,8 @@
 // true start state.
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "la_internal.cuh"
 #include "la_prefill_tc.cuh"
 #include "sm100.cuh"
@@ -686,6 +688,89 @@ size_t tc_workspace_bytes(int B, int H, int N, int d, int dv)
 cudaError_t launch_prefill_tc_kernelized(const PrefillArgs& a)
 {
     const TcSegments sg = tc_segments(a.B, a.H, a.N, a.d, a.dv);
+    const bool dec = a.mode == LA_DECAY;
+#define LA_TC(D, DV)                                                               \
+    if (a.d == D && a.dv == DV) return dec ? launch_tc<D, DV, true>(a, sg) : launch_tc<D, DV, false>(a, sg);
+    LA_TC(64, 64)
+    LA_TC(64, 128)
+    LA_TC(128, 64)
+    LA_TC(128, 128)
+#undef LA_TC
+    return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------
+// No-allocation variant.  Some callers cannot call cudaMalloc on their launch
+// path (an inference server that plans all device memory up front, a plugin
+// host that hands out no workspace, code that must not trigger the implicit
+// device synchronisation an allocation can cause).  For them the segment
+// summaries live in this fixed array instead of a caller workspace.  Every
+// GPU that loads the library holds it until the process exits.  All calls
+// share it: calls whose work overlaps on the GPU (two streams, or two host
+// threads) race on its contents and must be serialised by the caller.  The
+// kernels overwrite every byte they later read, so nothing needs clearing.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch for the current device, looked up once
+// per device with that device current.  In host code the symbol itself is
+// only a host-side stand-in and must never be handed to a kernel.
+void* noalloc_scratch_address(cudaError_t* err)
+{
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = -1;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+// Segment split that fits the fixed scratch: start from the usual split and
+// lengthen segments until chains * segments summaries fit.  G == 0 means the
+// problem is too large even with one segment per chain.
+TcSegments tc_segments_noalloc(int B, int H, int N, int d, int dv)
+{
+    TcSegments s = tc_segments(B, H, N, d, dv);
+    const size_t per_seg = (size_t)B * H * ((size_t)d * dv + d) * sizeof(float);
+    if (per_seg == 0 || N == 0) return s;
+    const size_t gmax = kNoAllocScratchBytes / per_seg;
+    if (gmax == 0) {
+        s.G = 0;
+        return s;
+    }
+    if ((size_t)s.G > gmax) {
+        long long L = ((long long)N + (long long)gmax - 1) / (long long)gmax;
+        L = ((L + C - 1) / C) * C;
+        s.L = (int)L;
+        s.G = (int)((N + L - 1) / L);
+    }
+    return s;
+}
+
+cudaError_t launch_prefill_tc_kernelized_noalloc(const PrefillArgs& in)
+{
+    const TcSegments sg = tc_segments_noalloc(in.B, in.H, in.N, in.d, in.dv);
+    if (sg.G == 0) return cudaErrorInvalidValue;
+    cudaError_t e;
+    void* scratch = noalloc_scratch_address(&e);
+    if (!scratch) return e;
+    PrefillArgs a = in;
+    a.workspace = scratch;
+    a.workspace_bytes = kNoAllocScratchBytes;
     const bool dec = a.mode == LA_DECAY;
 #define LA_TC(D, DV)                                                               \
     if (a.d == D && a.dv == DV) return dec ? launch_tc<D, DV, true>(a, sg) : launch_tc<D, DV, false>(a, sg);

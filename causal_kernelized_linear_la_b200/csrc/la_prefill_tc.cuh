@@ -16,6 +16,11 @@ TcSegments tc_segments(int B, int H, int N, int d, int dv);
 size_t tc_workspace_bytes(int B, int H, int N, int d, int dv);
 cudaError_t launch_prefill_tc_kernelized(const PrefillArgs& a);
 
+// Fixed scratch of the no-allocation entry point (la_prefill_noalloc).
+constexpr size_t kNoAllocScratchBytes = 16u << 20;
+TcSegments tc_segments_noalloc(int B, int H, int N, int d, int dv);
+cudaError_t launch_prefill_tc_kernelized_noalloc(const PrefillArgs& a);
+
 // Read (and clear) the device error word the tensor-core kernels set when a
 // bounded wait gives up.  Synchronises `stream`.
 unsigned int read_and_clear_device_error(cudaStream_t stream);

@@ -111,6 +111,37 @@ LA_API la_status la_prefill(const void* q, const void* k, const void* v,
                      int B, int H, int N, int d, int dv, const la_config* cfg);
 
 /*
+ * la_prefill_noalloc -- the bf16 tensor-core prefill of the kernelized modes
+ * (LA_PLAIN, LA_DECAY) for callers that cannot allocate device memory on
+ * their launch path: a server that plans all device memory before it starts,
+ * a plugin host that offers no workspace, or code that must avoid the device
+ * synchronisation an allocation may cause.  The pages have no counterpart;
+ * this is a service of this library.
+ *
+ * Arguments, layouts and results are those of la_prefill; cfg->workspace is
+ * ignored.  Instead of a caller workspace the call uses a fixed 16 MiB array
+ * of device memory inside the library, which every GPU that loads the
+ * library holds until the process exits.  The segment summaries of one call
+ * must fit in it: (B*H) * ceil(N / L) * (d*dv + d) * 4 bytes for a segment
+ * length L the call picks (at least 64); a problem that does not fit even
+ * with one segment per chain, i.e. B*H*(d*dv + d)*4 > 16 MiB, is rejected with
+ * LA_ERR_WORKSPACE before anything is launched.  Only cfg->dtype == LA_BF16
+ * with LA_PLAIN or LA_DECAY is served (LA_ERR_UNSUPPORTED otherwise; the
+ * other paths of la_prefill need no workspace at all).
+ *
+ * All calls in one process share the array and it keeps the last call's
+ * contents: calls whose work can overlap on the GPU (enqueued on different
+ * streams, or from different host threads) race on it and must be
+ * serialised by the caller.  Separate processes each have their own copy.  The first call on each device looks up the array's device
+ * address with that device current; make that first call before any stream
+ * capture on that device.
+ */
+LA_API la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
+                                    const float* gamma_or_alpha, const float* g,
+                                    void* out, float* S_out, float* z_out,
+                                    int B, int H, int N, int d, int dv, const la_config* cfg);
+
+/*
  * la_prefill_workspace_bytes -- device scratch la_prefill needs for these
  * sizes and this cfg (dtype, mode).  0 means no workspace is needed.  The
  * workspace carries per-segment state summaries between the kernels of one
