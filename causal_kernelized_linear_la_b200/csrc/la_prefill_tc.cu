@@ -26,6 +26,9 @@
 // (Delta S, Delta z); kernel B scans summaries into segment start states and
 // the final state; kernel C runs the chunk loop of every segment from its
 // true start state.
+//
+// Supported decay range on this path: gamma >= 0.3 (64 |log gamma| <= 80);
+// smaller gamma sets the device error word (la_prefill_check reports it).
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -39,9 +42,12 @@ namespace {
 
 using namespace sm100;
 
-constexpr int C = 64;            // tokens per chunk
-constexpr int kThreads = 128;    // one warpgroup: TMEM lanes 0..127
-constexpr int TILE = C * 64 * 2; // one 64-token x 64-element bf16 tile (8 KB)
+constexpr int C = 64;             // tokens per chunk
+constexpr int kThreads = 512;     // four warpgroups; each phase is split by columns
+constexpr int TILE = C * 64 * 2;  // one 64-row x 128-byte swizzled tile (8 KB)
+// The scaled-frame exponents (decay) stay within +-kFrameLimit in natural-log
+// units, far from the fp32 / bf16 overflow at ~88.
+constexpr float kFrameLimit = 40.f;
 
 // ---------------------------------------------------------------------------
 // Shared-memory plan of the chunk kernel (all tiles 1024-byte aligned).
@@ -50,22 +56,20 @@ struct ChunkPlan {
     static constexpr int STAGES = (D + DV > 128) ? 3 : 4;
     static constexpr int QB = C * D * 2, KB = C * D * 2, VB = C * DV * 2;
     static constexpr int STAGE = QB + KB + VB;
-    static constexpr int OFF_KT = STAGES * STAGE;
-    static constexpr int OFF_P = OFF_KT + (DECAY ? KB : 0);
-    static constexpr int OFF_SB = OFF_P + C * C * 2;
-    static constexpr int OFF_O = OFF_SB + D * DV * 2;
-    static constexpr int OFF_MISC = OFF_O + C * DV * 2;
-    // misc: rden[C], qsc[C], dtab[C], z[2][D], barriers, tmem base
-    static constexpr int OFF_RDEN = OFF_MISC;
-    static constexpr int OFF_QSC = OFF_RDEN + C * 4;
-    static constexpr int OFF_DTAB = OFF_QSC + C * 4;
-    static constexpr int OFF_Z = OFF_DTAB + C * 4;
-    static constexpr int OFF_BAR = OFF_Z + 2 * D * 4;
-    static constexpr int NBAR = STAGES + 3;
+    static constexpr int OFF_KH = STAGES * STAGE;                 // K^ (frame-weighted phi(K)), decay only
+    static constexpr int OFF_Q32 = OFF_KH + (DECAY ? KB : 0);     // Q^ fp32 [C][D], tf32 operand
+    static constexpr int OFF_P = OFF_Q32 + C * D * 4;             // P~ bf16 [C][C]
+    static constexpr int OFF_ONES = OFF_P + C * C * 2;            // bf16 [C][C], row 0 = 1
+    static constexpr int OFF_O = OFF_ONES + C * C * 2;            // output staging bf16 [C][DV]
+    static constexpr int OFF_RDEN = OFF_O + C * DV * 2;           // [C] 1 / denominator
+    static constexpr int OFF_DTAB = OFF_RDEN + C * 4;             // [C] gamma^k
+    static constexpr int OFF_BAR = OFF_DTAB + C * 4;
+    static constexpr int NBAR = STAGES + 5;                       // full[S], p, s, o, pt_full, o_free
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
-    static constexpr int BYTES = OFF_TMEM + 16 + 1024;  // + alignment slack
-    // TMEM columns
-    static constexpr uint32_t T_P = 0, T_O = 64, T_OI = 128, T_S = 256, T_COLS = 512;
+    static constexpr int BYTES = OFF_TMEM + 16 + 1024;            // + alignment slack
+    static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
+    // TMEM columns: scores, output^T, denominator row, state^T, normaliser row
+    static constexpr uint32_t T_P = 0, T_O = 64, T_DEN = 128, T_S = 256, T_Z = 384, T_COLS = 512;
 };
 
 template <int D, int DV>
@@ -73,10 +77,11 @@ struct SummaryPlan {
     static constexpr int STAGES = 4;
     static constexpr int KB = C * D * 2, VB = C * DV * 2;
     static constexpr int STAGE = KB + VB;
-    static constexpr int OFF_BAR = STAGES * STAGE;          // full[S], empty[S], done
+    static constexpr int OFF_ONES = STAGES * STAGE;
+    static constexpr int OFF_BAR = OFF_ONES + C * C * 2;           // full[S], empty[S], done
     static constexpr int OFF_TMEM = OFF_BAR + (2 * STAGES + 1) * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
-    static constexpr uint32_t T_COLS = DV < 32 ? 32 : DV;
+    static constexpr uint32_t T_S = 0, T_Z = 128, T_COLS = 256;
 };
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p)
@@ -86,31 +91,46 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* p)
 
 // Row of an accumulator that this thread owns after tcgen05.ld.32x32b, for a
 // tile of M rows (M = 128: lane i = row i; M = 64: rows 16w..16w+15 live in
-// lanes 32w..32w+15).  Returns -1 when the lane holds no row.
+// lanes 32w..32w+15).  `quad` is the warp's TMEM lane quadrant.  Returns -1
+// when the lane holds no row.
 template <int M>
-__device__ __forceinline__ int acc_row(int warp, int lane)
+__device__ __forceinline__ int acc_row(int quad, int lane)
 {
-    if (M == 128) return warp * 32 + lane;
-    return lane < 16 ? warp * 16 + lane : -1;
+    if (M == 128) return quad * 32 + lane;
+    return lane < 16 ? quad * 16 + lane : -1;
 }
 
-__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, int warp, uint32_t col)
+__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, int quad, uint32_t col)
 {
-    return base + ((uint32_t)(warp * 32) << 16) + col;
+    return base + ((uint32_t)(quad * 32) << 16) + col;
 }
 
-// phi on a 16-byte chunk of 8 bf16 values, scaled by w; returns the packed chunk.
-__device__ __forceinline__ uint4 phi_chunk(uint4 x, float w)
+__device__ __forceinline__ void unpack8(uint4 x, float (&f)[8])
 {
-    uint32_t in[4] = {x.x, x.y, x.z, x.w};
-    uint32_t out[4];
+    const uint32_t in[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&in[i]);
-        const float2 f = __bfloat1622float2(h);
-        out[i] = pack_bf16x2(w * phi_fast(f.x), w * phi_fast(f.y));
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[i]));
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
     }
-    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8], float w)
+{
+    return make_uint4(pack_bf16x2(w * f[0], w * f[1]), pack_bf16x2(w * f[2], w * f[3]),
+                      pack_bf16x2(w * f[4], w * f[5]), pack_bf16x2(w * f[6], w * f[7]));
+}
+
+// Constant A operand: a 64 x 64 bf16 tile whose row 0 is all ones.  One MMA
+// with it sums the rows of a B operand into accumulator row 0.
+__device__ __forceinline__ void init_ones_tile(unsigned char* tile, int tid, int nthreads)
+{
+    for (int e = tid; e < C * 8; e += nthreads) {
+        const int row = e / 8;
+        const uint32_t one2 = pack_bf16x2(1.f, 1.f);
+        reinterpret_cast<uint4*>(tile)[e] = row == 0 ? make_uint4(one2, one2, one2, one2) : make_uint4(0, 0, 0, 0);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -124,18 +144,20 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     using P = SummaryPlan<D, DV>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
+    unsigned char* ones = sm + P::OFF_ONES;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* empty = full + P::STAGES;
     uint64_t* done = empty + P::STAGES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, wg = warp >> 2;
     const int unit = blockIdx.x;
     const int chain = unit / G, seg = unit % G;
     const int t0 = seg * L, t1 = min(N, t0 + L);
     const int nch = (t1 - t0 + C - 1) / C;
     const float lam = DECAY ? logf(gamma[chain % H]) : 0.f;
-    const uint64_t pol = policy_evict_normal();
+    const uint64_t pol = policy_evict_last();  // the chunk kernel reads k, v again
 
     if (tid == 0) {
         for (int s = 0; s < P::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -143,11 +165,14 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, P::T_COLS);
+    init_ones_tile(ones, tid, kThreads);
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
+    int loads_issued = 0, loads_waited = 0, commits = 0;
     auto issue = [&](int c) {
         const int s = c % P::STAGES;
         unsigned char* st = sm + s * P::STAGE;
@@ -155,12 +180,12 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         for (int b = 0; b < D / 64; ++b) tma_load_3d(st + b * TILE, &tm_k, b * 64, t0 + c * C, chain, &full[s], pol);
         for (int b = 0; b < DV / 64; ++b)
             tma_load_3d(st + P::KB + b * TILE, &tm_v, b * 64, t0 + c * C, chain, &full[s], pol);
+        loads_issued = c + 1;
     };
     if (tid == 0)
         for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
 
     bool bad = false;
-    float zacc = 0.f;
     const int last = t1 - 1;
     for (int c = 0; c < nch; ++c) {
         const int s = c % P::STAGES;
@@ -168,6 +193,7 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         unsigned char* kt = sm + s * P::STAGE;
         unsigned char* vt = kt + P::KB;
         if (!mbar_wait(&full[s], ph, kErrTmaLoad)) bad = true;
+        else loads_waited = c + 1;
         // K~_t = gamma^(last - t) phi(k_t), zero past the end of the sequence
         const int tc0 = t0 + c * C;
         for (int e = tid; e < (D / 8) * C; e += kThreads) {
@@ -175,34 +201,30 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             uint4* p = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
             const int t = tc0 + row;
             const float w = t <= last ? (DECAY ? __expf((float)(last - t) * lam) : 1.f) : 0.f;
-            *p = phi_chunk(*p, w);
+            float f[8];
+            unpack8(*p, f);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) f[x] = phi_fast(f[x]);
+            *p = pack8(f, w);
         }
         fence_async_smem();
         tc_fence_before();
         if (__syncthreads_or(bad)) { bad = true; break; }
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(D, DV, 1, 1);
+            const uint32_t ka = smem_u32(kt), va = smem_u32(vt), oa = smem_u32(ones);
+            const uint32_t id_s = idesc_bf16_f32(D, DV, 1, 1);
+            const uint32_t id_z = idesc_bf16_f32(64, D, 0, 1);
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t a = sdesc_sw128(smem_u32(kt) + ks * 2048, TILE, 1024);
-                const uint64_t bb = sdesc_sw128(smem_u32(vt) + ks * 2048, TILE, 1024);
-                mma_bf16(tbase, a, bb, idesc, (c > 0 || ks > 0) ? 1u : 0u);
+                const uint64_t bk = sdesc_sw128(ka + ks * 2048, TILE, 1024);
+                mma_bf16(tbase + P::T_S, bk, sdesc_sw128(va + ks * 2048, TILE, 1024), id_s, (c > 0 || ks > 0));
+                mma_bf16(tbase + P::T_Z, sdesc_sw128(oa + ks * 32, 16, 1024), bk, id_z, (c > 0 || ks > 0));
             }
             mma_commit(&empty[s]);
             if (c == nch - 1) mma_commit(done);
+            commits = c + 1;
         }
-        // Delta z: column sums of the bf16 K~ the tensor core consumes
-        if (tid < D) {
-            const int b = tid / 64, col = tid % 64;
-            const unsigned char* base = kt + b * TILE;
-            float acc = 0.f;
-#pragma unroll 8
-            for (int r = 0; r < C; ++r)
-                acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + sw128_offset(r, col * 2)));
-            zacc += acc;
-        }
-        // refill this stage once every thread is done with it and the MMA has consumed it
         __syncthreads();
         if (tid == 0 && c + P::STAGES < nch) {
             if (!mbar_wait(&empty[s], ph, kErrMma)) bad = true;
@@ -213,19 +235,42 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     tc_fence_after();
     float* slot = ws + (size_t)unit * (D * DV + D);
     if (!bad) {
-        const int f = acc_row<D>(warp, lane);
+        const int f = acc_row<D>(quad, lane);
 #pragma unroll
-        for (int g = 0; g < DV / 16; ++g) {
+        for (int gg = 0; gg < DV / 64; ++gg) {
+            const int col0 = wg * (DV / 4) + gg * 16;
             float v[16];
-            tmem_ld16(tmem_addr(tbase, warp, g * 16), v);
+            tmem_ld16(tmem_addr(tbase, quad, P::T_S + col0), v);
             tmem_ld_wait();
             if (f >= 0) {
-                float4* dst = reinterpret_cast<float4*>(slot + (size_t)f * DV + g * 16);
+                float4* dst = reinterpret_cast<float4*>(slot + (size_t)f * DV + col0);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
         }
-        if (tid < D) slot[D * DV + tid] = zacc;
+        // Delta z: row 0 of the ones-row product, in lane 0 of quadrant 0
+        if (quad == 0) {
+#pragma unroll
+            for (int gg = 0; gg < D / 64; ++gg) {
+                const int col0 = wg * (D / 4) + gg * 16;
+                float v[16];
+                tmem_ld16(tmem_addr(tbase, 0, P::T_Z + col0), v);
+                tmem_ld_wait();
+                if (lane == 0) {
+                    float4* dst = reinterpret_cast<float4*>(slot + D * DV + col0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                }
+            }
+        }
+    }
+    if (bad && tid == 0) {
+        // Leave no copy or MMA in flight before releasing TMEM and exiting.
+        for (int cc = loads_waited; cc < loads_issued; ++cc)
+            mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
+        if (commits > 0)
+            mbar_wait(&empty[(commits - 1) % P::STAGES], ((commits - 1) / P::STAGES) & 1, kErrMma);
     }
     tc_fence_before();
     __syncthreads();
@@ -274,53 +319,84 @@ scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float
 
 // ---------------------------------------------------------------------------
 // Kernel C: the chunk loop of one (chain, segment) from its start state.
+//
+// The state is kept transposed in TMEM (S^T: lane = value index, column =
+// key feature), exactly the layout of the A operand of a tf32 MMA, so the
+// start-state read of every chunk is an MMA straight out of TMEM and the
+// state never passes through the CUDA cores.  The normaliser rides along as
+// row 0 of two small accumulators fed by a constant "ones row" tile.
+//
+// Decay uses a scaled frame: with r the frame's reference position, the
+// stored state is T = gamma^-(c0 - r) S(c0-1) at chunk start c0, key rows are
+// written as K^_t = gamma^-(t+1-r) phi(k_t) and query rows read as
+// Q^_t = gamma^(t+1-r) phi(q_t).  The frame moves (T is rescaled once) only
+// when |lambda| (t - r) would exceed kFrameLimit.
+//
+// Roles: warps 0..15 ("workers") run the epilogues and phi; lane 0 of warp 16
+// ("issuer") issues TMA and every MMA.  Chunk c, from barrier B1:
+//   issuer:  store o(c-1); MMA1 P = phi(Q)phi(K)^T; MMA3 O^T = S^T Q^^T and
+//            MMA3d den = z.Q^ (tf32, A in TMEM); MMA4 S^T += V^T K^ and
+//            MMA4d z += 1^T K^; prefetch; [wait P~] MMA2 O^T += V^T P~^T,
+//            MMA2d den += 1^T P~^T; release the staging tile
+//   workers: [P ready] mask/decay -> P~, signal;  phi(c+1) in place (overlaps
+//            the MMA batch);  [state carry done] frame move, Q^/K^ of c+1;
+//            [outputs ready] 1/den, o = O^T/den -> staging tile      -> B1
 template <int D, int DV, bool DECAY>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads + 32, 1)
 chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
              const float* __restrict__ gamma, const float* __restrict__ ws, int N, int H, int G, int L, float eps)
 {
     using P = ChunkPlan<D, DV, DECAY>;
+    constexpr int NCHK = (D / 8) * C / kThreads;  // 16-byte chunks of a Q (or K) tile per worker thread
+    static_assert(NCHK >= 1 && (D / 8) * C % kThreads == 0, "tile split");
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
-    unsigned char* ktil = sm + P::OFF_KT;
+    unsigned char* khat = sm + P::OFF_KH;
+    unsigned char* q32 = sm + P::OFF_Q32;
     unsigned char* ptil = sm + P::OFF_P;
-    unsigned char* sbt = sm + P::OFF_SB;
+    unsigned char* ones = sm + P::OFF_ONES;
     unsigned char* otil = sm + P::OFF_O;
     float* rden = reinterpret_cast<float*>(sm + P::OFF_RDEN);
-    float* qsc = reinterpret_cast<float*>(sm + P::OFF_QSC);
     float* dtab = reinterpret_cast<float*>(sm + P::OFF_DTAB);
-    float* zbuf = reinterpret_cast<float*>(sm + P::OFF_Z);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* bar_p = full + P::STAGES;
     uint64_t* bar_s = bar_p + 1;
     uint64_t* bar_o = bar_p + 2;
+    uint64_t* pt_full = bar_p + 3;
+    uint64_t* o_free = bar_p + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, wg = warp >> 2;
+    const bool worker = tid < kThreads;        // warps 0..15: epilogues and phi
+    const bool issuer = tid == kThreads;       // lane 0 of warp 16: TMA and MMA issue
     const int unit = blockIdx.x;
     const int chain = unit / G, seg = unit % G;
     const int t0 = seg * L, t1 = min(N, t0 + L);
     const int nch = (t1 - t0 + C - 1) / C;
     const float lam = DECAY ? logf(gamma[chain % H]) : 0.f;
     const uint64_t pol_in = policy_evict_first();
+    // One chunk's key weights reach gamma^-C; beyond e^80 they would overflow.
+    if (DECAY && tid == 0 && (float)C * fabsf(lam) > 80.f) atomicCAS(&g_device_error, 0u, (unsigned int)kErrRange);
 
     if (tid == 0) {
-        for (int s = 0; s < P::NBAR; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < P::STAGES + 3; ++s) mbar_init(&full[s], 1);
+        mbar_init(pt_full, kThreads / 32);
+        mbar_init(o_free, 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, P::T_COLS);
-    if (tid < C) {
-        dtab[tid] = DECAY ? __expf((float)tid * lam) : 1.f;        // gamma^(i-j)
-        qsc[tid] = DECAY ? __expf((float)(tid + 1) * lam) : 1.f;    // gamma^(i+1)
-    }
+    if (tid < C) dtab[tid] = DECAY ? __expf((float)tid * lam) : 1.f;   // gamma^(i-j)
+    if (worker) init_ones_tile(ones, tid, kThreads);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
-    // bookkeeping for the error path (meaningful in thread 0, which issues)
-    int loads_issued = 0, loads_waited = 0, commits = 0, commits_o = 0;
+    // bookkeeping for the error path (meaningful in the issuer)
+    int loads_issued = 0, commits = 0, commits_o = 0;
+    int ref = 0;  // frame reference position (segment-local)
     auto chunk_len = [&](int c) { return min(C, t1 - (t0 + c * C)); };
     auto issue = [&](int c) {
         const int s = c % P::STAGES;
@@ -334,265 +410,273 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (int b = 0; b < DV / 64; ++b)
             tma_load_3d(st + P::QB + P::KB + b * TILE, &tm_v, b * 64, y, chain, &full[s], pol_in);
     };
-    if (tid == 0)
-        for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
-
-    // Start state: fp32 into TMEM (pre-scaled by gamma^n of the first chunk,
-    // ready for MMA4 to accumulate onto), bf16 copy into smem for MMA3.
-    {
-        const float* slot = ws + (size_t)unit * (D * DV + D);
-        const int f = acc_row<D>(warp, lane);
-        const float dec0 = DECAY ? __expf((float)chunk_len(0) * lam) : 1.f;
-#pragma unroll
-        for (int g = 0; g < DV / 16; ++g) {
-            float v[16];
-            if (f >= 0) {
-                const float4* src = reinterpret_cast<const float4*>(slot + (size_t)f * DV + g * 16);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 x = src[q];
-                    v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
-                }
-                uint4 c0, c1;
-                c0.x = pack_bf16x2(v[0], v[1]); c0.y = pack_bf16x2(v[2], v[3]);
-                c0.z = pack_bf16x2(v[4], v[5]); c0.w = pack_bf16x2(v[6], v[7]);
-                c1.x = pack_bf16x2(v[8], v[9]); c1.y = pack_bf16x2(v[10], v[11]);
-                c1.z = pack_bf16x2(v[12], v[13]); c1.w = pack_bf16x2(v[14], v[15]);
-                unsigned char* blk = sbt + (g / 4) * (D * 128);
-                *reinterpret_cast<uint4*>(blk + sw128_offset(f, (g % 4) * 32)) = c0;
-                *reinterpret_cast<uint4*>(blk + sw128_offset(f, (g % 4) * 32 + 16)) = c1;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] *= dec0;
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = 0.f;
-            }
-            tmem_st16(tmem_addr(tbase, warp, P::T_S + g * 16), v);
-        }
-        tmem_st_wait();
-        if (tid < D) zbuf[tid] = slot[D * DV + tid];
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    bool bad = false;
-    for (int c = 0; c < nch; ++c) {
-        const int s = c % P::STAGES;
-        const uint32_t ph = (c / P::STAGES) & 1;
-        const uint32_t cp = c & 1;
+    // phi on load, part A: phi(q), phi(k) of chunk c into registers and, as
+    // bf16, back in place (the score MMA operands; K zeroed past the end).
+    float fq[NCHK][8], fk[NCHK][8];
+    auto phi_a = [&](int c) {
         const int n = chunk_len(c);
-        unsigned char* qt = sm + s * P::STAGE;
+        unsigned char* qt = sm + (c % P::STAGES) * P::STAGE;
         unsigned char* kt = qt + P::QB;
-        unsigned char* vt = kt + P::KB;
-        unsigned char* kst = DECAY ? ktil : kt;   // K~ used by MMA4 and for z
-        const float* zc = zbuf + cp * D;
-        float* zn = zbuf + (cp ^ 1) * D;
-
-        // 1. inputs landed; phi on load (K~ zeroed past the end of the sequence)
-        if (!mbar_wait(&full[s], ph, kErrTmaLoad)) bad = true;
-        else loads_waited = c + 1;
-        for (int e = tid; e < (D / 8) * C; e += kThreads) {
+#pragma unroll
+        for (int u = 0; u < NCHK; ++u) {
+            const int e = tid + u * kThreads;
             const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
             uint4* pq = reinterpret_cast<uint4*>(qt + b * TILE) + rem;
             uint4* pk = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
-            *pq = phi_chunk(*pq, 1.f);
-            const float valid = row < n ? 1.f : 0.f;
-            const uint4 raw = *pk;
-            *pk = phi_chunk(raw, valid);
+            unpack8(*pq, fq[u]);
+            unpack8(*pk, fk[u]);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) { fq[u][x] = phi_fast(fq[u][x]); fk[u][x] = phi_fast(fk[u][x]); }
+            *pq = pack8(fq[u], 1.f);
+            *pk = pack8(fk[u], row < n ? 1.f : 0.f);
+        }
+    };
+    // part B: the frame-weighted operands Q^ (fp32, tf32 MMA) and K^ (bf16).
+    auto phi_b = [&](int c) {
+        const int n = chunk_len(c);
+        const int c0 = c * C;
+#pragma unroll
+        for (int u = 0; u < NCHK; ++u) {
+            const int e = tid + u * kThreads;
+            const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
+            const int f0 = b * 64 + (((rem % 8) ^ (row & 7)) * 8);   // first feature of this 16-byte chunk
+            const float qw = DECAY ? __expf((float)(c0 + row + 1 - ref) * lam) : 1.f;
+            unsigned char* qrow = q32 + (f0 / 32) * TILE;
+            const int fb = (f0 % 32) * 4;
+            *reinterpret_cast<float4*>(qrow + sw128_offset(row, fb)) =
+                make_float4(qw * fq[u][0], qw * fq[u][1], qw * fq[u][2], qw * fq[u][3]);
+            *reinterpret_cast<float4*>(qrow + sw128_offset(row, fb + 16)) =
+                make_float4(qw * fq[u][4], qw * fq[u][5], qw * fq[u][6], qw * fq[u][7]);
             if (DECAY) {
-                const float w = row < n ? __expf((float)(n - 1 - row) * lam) : 0.f;
-                reinterpret_cast<uint4*>(ktil + b * TILE)[rem] = phi_chunk(raw, w);
+                const float kw = row < n ? __expf(-(float)(c0 + row + 1 - ref) * lam) : 0.f;
+                reinterpret_cast<uint4*>(khat + b * TILE)[rem] = pack8(fk[u], kw);
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(bad)) { bad = true; break; }
+    };
+    // Move the frame to position c0 (decay): S^T and z row times gamma^(c0 - ref).
+    auto frame_move = [&](int c0) {
+        const float m = __expf((float)(c0 - ref) * lam);
+#pragma unroll
+        for (int gg = 0; gg < D / 64; ++gg) {
+            const int col0 = wg * (D / 4) + gg * 16;
+            float v[16];
+            tmem_ld16(tmem_addr(tbase, quad, P::T_S + col0), v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 16; ++x) v[x] *= m;
+            tmem_st16(tmem_addr(tbase, quad, P::T_S + col0), v);
+            tmem_ld16(tmem_addr(tbase, quad, P::T_Z + col0), v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 16; ++x) v[x] *= m;
+            tmem_st16(tmem_addr(tbase, quad, P::T_Z + col0), v);
+        }
+        tmem_st_wait();
+    };
+    auto needs_move = [&](int c) {
+        if (!DECAY) return false;
+        return (float)(c * C + C - ref) * fabsf(lam) > kFrameLimit;
+    };
 
-        // 2. issue MMA1 (scores), MMA3 (start-state read), MMA4 (state carry)
-        if (tid == 0) {
+    if (issuer)
+        for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
+
+    // Start state, transposed into TMEM: S^T[j][f] = S[f][j]; z as row 0 of
+    // the normaliser accumulator (other rows zero).
+    if (worker) {
+        const float* slot = ws + (size_t)unit * (D * DV + D);
+        const int j = acc_row<DV>(quad, lane);
+#pragma unroll
+        for (int gg = 0; gg < D / 64; ++gg) {
+            const int col0 = wg * (D / 4) + gg * 16;
+            float v[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) v[x] = j >= 0 ? slot[(size_t)(col0 + x) * DV + j] : 0.f;
+            tmem_st16(tmem_addr(tbase, quad, P::T_S + col0), v);
+#pragma unroll
+            for (int x = 0; x < 16; ++x) v[x] = (quad == 0 && lane == 0) ? slot[D * DV + col0 + x] : 0.f;
+            tmem_st16(tmem_addr(tbase, quad, P::T_Z + col0), v);
+        }
+        tmem_st_wait();
+    }
+    bool bad = false;
+    if (!mbar_wait(&full[0], 0, kErrTmaLoad)) bad = true;
+    if (!bad && worker) {
+        phi_a(0);
+        phi_b(0);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    if (__syncthreads_or(bad)) bad = true;
+
+    for (int c = 0; c < nch && !bad; ++c) {
+        const int s = c % P::STAGES;
+        const uint32_t cp = c & 1;
+        unsigned char* qt = sm + s * P::STAGE;
+        unsigned char* kt = qt + P::QB;
+        unsigned char* vt = kt + P::KB;
+        unsigned char* kh = DECAY ? khat : kt;
+
+        if (issuer) {
             tc_fence_after();
-            const uint32_t qa = smem_u32(qt), ka = smem_u32(kt), va = smem_u32(vt);
+            if (c >= 1) {
+                for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (c - 1) * C, chain);
+                tma_store_commit();
+            }
+            const uint64_t dq = sdesc_sw128(smem_u32(qt), 16, 1024);      // K-major tiles
+            const uint64_t dk = sdesc_sw128(smem_u32(kt), 16, 1024);
+            const uint64_t dq32 = sdesc_sw128(smem_u32(q32), 16, 1024);
+            const uint64_t dones = sdesc_sw128(smem_u32(ones), 16, 1024);
+            const uint64_t dp = sdesc_sw128(smem_u32(ptil), 16, 1024);
+            const uint64_t dv_mn = sdesc_sw128(smem_u32(vt), TILE, 1024);  // MN-major tiles
+            const uint64_t dkh_mn = sdesc_sw128(smem_u32(kh), TILE, 1024);
             const uint32_t id1 = idesc_bf16_f32(64, 64, 0, 0);
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t off = (ks / 4) * TILE + (ks % 4) * 32;
-                mma_bf16(tbase + P::T_P, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), id1,
-                         ks > 0);
+                const uint32_t off = ((ks / 4) * TILE + (ks % 4) * 32) >> 4;
+                mma_bf16(tbase + P::T_P, dq + off, dk + off, id1, ks > 0);
             }
             mma_commit(bar_p);
-            const uint32_t id3 = idesc_bf16_f32(DV, 64, 1, 0);
-            const uint32_t oreg = DECAY ? P::T_OI : P::T_O;
+            // start-state read, tf32 with S^T / z row from TMEM (before MMA4 updates them)
+            const uint32_t id3 = idesc_tf32_f32(DV, 64, 0, 0);
+            const uint32_t id3d = idesc_tf32_f32(64, 64, 0, 0);
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint64_t a = sdesc_sw128(smem_u32(sbt) + ks * 2048, D * 128, 1024);
-                const uint64_t b = sdesc_sw128(qa + (ks / 4) * TILE + (ks % 4) * 32, 16, 1024);
-                mma_bf16(tbase + oreg, a, b, id3, ks > 0);
+            for (int ks = 0; ks < D / 8; ++ks) {
+                const uint64_t b = dq32 + (((ks / 4) * TILE + (ks % 4) * 32) >> 4);
+                mma_tf32_ts(tbase + P::T_O, tbase + P::T_S + ks * 8, b, id3, ks > 0);
+                mma_tf32_ts(tbase + P::T_DEN, tbase + P::T_Z + ks * 8, b, id3d, ks > 0);
             }
-            const uint32_t id4 = idesc_bf16_f32(D, DV, 1, 1);
-            const uint32_t kst_a = smem_u32(kst);
+            // state carry
+            const uint32_t id4 = idesc_bf16_f32(DV, D, 1, 1);
+            const uint32_t id4d = idesc_bf16_f32(64, D, 0, 1);
 #pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks)
-                mma_bf16(tbase + P::T_S, sdesc_sw128(kst_a + ks * 2048, TILE, 1024),
-                         sdesc_sw128(va + ks * 2048, TILE, 1024), id4, 1u);
+            for (int ks = 0; ks < C / 16; ++ks) {
+                const uint64_t bk = dkh_mn + ((ks * 2048) >> 4);
+                mma_bf16(tbase + P::T_S, dv_mn + ((ks * 2048) >> 4), bk, id4, 1u);
+                mma_bf16(tbase + P::T_Z, dones + ((ks * 32) >> 4), bk, id4d, 1u);
+            }
             mma_commit(bar_s);
             commits = c + 1;
-            // prefetch: the stage chunk c-1 used is free (its MMAs completed)
             if (c >= 1 && c - 1 + P::STAGES < nch) issue(c - 1 + P::STAGES);
-        }
-
-        // 3. scores -> P~ (mask, decay, bf16) and denominators
-        if (!mbar_wait(bar_p, cp, kErrMma)) bad = true;
-        tc_fence_after();
-        {
-            const int i = acc_row<64>(warp, lane);
-            float praw[64];
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, warp, P::T_P + g * 16), v);
-#pragma unroll
-                for (int x = 0; x < 16; ++x) praw[g * 16 + x] = v[x];
-            }
-            tmem_ld_wait();
-            if (i >= 0) {
-                float rs = 0.f;
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int j0 = cc * 8 + 2 * h;
-                        const float a = j0 <= i ? praw[j0] * dtab[i - j0] : 0.f;
-                        const float b = j0 + 1 <= i ? praw[j0 + 1] * dtab[i - j0 - 1] : 0.f;
-                        pk[h] = pack_bf16x2(a, b);
-                        const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[h]));
-                        rs += r.x + r.y;
-                    }
-                    *reinterpret_cast<uint4*>(ptil + sw128_offset(i, cc * 16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-                float qz = 0.f;
-#pragma unroll
-                for (int b = 0; b < D / 64; ++b)
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        const uint4 x = *reinterpret_cast<const uint4*>(qt + b * TILE + sw128_offset(i, cc * 16));
-                        const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h]));
-                            const int fi = b * 64 + cc * 8 + 2 * h;
-                            qz = fmaf(f.x, zc[fi], qz);
-                            qz = fmaf(f.y, zc[fi + 1], qz);
-                        }
-                    }
-                rden[i] = 1.f / (rs + qsc[i] * qz + eps);
-            }
-        }
-        if (tid == 0) tma_store_wait_read();   // staging tile free again
-        fence_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(bad)) { bad = true; break; }
-
-        // 4. MMA2: intra-chunk values
-        if (tid == 0) {
+            // intra-chunk values once the workers have written P~
+            if (!mbar_wait(pt_full, cp, kErrMma)) bad = true;
             tc_fence_after();
             const uint32_t id2 = idesc_bf16_f32(DV, 64, 1, 0);
-            const uint32_t va = smem_u32(vt), pa = smem_u32(ptil);
+            const uint32_t id2d = idesc_bf16_f32(64, 64, 0, 0);
 #pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks)
-                mma_bf16(tbase + P::T_O, sdesc_sw128(va + ks * 2048, TILE, 1024),
-                         sdesc_sw128(pa + ks * 32, 16, 1024), id2, (DECAY && ks == 0) ? 0u : 1u);
+            for (int ks = 0; ks < C / 16; ++ks) {
+                const uint64_t bp = dp + ((ks * 32) >> 4);
+                mma_bf16(tbase + P::T_O, dv_mn + ((ks * 2048) >> 4), bp, id2, 1u);
+                mma_bf16(tbase + P::T_DEN, dones + ((ks * 32) >> 4), bp, id2d, 1u);
+            }
             mma_commit(bar_o);
             commits_o = c + 1;
+            tma_store_wait_read();   // the staging tile may be rewritten
+            mbar_arrive(o_free);
         }
 
-        // 5. state carry done: bf16 copy of S for the next chunk's MMA3,
-        //    pre-scale for the next chunk's MMA4, normaliser update
-        if (!mbar_wait(bar_s, cp, kErrMma)) bad = true;
-        tc_fence_after();
-        {
-            const int f = acc_row<D>(warp, lane);
-            const float decn = (DECAY && c + 1 < nch) ? __expf((float)chunk_len(c + 1) * lam) : 1.f;
-#pragma unroll
-            for (int g = 0; g < DV / 16; ++g) {
+        if (worker) {
+            // scores -> P~: rows i (M=64 layout), columns split by warpgroup
+            if (!mbar_wait(bar_p, cp, kErrMma)) bad = true;
+            tc_fence_after();
+            {
+                const int i = acc_row<64>(quad, lane);
                 float v[16];
-                tmem_ld16(tmem_addr(tbase, warp, P::T_S + g * 16), v);
+                tmem_ld16(tmem_addr(tbase, quad, P::T_P + wg * 16), v);
                 tmem_ld_wait();
-                if (f >= 0) {
-                    uint4 c0, c1;
-                    c0.x = pack_bf16x2(v[0], v[1]); c0.y = pack_bf16x2(v[2], v[3]);
-                    c0.z = pack_bf16x2(v[4], v[5]); c0.w = pack_bf16x2(v[6], v[7]);
-                    c1.x = pack_bf16x2(v[8], v[9]); c1.y = pack_bf16x2(v[10], v[11]);
-                    c1.z = pack_bf16x2(v[12], v[13]); c1.w = pack_bf16x2(v[14], v[15]);
-                    unsigned char* blk = sbt + (g / 4) * (D * 128);
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(f, (g % 4) * 32)) = c0;
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(f, (g % 4) * 32 + 16)) = c1;
-                }
-                if (DECAY) {
+                if (i >= 0) {
+                    uint32_t pk[8];
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) v[x] *= decn;
-                    tmem_st16(tmem_addr(tbase, warp, P::T_S + g * 16), v);
-                }
-            }
-            if (DECAY) tmem_st_wait();
-            if (tid < D) {
-                const int b = tid / 64, col = tid % 64;
-                const unsigned char* base = kst + b * TILE;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int r = 0; r < C; ++r)
-                    acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + sw128_offset(r, col * 2)));
-                const float dec = DECAY ? __expf((float)n * lam) : 1.f;
-                zn[tid] = fmaf(dec, zc[tid], acc);
-            }
-        }
-        fence_async_smem();
-
-        // 6. outputs: o_i = (O_intra + gamma^(i+1) O_inter) / den_i -> staging -> TMA store
-        if (!mbar_wait(bar_o, cp, kErrMma)) bad = true;
-        tc_fence_after();
-        {
-            const int j = acc_row<DV>(warp, lane);
-            unsigned char* oblk = otil + (j >= 0 ? (j / 64) * TILE : 0);
-            const int jb = (j >= 0 ? (j % 64) : 0) * 2;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float v[16], w[16];
-                tmem_ld16(tmem_addr(tbase, warp, P::T_O + g * 16), v);
-                if (DECAY) tmem_ld16(tmem_addr(tbase, warp, P::T_OI + g * 16), w);
-                tmem_ld_wait();
-                if (j >= 0) {
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const int i = g * 16 + x;
-                        const float num = DECAY ? fmaf(qsc[i], w[x], v[x]) : v[x];
-                        *reinterpret_cast<__nv_bfloat16*>(oblk + sw128_offset(i, jb)) =
-                            __float2bfloat16_rn(num * rden[i]);
+                    for (int h = 0; h < 8; ++h) {
+                        const int j0 = wg * 16 + 2 * h;
+                        const float a = j0 <= i ? v[2 * h] * dtab[i - j0] : 0.f;
+                        const float b = j0 + 1 <= i ? v[2 * h + 1] * dtab[i - j0 - 1] : 0.f;
+                        pk[h] = pack_bf16x2(a, b);
                     }
+                    *reinterpret_cast<uint4*>(ptil + sw128_offset(i, wg * 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4*>(ptil + sw128_offset(i, wg * 32 + 16)) =
+                        make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pt_full);
+
+            // phi of the next chunk, overlapping the MMA batch of this one
+            const bool more = c + 1 < nch;
+            const bool move = more && needs_move(c + 1);
+            if (more) {
+                if (!mbar_wait(&full[(c + 1) % P::STAGES], ((c + 1) / P::STAGES) & 1, kErrTmaLoad)) bad = true;
+                else phi_a(c + 1);
+            }
+            // the state carry (and its reads of Q^ / K^) must be complete
+            if (!mbar_wait(bar_s, cp, kErrMma)) bad = true;
+            tc_fence_after();
+            if (move) {
+                frame_move((c + 1) * C);
+                ref = (c + 1) * C;
+            }
+            if (more) phi_b(c + 1);
+
+            // denominators: row 0 of the normaliser accumulator (lane 0, quadrant 0)
+            if (!mbar_wait(bar_o, cp, kErrMma)) bad = true;
+            tc_fence_after();
+            if (quad == 0) {
+                float v[16];
+                tmem_ld16(tmem_addr(tbase, 0, P::T_DEN + wg * 16), v);
+                tmem_ld_wait();
+                float mine = 0.f;
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    const float t = __shfl_sync(0xffffffffu, v[x], 0);
+                    if (lane == x) mine = t;
+                }
+                if (lane < 16) rden[wg * 16 + lane] = __frcp_rn(mine + eps);
+            }
+            named_bar(1 + wg, 128);   // this warpgroup's 16 denominators are in smem
+            if (!mbar_wait(o_free, cp, kErrMma)) bad = true;
+            // outputs o_i = O^T[:, i] / den_i -> staging tile; adjacent value
+            // columns are paired into one 4-byte store
+            {
+                const int j = acc_row<DV>(quad, lane);
+                float v[16];
+                tmem_ld16(tmem_addr(tbase, quad, P::T_O + wg * 16), v);
+                tmem_ld_wait();
+                unsigned char* oblk = otil + (j >= 0 ? (j / 64) * TILE : 0);
+                const int jb = (j >= 0 ? (j % 64) : 0) * 2;
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    const int i = wg * 16 + x;
+                    const float val = v[x] * rden[i];
+                    const float nxt = __shfl_down_sync(0xffffffffu, val, 1);
+                    if (j >= 0 && (j & 1) == 0)
+                        *reinterpret_cast<uint32_t*>(oblk + sw128_offset(i, jb)) = pack_bf16x2(val, nxt);
                 }
             }
         }
         fence_async_smem();
         tc_fence_before();
-        if (__syncthreads_or(bad)) { bad = true; break; }
-        if (tid == 0) {
-            for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + c * C, chain);
+        if (__syncthreads_or(bad)) { bad = true; break; }                         // B1
+    }
+    if (issuer) {
+        if (!bad && nch > 0) {
+            tc_fence_after();
+            for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (nch - 1) * C, chain);
             tma_store_commit();
         }
-    }
-    if (tid == 0) tma_store_wait_all();
-    if (bad && tid == 0) {
-        // Leave no copy or MMA in flight before releasing TMEM and exiting:
-        // wait (bounded) for every issued load not yet consumed and for the
-        // last commit of each MMA barrier.
-        for (int cc = loads_waited; cc < loads_issued; ++cc)
-            mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
-        if (commits > 0) {
-            const uint32_t last = (commits - 1) & 1;
-            mbar_wait(bar_p, last, kErrMma);
-            mbar_wait(bar_s, last, kErrMma);
-            if (commits_o > 0) mbar_wait(bar_o, (commits_o - 1) & 1, kErrMma);
+        tma_store_wait_all();
+        if (bad) {
+            // Leave no copy or MMA in flight before releasing TMEM and exiting:
+            // only the last STAGES loads can still be in flight.
+            for (int cc = max(0, loads_issued - P::STAGES); cc < loads_issued; ++cc)
+                mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
+            if (commits > 0) {
+                const uint32_t last = (commits - 1) & 1;
+                mbar_wait(bar_p, last, kErrMma);
+                mbar_wait(bar_s, last, kErrMma);
+                if (commits_o > 0) mbar_wait(bar_o, (commits_o - 1) & 1, kErrMma);
+            }
         }
     }
     tc_fence_before();
@@ -659,7 +743,7 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     const int sc = ChunkPlan<D, DV, DECAY>::BYTES;
     e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, sc);
     if (e != cudaSuccess) return e;
-    kc<<<units, kThreads, sc, a.stream>>>(mq, mk, mv, mo, a.gamma, ws, a.N, a.H, sg.G, sg.L, a.eps);
+    kc<<<units, kThreads + 32, sc, a.stream>>>(mq, mk, mv, mo, a.gamma, ws, a.N, a.H, sg.G, sg.L, a.eps);
     return cudaGetLastError();
 }
 
@@ -670,12 +754,22 @@ TcSegments tc_segments(int B, int H, int N, int d, int dv)
     (void)d; (void)dv;
     TcSegments s;
     const long long chains = (long long)B * H;
-    const long long target = 4LL * 148;  // about four CTAs per SM over the launch
-    long long L = chains > 0 ? (N * chains + target - 1) / target : N;
-    L = ((L + C - 1) / C) * C;
+    if (N <= 0 || chains <= 0) return s;
+    // One CTA per SM runs one segment at a time.  Prefer whole waves of long
+    // segments: G segments per chain with chains * G close to a multiple of
+    // the SM count, and segments of at most kMaxSeg tokens.
+    constexpr long long kSMs = 148, kMaxSeg = 4096;
+    long long G = 1, L = N;
+    for (long long waves = 1;; ++waves) {
+        G = waves * kSMs / chains;
+        if (G < 1) G = 1;
+        L = (N + G - 1) / G;
+        L = ((L + C - 1) / C) * C;
+        if (L <= kMaxSeg || L <= C) break;
+    }
     if (L < 2 * C) L = 2 * C;
     s.L = (int)L;
-    s.G = N > 0 ? (int)((N + L - 1) / L) : 0;
+    s.G = (int)((N + L - 1) / L);
     return s;
 }
 

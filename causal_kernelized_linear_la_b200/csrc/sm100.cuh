@@ -19,14 +19,17 @@ namespace sm100 {
 // la_prefill_check).  Non-zero: which wait gave up first.
 static __device__ unsigned int g_device_error = 0;
 
-// Each try_wait can suspend the thread for a while; this bounds a wait to
-// well under a second on B200 while never tripping on legitimate latency.
-constexpr uint32_t kSpinLimit = 1u << 24;
+// Each try_wait suspends the thread until the phase completes or a hinted
+// time (kSuspendNs) passes; kSpinLimit such waits bound a wait to about a
+// second, far above any legitimate latency.
+constexpr uint32_t kSuspendNs = 100000;
+constexpr uint32_t kSpinLimit = 10000;
 
 enum WaitSite : unsigned int {
     kErrTmaLoad = 1,
     kErrMma = 2,
     kErrLookback = 3,
+    kErrRange = 4,   // an input outside the range a kernel supports
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
@@ -52,15 +55,20 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes)
                  : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -165,6 +173,20 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::tf32 (fp32 containers, tf32
+// multiply, fp32 accumulate).  A is read from TMEM: lane = row, one 32-bit
+// column per K element.
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on an mbarrier once all previously issued tcgen05 ops of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar)
 {
@@ -180,6 +202,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
     return (1u << 4)            // D format: f32
            | (1u << 7)          // A format: bf16
            | (1u << 10)         // B format: bf16
+           | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::tf32 with fp32 D (A, B K-major unless flagged).
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N, int a_mn, int b_mn)
+{
+    return (1u << 4)            // D format: f32
+           | (2u << 7)          // A format: tf32
+           | (2u << 10)         // B format: tf32
            | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
 }
@@ -245,6 +277,12 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t byte_in_row)
 {
     return row * 128u + ((((byte_in_row >> 4) ^ (row & 7u)) << 4) | (byte_in_row & 15u));
+}
+
+// Named barrier over `count` threads (a multiple of 32), id 1..15.
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
