@@ -110,7 +110,10 @@ la_status la_prefill(const void* q, const void* k, const void* v,
     a.workspace = cfg->workspace; a.workspace_bytes = cfg->workspace_bytes;
 
     if (N == 0) return la::write_start_state(a);
-    if (delta) return la::from_cuda(la::launch_prefill_simt_gated_delta(a));
+    if (delta) {
+        if (a.dtype == LA_BF16 && a.dv % 64 == 0) return la::from_cuda(la::launch_prefill_tc_gated_delta(a));
+        return la::from_cuda(la::launch_prefill_simt_gated_delta(a));
+    }
     if (la::uses_tc_kernelized(a.dtype, a.mode)) return la::from_cuda(la::launch_prefill_tc_kernelized(a));
     return la::from_cuda(la::launch_prefill_simt_kernelized(a));
 }
@@ -210,7 +213,10 @@ la_status la_prefill_check(const void* workspace, void* stream)
     (void)workspace;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return LA_ERR_CUDA;
-    if (la::read_and_clear_device_error(s) != 0) return LA_ERR_TIMEOUT;
+    const unsigned int e1 = la::read_and_clear_device_error(s);
+    const unsigned int e2 = la::read_and_clear_device_error_gdelta(s);
+    if (e1 == 4u || e2 == 4u) return LA_ERR_UNSUPPORTED;
+    if (e1 != 0 || e2 != 0) return LA_ERR_TIMEOUT;
     return LA_OK;
 }
 

@@ -84,43 +84,6 @@ struct SummaryPlan {
     static constexpr uint32_t T_S = 0, T_Z = 128, T_COLS = 256;
 };
 
-__device__ __forceinline__ unsigned char* align1024(unsigned char* p)
-{
-    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// Row of an accumulator that this thread owns after tcgen05.ld.32x32b, for a
-// tile of M rows (M = 128: lane i = row i; M = 64: rows 16w..16w+15 live in
-// lanes 32w..32w+15).  `quad` is the warp's TMEM lane quadrant.  Returns -1
-// when the lane holds no row.
-template <int M>
-__device__ __forceinline__ int acc_row(int quad, int lane)
-{
-    if (M == 128) return quad * 32 + lane;
-    return lane < 16 ? quad * 16 + lane : -1;
-}
-
-__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, int quad, uint32_t col)
-{
-    return base + ((uint32_t)(quad * 32) << 16) + col;
-}
-
-__device__ __forceinline__ void unpack8(uint4 x, float (&f)[8])
-{
-    const uint32_t in[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[i]));
-        f[2 * i] = t.x;
-        f[2 * i + 1] = t.y;
-    }
-}
-
-__device__ __forceinline__ uint4 pack8(const float (&f)[8], float w)
-{
-    return make_uint4(pack_bf16x2(w * f[0], w * f[1]), pack_bf16x2(w * f[2], w * f[3]),
-                      pack_bf16x2(w * f[4], w * f[5]), pack_bf16x2(w * f[6], w * f[7]));
-}
 
 // Constant A operand: a 64 x 64 bf16 tile whose row 0 is all ones.  One MMA
 // with it sums the rows of a B operand into accumulator row 0.
@@ -700,6 +663,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
+}  // namespace
+
 // 3-D map over a bf16 [chains][N][inner] tensor; box = 64 elements x 64 rows,
 // 128-byte swizzle; rows past N read as zero and are not written.
 bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains)
@@ -714,6 +679,8 @@ bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains)
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int D, int DV, bool DECAY>
 cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)

@@ -1,6 +1,8 @@
 // Host-side interface of the tensor-core prefill kernels.
 #pragma once
 
+#include <cuda.h>
+
 #include "la_internal.cuh"
 
 namespace la {
@@ -20,6 +22,14 @@ cudaError_t launch_prefill_tc_kernelized(const PrefillArgs& a);
 constexpr size_t kNoAllocScratchBytes = 16u << 20;
 TcSegments tc_segments_noalloc(int B, int H, int N, int d, int dv);
 cudaError_t launch_prefill_tc_kernelized_noalloc(const PrefillArgs& a);
+
+// 3-D TMA map over a bf16 [chains][N][inner] tensor (box 64 x 64 rows,
+// 128-byte swizzle, zero fill past N).
+bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains);
+
+// Gated-delta prefill on the tensor cores (bf16 inputs).
+cudaError_t launch_prefill_tc_gated_delta(const PrefillArgs& a);
+unsigned int read_and_clear_device_error_gdelta(cudaStream_t stream);
 
 // Read (and clear) the device error word the tensor-core kernels set when a
 // bounded wait gives up.  Synchronises `stream`.

@@ -8,6 +8,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -289,6 +290,49 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// ---- tile and accumulator helpers shared by the tensor-core kernels -------
+
+// A 64-row x 128-byte swizzled tile: 64 tokens x 64 bf16 (or x 32 fp32).
+constexpr int kTileBytes = 64 * 128;
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p)
+{
+    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Row of an accumulator that this thread owns after tcgen05.ld.32x32b, for a
+// tile of M rows (M = 128: lane i = row i; M = 64: rows 16w..16w+15 live in
+// lanes 32w..32w+15).  `quad` is the warp's TMEM lane quadrant.  Returns -1
+// when the lane holds no row.
+template <int M>
+__device__ __forceinline__ int acc_row(int quad, int lane)
+{
+    if (M == 128) return quad * 32 + lane;
+    return lane < 16 ? quad * 16 + lane : -1;
+}
+
+__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, int quad, uint32_t col)
+{
+    return base + ((uint32_t)(quad * 32) << 16) + col;
+}
+
+__device__ __forceinline__ void unpack8(uint4 x, float (&f)[8])
+{
+    const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[i]));
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8], float w)
+{
+    return make_uint4(pack_bf16x2(w * f[0], w * f[1]), pack_bf16x2(w * f[2], w * f[3]),
+                      pack_bf16x2(w * f[4], w * f[5]), pack_bf16x2(w * f[6], w * f[7]));
 }
 
 }  // namespace sm100
