@@ -59,17 +59,25 @@ struct ChunkPlan {
     static constexpr int OFF_KH = STAGES * STAGE;                 // K^ (frame-weighted phi(K)), decay only
     static constexpr int OFF_Q32 = OFF_KH + (DECAY ? KB : 0);     // Q^ fp32 [C][D], tf32 operand
     static constexpr int OFF_P = OFF_Q32 + C * D * 4;             // P~ bf16 [C][C]
-    static constexpr int OFF_ONES = OFF_P + C * C * 2;            // bf16 [C][C], row 0 = 1
-    static constexpr int OFF_O = OFF_ONES + C * C * 2;            // output staging bf16 [C][DV]
-    static constexpr int OFF_RDEN = OFF_O + C * DV * 2;           // [C] 1 / denominator
+    // The ones-row A operand of the normaliser MMA: only its row 0 (128
+    // bytes) must hold ones; rows 1..63 feed accumulator rows that are never
+    // read, so they overlap the small vectors below and the staging tile.
+    static constexpr int OFF_ONES = OFF_P + C * C * 2;
+    static constexpr int OFF_RDEN = OFF_ONES + 128;               // [C] 1 / denominator
     static constexpr int OFF_DTAB = OFF_RDEN + C * 4;             // [C] gamma^k
-    static constexpr int OFF_BAR = OFF_DTAB + C * 4;
+    static constexpr int OFF_O = OFF_ONES + 1024;                 // output staging bf16 [C][DV]
+    static constexpr int OFF_RSP = OFF_O + C * DV * 2;            // [4][C] row sums of P~ per warpgroup
+    static constexpr int OFF_DINT = OFF_RSP + 4 * C * 4;          // [2][C] Q^ . z per chunk parity
+    static constexpr int OFF_ZS = OFF_DINT + 2 * C * 4;           // [2][D] z at chunk start per parity
+    static constexpr int OFF_BAR = OFF_ZS + 2 * D * 4;
     static constexpr int NBAR = STAGES + 5;                       // full[S], p, s, o, pt_full, o_free
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;            // + alignment slack
+    static_assert(OFF_DTAB + C * 4 <= OFF_O, "vectors overlap the staging tile");
+    static_assert(OFF_ONES + 8 * 1024 <= OFF_RSP, "ones operand must stay inside the plan");
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
-    // TMEM columns: scores, output^T, denominator row, state^T, normaliser row
-    static constexpr uint32_t T_P = 0, T_O = 64, T_DEN = 128, T_S = 256, T_Z = 384, T_COLS = 512;
+    // TMEM columns: scores, output^T, state^T, normaliser row
+    static constexpr uint32_t T_P = 0, T_O = 64, T_S = 128, T_Z = 256, T_COLS = 512;
 };
 
 template <int D, int DV>
@@ -167,7 +175,10 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             float f[8];
             unpack8(*p, f);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) f[x] = phi_fast(f[x]);
+            for (int x = 0; x < 8; x += 2) {
+                const float2 y = phi2_fast(f[x], f[x + 1]);
+                f[x] = y.x; f[x + 1] = y.y;
+            }
             *p = pack8(f, w);
         }
         fence_async_smem();
@@ -188,10 +199,12 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             if (c == nch - 1) mma_commit(done);
             commits = c + 1;
         }
+        // refill the stage chunk c-1 used: its MMA was issued a whole chunk ago
         __syncthreads();
-        if (tid == 0 && c + P::STAGES < nch) {
-            if (!mbar_wait(&empty[s], ph, kErrMma)) bad = true;
-            else issue(c + P::STAGES);
+        if (tid == 0 && c >= 1 && c - 1 + P::STAGES < nch) {
+            const int sp = (c - 1) % P::STAGES;
+            if (!mbar_wait(&empty[sp], ((c - 1) / P::STAGES) & 1, kErrMma)) bad = true;
+            else issue(c - 1 + P::STAGES);
         }
     }
     if (!bad && !mbar_wait(done, 0, kErrMma)) bad = true;
@@ -286,8 +299,9 @@ scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float
 // The state is kept transposed in TMEM (S^T: lane = value index, column =
 // key feature), exactly the layout of the A operand of a tf32 MMA, so the
 // start-state read of every chunk is an MMA straight out of TMEM and the
-// state never passes through the CUDA cores.  The normaliser rides along as
-// row 0 of two small accumulators fed by a constant "ones row" tile.
+// state never passes through the CUDA cores.  The normaliser z is carried as
+// row 0 of a small accumulator fed by a constant "ones row" tile; the
+// denominators (row sums of P~ plus Q^.z) are formed on the CUDA cores.
 //
 // Decay uses a scaled frame: with r the frame's reference position, the
 // stored state is T = gamma^-(c0 - r) S(c0-1) at chunk start c0, key rows are
@@ -297,13 +311,13 @@ scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float
 //
 // Roles: warps 0..15 ("workers") run the epilogues and phi; lane 0 of warp 16
 // ("issuer") issues TMA and every MMA.  Chunk c, from barrier B1:
-//   issuer:  store o(c-1); MMA1 P = phi(Q)phi(K)^T; MMA3 O^T = S^T Q^^T and
-//            MMA3d den = z.Q^ (tf32, A in TMEM); MMA4 S^T += V^T K^ and
-//            MMA4d z += 1^T K^; prefetch; [wait P~] MMA2 O^T += V^T P~^T,
-//            MMA2d den += 1^T P~^T; release the staging tile
-//   workers: [P ready] mask/decay -> P~, signal;  phi(c+1) in place (overlaps
-//            the MMA batch);  [state carry done] frame move, Q^/K^ of c+1;
-//            [outputs ready] 1/den, o = O^T/den -> staging tile      -> B1
+//   issuer:  store o(c-1); MMA1 P = phi(Q)phi(K)^T; MMA3 O^T = S^T Q^^T
+//            (tf32, A in TMEM); MMA4 S^T += V^T K^ and MMA4d z += 1^T K^;
+//            prefetch; [wait P~] MMA2 O^T += V^T P~^T; release the staging tile
+//   workers: [P ready] mask/decay -> P~ and its row sums, signal;  phi(c+1)
+//            in place (overlaps the MMA batch);  [state carry done] frame
+//            move, z of c+1, Q^/K^ of c+1 and Q^.z;  [outputs ready] 1/den,
+//            o = O^T/den -> staging tile                              -> B1
 template <int D, int DV, bool DECAY>
 __global__ void __launch_bounds__(kThreads + 32, 1)
 chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -322,6 +336,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     unsigned char* otil = sm + P::OFF_O;
     float* rden = reinterpret_cast<float*>(sm + P::OFF_RDEN);
     float* dtab = reinterpret_cast<float*>(sm + P::OFF_DTAB);
+    float* rsp = reinterpret_cast<float*>(sm + P::OFF_RSP);
+    float* dint = reinterpret_cast<float*>(sm + P::OFF_DINT);
+    float* zs = reinterpret_cast<float*>(sm + P::OFF_ZS);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* bar_p = full + P::STAGES;
     uint64_t* bar_s = bar_p + 1;
@@ -351,7 +368,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     if (warp == 0) tmem_alloc(tmem_slot, P::T_COLS);
     if (tid < C) dtab[tid] = DECAY ? __expf((float)tid * lam) : 1.f;   // gamma^(i-j)
-    if (worker) init_ones_tile(ones, tid, kThreads);
+    if (tid < 8) {
+        const uint32_t one2 = pack_bf16x2(1.f, 1.f);
+        reinterpret_cast<uint4*>(ones)[tid] = make_uint4(one2, one2, one2, one2);   // row 0 only
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -389,15 +409,23 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             unpack8(*pq, fq[u]);
             unpack8(*pk, fk[u]);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) { fq[u][x] = phi_fast(fq[u][x]); fk[u][x] = phi_fast(fk[u][x]); }
+            for (int x = 0; x < 8; x += 2) {
+                const float2 a = phi2_fast(fq[u][x], fq[u][x + 1]);
+                const float2 b = phi2_fast(fk[u][x], fk[u][x + 1]);
+                fq[u][x] = a.x; fq[u][x + 1] = a.y;
+                fk[u][x] = b.x; fk[u][x + 1] = b.y;
+            }
             *pq = pack8(fq[u], 1.f);
             *pk = pack8(fk[u], row < n ? 1.f : 0.f);
         }
     };
-    // part B: the frame-weighted operands Q^ (fp32, tf32 MMA) and K^ (bf16).
+    // part B: the frame-weighted operands Q^ (fp32, tf32 MMA) and K^ (bf16),
+    // and Q^ . z(c) for the denominators (8 consecutive threads share a row).
     auto phi_b = [&](int c) {
         const int n = chunk_len(c);
         const int c0 = c * C;
+        const float* zc = zs + (c & 1) * D;
+        float qz = 0.f;
 #pragma unroll
         for (int u = 0; u < NCHK; ++u) {
             const int e = tid + u * kThreads;
@@ -410,11 +438,17 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 make_float4(qw * fq[u][0], qw * fq[u][1], qw * fq[u][2], qw * fq[u][3]);
             *reinterpret_cast<float4*>(qrow + sw128_offset(row, fb + 16)) =
                 make_float4(qw * fq[u][4], qw * fq[u][5], qw * fq[u][6], qw * fq[u][7]);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) qz = fmaf(qw * fq[u][x], zc[f0 + x], qz);
             if (DECAY) {
                 const float kw = row < n ? __expf(-(float)(c0 + row + 1 - ref) * lam) : 0.f;
                 reinterpret_cast<uint4*>(khat + b * TILE)[rem] = pack8(fk[u], kw);
             }
         }
+        qz += __shfl_xor_sync(0xffffffffu, qz, 1);
+        qz += __shfl_xor_sync(0xffffffffu, qz, 2);
+        qz += __shfl_xor_sync(0xffffffffu, qz, 4);
+        if ((tid & 7) == 0) dint[(c & 1) * C + tid / 8] = qz;   // row tid/8 for every u
     };
     // Move the frame to position c0 (decay): S^T and z row times gamma^(c0 - ref).
     auto frame_move = [&](int c0) {
@@ -435,6 +469,24 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tmem_st16(tmem_addr(tbase, quad, P::T_Z + col0), v);
         }
         tmem_st_wait();
+    };
+    // z at the start of chunk c (row 0 of the normaliser accumulator, lane 0
+    // of quadrant 0) into zs[c & 1]; the caller synchronises the workers.
+    auto z_to_smem = [&](int c) {
+        if (quad == 0) {
+#pragma unroll
+            for (int gg = 0; gg < D / 64; ++gg) {
+                const int col0 = wg * (D / 4) + gg * 16;
+                float v[16];
+                tmem_ld16(tmem_addr(tbase, 0, P::T_Z + col0), v);
+                tmem_ld_wait();
+                if (lane == 0) {
+                    float4* dst = reinterpret_cast<float4*>(zs + (c & 1) * D + col0);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                }
+            }
+        }
     };
     auto needs_move = [&](int c) {
         if (!DECAY) return false;
@@ -461,6 +513,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tmem_st16(tmem_addr(tbase, quad, P::T_Z + col0), v);
         }
         tmem_st_wait();
+        if (tid < D) zs[tid] = slot[D * DV + tid];
+        named_bar(5, kThreads);
     }
     bool bad = false;
     if (!mbar_wait(&full[0], 0, kErrTmaLoad)) bad = true;
@@ -500,14 +554,12 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mma_bf16(tbase + P::T_P, dq + off, dk + off, id1, ks > 0);
             }
             mma_commit(bar_p);
-            // start-state read, tf32 with S^T / z row from TMEM (before MMA4 updates them)
+            // start-state read, tf32 with S^T from TMEM (before MMA4 updates it)
             const uint32_t id3 = idesc_tf32_f32(DV, 64, 0, 0);
-            const uint32_t id3d = idesc_tf32_f32(64, 64, 0, 0);
 #pragma unroll
             for (int ks = 0; ks < D / 8; ++ks) {
                 const uint64_t b = dq32 + (((ks / 4) * TILE + (ks % 4) * 32) >> 4);
                 mma_tf32_ts(tbase + P::T_O, tbase + P::T_S + ks * 8, b, id3, ks > 0);
-                mma_tf32_ts(tbase + P::T_DEN, tbase + P::T_Z + ks * 8, b, id3d, ks > 0);
             }
             // state carry
             const uint32_t id4 = idesc_bf16_f32(DV, D, 1, 1);
@@ -525,13 +577,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (!mbar_wait(pt_full, cp, kErrMma)) bad = true;
             tc_fence_after();
             const uint32_t id2 = idesc_bf16_f32(DV, 64, 1, 0);
-            const uint32_t id2d = idesc_bf16_f32(64, 64, 0, 0);
 #pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t bp = dp + ((ks * 32) >> 4);
-                mma_bf16(tbase + P::T_O, dv_mn + ((ks * 2048) >> 4), bp, id2, 1u);
-                mma_bf16(tbase + P::T_DEN, dones + ((ks * 32) >> 4), bp, id2d, 1u);
-            }
+            for (int ks = 0; ks < C / 16; ++ks)
+                mma_bf16(tbase + P::T_O, dv_mn + ((ks * 2048) >> 4), dp + ((ks * 32) >> 4), id2, 1u);
             mma_commit(bar_o);
             commits_o = c + 1;
             tma_store_wait_read();   // the staging tile may be rewritten
@@ -549,13 +597,17 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tmem_ld_wait();
                 if (i >= 0) {
                     uint32_t pk[8];
+                    float rs = 0.f;
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
                         const int j0 = wg * 16 + 2 * h;
                         const float a = j0 <= i ? v[2 * h] * dtab[i - j0] : 0.f;
                         const float b = j0 + 1 <= i ? v[2 * h + 1] * dtab[i - j0 - 1] : 0.f;
                         pk[h] = pack_bf16x2(a, b);
+                        const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[h]));
+                        rs += r.x + r.y;   // the row sum of exactly the values the MMA uses
                     }
+                    rsp[wg * C + i] = rs;
                     *reinterpret_cast<uint4*>(ptil + sw128_offset(i, wg * 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     *reinterpret_cast<uint4*>(ptil + sw128_offset(i, wg * 32 + 16)) =
                         make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -580,41 +632,46 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 frame_move((c + 1) * C);
                 ref = (c + 1) * C;
             }
-            if (more) phi_b(c + 1);
+            if (more) {
+                z_to_smem(c + 1);
+                named_bar(5, kThreads);   // z(c+1) and every row sum of P~(c) are in smem
+                phi_b(c + 1);
+            } else {
+                named_bar(5, kThreads);
+            }
 
             // denominators: row 0 of the normaliser accumulator (lane 0, quadrant 0)
             if (!mbar_wait(bar_o, cp, kErrMma)) bad = true;
             tc_fence_after();
-            if (quad == 0) {
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, 0, P::T_DEN + wg * 16), v);
-                tmem_ld_wait();
-                float mine = 0.f;
-#pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const float t = __shfl_sync(0xffffffffu, v[x], 0);
-                    if (lane == x) mine = t;
-                }
-                if (lane < 16) rden[wg * 16 + lane] = __frcp_rn(mine + eps);
+            if (quad == 0 && lane < 16) {
+                const int i = wg * 16 + lane;
+                const float den = rsp[i] + rsp[C + i] + rsp[2 * C + i] + rsp[3 * C + i] + dint[cp * C + i];
+                rden[i] = __frcp_rn(den + eps);
             }
             named_bar(1 + wg, 128);   // this warpgroup's 16 denominators are in smem
             if (!mbar_wait(o_free, cp, kErrMma)) bad = true;
-            // outputs o_i = O^T[:, i] / den_i -> staging tile; adjacent value
-            // columns are paired into one 4-byte store
+            // outputs o_i = O^T[:, i] / den_i -> staging tile (one value column per thread)
             {
                 const int j = acc_row<DV>(quad, lane);
-                float v[16];
+                float v[16], r[16];
                 tmem_ld16(tmem_addr(tbase, quad, P::T_O + wg * 16), v);
-                tmem_ld_wait();
-                unsigned char* oblk = otil + (j >= 0 ? (j / 64) * TILE : 0);
-                const int jb = (j >= 0 ? (j % 64) : 0) * 2;
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const int i = wg * 16 + x;
-                    const float val = v[x] * rden[i];
-                    const float nxt = __shfl_down_sync(0xffffffffu, val, 1);
-                    if (j >= 0 && (j & 1) == 0)
-                        *reinterpret_cast<uint32_t*>(oblk + sw128_offset(i, jb)) = pack_bf16x2(val, nxt);
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 t = reinterpret_cast<const float4*>(rden + wg * 16)[q4];
+                    r[4 * q4] = t.x; r[4 * q4 + 1] = t.y; r[4 * q4 + 2] = t.z; r[4 * q4 + 3] = t.w;
+                }
+                tmem_ld_wait();
+                if (j >= 0) {
+                    // element (i, j) of the swizzled staging tile: 16-byte chunk
+                    // (j % 64) / 8 of row i, XOR (i % 8); i % 8 == x % 8 here
+                    unsigned char* base = otil + (j / 64) * TILE + (j % 8) * 2;
+                    const int cj = (j % 64) >> 3;
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        const int i = wg * 16 + x;
+                        *reinterpret_cast<__nv_bfloat16*>(base + i * 128 + ((cj ^ (x & 7)) << 4)) =
+                            __float2bfloat16_rn(v[x] * r[x]);
+                    }
                 }
             }
         }

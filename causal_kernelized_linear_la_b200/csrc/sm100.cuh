@@ -9,6 +9,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -290,6 +291,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// elu(x) + 1 for a pair of values, the exponential of the non-positive part
+// evaluated two at a time by ex2.approx.f16x2: the argument min(x,0)*log2(e)
+// carries an 11-bit mantissa in fp16, finer than the bf16 rounding applied to
+// the result.  Arguments below fp16 range give 0, i.e. phi ~ e^x < 2^-24.
+__device__ __forceinline__ float2 phi2_fast(float x0, float x1)
+{
+    constexpr float kLog2e = 1.4426950408889634f;
+    const __half2 a = __floats2half2_rn(fminf(x0, 0.f) * kLog2e, fminf(x1, 0.f) * kLog2e);
+    uint32_t ai = *reinterpret_cast<const uint32_t*>(&a), ei;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(ei) : "r"(ai));
+    const float2 e = __half22float2(*reinterpret_cast<const __half2*>(&ei));
+    return make_float2(fmaxf(x0, 0.f) + e.x, fmaxf(x1, 0.f) + e.y);
 }
 
 // ---- tile and accumulator helpers shared by the tensor-core kernels -------
