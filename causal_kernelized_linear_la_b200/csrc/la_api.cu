@@ -65,6 +65,7 @@ size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_c
 {
     if (!cfg || B <= 0 || H <= 0 || N <= 0 || !la::head_ok(d) || !la::head_ok(dv)) return 0;
     if (la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return la::tc_workspace_bytes(B, H, N, d, dv);
+    if (cfg->dtype == LA_BF16 && cfg->mode == LA_GATED_DELTA) return la::gd_workspace_bytes(B, H, N, d, dv);
     return 0;
 }
 
@@ -111,7 +112,7 @@ la_status la_prefill(const void* q, const void* k, const void* v,
 
     if (N == 0) return la::write_start_state(a);
     if (delta) {
-        if (a.dtype == LA_BF16 && a.dv % 64 == 0) return la::from_cuda(la::launch_prefill_tc_gated_delta(a));
+        if (a.dtype == LA_BF16) return la::from_cuda(la::launch_prefill_tc_gated_delta(a));
         return la::from_cuda(la::launch_prefill_simt_gated_delta(a));
     }
     if (la::uses_tc_kernelized(a.dtype, a.mode)) return la::from_cuda(la::launch_prefill_tc_kernelized(a));

@@ -27,7 +27,9 @@ cudaError_t launch_prefill_tc_kernelized_noalloc(const PrefillArgs& a);
 // 128-byte swizzle, zero fill past N).
 bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains);
 
-// Gated-delta prefill on the tensor cores (bf16 inputs).
+// Gated-delta prefill on the tensor cores (bf16 inputs).  The workspace holds
+// the per-chunk operands the parallel pass hands to the sequential pass.
+size_t gd_workspace_bytes(int B, int H, int N, int d, int dv);
 cudaError_t launch_prefill_tc_gated_delta(const PrefillArgs& a);
 unsigned int read_and_clear_device_error_gdelta(cudaStream_t stream);
 

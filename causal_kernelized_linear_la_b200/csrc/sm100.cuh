@@ -307,6 +307,18 @@ __device__ __forceinline__ float2 phi2_fast(float x0, float x1)
     return make_float2(fmaxf(x0, 0.f) + e.x, fmaxf(x1, 0.f) + e.y);
 }
 
+// ---- cp.async (4-byte global -> shared) ---------------------------------------
+
+// Asynchronous 4-byte copy; src_bytes = 0 stores zero and reads nothing.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until this thread's cp.async groups are complete.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // ---- tile and accumulator helpers shared by the tensor-core kernels -------
 
 // A 64-row x 128-byte swizzled tile: 64 tokens x 64 bf16 (or x 32 fp32).

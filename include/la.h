@@ -127,7 +127,7 @@ LA_API la_status la_prefill(const void* q, const void* k, const void* v,
  * with one segment per chain, i.e. B*H*(d*dv + d)*4 > 16 MiB, is rejected with
  * LA_ERR_WORKSPACE before anything is launched.  Only cfg->dtype == LA_BF16
  * with LA_PLAIN or LA_DECAY is served (LA_ERR_UNSUPPORTED otherwise; the
- * other paths of la_prefill need no workspace at all).
+ * f32 paths need no workspace, and the gated delta rule's grows with N).
  *
  * All calls in one process share the array and it keeps the last call's
  * contents: calls whose work can overlap on the GPU (enqueued on different
@@ -144,9 +144,12 @@ LA_API la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
 /*
  * la_prefill_workspace_bytes -- device scratch la_prefill needs for these
  * sizes and this cfg (dtype, mode).  0 means no workspace is needed.  The
- * workspace carries per-segment state summaries between the kernels of one
- * call; its content need not be initialised and is dead after the call's
- * work completes.  Two calls in flight at once need two workspaces.
+ * workspace carries data between the kernels of one call: per-segment state
+ * summaries for bf16 LA_PLAIN / LA_DECAY, and for bf16 LA_GATED_DELTA the
+ * per-chunk operands (-W, T' and the masked score block, bf16, ceil(N/64)*64
+ * rows of d + 128 values per chain).  Its content need not be initialised and
+ * is dead after the call's work completes.  Two calls in flight at once need
+ * two workspaces.
  */
 LA_API size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_config* cfg);
 
