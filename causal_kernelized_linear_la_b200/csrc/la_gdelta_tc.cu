@@ -19,11 +19,16 @@
 //   gd_prep_kernel   every (chain, chunk) in parallel: the score blocks
 //                    [K;Q]K^T, A and P~, T = (I + A)^{-1} on the CUDA cores in
 //                    fp32 (blocked forward substitution), T', W = T' diag(b) K.
-//                    Writes -W, T' and P~ (bf16) to the workspace.
+//                    Writes -W, diag(b) Q, T' and P~ (bf16) to the workspace.
 //   gd_chain_kernel  one CTA per (chain, 64 value columns), chunks in order:
-//                    U = T' V + (-W) S and Q S, then P~ U and the state update,
-//                    all on the tensor cores; the CUDA cores only convert U and
-//                    S to bf16 operands, scale S by b_C and write the output.
+//                    U = T' V + (-W) S and diag(b) Q S, then P~ U and the state
+//                    update, all on the tensor cores; the CUDA cores only
+//                    convert U and S to bf16 operands, scale S by b_C and write
+//                    the output.  A tcgen05.mma costs about the same to issue
+//                    at M = 64 as at M = 128, so operands that share a B are
+//                    stacked into M = 128: [T'; 0] V, [-W; diag(b) Q] S and
+//                    [0; P~] U leave U in accumulator rows 0-63 and the whole
+//                    output in rows 64-127.
 // The columns of S evolve independently under the delta rule, so value tiles
 // need no communication.
 #include <algorithm>
@@ -45,6 +50,27 @@ constexpr int kThreads = 256;    // two warpgroups
 constexpr int TILE = kTileBytes; // 64 rows x 128 bytes
 // log alpha is clamped here so that alpha = 0 (a full reset) never forms inf - inf
 constexpr float kLogAlphaMin = -80.f;
+
+// fp32 -> tf32 (round to nearest, ties away) for the warp-level MMA below.
+__device__ __forceinline__ uint32_t to_tf32(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D (16x8, fp32) += A (16x8, tf32, row-major) * B (8x8, tf32, column-major):
+// the warp-level m16n8k8 MMA, used for the 16 x 16 block products of the
+// triangular solve (too small to fill a tcgen05 tile).  Fragments: with
+// g = lane / 4, t = lane % 4, a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]},
+// b = {B[t][g], B[t+4][g]}, d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
 // Within-chunk inclusive log decay for the two tokens 2*lane, 2*lane + 1 of a
 // chunk (one warp covers the chunk).  Tokens past the sequence end count as
@@ -80,9 +106,10 @@ struct PrepPlan {
     static constexpr int OFF_A = OFF_P + TILE;              // A fp32 [C][C+1]; later the -W staging tiles
     static constexpr int TS = C + 4;                        // row stride of T (16-byte aligned rows)
     static constexpr int OFF_TM = OFF_A + C * (C + 1) * 4;  // T fp32 [C][TS]
-    static constexpr int OFF_X = OFF_TM + C * TS * 4;       // off-diagonal scratch fp32 [3][16][16]
-    static constexpr int OFF_VEC = OFF_X + 3 * 16 * 16 * 4; // L[C], b[C], g[C], staged alpha/g [2][2][C]
-    static constexpr int OFF_BAR = OFF_VEC + 7 * C * 4;
+    static constexpr int OFF_X = OFF_TM + C * TS * 4;       // per-warp 16 x 8 block scratch, fp32 [8][16][9]
+    // L[C], b[C], g[C], staged alpha/g [2][2][C], e^{L-L_m}[C], e^{L_m-L}[C], flag
+    static constexpr int OFF_VEC = OFF_X + 8 * 16 * 9 * 4;
+    static constexpr int OFF_BAR = OFF_VEC + 9 * C * 4 + 16;
     static constexpr int OFF_TMEM = OFF_BAR + 3 * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(NB * TILE <= C * (C + 1) * 4, "-W staging fits over A");
@@ -94,8 +121,9 @@ struct PrepPlan {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_t,
-               const __grid_constant__ CUtensorMap tm_p, const float* __restrict__ alpha,
+               const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qb,
+               const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_p,
+               const float* __restrict__ alpha,
                const float* __restrict__ gate, int N, int chains)
 {
     using P = PrepPlan<D>;
@@ -113,6 +141,9 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float* bv = Lv + C;
     float* gv = Lv + 2 * C;
     float* avec = Lv + 3 * C;   // [2][2][C]: alpha, g of two work items
+    float* ef = Lv + 7 * C;     // e^{L_t - L_m}, m the chunk's middle token
+    float* eg = Lv + 8 * C;     // e^{L_m - L_t}
+    int* factored = reinterpret_cast<int*>(Lv + 9 * C);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* bar1 = full + 1;
     uint64_t* bar2 = full + 2;
@@ -204,6 +235,19 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             bv[2 * lane + 1] = __expf(Lb);
             gv[2 * lane] = av[C + 2 * lane];
             gv[2 * lane + 1] = av[C + 2 * lane + 1];
+            // e^{L_t - L_j} = e^{L_t - L_m} e^{L_m - L_j} while both factors stay finite
+            const float Lm = __shfl_sync(0xffffffffu, Lb, C / 4 - 1);
+            float lo = fminf(La, Lb), hi = fmaxf(La, Lb);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+            }
+            ef[2 * lane] = __expf(La - Lm);
+            ef[2 * lane + 1] = __expf(Lb - Lm);
+            eg[2 * lane] = __expf(Lm - La);
+            eg[2 * lane + 1] = __expf(Lm - Lb);
+            if (lane == 0) *factored = (hi - Lm <= 80.f && Lm - lo <= 80.f) ? 1 : 0;
             __syncwarp();
             if (next < items) stage_vectors(next, (it + 1) & 1);
         }
@@ -226,35 +270,60 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tmem_ld16(tmem_addr(tbase, quad, P::T_KQ + wg * 32), *reinterpret_cast<float(*)[16]>(v));
             tmem_ld16(tmem_addr(tbase, quad, P::T_KQ + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
             tmem_ld_wait();
+            const bool fact = *factored != 0;
             if (r < 64) {
-                const float gr = gv[r], Lr = Lv[r];
+                const float gr = gv[r], Lr = Lv[r], sr = gr * ef[r];
+                if (fact) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    const int j = wg * 32 + x;
-                    As[r * (C + 1) + j] = j < r ? gr * __expf(Lr - Lv[j]) * v[x] : 0.f;
+                    for (int x = 0; x < 32; ++x) {
+                        const int j = wg * 32 + x;
+                        As[r * (C + 1) + j] = j < r ? sr * eg[j] * v[x] : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                        const int j = wg * 32 + x;
+                        As[r * (C + 1) + j] = j < r ? gr * __expf(Lr - Lv[j]) * v[x] : 0.f;
+                    }
                 }
             } else {
                 const int i = r - 64;
-                const float Li = Lv[i];
+                const float Li = Lv[i], si = ef[i];
                 uint32_t pk[16];
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
                     const int j = wg * 32 + 2 * h;
-                    const float a = j <= i ? __expf(Li - Lv[j]) * v[2 * h] : 0.f;
-                    const float b = j + 1 <= i ? __expf(Li - Lv[j + 1]) * v[2 * h + 1] : 0.f;
+                    const float e0 = fact ? si * eg[j] : __expf(Li - Lv[j]);
+                    const float e1 = fact ? si * eg[j + 1] : __expf(Li - Lv[j + 1]);
+                    const float a = j <= i ? e0 * v[2 * h] : 0.f;
+                    const float b = j + 1 <= i ? e1 * v[2 * h + 1] : 0.f;
                     pk[h] = pack_bf16x2(a, b);
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     *reinterpret_cast<uint4*>(ptile + sw128_offset(i, wg * 64 + q * 16)) =
                         make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                // diag(b) Q in place for row i (M1, its reader, is complete).  The
+                // whole row takes one factor, so any chunk order works: rotating it
+                // by the row keeps the 32 rows of a warp on distinct banks.
+                const float bi = bv[i];
+#pragma unroll
+                for (int q = wg; q < NB * 8; q += 2) {
+                    const int chunk = (q + i) & 7;
+                    uint4* pq = reinterpret_cast<uint4*>(sm + (2 * (q / 8) + 1) * TILE + i * 128 + chunk * 16);
+                    float f[8];
+                    unpack8(*pq, f);
+                    *pq = pack8(f, bi);
+                }
             }
         }
         fence_async_smem();
         tc_fence_before();
         if (__syncthreads_or(bad)) { bad = true; break; }
-        // M1 is complete and Kb built: the K/Q tiles take the next item
-        if (tid == 0 && next < items) issue(next);
+        if (tid == 0) {
+            for (int b = 0; b < NB; ++b) tma_store_3d(&tm_qb, sm + (2 * b + 1) * TILE, b * 64, c * C, chain);
+            tma_store_commit();
+        }
 
         // T = (I + A)^{-1}: diagonal 16 x 16 blocks (one thread per column) ...
         constexpr int TSt = P::TS;
@@ -272,61 +341,65 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int i = 0; i < 16; ++i) Tm[(16 * a + i) * TSt + 16 * a + l] = x[i];
         }
         __syncthreads();
-        // ... then block diagonals k = 1..3: X_ab = sum_{c=b}^{a-1} A_ac T_cb, T_ab = -T_aa X_ab.
-        // A thread computes one row and four columns of a block (the A element
-        // it loads feeds four FMAs; rows of T are read as 16-byte vectors).
+        // ... then block diagonals k = 1..3: X_ab = sum_{c=b}^{a-1} A_ac T_cb and
+        // T_ab = -T_aa X_ab, as tf32 warp MMAs; warp w takes pair b = w / 2 of the
+        // level and the 8 columns (w % 2) of its block.
+        {
+            const int g = lane >> 2, t4 = lane & 3;
+            float* Xw = Xs + warp * 16 * 9;
 #pragma unroll
-        for (int k = 1; k <= 3; ++k) {
-            const int nblk = 4 - k;
-            const bool active = tid < nblk * 64;
-            const int b = tid / 64, a = b + k, i = (tid % 64) / 4, j0 = (tid % 4) * 4;
-            if (active) {
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int cc = 0; cc < 3; ++cc) {
-                    const int cb = b + cc;
-                    if (cc < k) {
-#pragma unroll
-                        for (int m = 0; m < 16; ++m) {
-                            const float av = As[(16 * a + i) * (C + 1) + 16 * cb + m];
-                            const float4 tv = *reinterpret_cast<const float4*>(&Tm[(16 * cb + m) * TSt + 16 * b + j0]);
-                            x.x = fmaf(av, tv.x, x.x);
-                            x.y = fmaf(av, tv.y, x.y);
-                            x.z = fmaf(av, tv.z, x.z);
-                            x.w = fmaf(av, tv.w, x.w);
-                        }
+            for (int k = 1; k <= 3; ++k) {
+                if (warp < 2 * (4 - k)) {
+                    const int b = warp >> 1, a = b + k, n0 = 16 * b + 8 * (warp & 1);
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int kc = 16 * b; kc < 16 * a; kc += 8) {
+                        const float* Ap = As + (16 * a) * (C + 1) + kc;
+                        const uint32_t af[4] = {to_tf32(Ap[g * (C + 1) + t4]), to_tf32(Ap[(g + 8) * (C + 1) + t4]),
+                                                to_tf32(Ap[g * (C + 1) + t4 + 4]),
+                                                to_tf32(Ap[(g + 8) * (C + 1) + t4 + 4])};
+                        const float* Bp = Tm + kc * TSt + n0;
+                        mma_16x8x8_tf32(x, af, to_tf32(Bp[t4 * TSt + g]), to_tf32(Bp[(t4 + 4) * TSt + g]));
                     }
-                }
-                *reinterpret_cast<float4*>(&Xs[(b * 16 + i) * 16 + j0]) = x;
-            }
-            __syncthreads();
-            if (active) {
-                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+                    Xw[g * 9 + 2 * t4] = x[0];
+                    Xw[g * 9 + 2 * t4 + 1] = x[1];
+                    Xw[(g + 8) * 9 + 2 * t4] = x[2];
+                    Xw[(g + 8) * 9 + 2 * t4 + 1] = x[3];
+                    __syncwarp();
+                    float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    if (m <= i) {
-                        const float tv = Tm[(16 * a + i) * TSt + 16 * a + m];
-                        const float4 xv = *reinterpret_cast<const float4*>(&Xs[(b * 16 + m) * 16 + j0]);
-                        y.x = fmaf(tv, xv.x, y.x);
-                        y.y = fmaf(tv, xv.y, y.y);
-                        y.z = fmaf(tv, xv.z, y.z);
-                        y.w = fmaf(tv, xv.w, y.w);
+                    for (int kk = 0; kk < 16; kk += 8) {
+                        const float* Ap = Tm + (16 * a) * TSt + 16 * a + kk;
+                        const uint32_t af[4] = {to_tf32(Ap[g * TSt + t4]), to_tf32(Ap[(g + 8) * TSt + t4]),
+                                                to_tf32(Ap[g * TSt + t4 + 4]), to_tf32(Ap[(g + 8) * TSt + t4 + 4])};
+                        mma_16x8x8_tf32(y, af, to_tf32(Xw[(kk + t4) * 9 + g]), to_tf32(Xw[(kk + t4 + 4) * 9 + g]));
                     }
+                    float* Dp = Tm + (16 * a) * TSt + n0;
+                    Dp[g * TSt + 2 * t4] = -y[0];
+                    Dp[g * TSt + 2 * t4 + 1] = -y[1];
+                    Dp[(g + 8) * TSt + 2 * t4] = -y[2];
+                    Dp[(g + 8) * TSt + 2 * t4 + 1] = -y[3];
+                    __syncwarp();
                 }
-                *reinterpret_cast<float4*>(&Tm[(16 * a + i) * TSt + 16 * b + j0]) =
-                    make_float4(-y.x, -y.y, -y.z, -y.w);
+                __syncthreads();
             }
-            __syncthreads();
+        }
+        // the diag(b) Q store has long read its tiles: K/Q take the next item
+        if (tid == 0 && next < items) {
+            tma_store_wait_read();
+            issue(next);
         }
         // T' = T diag(g), bf16, K-major A operand of M2 (T is unit lower triangular)
         for (int e = tid; e < C * 8; e += kThreads) {
             const int i = e / 8, cc = e % 8;
+            const float4 t0 = *reinterpret_cast<const float4*>(&Tm[i * TSt + cc * 8]);
+            const float4 t1 = *reinterpret_cast<const float4*>(&Tm[i * TSt + cc * 8 + 4]);
+            const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
             uint32_t pk[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 const int j = cc * 8 + 2 * h;
-                const float a = j <= i ? Tm[i * TSt + j] * gv[j] : 0.f;
-                const float b = j + 1 <= i ? Tm[i * TSt + j + 1] * gv[j + 1] : 0.f;
+                const float a = j <= i ? tv[2 * h] * gv[j] : 0.f;
+                const float b = j + 1 <= i ? tv[2 * h + 1] * gv[j + 1] : 0.f;
                 pk[h] = pack_bf16x2(a, b);
             }
             *reinterpret_cast<uint4*>(ttile + sw128_offset(i, cc * 16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -356,20 +429,22 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         {
             const int i = acc_row<64>(quad, lane);
 #pragma unroll
-            for (int gg = 0; gg < D / 32; ++gg) {
+            for (int gg = 0; gg < D / 32; gg += 2) {
                 const int col0 = wg * (D / 2) + gg * 16;
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_W + col0), v);
+                float v[32];
+                tmem_ld16(tmem_addr(tbase, quad, P::T_W + col0), *reinterpret_cast<float(*)[16]>(v));
+                tmem_ld16(tmem_addr(tbase, quad, P::T_W + col0 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
                 tmem_ld_wait();
                 if (i >= 0) {
                     unsigned char* blk = wstage + (col0 / 64) * TILE;
                     const int byte0 = (col0 % 64) * 2;
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(i, byte0)) =
-                        make_uint4(pack_bf16x2(-v[0], -v[1]), pack_bf16x2(-v[2], -v[3]), pack_bf16x2(-v[4], -v[5]),
-                                   pack_bf16x2(-v[6], -v[7]));
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(i, byte0 + 16)) =
-                        make_uint4(pack_bf16x2(-v[8], -v[9]), pack_bf16x2(-v[10], -v[11]),
-                                   pack_bf16x2(-v[12], -v[13]), pack_bf16x2(-v[14], -v[15]));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float* w = v + 8 * q;
+                        *reinterpret_cast<uint4*>(blk + sw128_offset(i, byte0 + 16 * q)) =
+                            make_uint4(pack_bf16x2(-w[0], -w[1]), pack_bf16x2(-w[2], -w[3]),
+                                       pack_bf16x2(-w[4], -w[5]), pack_bf16x2(-w[6], -w[7]));
+                    }
                 }
             }
         }
@@ -404,27 +479,33 @@ template <int D>
 struct ChainPlan {
     static constexpr int STAGES = 2;
     static constexpr int NB = D / 64;
-    // stage: K[NB] Q[NB] -W[NB] T' P~ V
-    static constexpr int O_K = 0, O_Q = NB * TILE, O_W = 2 * NB * TILE, O_T = 3 * NB * TILE;
-    static constexpr int O_P = O_T + TILE, O_V = O_P + TILE;
-    static constexpr int STAGE = O_V + TILE;                // all of it arrives by TMA
+    // stage: K[NB] | -W_0 Qb_0 -W_1 Qb_1 ... | T' Z P~ | V   (Z: a zero tile, never loaded)
+    // [-W_b; Qb_b], [T'; Z] and [Z; P~] are M = 128 K-major A operands.
+    static constexpr int O_K = 0, O_WQ = NB * TILE, O_T = 3 * NB * TILE;
+    static constexpr int O_Z = O_T + TILE, O_P = O_Z + TILE, O_V = O_P + TILE;
+    static constexpr int STAGE = O_V + TILE;
+    static constexpr int LOAD_BYTES = STAGE - TILE;         // all but Z arrives by TMA
     static constexpr int OFF_SB = STAGES * STAGE;           // S bf16 [D][64], MN-major B operand
     static constexpr int OFF_U = OFF_SB + NB * TILE;        // U bf16 [C][64], MN-major B operand
     static constexpr int OFF_UH = OFF_U + TILE;             // diag(b_C / b) U
     static constexpr int OFF_O = OFF_UH + TILE;             // output staging
-    static constexpr int OFF_VEC = OFF_O + TILE;            // b[3][C], r[3][C], staged alpha [2][C]
-    static constexpr int OFF_BAR = OFF_VEC + 8 * C * 4;
-    static constexpr int NBAR = STAGES + 2;
+    static constexpr int OFF_VEC = OFF_O + TILE;            // r[3][C], staged alpha [2][C], b_C [3]
+    static constexpr int OFF_BAR = OFF_VEC + 6 * C * 4 + 16;
+    // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready s_ready ostage_full ostage_empty drain
+    static constexpr int NBAR = 16;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
-    // TMEM columns: U, Q S (two buffers), P~ U (two buffers), state (rows = key feature)
-    static constexpr uint32_t T_U = 0, T_O1 = 64, T_O2 = 192, T_S = 320, T_COLS = 512;
+    // TMEM columns: [U; O] (M = 128, two buffers), state (rows = key feature)
+    static constexpr uint32_t T_UO = 0, T_S = 128, T_COLS = 256;
 };
 
+constexpr int kConv = 256;                   // converter threads (warps 0-7)
+constexpr int kChainThreads = kConv + 64;    // + MMA issuer warp 8 + TMA warp 9
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(kChainThreads, 1)
+gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                 const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_p,
                 const __grid_constant__ CUtensorMap tm_o, const float* __restrict__ alpha,
@@ -438,304 +519,313 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     unsigned char* utile = sm + P::OFF_U;
     unsigned char* uhtile = sm + P::OFF_UH;
     unsigned char* ostage = sm + P::OFF_O;
-    float* vb_b = reinterpret_cast<float*>(sm + P::OFF_VEC);   // [3][C] b_i
-    float* vb_r = vb_b + 3 * C;                                // [3][C] b_C / b_i
-    float* abuf = vb_b + 6 * C;                                // [2][C] staged alpha
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
-    uint64_t* bar3 = full + P::STAGES;
-    uint64_t* bar4 = bar3 + 1;
+    float* vb_r = reinterpret_cast<float*>(sm + P::OFF_VEC);   // [3][C] b_C / b_i
+    float* abuf = vb_r + 3 * C;                                // [2][C] staged alpha
+    float* vb_c = vb_r + 5 * C;                                // [3] b_C
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
+    uint64_t* full = bars;          // TMA -> issuer, per stage
+    uint64_t* empty = bars + 2;     // issuer (commit) -> TMA, per stage
+    uint64_t* uo_full = bars + 4;   // issuer: [U; Qb S] complete, per TMEM buffer
+    uint64_t* o_full = bars + 6;    // issuer: output accumulator complete, per TMEM buffer
+    uint64_t* o_read = bars + 8;    // converters: output accumulator read, per TMEM buffer
+    uint64_t* s_full = bars + 10;   // issuer: state update complete
+    uint64_t* u_ready = bars + 11;  // converters: U operands written, state scaled
+    uint64_t* s_ready = bars + 12;  // converters: bf16 state written
+    uint64_t* os_full = bars + 13;  // converters: output staging written
+    uint64_t* os_empty = bars + 14; // TMA: output staging read by its store
+    uint64_t* drain = bars + 15;    // issuer: every MMA it issued is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, wg = warp >> 2;
+    const int quad = warp & 3, wg = (warp >> 2) & 1;
     const int ntile = dv / DVT;
     const int chain = blockIdx.x / ntile, j0 = (blockIdx.x % ntile) * DVT;
     const int nch = (N + C - 1) / C;
-    const float* al = alpha + (size_t)chain * N;
-    const uint64_t pol_once = policy_evict_first();
-    const uint64_t pol_shared = ntile > 1 ? policy_evict_normal() : policy_evict_first();
 
     if (tid == 0) {
-        for (int s = 0; s < P::NBAR; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&uo_full[s], 1);
+            mbar_init(&o_full[s], 1);
+            mbar_init(&o_read[s], 128);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(u_ready, kConv);
+        mbar_init(s_ready, kConv);
+        mbar_init(os_full, 128);
+        mbar_init(os_empty, 1);
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
+    // zero tiles of both stages (rows 64-127 of [T'; Z], rows 0-63 of [Z; P~])
+    for (int s = 0; s < P::STAGES; ++s)
+        for (int e = tid; e < TILE / 16; e += kChainThreads)
+            reinterpret_cast<uint4*>(sm + s * P::STAGE + P::O_Z)[e] = make_uint4(0u, 0u, 0u, 0u);
     if (warp == 0) tmem_alloc(tmem_slot, P::T_COLS);
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
-    int loads_issued = 0, commits3 = 0, commits4 = 0;
-    auto issue = [&](int c) {
-        const int s = c % P::STAGES;
-        unsigned char* st = sm + s * P::STAGE;
-        const int y = c * C;
-        mbar_expect_tx(&full[s], P::STAGE);
-        for (int b = 0; b < NB; ++b) {
-            tma_load_3d(st + P::O_K + b * TILE, &tm_k, b * 64, y, chain, &full[s], pol_shared);
-            tma_load_3d(st + P::O_Q + b * TILE, &tm_q, b * 64, y, chain, &full[s], pol_shared);
-            tma_load_3d(st + P::O_W + b * TILE, &tm_w, b * 64, y, chain, &full[s], pol_shared);
+    if (warp == 9) {
+        // ---------------- TMA: stage loads and output stores ----------------
+        if (lane == 0) {
+            const uint64_t pol_once = policy_evict_first();
+            const uint64_t pol_shared = ntile > 1 ? policy_evict_normal() : policy_evict_first();
+            int loads = 0, stores = 0;
+            auto issue = [&](int c) {
+                const int s = c % P::STAGES;
+                unsigned char* st = sm + s * P::STAGE;
+                const int y = c * C;
+                mbar_expect_tx(&full[s], P::LOAD_BYTES);
+                for (int b = 0; b < NB; ++b) {
+                    tma_load_3d(st + P::O_K + b * TILE, &tm_k, b * 64, y, chain, &full[s], pol_shared);
+                    tma_load_3d(st + P::O_WQ + (2 * b) * TILE, &tm_w, b * 64, y, chain, &full[s], pol_shared);
+                    tma_load_3d(st + P::O_WQ + (2 * b + 1) * TILE, &tm_qb, b * 64, y, chain, &full[s], pol_shared);
+                }
+                tma_load_3d(st + P::O_T, &tm_t, 0, y, chain, &full[s], pol_shared);
+                tma_load_3d(st + P::O_P, &tm_p, 0, y, chain, &full[s], pol_shared);
+                tma_load_3d(st + P::O_V, &tm_v, j0, y, chain, &full[s], pol_once);
+                loads = c + 1;
+            };
+            auto store = [&](int c) {
+                tma_store_3d(&tm_o, ostage, j0, c * C, chain);
+                tma_store_commit();
+                tma_store_wait_read();
+                mbar_arrive(os_empty);
+                stores = c + 1;
+            };
+            for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                if (c >= 1) {
+                    ok = mbar_wait(os_full, (c - 1) & 1, kErrMma);
+                    if (!ok) break;
+                    store(c - 1);
+                }
+                if (c + P::STAGES < nch) {
+                    ok = mbar_wait(&empty[c % P::STAGES], (c / P::STAGES) & 1, kErrMma);
+                    if (ok) issue(c + P::STAGES);
+                }
+            }
+            if (ok && mbar_wait(os_full, (nch - 1) & 1, kErrMma)) store(nch - 1);
+            tma_store_wait_all();
+            // loads in flight must land before the block exits
+            for (int c = max(0, loads - P::STAGES); c < loads; ++c)
+                mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad);
+            (void)stores;
         }
-        tma_load_3d(st + P::O_T, &tm_t, 0, y, chain, &full[s], pol_shared);
-        tma_load_3d(st + P::O_P, &tm_p, 0, y, chain, &full[s], pol_shared);
-        tma_load_3d(st + P::O_V, &tm_v, j0, y, chain, &full[s], pol_once);
-        loads_issued = c + 1;
-    };
-    // warp 1: alpha of chunk c into staging buffer c & 1
-    auto stage_alpha = [&](int c) {
-        float* dst = abuf + (c & 1) * C;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int j = 2 * lane + h, t = c * C + j;
-            const bool ok = t < N;
-            cp_async4(dst + j, ok ? al + t : al, ok ? 4u : 0u);
-        }
-        cp_async_commit();
-    };
-    // warp 1: b_i and b_C / b_i of chunk c into vector buffer c % 3
-    auto chunk_vectors = [&](int c) {
-        cp_async_wait_all();
-        const float* a = abuf + (c & 1) * C;
-        const int t = c * C + 2 * lane;
-        float La, Lb, Lc;
-        chunk_logdecay(a[2 * lane], a[2 * lane + 1], t < N, t + 1 < N, lane, La, Lb, Lc);
-        float* b = vb_b + (c % 3) * C;
-        float* r = vb_r + (c % 3) * C;
-        b[2 * lane] = __expf(La);
-        b[2 * lane + 1] = __expf(Lb);
-        r[2 * lane] = __expf(Lc - La);
-        r[2 * lane + 1] = __expf(Lc - Lb);
         __syncwarp();
-    };
-    // output rows of chunk cc: o_i = b_i (Q S)_i + (P~ U)_i  -> bf16 staging
-    auto output_tile = [&](int cc) {
-        const int i = acc_row<64>(quad, lane);
-        const float* b = vb_b + (cc % 3) * C;
-        const float bi = i >= 0 ? b[i] : 0.f;
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-            const int col0 = wg * 32 + gg * 16;
-            float x1[16], x2[16];
-            tmem_ld16(tmem_addr(tbase, quad, P::T_O1 + (cc & 1) * 64 + col0), x1);
-            tmem_ld16(tmem_addr(tbase, quad, P::T_O2 + (cc & 1) * 64 + col0), x2);
-            tmem_ld_wait();
-            if (i >= 0) {
-                float o[16];
-#pragma unroll
-                for (int x = 0; x < 16; ++x) o[x] = fmaf(bi, x1[x], x2[x]);
-                *reinterpret_cast<uint4*>(ostage + sw128_offset(i, col0 * 2)) =
-                    make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                               pack_bf16x2(o[6], o[7]));
-                *reinterpret_cast<uint4*>(ostage + sw128_offset(i, col0 * 2 + 16)) =
-                    make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
-                               pack_bf16x2(o[14], o[15]));
-            }
-        }
-    };
-
-    if (tid == 0)
-        for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
-    if (warp == 1) {
-        stage_alpha(0);
-        chunk_vectors(0);
-        if (nch > 1) stage_alpha(1);
-    }
-
-    // start state slice S[:, j0:j0+64] into TMEM (rows = key feature) and bf16 smem
-    {
-        const int f = acc_row<D>(quad, lane);
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-            const int col0 = wg * 32 + gg * 16;
-            float v[16];
-#pragma unroll
-            for (int x = 0; x < 16; ++x)
-                v[x] = (f >= 0 && S0) ? S0[((size_t)chain * D + f) * dv + j0 + col0 + x] : 0.f;
-            if (f >= 0) {
-                *reinterpret_cast<uint4*>(sbt + sw128_offset(f, col0 * 2)) =
-                    make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                               pack_bf16x2(v[6], v[7]));
-                *reinterpret_cast<uint4*>(sbt + sw128_offset(f, col0 * 2 + 16)) =
-                    make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                               pack_bf16x2(v[14], v[15]));
-            }
-            tmem_st16(tmem_addr(tbase, quad, P::T_S + col0), v);
-        }
-        tmem_st_wait();
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    bool bad = false;
-    for (int c = 0; c < nch; ++c) {
-        const int s = c % P::STAGES;
-        const uint32_t cp = c & 1;
-        unsigned char* st = sm + s * P::STAGE;
-
-        // U = T' V + (-W) S;  Q S  (both read the bf16 copy of S)
-        if (tid == 0) {
-            if (!mbar_wait(&full[s], (c / P::STAGES) & 1, kErrTmaLoad)) {
-                bad = true;
-            } else {
+    } else if (warp == 8) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                const int s = c % P::STAGES;
+                const uint32_t cp = c & 1;
+                unsigned char* st = sm + s * P::STAGE;
+                const uint32_t tuo = tbase + P::T_UO + cp * 64;
+                const uint32_t id = idesc_bf16_f32(128, 64, 0, 1);
+                ok = mbar_wait(&full[s], (c / P::STAGES) & 1, kErrTmaLoad);
+                if (ok && c >= 2) ok = mbar_wait(&o_read[cp], ((c - 2) / 2) & 1, kErrMma);
+                if (!ok) break;
                 tc_fence_after();
-                const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
+                // [U; O] = [T'; 0] V
                 const uint64_t dt = sdesc_sw128(smem_u32(st + P::O_T), 16, 1024);
                 const uint64_t dvv = sdesc_sw128(smem_u32(st + P::O_V), TILE, 1024);
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tbase + P::T_U, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id, ks > 0);
-                const uint64_t dw = sdesc_sw128(smem_u32(st + P::O_W), 16, 1024);
-                const uint64_t dq = sdesc_sw128(smem_u32(st + P::O_Q), 16, 1024);
+                    mma_bf16(tuo, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id, ks > 0);
+                // [U; O] += [-W; Qb] S once the bf16 state is in place
+                ok = mbar_wait(s_ready, c & 1, kErrMma);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t dwq = sdesc_sw128(smem_u32(st + P::O_WQ), 16, 1024);
                 const uint64_t ds = sdesc_sw128(smem_u32(sbt), TILE, 1024);
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = ((ks / 4) * TILE + (ks % 4) * 32) >> 4;
-                    const uint64_t b = ds + ((ks * 2048) >> 4);
-                    mma_bf16(tbase + P::T_U, dw + off, b, id, 1u);
-                    mma_bf16(tbase + P::T_O1 + cp * 64, dq + off, b, id, ks > 0);
-                }
-                mma_commit(bar3);
-                commits3 = c + 1;
-            }
-        }
-        // S *= b_C in TMEM (the MMAs above read only the bf16 copy)
-        {
-            const float bc = vb_b[(c % 3) * C + C - 1];
+                for (int ks = 0; ks < D / 16; ++ks)
+                    mma_bf16(tuo, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4), ds + ((ks * 2048) >> 4), id,
+                             1u);
+                mma_commit(&uo_full[cp]);
+                // S += K^T diag(b_C / b) U, then O += [0; P~] U
+                ok = mbar_wait(u_ready, c & 1, kErrMma);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t ids = idesc_bf16_f32(D, 64, 1, 1);
+                const uint64_t dk = sdesc_sw128(smem_u32(st + P::O_K), TILE, 1024);
+                const uint64_t duh = sdesc_sw128(smem_u32(uhtile), TILE, 1024);
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-                const int col0 = wg * 32 + gg * 16;
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_S + col0), v);
-                tmem_ld_wait();
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tbase + P::T_S, dk + ((ks * 2048) >> 4), duh + ((ks * 2048) >> 4), ids, 1u);
+                mma_commit(s_full);
+                const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
+                const uint64_t du = sdesc_sw128(smem_u32(utile), TILE, 1024);
 #pragma unroll
-                for (int x = 0; x < 16; ++x) v[x] *= bc;
-                tmem_st16(tmem_addr(tbase, quad, P::T_S + col0), v);
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tuo, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, 1u);
+                mma_commit(&o_full[cp]);
+                mma_commit(&empty[s]);
             }
-            tmem_st_wait();
+            // every MMA issued must complete before TMEM is released
+            mma_commit(drain);
+            mbar_wait(drain, 0, kErrMma);
         }
-        // output of the previous chunk (its accumulators are complete)
-        if (c >= 1) output_tile(c - 1);
-        if (warp == 1 && c + 1 < nch) {
-            chunk_vectors(c + 1);
-            if (c + 2 < nch) stage_alpha(c + 2);
-        }
-
-        // U -> bf16 (MN-major B operand) and diag(b_C / b) U
-        if (!mbar_wait(bar3, cp, kErrMma)) bad = true;
-        tc_fence_after();
-        {
-            const int i = acc_row<64>(quad, lane);
-            const float ri = i >= 0 ? vb_r[(c % 3) * C + i] : 0.f;
+        __syncwarp();
+    } else {
+        // ---------------- converters (warps 0-7) ----------------
+        const float* al = alpha + (size_t)chain * N;
+        // warp 1: alpha of chunk c into staging buffer c & 1
+        auto stage_alpha = [&](int c) {
+            float* dst = abuf + (c & 1) * C;
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-                const int col0 = wg * 32 + gg * 16;
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_U + col0), v);
-                tmem_ld_wait();
-                if (i >= 0) {
-                    *reinterpret_cast<uint4*>(utile + sw128_offset(i, col0 * 2)) =
-                        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                   pack_bf16x2(v[6], v[7]));
-                    *reinterpret_cast<uint4*>(utile + sw128_offset(i, col0 * 2 + 16)) =
-                        make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                                   pack_bf16x2(v[14], v[15]));
-                    *reinterpret_cast<uint4*>(uhtile + sw128_offset(i, col0 * 2)) =
-                        make_uint4(pack_bf16x2(ri * v[0], ri * v[1]), pack_bf16x2(ri * v[2], ri * v[3]),
-                                   pack_bf16x2(ri * v[4], ri * v[5]), pack_bf16x2(ri * v[6], ri * v[7]));
-                    *reinterpret_cast<uint4*>(uhtile + sw128_offset(i, col0 * 2 + 16)) =
-                        make_uint4(pack_bf16x2(ri * v[8], ri * v[9]), pack_bf16x2(ri * v[10], ri * v[11]),
-                                   pack_bf16x2(ri * v[12], ri * v[13]), pack_bf16x2(ri * v[14], ri * v[15]));
-                }
+            for (int h = 0; h < 2; ++h) {
+                const int j = 2 * lane + h, t = c * C + j;
+                const bool ok = t < N;
+                cp_async4(dst + j, ok ? al + t : al, ok ? 4u : 0u);
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(bad)) { bad = true; break; }
-
-        // P~ U (onto its own accumulator);  S += K^T diag(b_C / b) U
-        if (tid == 0) {
+            cp_async_commit();
+        };
+        // warp 1: b_C / b_i and b_C of chunk c into vector buffer c % 3
+        auto chunk_vectors = [&](int c) {
+            cp_async_wait_all();
+            const float* a = abuf + (c & 1) * C;
+            const int t = c * C + 2 * lane;
+            float La, Lb, Lc;
+            chunk_logdecay(a[2 * lane], a[2 * lane + 1], t < N, t + 1 < N, lane, La, Lb, Lc);
+            float* r = vb_r + (c % 3) * C;
+            r[2 * lane] = __expf(Lc - La);
+            r[2 * lane + 1] = __expf(Lc - Lb);
+            if (lane == 0) vb_c[c % 3] = __expf(Lc);
+            __syncwarp();
+        };
+        bool bad = false;
+        // output rows of chunk cc (accumulator rows 64-127, warps of quadrants 2, 3) -> staging
+        auto output_tile = [&](int cc) {
+            if (quad < 2) return;
+            if (!mbar_wait(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
+            if (cc >= 1 && !mbar_wait(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
             tc_fence_after();
-            if (c >= 1) {
-                tma_store_3d(&tm_o, ostage, j0, (c - 1) * C, chain);
-                tma_store_commit();
-            }
-            const uint32_t ido = idesc_bf16_f32(64, 64, 0, 1);
-            const uint32_t ids = idesc_bf16_f32(D, 64, 1, 1);
-            const uint64_t dp = sdesc_sw128(smem_u32(st + P::O_P), 16, 1024);
-            const uint64_t dk = sdesc_sw128(smem_u32(st + P::O_K), TILE, 1024);
-            const uint64_t du = sdesc_sw128(smem_u32(utile), TILE, 1024);
-            const uint64_t duh = sdesc_sw128(smem_u32(uhtile), TILE, 1024);
+            const int i = quad * 32 + lane - 64;
+            float o[32];
+            tmem_ld16(tmem_addr(tbase, quad, P::T_UO + (cc & 1) * 64 + wg * 32), *reinterpret_cast<float(*)[16]>(o));
+            tmem_ld16(tmem_addr(tbase, quad, P::T_UO + (cc & 1) * 64 + wg * 32 + 16),
+                      *reinterpret_cast<float(*)[16]>(o + 16));
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&o_read[cc & 1]);
 #pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                mma_bf16(tbase + P::T_O2 + cp * 64, dp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), ido, ks > 0);
-                mma_bf16(tbase + P::T_S, dk + ((ks * 2048) >> 4), duh + ((ks * 2048) >> 4), ids, 1u);
-            }
-            mma_commit(bar4);
-            commits4 = c + 1;
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(ostage + sw128_offset(i, wg * 64 + q * 16)) =
+                    make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                               pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+            fence_async_smem();
+            mbar_arrive(os_full);
+        };
+
+        if (warp == 1) {
+            stage_alpha(0);
+            chunk_vectors(0);
+            if (nch > 1) stage_alpha(1);
         }
-        if (!mbar_wait(bar4, cp, kErrMma)) bad = true;
-        tc_fence_after();
-        if (tid == 0) {
-            if (c + P::STAGES < nch) issue(c + P::STAGES);   // this stage is free again
-            tma_store_wait_read();                           // the staging tile is rewritten next chunk
-        }
-        // next chunk's bf16 S
+        named_bar(1, kConv);
+        // start state slice S[:, j0:j0+64]: bf16 copy for the first read, b_C-scaled fp32 in TMEM
         {
             const int f = acc_row<D>(quad, lane);
+            const float bc = vb_c[0];
+            float v[32];
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-                const int col0 = wg * 32 + gg * 16;
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_S + col0), v);
+            for (int x = 0; x < 32; ++x)
+                v[x] = (f >= 0 && S0) ? S0[((size_t)chain * D + f) * dv + j0 + wg * 32 + x] : 0.f;
+            if (f >= 0) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(sbt + sw128_offset(f, wg * 64 + q * 16)) =
+                        make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+            }
+            fence_async_smem();
+            mbar_arrive(s_ready);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] *= bc;
+            tmem_st16(tmem_addr(tbase, quad, P::T_S + wg * 32), *reinterpret_cast<float(*)[16]>(v));
+            tmem_st16(tmem_addr(tbase, quad, P::T_S + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+            tmem_st_wait();
+        }
+
+        for (int c = 0; c < nch; ++c) {
+            const uint32_t cp = c & 1;
+            // output of the previous chunk, while [U; O] of this one is computed
+            if (c >= 1) output_tile(c - 1);
+            if (warp == 1 && c + 1 < nch) {
+                chunk_vectors(c + 1);
+                if (c + 2 < nch) stage_alpha(c + 2);
+            }
+            if (named_bar_or(1, kConv, bad)) { bad = true; break; }
+
+            // U (rows 0-63) -> bf16 (MN-major B operand) and diag(b_C / b) U
+            if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
+            tc_fence_after();
+            if (quad < 2) {
+                const int i = quad * 32 + lane;
+                const float ri = vb_r[(c % 3) * C + i];
+                float v[32];
+                tmem_ld16(tmem_addr(tbase, quad, P::T_UO + cp * 64 + wg * 32), *reinterpret_cast<float(*)[16]>(v));
+                tmem_ld16(tmem_addr(tbase, quad, P::T_UO + cp * 64 + wg * 32 + 16),
+                          *reinterpret_cast<float(*)[16]>(v + 16));
                 tmem_ld_wait();
-                if (f >= 0) {
-                    *reinterpret_cast<uint4*>(sbt + sw128_offset(f, col0 * 2)) =
-                        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                   pack_bf16x2(v[6], v[7]));
-                    *reinterpret_cast<uint4*>(sbt + sw128_offset(f, col0 * 2 + 16)) =
-                        make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                                   pack_bf16x2(v[14], v[15]));
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float* w = v + 8 * q;
+                    *reinterpret_cast<uint4*>(utile + sw128_offset(i, wg * 64 + q * 16)) =
+                        make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]),
+                                   pack_bf16x2(w[6], w[7]));
+                    *reinterpret_cast<uint4*>(uhtile + sw128_offset(i, wg * 64 + q * 16)) =
+                        make_uint4(pack_bf16x2(ri * w[0], ri * w[1]), pack_bf16x2(ri * w[2], ri * w[3]),
+                                   pack_bf16x2(ri * w[4], ri * w[5]), pack_bf16x2(ri * w[6], ri * w[7]));
+                }
+                fence_async_smem();
+            }
+            tc_fence_before();
+            mbar_arrive(u_ready);
+
+            // state: bf16 copy for the next chunk, then scale by its b_C in TMEM
+            if (!mbar_wait(s_full, c & 1, kErrMma)) bad = true;
+            tc_fence_after();
+            {
+                const int f = acc_row<D>(quad, lane);
+                float v[32];
+                tmem_ld16(tmem_addr(tbase, quad, P::T_S + wg * 32), *reinterpret_cast<float(*)[16]>(v));
+                tmem_ld16(tmem_addr(tbase, quad, P::T_S + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+                tmem_ld_wait();
+                if (c + 1 < nch) {
+                    if (f >= 0) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            *reinterpret_cast<uint4*>(sbt + sw128_offset(f, wg * 64 + q * 16)) = make_uint4(
+                                pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                    }
+                    fence_async_smem();
+                    mbar_arrive(s_ready);
+                    const float bc = vb_c[(c + 1) % 3];
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) v[x] *= bc;
+                    tmem_st16(tmem_addr(tbase, quad, P::T_S + wg * 32), *reinterpret_cast<float(*)[16]>(v));
+                    tmem_st16(tmem_addr(tbase, quad, P::T_S + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+                    tmem_st_wait();
+                } else if (f >= 0 && !bad) {
+                    // final state slice
+                    float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)chain * D + f) * dv + j0 + wg * 32);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                 }
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(bad)) { bad = true; break; }
-    }
-    if (!bad) {
-        // last output tile and the final state slice
-        output_tile(nch - 1);
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_3d(&tm_o, ostage, j0, (nch - 1) * C, chain);
-            tma_store_commit();
-        }
-        const int f = acc_row<D>(quad, lane);
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-            const int col0 = wg * 32 + gg * 16;
-            float v[16];
-            tmem_ld16(tmem_addr(tbase, quad, P::T_S + col0), v);
-            tmem_ld_wait();
-            if (f >= 0) {
-                float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)chain * D + f) * dv + j0 + col0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            }
-        }
-    }
-    if (warp == 1) cp_async_wait_all();
-    if (tid == 0) {
-        tma_store_wait_all();
-        if (bad) {
-            for (int cc = max(0, loads_issued - P::STAGES); cc < loads_issued; ++cc)
-                mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
-            if (commits3 > 0) mbar_wait(bar3, (commits3 - 1) & 1, kErrMma);
-            if (commits4 > 0) mbar_wait(bar4, (commits4 - 1) & 1, kErrMma);
-        }
+        if (!bad) output_tile(nch - 1);
+        if (warp == 1) cp_async_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -756,15 +846,16 @@ cudaError_t launch_gd(const PrefillArgs& a)
     const int chains = a.B * a.H;
     const int nch = (a.N + C - 1) / C;
     const int npad = nch * C;
-    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
-    unsigned char* wneg = ws;
-    unsigned char* tp = wneg + (size_t)chains * npad * D * 2;
+    // workspace: -W and diag(b) Q [chains][npad][D], T' and P~ [chains][npad][C], all bf16
+    unsigned char* wneg = static_cast<unsigned char*>(a.workspace);
+    unsigned char* qb = wneg + (size_t)chains * npad * D * 2;
+    unsigned char* tp = qb + (size_t)chains * npad * D * 2;
     unsigned char* pp = tp + (size_t)chains * npad * C * 2;
-    CUtensorMap mq, mk, mv, mo, mw, mt, mp;
+    CUtensorMap mq, mk, mv, mo, mw, mqb, mt, mp;
     if (!make_map(&mq, a.q, D, a.N, chains) || !make_map(&mk, a.k, D, a.N, chains) ||
         !make_map(&mv, a.v, a.dv, a.N, chains) || !make_map(&mo, a.out, a.dv, a.N, chains) ||
-        !make_map(&mw, wneg, D, npad, chains) || !make_map(&mt, tp, C, npad, chains) ||
-        !make_map(&mp, pp, C, npad, chains))
+        !make_map(&mw, wneg, D, npad, chains) || !make_map(&mqb, qb, D, npad, chains) ||
+        !make_map(&mt, tp, C, npad, chains) || !make_map(&mp, pp, C, npad, chains))
         return cudaErrorInvalidValue;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
@@ -775,7 +866,7 @@ cudaError_t launch_gd(const PrefillArgs& a)
     if (e != cudaSuccess) return e;
     const long long items = (long long)chains * nch;
     const int g1 = (int)std::min<long long>(items, 2LL * sms);
-    k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mt, mp, a.alpha, a.g, a.N, chains);
+    k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mqb, mt, mp, a.alpha, a.g, a.N, chains);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -783,7 +874,7 @@ cudaError_t launch_gd(const PrefillArgs& a)
     const int s2 = ChainPlan<D>::BYTES;
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
     if (e != cudaSuccess) return e;
-    k2<<<chains * (a.dv / DVT), kThreads, s2, a.stream>>>(mq, mk, mv, mw, mt, mp, mo, a.alpha, a.S0, a.S_out,
+    k2<<<chains * (a.dv / DVT), kChainThreads, s2, a.stream>>>(mqb, mk, mv, mw, mt, mp, mo, a.alpha, a.S0, a.S_out,
                                                            a.N, a.dv);
     return cudaGetLastError();
 }
@@ -794,7 +885,7 @@ size_t gd_workspace_bytes(int B, int H, int N, int d, int dv)
 {
     (void)dv;
     const size_t npad = (size_t)((N + C - 1) / C) * C;
-    return (size_t)B * H * npad * (size_t)(d + 2 * C) * 2;
+    return (size_t)B * H * npad * (size_t)(2 * d + 2 * C) * 2;
 }
 
 cudaError_t launch_prefill_tc_gated_delta(const PrefillArgs& a)
