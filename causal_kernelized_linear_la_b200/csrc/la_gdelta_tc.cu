@@ -12,14 +12,15 @@
 // With T = (I + A)^{-1}, T' = T diag(g):
 //   W = T' diag(b) K,  U = T' V - W S
 //   O = diag(b) Q S + P~ U,   P~_tj = e^{L_t-L_j} (q_t . k_j) [j <= t]
-//   S_next = b_C S + K^T diag(b_C / b) U
+//   S_next = b_C S + K~^T U,   K~ = diag(b_C / b) K
 // Substituting back reproduces the token recurrence exactly (up to rounding).
 //
 // Only U and S_next depend on the state, so the work splits in two launches:
 //   gd_prep_kernel   every (chain, chunk) in parallel: the score blocks
 //                    [K;Q]K^T, A and P~, T = (I + A)^{-1} on the CUDA cores in
 //                    fp32 (blocked forward substitution), T', W = T' diag(b) K.
-//                    Writes -W, diag(b) Q, T' and P~ (bf16) to the workspace.
+//                    Writes -W, diag(b) Q, diag(b_C / b) K, T' and P~ (bf16) to
+//                    the workspace.
 //   gd_chain_kernel  one CTA per (chain, 64 value columns), chunks in order:
 //                    U = T' V + (-W) S and diag(b) Q S, then P~ U and the state
 //                    update, all on the tensor cores; the CUDA cores only
@@ -28,7 +29,11 @@
 //                    at M = 64 as at M = 128, so operands that share a B are
 //                    stacked into M = 128: [T'; 0] V, [-W; diag(b) Q] S and
 //                    [0; P~] U leave U in accumulator rows 0-63 and the whole
-//                    output in rows 64-127.
+//                    output in rows 64-127.  Issue itself is slow (tens of
+//                    cycles per MMA), so two warps issue, each half of every
+//                    contraction on the chain into its own TMEM accumulator
+//                    (the converters add the pair when they read it out); one
+//                    also issues the next chunk's T' V, the other P~ U.
 // The columns of S evolve independently under the delta rule, so value tiles
 // need no communication.
 #include <algorithm>
@@ -107,9 +112,9 @@ struct PrepPlan {
     static constexpr int TS = C + 4;                        // row stride of T (16-byte aligned rows)
     static constexpr int OFF_TM = OFF_A + C * (C + 1) * 4;  // T fp32 [C][TS]
     static constexpr int OFF_X = OFF_TM + C * TS * 4;       // per-warp 16 x 8 block scratch, fp32 [8][16][9]
-    // L[C], b[C], g[C], staged alpha/g [2][2][C], e^{L-L_m}[C], e^{L_m-L}[C], flag
+    // L[C], b[C], g[C], staged alpha/g [2][2][C], e^{L-L_m}[C], e^{L_m-L}[C], b_C/b[C], flag
     static constexpr int OFF_VEC = OFF_X + 8 * 16 * 9 * 4;
-    static constexpr int OFF_BAR = OFF_VEC + 9 * C * 4 + 16;
+    static constexpr int OFF_BAR = OFF_VEC + 10 * C * 4 + 16;
     static constexpr int OFF_TMEM = OFF_BAR + 3 * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(NB * TILE <= C * (C + 1) * 4, "-W staging fits over A");
@@ -122,8 +127,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qb,
-               const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_p,
-               const float* __restrict__ alpha,
+               const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_t,
+               const __grid_constant__ CUtensorMap tm_p, const float* __restrict__ alpha,
                const float* __restrict__ gate, int N, int chains)
 {
     using P = PrepPlan<D>;
@@ -143,7 +148,8 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float* avec = Lv + 3 * C;   // [2][2][C]: alpha, g of two work items
     float* ef = Lv + 7 * C;     // e^{L_t - L_m}, m the chunk's middle token
     float* eg = Lv + 8 * C;     // e^{L_m - L_t}
-    int* factored = reinterpret_cast<int*>(Lv + 9 * C);
+    float* kr = Lv + 9 * C;     // b_C / b_t
+    int* factored = reinterpret_cast<int*>(Lv + 10 * C);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* bar1 = full + 1;
     uint64_t* bar2 = full + 2;
@@ -243,6 +249,8 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
                 hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
             }
+            kr[2 * lane] = __expf(Lc - La);
+            kr[2 * lane + 1] = __expf(Lc - Lb);
             ef[2 * lane] = __expf(La - Lm);
             ef[2 * lane + 1] = __expf(Lb - Lm);
             eg[2 * lane] = __expf(Lm - La);
@@ -260,6 +268,7 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             unpack8(reinterpret_cast<const uint4*>(sm + (2 * b) * TILE)[rem], f);
             reinterpret_cast<uint4*>(kbt + b * TILE)[rem] = pack8(f, bv[row]);
         }
+        __syncthreads();   // raw K is rewritten in place below
 
         // score blocks -> A (fp32, strictly lower, gated and decayed) and P~ (bf16)
         if (!mbar_wait(bar1, ph, kErrMma)) bad = true;
@@ -290,38 +299,63 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int i = r - 64;
                 const float Li = Lv[i], si = ef[i];
                 uint32_t pk[16];
+                if (fact) {
 #pragma unroll
-                for (int h = 0; h < 16; ++h) {
-                    const int j = wg * 32 + 2 * h;
-                    const float e0 = fact ? si * eg[j] : __expf(Li - Lv[j]);
-                    const float e1 = fact ? si * eg[j + 1] : __expf(Li - Lv[j + 1]);
-                    const float a = j <= i ? e0 * v[2 * h] : 0.f;
-                    const float b = j + 1 <= i ? e1 * v[2 * h + 1] : 0.f;
-                    pk[h] = pack_bf16x2(a, b);
+                    for (int h = 0; h < 16; ++h) {
+                        const int j = wg * 32 + 2 * h;
+                        const float a = j <= i ? si * eg[j] * v[2 * h] : 0.f;
+                        const float b = j + 1 <= i ? si * eg[j + 1] * v[2 * h + 1] : 0.f;
+                        pk[h] = pack_bf16x2(a, b);
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) {
+                        const int j = wg * 32 + 2 * h;
+                        const float a = j <= i ? __expf(Li - Lv[j]) * v[2 * h] : 0.f;
+                        const float b = j + 1 <= i ? __expf(Li - Lv[j + 1]) * v[2 * h + 1] : 0.f;
+                        pk[h] = pack_bf16x2(a, b);
+                    }
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     *reinterpret_cast<uint4*>(ptile + sw128_offset(i, wg * 64 + q * 16)) =
                         make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                // diag(b) Q in place for row i (M1, its reader, is complete).  The
-                // whole row takes one factor, so any chunk order works: rotating it
-                // by the row keeps the 32 rows of a warp on distinct banks.
-                const float bi = bv[i];
+            }
+            // diag(b) Q and diag(b_C / b) K in place (M1, their reader, is complete;
+            // Kb is built): the four threads that own row rq = r % 64 (both row
+            // halves, both column halves) take a quarter of its 16-byte chunks each.
+            // A row takes one factor, so any chunk order works: rotating it by the
+            // row keeps a warp's 32 rows on distinct banks.  Loads go first.
+            const int rq = r & 63, slot = (r >> 6) * 2 + wg;
+            const float bq = bv[rq], kq = kr[rq];
+            constexpr int PER = NB * 2;
+            uint4 xq[PER], xk[PER];
 #pragma unroll
-                for (int q = wg; q < NB * 8; q += 2) {
-                    const int chunk = (q + i) & 7;
-                    uint4* pq = reinterpret_cast<uint4*>(sm + (2 * (q / 8) + 1) * TILE + i * 128 + chunk * 16);
-                    float f[8];
-                    unpack8(*pq, f);
-                    *pq = pack8(f, bi);
-                }
+            for (int n = 0; n < PER; ++n) {
+                const int q = slot + 4 * n, chunk = ((q & 7) + rq) & 7;
+                const int off = rq * 128 + chunk * 16;
+                xq[n] = *reinterpret_cast<const uint4*>(sm + (2 * (q / 8) + 1) * TILE + off);
+                xk[n] = *reinterpret_cast<const uint4*>(sm + (2 * (q / 8)) * TILE + off);
+            }
+#pragma unroll
+            for (int n = 0; n < PER; ++n) {
+                const int q = slot + 4 * n, chunk = ((q & 7) + rq) & 7;
+                const int off = rq * 128 + chunk * 16;
+                float f[8];
+                unpack8(xq[n], f);
+                *reinterpret_cast<uint4*>(sm + (2 * (q / 8) + 1) * TILE + off) = pack8(f, bq);
+                unpack8(xk[n], f);
+                *reinterpret_cast<uint4*>(sm + (2 * (q / 8)) * TILE + off) = pack8(f, kq);
             }
         }
         fence_async_smem();
         tc_fence_before();
         if (__syncthreads_or(bad)) { bad = true; break; }
         if (tid == 0) {
-            for (int b = 0; b < NB; ++b) tma_store_3d(&tm_qb, sm + (2 * b + 1) * TILE, b * 64, c * C, chain);
+            for (int b = 0; b < NB; ++b) {
+                tma_store_3d(&tm_qb, sm + (2 * b + 1) * TILE, b * 64, c * C, chain);
+                tma_store_3d(&tm_kt, sm + (2 * b) * TILE, b * 64, c * C, chain);
+            }
             tma_store_commit();
         }
 
@@ -383,7 +417,7 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 __syncthreads();
             }
         }
-        // the diag(b) Q store has long read its tiles: K/Q take the next item
+        // the diag(b) Q and K~ stores have long read their tiles: K/Q take the next item
         if (tid == 0 && next < items) {
             tma_store_wait_read();
             issue(next);
@@ -479,7 +513,7 @@ template <int D>
 struct ChainPlan {
     static constexpr int STAGES = 2;
     static constexpr int NB = D / 64;
-    // stage: K[NB] | -W_0 Qb_0 -W_1 Qb_1 ... | T' Z P~ | V   (Z: a zero tile, never loaded)
+    // stage: K~[NB] | -W_0 Qb_0 -W_1 Qb_1 ... | T' Z P~ | V   (Z: a zero tile, never loaded)
     // [-W_b; Qb_b], [T'; Z] and [Z; P~] are M = 128 K-major A operands.
     static constexpr int O_K = 0, O_WQ = NB * TILE, O_T = 3 * NB * TILE;
     static constexpr int O_Z = O_T + TILE, O_P = O_Z + TILE, O_V = O_P + TILE;
@@ -487,21 +521,23 @@ struct ChainPlan {
     static constexpr int LOAD_BYTES = STAGE - TILE;         // all but Z arrives by TMA
     static constexpr int OFF_SB = STAGES * STAGE;           // S bf16 [D][64], MN-major B operand
     static constexpr int OFF_U = OFF_SB + NB * TILE;        // U bf16 [C][64], MN-major B operand
-    static constexpr int OFF_UH = OFF_U + TILE;             // diag(b_C / b) U
-    static constexpr int OFF_O = OFF_UH + TILE;             // output staging
-    static constexpr int OFF_VEC = OFF_O + TILE;            // r[3][C], staged alpha [2][C], b_C [3]
-    static constexpr int OFF_BAR = OFF_VEC + 6 * C * 4 + 16;
-    // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready s_ready ostage_full ostage_empty drain
-    static constexpr int NBAR = 16;
+    static constexpr int OFF_O = OFF_U + TILE;              // output staging
+    static constexpr int OFF_VEC = OFF_O + TILE;            // staged alpha [2][C], b_C [3]
+    static constexpr int OFF_BAR = OFF_VEC + 2 * C * 4 + 16;
+    // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready s_ready ostage_full ostage_empty
+    // drain[2]
+    static constexpr int NBAR = 17;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
-    // TMEM columns: [U; O] (M = 128, two buffers), state (rows = key feature)
-    static constexpr uint32_t T_UO = 0, T_S = 128, T_COLS = 256;
+    // TMEM columns: the two issuers' partial [U; O] accumulators (two buffers each)
+    // and partial states; U, O and S are the sums of the pairs.
+    static constexpr uint32_t T_X1 = 0, T_X2 = 128, T_S1 = 256, T_S2 = 320, T_COLS = 512;
+    static constexpr int KS_HALF = D / 32;                   // K-steps of (-W) S per issuer
 };
 
 constexpr int kConv = 256;                   // converter threads (warps 0-7)
-constexpr int kChainThreads = kConv + 64;    // + MMA issuer warp 8 + TMA warp 9
+constexpr int kChainThreads = kConv + 96;    // + issuer warps 8 and 10, TMA warp 9
 
 template <int D>
 __global__ void __launch_bounds__(kChainThreads, 1)
@@ -517,23 +553,21 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
     unsigned char* sm = align1024(smem_raw);
     unsigned char* sbt = sm + P::OFF_SB;
     unsigned char* utile = sm + P::OFF_U;
-    unsigned char* uhtile = sm + P::OFF_UH;
     unsigned char* ostage = sm + P::OFF_O;
-    float* vb_r = reinterpret_cast<float*>(sm + P::OFF_VEC);   // [3][C] b_C / b_i
-    float* abuf = vb_r + 3 * C;                                // [2][C] staged alpha
-    float* vb_c = vb_r + 5 * C;                                // [3] b_C
+    float* abuf = reinterpret_cast<float*>(sm + P::OFF_VEC);   // [2][C] staged alpha
+    float* vb_c = abuf + 2 * C;                                // [3] b_C
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
-    uint64_t* full = bars;          // TMA -> issuer, per stage
-    uint64_t* empty = bars + 2;     // issuer (commit) -> TMA, per stage
-    uint64_t* uo_full = bars + 4;   // issuer: [U; Qb S] complete, per TMEM buffer
-    uint64_t* o_full = bars + 6;    // issuer: output accumulator complete, per TMEM buffer
-    uint64_t* o_read = bars + 8;    // converters: output accumulator read, per TMEM buffer
-    uint64_t* s_full = bars + 10;   // issuer: state update complete
-    uint64_t* u_ready = bars + 11;  // converters: U operands written, state scaled
+    uint64_t* full = bars;          // TMA -> issuers, per stage
+    uint64_t* empty = bars + 2;     // both issuers (commit) -> TMA, per stage
+    uint64_t* uo_full = bars + 4;   // both issuers: [U; Qb S] partials complete, per TMEM buffer
+    uint64_t* o_full = bars + 6;    // issuer B: output partial complete, per TMEM buffer
+    uint64_t* o_read = bars + 8;    // converters: output partials read, per TMEM buffer
+    uint64_t* s_full = bars + 10;   // both issuers: state update partials complete
+    uint64_t* u_ready = bars + 11;  // converters: U in place, state rescaled
     uint64_t* s_ready = bars + 12;  // converters: bf16 state written
     uint64_t* os_full = bars + 13;  // converters: output staging written
     uint64_t* os_empty = bars + 14; // TMA: output staging read by its store
-    uint64_t* drain = bars + 15;    // issuer: every MMA it issued is complete
+    uint64_t* drain = bars + 15;    // [2] issuers: every MMA each issued is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -545,17 +579,17 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-            mbar_init(&uo_full[s], 1);
+            mbar_init(&empty[s], 2);
+            mbar_init(&uo_full[s], 2);
             mbar_init(&o_full[s], 1);
             mbar_init(&o_read[s], 128);
+            mbar_init(&drain[s], 1);
         }
-        mbar_init(s_full, 1);
+        mbar_init(s_full, 2);
         mbar_init(u_ready, kConv);
         mbar_init(s_ready, kConv);
         mbar_init(os_full, 128);
         mbar_init(os_empty, 1);
-        mbar_init(drain, 1);
         fence_mbar_init();
     }
     // zero tiles of both stages (rows 64-127 of [T'; Z], rows 0-63 of [Z; P~])
@@ -574,7 +608,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
         if (lane == 0) {
             const uint64_t pol_once = policy_evict_first();
             const uint64_t pol_shared = ntile > 1 ? policy_evict_normal() : policy_evict_first();
-            int loads = 0, stores = 0;
+            int loads = 0;
             auto issue = [&](int c) {
                 const int s = c % P::STAGES;
                 unsigned char* st = sm + s * P::STAGE;
@@ -590,14 +624,27 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
                 tma_load_3d(st + P::O_V, &tm_v, j0, y, chain, &full[s], pol_once);
                 loads = c + 1;
             };
+            // two stages give a load about one chunk of lead time; pulling the
+            // operands of the chunk two further ahead into L2 hides the rest
+            auto prefetch = [&](int c) {
+                const int y = c * C;
+                for (int b = 0; b < NB; ++b) {
+                    tma_prefetch_3d(&tm_k, b * 64, y, chain);
+                    tma_prefetch_3d(&tm_w, b * 64, y, chain);
+                    tma_prefetch_3d(&tm_qb, b * 64, y, chain);
+                }
+                tma_prefetch_3d(&tm_t, 0, y, chain);
+                tma_prefetch_3d(&tm_p, 0, y, chain);
+                tma_prefetch_3d(&tm_v, j0, y, chain);
+            };
             auto store = [&](int c) {
                 tma_store_3d(&tm_o, ostage, j0, c * C, chain);
                 tma_store_commit();
                 tma_store_wait_read();
                 mbar_arrive(os_empty);
-                stores = c + 1;
             };
             for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
+            for (int c = P::STAGES; c < min(nch, 2 * P::STAGES); ++c) prefetch(c);
             bool ok = true;
             for (int c = 0; c < nch && ok; ++c) {
                 if (c >= 1) {
@@ -608,6 +655,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
                 if (c + P::STAGES < nch) {
                     ok = mbar_wait(&empty[c % P::STAGES], (c / P::STAGES) & 1, kErrMma);
                     if (ok) issue(c + P::STAGES);
+                    if (ok && c + 2 * P::STAGES < nch) prefetch(c + 2 * P::STAGES);
                 }
             }
             if (ok && mbar_wait(os_full, (nch - 1) & 1, kErrMma)) store(nch - 1);
@@ -615,62 +663,82 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
             // loads in flight must land before the block exits
             for (int c = max(0, loads - P::STAGES); c < loads; ++c)
                 mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad);
-            (void)stores;
         }
         __syncwarp();
-    } else if (warp == 8) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == 8 || warp == 10) {
+        // ---------------- MMA issuers ----------------
+        // Issuer A (warp 8): X1 = [T'; 0] V (one chunk ahead), X1 += [-W; Qb] S over
+        // the first half of the features, S1 += K~^T U over the first 32 tokens.
+        // Issuer B (warp 10): X2 = [-W; Qb] S over the second half, S2 = K~^T U
+        // over the last 32 tokens, X2 += [0; P~] U.  U = X1 + X2 (rows 0-63),
+        // O = X1 + X2 (rows 64-127), S = S1 + S2.
         if (lane == 0) {
-            bool ok = true;
-            for (int c = 0; c < nch && ok; ++c) {
-                const int s = c % P::STAGES;
-                const uint32_t cp = c & 1;
-                unsigned char* st = sm + s * P::STAGE;
-                const uint32_t tuo = tbase + P::T_UO + cp * 64;
-                const uint32_t id = idesc_bf16_f32(128, 64, 0, 1);
-                ok = mbar_wait(&full[s], (c / P::STAGES) & 1, kErrTmaLoad);
-                if (ok && c >= 2) ok = mbar_wait(&o_read[cp], ((c - 2) / 2) & 1, kErrMma);
-                if (!ok) break;
+            const bool A = warp == 8;
+            const uint32_t id = idesc_bf16_f32(128, 64, 0, 1);
+            const uint32_t ids = idesc_bf16_f32(D, 64, 1, 1);
+            const uint64_t ds = sdesc_sw128(smem_u32(sbt), TILE, 1024);
+            const uint64_t du = sdesc_sw128(smem_u32(utile), TILE, 1024);
+            const uint32_t tx = tbase + (A ? P::T_X1 : P::T_X2);
+            const uint32_t tsp = tbase + (A ? P::T_S1 : P::T_S2);
+            auto ready = [&](int c) {   // stage c loaded and TMEM buffer c & 1 read out
+                if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) return false;
+                if (c >= 2 && !mbar_wait(&o_read[c & 1], ((c - 2) / 2) & 1, kErrMma)) return false;
+                return true;
+            };
+            auto m0 = [&](int c) {
+                if (!ready(c)) return false;
                 tc_fence_after();
-                // [U; O] = [T'; 0] V
+                unsigned char* st = sm + (c % P::STAGES) * P::STAGE;
                 const uint64_t dt = sdesc_sw128(smem_u32(st + P::O_T), 16, 1024);
                 const uint64_t dvv = sdesc_sw128(smem_u32(st + P::O_V), TILE, 1024);
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tuo, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id, ks > 0);
-                // [U; O] += [-W; Qb] S once the bf16 state is in place
-                ok = mbar_wait(s_ready, c & 1, kErrMma);
-                if (!ok) break;
+                    mma_bf16(tx + (c & 1) * 64, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id, ks > 0);
+                return true;
+            };
+            bool ok = A ? m0(0) : true;
+            for (int c = 0; c < nch && ok; ++c) {
+                const int s = c % P::STAGES;
+                const uint32_t cp = c & 1;
+                unsigned char* st = sm + s * P::STAGE;
+                const uint32_t txc = tx + cp * 64;
+                if (!A && !(ok = ready(c))) break;
+                if (!(ok = mbar_wait(s_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
                 const uint64_t dwq = sdesc_sw128(smem_u32(st + P::O_WQ), 16, 1024);
-                const uint64_t ds = sdesc_sw128(smem_u32(sbt), TILE, 1024);
+                const int k0 = A ? 0 : P::KS_HALF;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    mma_bf16(tuo, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4), ds + ((ks * 2048) >> 4), id,
-                             1u);
+                for (int kk = 0; kk < P::KS_HALF; ++kk) {
+                    const int ks = k0 + kk;
+                    mma_bf16(txc, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4), ds + ((ks * 2048) >> 4), id,
+                             (A || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(&uo_full[cp]);
-                // S += K^T diag(b_C / b) U, then O += [0; P~] U
-                ok = mbar_wait(u_ready, c & 1, kErrMma);
-                if (!ok) break;
+                if (!(ok = mbar_wait(u_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
-                const uint32_t ids = idesc_bf16_f32(D, 64, 1, 1);
                 const uint64_t dk = sdesc_sw128(smem_u32(st + P::O_K), TILE, 1024);
-                const uint64_t duh = sdesc_sw128(smem_u32(uhtile), TILE, 1024);
+                const int t0 = A ? 0 : 2;
 #pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tbase + P::T_S, dk + ((ks * 2048) >> 4), duh + ((ks * 2048) >> 4), ids, 1u);
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int ks = t0 + kk;
+                    mma_bf16(tsp, dk + ((ks * 2048) >> 4), du + ((ks * 2048) >> 4), ids, (A || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(s_full);
-                const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
-                const uint64_t du = sdesc_sw128(smem_u32(utile), TILE, 1024);
+                if (A) {
+                    mma_commit(&empty[s]);
+                    if (c + 1 < nch) ok = m0(c + 1);
+                } else {
+                    const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
 #pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tuo, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, 1u);
-                mma_commit(&o_full[cp]);
-                mma_commit(&empty[s]);
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_bf16(txc, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, 1u);
+                    mma_commit(&o_full[cp]);
+                    mma_commit(&empty[s]);
+                }
             }
             // every MMA issued must complete before TMEM is released
-            mma_commit(drain);
-            mbar_wait(drain, 0, kErrMma);
+            mma_commit(&drain[A ? 0 : 1]);
+            mbar_wait(&drain[A ? 0 : 1], 0, kErrMma);
         }
         __syncwarp();
     } else {
@@ -687,21 +755,29 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
             }
             cp_async_commit();
         };
-        // warp 1: b_C / b_i and b_C of chunk c into vector buffer c % 3
+        // warp 1: b_C of chunk c into vector buffer c % 3
         auto chunk_vectors = [&](int c) {
             cp_async_wait_all();
             const float* a = abuf + (c & 1) * C;
             const int t = c * C + 2 * lane;
             float La, Lb, Lc;
             chunk_logdecay(a[2 * lane], a[2 * lane + 1], t < N, t + 1 < N, lane, La, Lb, Lc);
-            float* r = vb_r + (c % 3) * C;
-            r[2 * lane] = __expf(Lc - La);
-            r[2 * lane + 1] = __expf(Lc - Lb);
             if (lane == 0) vb_c[c % 3] = __expf(Lc);
             __syncwarp();
         };
         bool bad = false;
-        // output rows of chunk cc (accumulator rows 64-127, warps of quadrants 2, 3) -> staging
+        // 32 columns of accumulator rows of this warp's quadrant: X1 + X2
+        auto ld_sum = [&](uint32_t col, float (&v)[32]) {
+            float w[32];
+            tmem_ld16(tmem_addr(tbase, quad, P::T_X1 + col), *reinterpret_cast<float(*)[16]>(v));
+            tmem_ld16(tmem_addr(tbase, quad, P::T_X1 + col + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+            tmem_ld16(tmem_addr(tbase, quad, P::T_X2 + col), *reinterpret_cast<float(*)[16]>(w));
+            tmem_ld16(tmem_addr(tbase, quad, P::T_X2 + col + 16), *reinterpret_cast<float(*)[16]>(w + 16));
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] += w[x];
+        };
+        // output rows of chunk cc (accumulator rows 64-127, quadrants 2 and 3) -> staging
         auto output_tile = [&](int cc) {
             if (quad < 2) return;
             if (!mbar_wait(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
@@ -709,10 +785,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
             tc_fence_after();
             const int i = quad * 32 + lane - 64;
             float o[32];
-            tmem_ld16(tmem_addr(tbase, quad, P::T_UO + (cc & 1) * 64 + wg * 32), *reinterpret_cast<float(*)[16]>(o));
-            tmem_ld16(tmem_addr(tbase, quad, P::T_UO + (cc & 1) * 64 + wg * 32 + 16),
-                      *reinterpret_cast<float(*)[16]>(o + 16));
-            tmem_ld_wait();
+            ld_sum((cc & 1) * 64 + wg * 32, o);
             tc_fence_before();
             mbar_arrive(&o_read[cc & 1]);
 #pragma unroll
@@ -730,7 +803,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
             if (nch > 1) stage_alpha(1);
         }
         named_bar(1, kConv);
-        // start state slice S[:, j0:j0+64]: bf16 copy for the first read, b_C-scaled fp32 in TMEM
+        // start state slice S[:, j0:j0+64]: bf16 copy for the first read, b_C-scaled fp32 in S1
         {
             const int f = acc_row<D>(quad, lane);
             const float bc = vb_c[0];
@@ -749,14 +822,15 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
             mbar_arrive(s_ready);
 #pragma unroll
             for (int x = 0; x < 32; ++x) v[x] *= bc;
-            tmem_st16(tmem_addr(tbase, quad, P::T_S + wg * 32), *reinterpret_cast<float(*)[16]>(v));
-            tmem_st16(tmem_addr(tbase, quad, P::T_S + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+            tmem_st16(tmem_addr(tbase, quad, P::T_S1 + wg * 32), *reinterpret_cast<float(*)[16]>(v));
+            tmem_st16(tmem_addr(tbase, quad, P::T_S1 + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
             tmem_st_wait();
         }
 
         for (int c = 0; c < nch; ++c) {
             const uint32_t cp = c & 1;
-            // output of the previous chunk, while [U; O] of this one is computed
+            // off the chain, while [U; O] of this chunk is computed: the previous
+            // chunk's output and the next chunk's decay vector
             if (c >= 1) output_tile(c - 1);
             if (warp == 1 && c + 1 < nch) {
                 chunk_vectors(c + 1);
@@ -764,41 +838,36 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
             }
             if (named_bar_or(1, kConv, bad)) { bad = true; break; }
 
-            // U (rows 0-63) -> bf16 (MN-major B operand) and diag(b_C / b) U
+            // U (rows 0-63) -> bf16 (MN-major B operand)
             if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
             tc_fence_after();
             if (quad < 2) {
                 const int i = quad * 32 + lane;
-                const float ri = vb_r[(c % 3) * C + i];
                 float v[32];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_UO + cp * 64 + wg * 32), *reinterpret_cast<float(*)[16]>(v));
-                tmem_ld16(tmem_addr(tbase, quad, P::T_UO + cp * 64 + wg * 32 + 16),
-                          *reinterpret_cast<float(*)[16]>(v + 16));
-                tmem_ld_wait();
+                ld_sum(cp * 64 + wg * 32, v);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float* w = v + 8 * q;
+                for (int q = 0; q < 4; ++q)
                     *reinterpret_cast<uint4*>(utile + sw128_offset(i, wg * 64 + q * 16)) =
-                        make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]),
-                                   pack_bf16x2(w[6], w[7]));
-                    *reinterpret_cast<uint4*>(uhtile + sw128_offset(i, wg * 64 + q * 16)) =
-                        make_uint4(pack_bf16x2(ri * w[0], ri * w[1]), pack_bf16x2(ri * w[2], ri * w[3]),
-                                   pack_bf16x2(ri * w[4], ri * w[5]), pack_bf16x2(ri * w[6], ri * w[7]));
-                }
+                        make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
                 fence_async_smem();
             }
             tc_fence_before();
             mbar_arrive(u_ready);
 
-            // state: bf16 copy for the next chunk, then scale by its b_C in TMEM
+            // state S = S1 + S2: bf16 copy for the next chunk, then S1 = b_C S
             if (!mbar_wait(s_full, c & 1, kErrMma)) bad = true;
             tc_fence_after();
             {
                 const int f = acc_row<D>(quad, lane);
-                float v[32];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_S + wg * 32), *reinterpret_cast<float(*)[16]>(v));
-                tmem_ld16(tmem_addr(tbase, quad, P::T_S + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+                float v[32], w[32];
+                tmem_ld16(tmem_addr(tbase, quad, P::T_S1 + wg * 32), *reinterpret_cast<float(*)[16]>(v));
+                tmem_ld16(tmem_addr(tbase, quad, P::T_S1 + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+                tmem_ld16(tmem_addr(tbase, quad, P::T_S2 + wg * 32), *reinterpret_cast<float(*)[16]>(w));
+                tmem_ld16(tmem_addr(tbase, quad, P::T_S2 + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(w + 16));
                 tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] += w[x];
                 if (c + 1 < nch) {
                     if (f >= 0) {
 #pragma unroll
@@ -808,12 +877,13 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
                                 pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
                     }
                     fence_async_smem();
+                    tc_fence_before();
                     mbar_arrive(s_ready);
                     const float bc = vb_c[(c + 1) % 3];
 #pragma unroll
                     for (int x = 0; x < 32; ++x) v[x] *= bc;
-                    tmem_st16(tmem_addr(tbase, quad, P::T_S + wg * 32), *reinterpret_cast<float(*)[16]>(v));
-                    tmem_st16(tmem_addr(tbase, quad, P::T_S + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+                    tmem_st16(tmem_addr(tbase, quad, P::T_S1 + wg * 32), *reinterpret_cast<float(*)[16]>(v));
+                    tmem_st16(tmem_addr(tbase, quad, P::T_S1 + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
                     tmem_st_wait();
                 } else if (f >= 0 && !bad) {
                     // final state slice
@@ -846,15 +916,18 @@ cudaError_t launch_gd(const PrefillArgs& a)
     const int chains = a.B * a.H;
     const int nch = (a.N + C - 1) / C;
     const int npad = nch * C;
-    // workspace: -W and diag(b) Q [chains][npad][D], T' and P~ [chains][npad][C], all bf16
+    // workspace: -W, diag(b) Q, diag(b_C / b) K [chains][npad][D], T' and P~
+    // [chains][npad][C], all bf16
     unsigned char* wneg = static_cast<unsigned char*>(a.workspace);
     unsigned char* qb = wneg + (size_t)chains * npad * D * 2;
-    unsigned char* tp = qb + (size_t)chains * npad * D * 2;
+    unsigned char* kt = qb + (size_t)chains * npad * D * 2;
+    unsigned char* tp = kt + (size_t)chains * npad * D * 2;
     unsigned char* pp = tp + (size_t)chains * npad * C * 2;
-    CUtensorMap mq, mk, mv, mo, mw, mqb, mt, mp;
+    CUtensorMap mq, mk, mv, mo, mw, mqb, mkt, mt, mp;
     if (!make_map(&mq, a.q, D, a.N, chains) || !make_map(&mk, a.k, D, a.N, chains) ||
         !make_map(&mv, a.v, a.dv, a.N, chains) || !make_map(&mo, a.out, a.dv, a.N, chains) ||
         !make_map(&mw, wneg, D, npad, chains) || !make_map(&mqb, qb, D, npad, chains) ||
+        !make_map(&mkt, kt, D, npad, chains) ||
         !make_map(&mt, tp, C, npad, chains) || !make_map(&mp, pp, C, npad, chains))
         return cudaErrorInvalidValue;
     const int sms = sm_count();
@@ -866,7 +939,7 @@ cudaError_t launch_gd(const PrefillArgs& a)
     if (e != cudaSuccess) return e;
     const long long items = (long long)chains * nch;
     const int g1 = (int)std::min<long long>(items, 2LL * sms);
-    k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mqb, mt, mp, a.alpha, a.g, a.N, chains);
+    k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mqb, mkt, mt, mp, a.alpha, a.g, a.N, chains);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -874,7 +947,7 @@ cudaError_t launch_gd(const PrefillArgs& a)
     const int s2 = ChainPlan<D>::BYTES;
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
     if (e != cudaSuccess) return e;
-    k2<<<chains * (a.dv / DVT), kChainThreads, s2, a.stream>>>(mqb, mk, mv, mw, mt, mp, mo, a.alpha, a.S0, a.S_out,
+    k2<<<chains * (a.dv / DVT), kChainThreads, s2, a.stream>>>(mqb, mkt, mv, mw, mt, mp, mo, a.alpha, a.S0, a.S_out,
                                                            a.N, a.dv);
     return cudaGetLastError();
 }
@@ -885,7 +958,7 @@ size_t gd_workspace_bytes(int B, int H, int N, int d, int dv)
 {
     (void)dv;
     const size_t npad = (size_t)((N + C - 1) / C) * C;
-    return (size_t)B * H * npad * (size_t)(2 * d + 2 * C) * 2;
+    return (size_t)B * H * npad * (size_t)(3 * d + 2 * C) * 2;
 }
 
 cudaError_t launch_prefill_tc_gated_delta(const PrefillArgs& a)

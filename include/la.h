@@ -146,8 +146,8 @@ LA_API la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
  * sizes and this cfg (dtype, mode).  0 means no workspace is needed.  The
  * workspace carries data between the kernels of one call: per-segment state
  * summaries for bf16 LA_PLAIN / LA_DECAY, and for bf16 LA_GATED_DELTA the
- * per-chunk operands (-W, diag(b) q, T' and the masked score block, bf16,
- * ceil(N/64)*64 rows of 2d + 128 values per chain).  Its content need not be initialised and
+ * per-chunk operands (-W, diag(b) q, diag(b_C/b) k, T' and the masked score
+ * block, bf16, ceil(N/64)*64 rows of 3d + 128 values per chain).  Its content need not be initialised and
  * is dead after the call's work completes.  Two calls in flight at once need
  * two workspaces.
  */

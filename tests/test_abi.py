@@ -92,7 +92,7 @@ def test_workspace_query_is_host_only():
 
 
 def test_gated_delta_workspace_size():
-    # bf16 gated delta: per chain ceil(N/64)*64 rows of 2d + 128 bf16 values; f32 needs none
+    # bf16 gated delta: per chain ceil(N/64)*64 rows of 3d + 128 bf16 values; f32 needs none
     n = la.la_prefill_workspace_bytes(1, 32, 1000, 128, 128, "bf16", "gated_delta")
-    assert n == 32 * 1024 * (2 * 128 + 128) * 2
+    assert n == 32 * 1024 * (3 * 128 + 128) * 2
     assert la.la_prefill_workspace_bytes(1, 32, 1000, 128, 128, "f32", "gated_delta") == 0
