@@ -53,7 +53,10 @@ constexpr float kFrameLimit = 40.f;
 // Shared-memory plan of the chunk kernel (all tiles 1024-byte aligned).
 template <int D, int DV, bool DECAY>
 struct ChunkPlan {
-    static constexpr int STAGES = (D + DV > 128) ? 3 : 4;
+    // d = dv = 64: two CTAs share an SM (three stages, 256 TMEM columns, at
+    // most 60 registers a thread), so one CTA's waits hide behind the other's work
+    static constexpr bool TWO_PER_SM = D == 64 && DV == 64;
+    static constexpr int STAGES = TWO_PER_SM ? (DECAY ? 2 : 3) : (D + DV > 128) ? 3 : 4;
     static constexpr int QB = C * D * 2, KB = C * D * 2, VB = C * DV * 2;
     static constexpr int STAGE = QB + KB + VB;
     static constexpr int OFF_KH = STAGES * STAGE;                 // K^ (frame-weighted phi(K)), decay only
@@ -77,7 +80,9 @@ struct ChunkPlan {
     static_assert(OFF_ONES + 8 * 1024 <= OFF_RSP, "ones operand must stay inside the plan");
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
     // TMEM columns: scores, output^T, state^T, normaliser row
-    static constexpr uint32_t T_P = 0, T_O = 64, T_S = 128, T_Z = 256, T_COLS = 512;
+    static constexpr uint32_t T_P = 0, T_O = 64, T_S = 128;
+    static constexpr uint32_t T_Z = TWO_PER_SM ? 192 : 256, T_COLS = TWO_PER_SM ? 256 : 512;
+    static_assert(!TWO_PER_SM || 2 * (BYTES + 1024) <= 233472, "two CTAs per SM");
 };
 
 template <int D, int DV>
@@ -319,7 +324,7 @@ scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float
 //            move, z of c+1, Q^/K^ of c+1 and Q^.z;  [outputs ready] 1/den,
 //            o = O^T/den -> staging tile                              -> B1
 template <int D, int DV, bool DECAY>
-__global__ void __launch_bounds__(kThreads + 32, 1)
+__global__ void __launch_bounds__(kThreads + 32, ChunkPlan<D, DV, DECAY>::TWO_PER_SM ? 2 : 1)
 chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
              const float* __restrict__ gamma, const float* __restrict__ ws, int N, int H, int G, int L, float eps)
@@ -775,14 +780,15 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
 
 TcSegments tc_segments(int B, int H, int N, int d, int dv)
 {
-    (void)d; (void)dv;
     TcSegments s;
     const long long chains = (long long)B * H;
     if (N <= 0 || chains <= 0) return s;
-    // One CTA per SM runs one segment at a time.  Prefer whole waves of long
-    // segments: G segments per chain with chains * G close to a multiple of
-    // the SM count, and segments of at most kMaxSeg tokens.
-    constexpr long long kSMs = 148, kMaxSeg = 4096;
+    // One CTA (two for d = dv = 64) per SM runs one segment at a time.  Prefer
+    // whole waves of long segments: G segments per chain with chains * G close
+    // to a multiple of the resident CTA count, and segments of at most kMaxSeg
+    // tokens.
+    constexpr long long kMaxSeg = 4096;
+    const long long kSMs = (d == 64 && dv == 64) ? 2 * 148 : 148;
     long long G = 1, L = N;
     for (long long waves = 1;; ++waves) {
         G = waves * kSMs / chains;
