@@ -30,6 +30,7 @@ MODES = {"plain": 0, "decay": 1, "gated_delta": 2}
 
 # Symbols the library exports; the header include/la.h declares exactly these.
 EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
+           "la_set_stage_events",
            "la_prefill_check", "la_status_string", "la_version")
 
 
@@ -69,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.la_gated_delta_decode_step.restype = i
         L.la_prefill_check.argtypes = [vp, vp]
         L.la_prefill_check.restype = i
+        L.la_set_stage_events.argtypes = [ctypes.POINTER(vp), i]
+        L.la_set_stage_events.restype = i
         L.la_status_string.argtypes = [i]
         L.la_status_string.restype = ctypes.c_char_p
         L.la_version.argtypes = []
@@ -192,6 +195,17 @@ def la_gated_delta_decode_step(q, k, v, alpha, g, S, out=None, stream=None):
     if rc != LA_OK:
         raise LaError(rc, "la_gated_delta_decode_step")
     return out
+
+
+def la_set_stage_events(events=None):
+    """Profiling hook: record torch.cuda.Event events[i] after the i-th kernel
+    of every later call (None or [] turns it off).  The events must have been
+    recorded once (so that they exist) and stay alive while the hook is set."""
+    events = list(events or [])
+    arr = (ctypes.c_void_p * max(1, len(events)))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    rc = lib().la_set_stage_events(arr, len(events))
+    if rc != LA_OK:
+        raise LaError(rc, "la_set_stage_events")
 
 
 def la_prefill_check(workspace=None, stream=None):

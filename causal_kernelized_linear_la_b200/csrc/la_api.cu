@@ -11,9 +11,19 @@ namespace {
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool head_ok(int x) { return x == 64 || x == 128; }
 
+// Stage events of la_set_stage_events (process-wide; see la.h).
+constexpr int kMaxStageEvents = 8;
+cudaEvent_t g_stage_events[kMaxStageEvents];
+int g_stage_count = 0;
+
 la_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
 
 }  // namespace
+
+void stage_mark(int i, cudaStream_t stream)
+{
+    if (i < g_stage_count) cudaEventRecord(g_stage_events[i], stream);
+}
 
 // bf16 kernelized prefill runs on the tensor cores; fp32 inputs stay on the
 // fp32 SIMT kernels (bf16 operands could not meet a 1e-4 error bound).
@@ -207,6 +217,16 @@ la_status la_gated_delta_decode_step(const void* q, const void* k, const void* v
     a.B = B; a.H = H; a.d = d; a.dv = dv; a.dtype = cfg->dtype;
     a.stream = static_cast<cudaStream_t>(cfg->stream);
     return la::from_cuda(la::launch_decode_gated_delta(a));
+}
+
+la_status la_set_stage_events(void* const* events, int n)
+{
+    if (n < 0 || n > la::kMaxStageEvents || (n > 0 && !events)) return LA_ERR_INVALID;
+    for (int i = 0; i < n; ++i)
+        if (!events[i]) return LA_ERR_INVALID;
+    for (int i = 0; i < n; ++i) la::g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    la::g_stage_count = n;
+    return LA_OK;
 }
 
 la_status la_prefill_check(const void* workspace, void* stream)

@@ -195,7 +195,9 @@ cudaError_t launch_kz(const DecodeArgs& a)
     const long long n = (long long)a.B * a.H;
     decode_kernelized<T, D, DV><<<(unsigned)n, kThreads, 0, a.stream>>>(
         (const T*)a.q, (const T*)a.k, (const T*)a.v, a.S, a.z, (T*)a.out, a.eps);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) stage_mark(0, a.stream);
+    return e;
 }
 
 template <typename T, int D, int DV>
@@ -204,7 +206,9 @@ cudaError_t launch_gd(const DecodeArgs& a)
     const long long n = (long long)a.B * a.H;
     decode_gated_delta<T, D, DV><<<(unsigned)n, kThreads, 0, a.stream>>>(
         (const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.g, a.S, (T*)a.out);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) stage_mark(0, a.stream);
+    return e;
 }
 
 }  // namespace

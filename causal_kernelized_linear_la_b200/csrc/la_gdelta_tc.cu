@@ -942,6 +942,7 @@ cudaError_t launch_gd(const PrefillArgs& a)
     k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mqb, mkt, mt, mp, a.alpha, a.g, a.N, chains);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    stage_mark(0, a.stream);
 
     auto k2 = gd_chain_kernel<D>;
     const int s2 = ChainPlan<D>::BYTES;
@@ -949,7 +950,9 @@ cudaError_t launch_gd(const PrefillArgs& a)
     if (e != cudaSuccess) return e;
     k2<<<chains * (a.dv / DVT), kChainThreads, s2, a.stream>>>(mqb, mkt, mv, mw, mt, mp, mo, a.alpha, a.S0, a.S_out,
                                                            a.N, a.dv);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stage_mark(1, a.stream);
+    return cudaSuccess;
 }
 
 }  // namespace

@@ -75,4 +75,8 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Profiling hook (la_set_stage_events): record the caller's i-th event on
+// `stream` right after a call's i-th kernel launch, if one is set.
+void stage_mark(int i, cudaStream_t stream);
+
 }  // namespace la

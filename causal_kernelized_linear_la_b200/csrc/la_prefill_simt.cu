@@ -156,7 +156,9 @@ cudaError_t launch_kernelized_t(const PrefillArgs& a)
     dim3 grid(a.B * a.H, a.dv / DVT);
     kern<<<grid, kThreads, smem, a.stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.gamma, a.S0, a.z0,
                                              (T*)a.out, a.S_out, a.z_out, a.H, a.N, a.dv, a.eps);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stage_mark(0, a.stream);
+    return cudaSuccess;
 }
 
 // ---------------------------------------------------------------------------
@@ -243,7 +245,9 @@ cudaError_t launch_gdelta_t(const PrefillArgs& a)
     dim3 grid(a.B * a.H, (a.dv + threads - 1) / threads);
     gated_delta_token_simt<T, D><<<grid, threads, 0, a.stream>>>(
         (const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.g, a.S0, (T*)a.out, a.S_out, a.N, a.dv);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) stage_mark(0, a.stream);
+    return e;
 }
 
 }  // namespace

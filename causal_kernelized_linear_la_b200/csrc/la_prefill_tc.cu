@@ -761,19 +761,23 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     if (e != cudaSuccess) return e;
     ka<<<units, kThreads, sa, a.stream>>>(mk, mv, a.gamma, ws, a.N, a.H, sg.G, sg.L);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stage_mark(0, a.stream);
 
     constexpr int SLOT = D * DV + D;
     dim3 gs(chains, (SLOT + 255) / 256);
     scan_kernel<D, DV, DECAY><<<gs, 256, 0, a.stream>>>(ws, a.gamma, a.S0, a.z0, a.S_out, a.z_out, a.N, a.H,
                                                         sg.G, sg.L);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stage_mark(1, a.stream);
 
     auto kc = chunk_kernel<D, DV, DECAY>;
     const int sc = ChunkPlan<D, DV, DECAY>::BYTES;
     e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, sc);
     if (e != cudaSuccess) return e;
     kc<<<units, kThreads + 32, sc, a.stream>>>(mq, mk, mv, mo, a.gamma, ws, a.N, a.H, sg.G, sg.L, a.eps);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stage_mark(2, a.stream);
+    return cudaSuccess;
 }
 
 }  // namespace

@@ -186,6 +186,21 @@ LA_API la_status la_gated_delta_decode_step(const void* q, const void* k, const 
                                      int B, int H, int d, int dv, const la_config* cfg);
 
 /*
+ * la_set_stage_events -- profiling hook, off by default.  With n > 0, every
+ * later la_prefill / la_decode_step / la_gated_delta_decode_step records
+ * events[i] on its cfg->stream right after launching its i-th kernel
+ * (i < n; a call launches 1 to 3 kernels: bf16 LA_PLAIN/LA_DECAY prefill =
+ * segment summaries, scan, chunk loop; bf16 LA_GATED_DELTA prefill = chunk
+ * prep, chain; every other path one kernel).  events are cudaEvent_t handles
+ * owned by the caller, who must keep them alive while the hook is set; n = 0
+ * turns it off.  The setting is process-wide and not thread-safe: set it
+ * only while no other thread launches through this library.  Returns
+ * LA_ERR_INVALID for n outside 0..8 or a NULL handle.  Not from the pages: a
+ * service for timing each kernel of a call with CUDA events.
+ */
+LA_API la_status la_set_stage_events(void* const* events, int n);
+
+/*
  * la_prefill_check -- wait for the work enqueued on `stream` and report any
  * device-side error recorded in `workspace` by the last la_prefill that used
  * it (LA_ERR_TIMEOUT if a bounded wait between cooperating blocks gave up).

@@ -96,3 +96,15 @@ def test_gated_delta_workspace_size():
     n = la.la_prefill_workspace_bytes(1, 32, 1000, 128, 128, "bf16", "gated_delta")
     assert n == 32 * 1024 * (3 * 128 + 128) * 2
     assert la.la_prefill_workspace_bytes(1, 32, 1000, 128, 128, "f32", "gated_delta") == 0
+
+
+def test_stage_events_validation():
+    # host-only: argument checks of the profiling hook, no CUDA call is made
+    L = la.lib()
+    c = ctypes.c_void_p
+    assert L.la_set_stage_events(None, 1) == la.LA_ERR_INVALID
+    arr = (c * 1)(c(0))
+    assert L.la_set_stage_events(arr, 1) == la.LA_ERR_INVALID      # NULL handle
+    assert L.la_set_stage_events(arr, 9) == la.LA_ERR_INVALID      # more than 8
+    assert L.la_set_stage_events(None, -1) == la.LA_ERR_INVALID
+    assert L.la_set_stage_events(None, 0) == la.LA_OK              # off
