@@ -311,7 +311,8 @@ def run_gpu(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     hbm_peak, tc_peak, peak_kind = _measured_peaks()
     spec = inputs.WORKLOADS[args.workload]
-    p = inputs.make_workload(args.workload, seed=rank_seed(spec["seed"], rank))
+    over = {"N": args.seq_len} if args.seq_len else {}
+    p = inputs.make_workload(args.workload, seed=rank_seed(spec["seed"], rank), **over)
     u = prefill_units(p)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
@@ -371,6 +372,8 @@ def run_gpu(args, world, rank, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk_sum,
     }
+    if args.seq_len:
+        line["config"]["note"] = "seq_len overridden for profiling; not the benchmark configuration"
     if extra:
         line["other_workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -555,6 +558,9 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="profiling aid: the workload with this many tokens per chain instead of its own "
+                         "(the line's config says so); not a benchmark configuration")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     args.steps = max(1, args.steps)
