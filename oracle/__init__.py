@@ -16,6 +16,8 @@ return float64 arrays:
   ("Efficient attention variants" §7.4).
 * ``decode_step(q, k, v, S, z, eps)`` -> ``(o, S, z)``: one application of the
   kernelized loop body (gamma = 1) to a given state and one token.
+* ``causal_conv(x, w, cache=None)`` -> ``(y, cache_out)``: the short causal
+  convolution with its conv cache ("What Is Linear Attention?" §5.4).
 
 Parity status: every function is pinned by tests under ``tests/`` (none is
 "parity unpinned").
@@ -74,6 +76,8 @@ def _bind(lib):
     lib.la_oracle_kernelized.restype = None
     lib.la_oracle_gated_delta.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I]
     lib.la_oracle_gated_delta.restype = None
+    lib.la_oracle_causal_conv.argtypes = [P, P, P, P, P, I, I, I, I, I]
+    lib.la_oracle_causal_conv.restype = None
     lib.la_oracle_threads.argtypes = []
     lib.la_oracle_threads.restype = I
 
@@ -142,3 +146,19 @@ def gated_delta_step(q, k, v, alpha, g, S):
                         np.asarray(v)[:, :, None, :], np.asarray(alpha)[:, :, None],
                         np.asarray(g)[:, :, None], S)
     return o[:, :, 0, :], S1
+
+
+def causal_conv(x, w, cache=None):
+    """x [B,H,N,d], w [H,d,W], cache [B,H,W-1,d] or None (zero history)
+    -> (y [B,H,N,d], cache_out [B,H,W-1,d])."""
+    x, w, cache = _f64(x), _f64(w), _f64(cache)
+    B, H, N, d = x.shape
+    W = w.shape[-1]
+    assert w.shape == (H, d, W) and W >= 1
+    if cache is not None:
+        assert cache.shape == (B, H, W - 1, d)
+    y = np.empty((B, H, N, d))
+    cache_out = np.empty((B, H, W - 1, d))
+    _load().la_oracle_causal_conv(_ptr(x), _ptr(w), _ptr(cache), _ptr(y), _ptr(cache_out) if W > 1 else None,
+                                  B, H, N, d, W)
+    return y, cache_out

@@ -152,6 +152,37 @@ void la_oracle_gated_delta(const double* q, const double* k, const double* v,
     }
 }
 
+/* Short causal convolution ("What Is Linear Attention?" §5.4): a window of the
+ * last w tokens, one filter per (head, channel), no activation.  With the
+ * previous w-1 inputs of the chain as the window's history (cache; zero when
+ * absent), xh = [cache; x] and
+ *     y_t[c] = sum_{i=0}^{w-1} W[h][c][i] * xh[t + i][c]      (xh[t + w-1] = x_t)
+ * and the new cache is the last w-1 rows of xh. */
+void la_oracle_causal_conv(const double* x, const double* W, const double* cache,
+                           double* y, double* cache_out, int B, int H, int N, int d, int w)
+{
+    const int chains = B * H, hist = w - 1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int ch = 0; ch < chains; ++ch) {
+        const int h = ch % H;
+        const double* xc = x + (size_t)ch * N * d;
+        const double* cc = cache ? cache + (size_t)ch * hist * d : NULL;
+        /* row r of the history-extended sequence, channel c */
+#define XH(r, c) ((r) < hist ? (cc ? cc[(size_t)(r) * d + (c)] : 0.0) : xc[(size_t)((r) - hist) * d + (c)])
+        for (int t = 0; t < N; ++t)
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int i = 0; i < w; ++i) acc += W[((size_t)h * d + c) * w + i] * XH(t + i, c);
+                y[((size_t)ch * N + t) * d + c] = acc;
+            }
+        if (cache_out)
+            for (int r = 0; r < hist; ++r)
+                for (int c = 0; c < d; ++c)
+                    cache_out[((size_t)ch * hist + r) * d + c] = XH(N + r, c);
+#undef XH
+    }
+}
+
 int la_oracle_threads(void)
 {
 #ifdef _OPENMP

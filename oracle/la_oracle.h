@@ -46,6 +46,13 @@ void la_oracle_gated_delta(const double* q, const double* k, const double* v,
                            double* o, double* S_out,
                            int B, int H, int N, int d, int dv);
 
+/* Short causal convolution ("What Is Linear Attention?" §5.4): x [B,H,N,d],
+ * W [H,d,w], cache [B,H,w-1,d] or NULL (zero history) -> y [B,H,N,d] and, if
+ * cache_out is not NULL, the last w-1 inputs [B,H,w-1,d].  Weight i multiplies
+ * the input w-1-i tokens back (the last weight the current token). */
+void la_oracle_causal_conv(const double* x, const double* W, const double* cache,
+                           double* y, double* cache_out, int B, int H, int N, int d, int w);
+
 /* Number of OpenMP threads the oracle will use. */
 int la_oracle_threads(void);
 

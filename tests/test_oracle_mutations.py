@@ -22,6 +22,11 @@ MUTANTS = {
     "delta_reads_with_key": ("for (int i = 0; i < d; ++i) s += S[(size_t)i * dv + j] * qt[i];",
                              "for (int i = 0; i < d; ++i) s += S[(size_t)i * dv + j] * kt[i];"),
     "delta_gate_dropped": ("gt * kt[i] * (vt[j]", "kt[i] * (vt[j]"),
+    "conv_reversed_taps": ("W[((size_t)h * d + c) * w + i] * XH(t + i, c)",
+                           "W[((size_t)h * d + c) * w + (w - 1 - i)] * XH(t + i, c)"),
+    "conv_window_off_by_one": ("acc += W[((size_t)h * d + c) * w + i] * XH(t + i, c);",
+                               "acc += W[((size_t)h * d + c) * w + i] * XH(t + i + 1 < N + hist ? t + i + 1 : t + i, c);"),
+    "conv_cache_ignored": ("(cc ? cc[(size_t)(r) * d + (c)] : 0.0)", "0.0"),
 }
 
 

@@ -293,3 +293,83 @@ def test_phi_is_elu_plus_one():
     np.testing.assert_allclose(z[0, 0], ref, rtol=1e-15, atol=4e-16)
     neg = x < 0
     np.testing.assert_allclose(S[0, 0, neg, 0], np.exp(x[neg]), rtol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Short causal convolution with conv cache ([A] §5.4: x'_t = Conv(x_{t-w:t});
+# a "conv cache" keeps the recent tokens' window for decoding).
+
+@pytest.mark.parametrize("W", [1, 2, 4, 5])
+def test_conv_equals_numpy_convolve(W):
+    # With zero history, output channel c of a chain is the full linear
+    # convolution of the channel with its filter, truncated to N (numpy's
+    # convolve reverses the kernel, so the filter is passed reversed: the last
+    # weight meets the current token).
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((2, 3, 37, 6))
+    w = rng.standard_normal((3, 6, W))
+    y, _ = oracle.causal_conv(x, w)
+    for b in range(2):
+        for h in range(3):
+            for c in range(6):
+                ref = np.convolve(x[b, h, :, c], w[h, c, ::-1])[:37]
+                np.testing.assert_allclose(y[b, h, :, c], ref, rtol=0, atol=1e-12)
+
+
+def test_conv_impulse_response():
+    # A unit impulse at token t0 of one channel answers with the filter
+    # reversed: y_{t0+j} = w[W-1-j] for j < W, and nothing before t0 (causality).
+    W, N, t0 = 4, 12, 5
+    x = np.zeros((1, 1, N, 2))
+    x[0, 0, t0, 1] = 1.0
+    w = np.array([[[0.0, 0.0, 0.0, 0.0], [0.5, -1.5, 2.0, 3.0]]])
+    y, _ = oracle.causal_conv(x, w)
+    expect = np.zeros(N)
+    for j in range(W):
+        expect[t0 + j] = w[0, 1, W - 1 - j]
+    np.testing.assert_array_equal(y[0, 0, :, 1], expect)
+    np.testing.assert_array_equal(y[0, 0, :, 0], np.zeros(N))
+
+
+@pytest.mark.parametrize("n1", [0, 1, 2, 9, 30])
+def test_conv_cache_continues_the_sequence(n1):
+    # Splitting a sequence anywhere and carrying the cache gives the same outputs
+    # and the same final cache as one pass, bit for bit (the same products in the
+    # same order); the cache is the last W-1 inputs of the history-extended sequence.
+    rng = np.random.default_rng(8)
+    W, N = 4, 30
+    x = rng.standard_normal((2, 2, N, 5))
+    w = rng.standard_normal((2, 5, W))
+    c0 = rng.standard_normal((2, 2, W - 1, 5))
+    y, c = oracle.causal_conv(x, w, c0)
+    ya, ca = oracle.causal_conv(x[:, :, :n1], w, c0)
+    yb, cb = oracle.causal_conv(x[:, :, n1:], w, ca)
+    np.testing.assert_array_equal(np.concatenate([ya, yb], axis=2), y)
+    np.testing.assert_array_equal(cb, c)
+    xh = np.concatenate([c0, x], axis=2)
+    np.testing.assert_array_equal(c, xh[:, :, -(W - 1):])
+    # decoding token by token is the same again
+    cc = c0
+    for t in range(N):
+        yt, cc = oracle.causal_conv(x[:, :, t:t + 1], w, cc)
+        np.testing.assert_array_equal(yt[:, :, 0], y[:, :, t])
+
+
+def test_conv_short_sequence_keeps_old_cache_rows():
+    # N < W-1: the new cache still holds W-1-N of the old cache rows, shifted.
+    rng = np.random.default_rng(9)
+    W = 5
+    x = rng.standard_normal((1, 1, 2, 3))
+    w = rng.standard_normal((1, 3, W))
+    c0 = rng.standard_normal((1, 1, W - 1, 3))
+    _, c = oracle.causal_conv(x, w, c0)
+    np.testing.assert_array_equal(c[0, 0, :2], c0[0, 0, 2:])
+    np.testing.assert_array_equal(c[0, 0, 2:], x[0, 0])
+
+
+def test_conv_width_one_is_a_channel_scale():
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((2, 2, 7, 4))
+    w = rng.standard_normal((2, 4, 1))
+    y, _ = oracle.causal_conv(x, w)
+    np.testing.assert_allclose(y, x * w[None, :, None, :, 0], rtol=0, atol=1e-15)
