@@ -471,6 +471,34 @@ def time_kernels(p, steps, torch, la, flush):
     return {n: sum(t) / len(t) for n, t in zip(names, per)}
 
 
+def time_conv(torch, la, rank, flush, hbm_peak, B=4, H=8, N=4096, d=64, w=4, steps=20):
+    """The short causal convolution (with conv cache) over one q-shaped bf16
+    stream of the headline workload's size, filter width 4: device time per
+    call, L2 flushed before each, and its bytes against HBM."""
+    g = torch.Generator(device="cpu").manual_seed(rank_seed(77, rank))
+    x = (torch.randn((B, H, N, d), generator=g) / 8).to(torch.bfloat16).cuda()
+    wt = (torch.randn((H, d, w), generator=g) / 2).cuda()
+    c0 = torch.randn((B, H, w - 1, d), generator=g).to(torch.bfloat16).cuda()
+    out = torch.empty_like(x)
+    c1 = torch.empty_like(c0)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        flush.fill_(1)
+        la.la_causal_conv(x, wt, c0, out=out, cache_out=c1)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        flush.fill_(1)
+        a.record(stream)
+        la.la_causal_conv(x, wt, c0, out=out, cache_out=c1)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    nbytes = 2 * x.numel() * 2 + wt.numel() * 4 + 2 * c0.numel() * 2
+    return {"shape": f"x [B={B},H={H},N={N},d={d}] bf16, w={w}", "ms": ms,
+            "tokens_per_s": B * N / (ms / 1e3), "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+            "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak}
+
+
 def run_extra(args, torch, la, rank, flush):
     """Device-timed numbers for the other workloads (not the headline line)."""
     res = {}
@@ -484,6 +512,7 @@ def run_extra(args, torch, la, rank, flush):
         res[name] = {"tokens_per_s": u["tokens"] / (ms / 1e3), "ms": ms,
                      "hbm_frac": u["bytes"] / (ms / 1e3) / 1e9 / hbm_peak, "dtype": path_dtype(p)}
         del p
+    res["conv"] = time_conv(torch, la, rank, flush, hbm_peak)
     dspec = inputs.WORKLOADS["decode"]
     dms = time_decode(1000, 20, torch, la, rank_seed(dspec["seed"], rank))
     du = decode_units(dspec["S"], dspec["H"], dspec["d"], dspec["dv"])

@@ -30,7 +30,7 @@ MODES = {"plain": 0, "decay": 1, "gated_delta": 2}
 
 # Symbols the library exports; the header include/la.h declares exactly these.
 EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
-           "la_set_stage_events",
+           "la_set_stage_events", "la_causal_conv",
            "la_prefill_check", "la_status_string", "la_version")
 
 
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.la_gated_delta_decode_step.restype = i
         L.la_prefill_check.argtypes = [vp, vp]
         L.la_prefill_check.restype = i
+        L.la_causal_conv.argtypes = [vp] * 5 + [i] * 5 + [cfgp]
+        L.la_causal_conv.restype = i
         L.la_set_stage_events.argtypes = [ctypes.POINTER(vp), i]
         L.la_set_stage_events.restype = i
         L.la_status_string.argtypes = [i]
@@ -195,6 +197,31 @@ def la_gated_delta_decode_step(q, k, v, alpha, g, S, out=None, stream=None):
     if rc != LA_OK:
         raise LaError(rc, "la_gated_delta_decode_step")
     return out
+
+
+def la_causal_conv(x, weight, cache=None, out=None, cache_out=None, stream=None):
+    """Short causal convolution with conv cache on device tensors.
+    x [B,H,N,d] bf16/fp32, weight [H,d,w] fp32, cache [B,H,w-1,d] or None.
+    Returns (out, cache_out); cache_out is allocated when not given."""
+    if x.dim() != 4 or weight.dim() != 3:
+        raise ValueError("x must be [B,H,N,d] and weight [H,d,w]")
+    torch = _torch()
+    B, H, N, d = x.shape
+    w = weight.shape[-1]
+    if weight.shape != (H, d, w) or weight.dtype != torch.float32:
+        raise ValueError("weight must be fp32 [H,d,w]")
+    dev = x.device
+    if out is None:
+        out = torch.empty_like(x)
+    if cache_out is None and w > 1:
+        cache_out = torch.empty((B, H, w - 1, d), device=dev, dtype=x.dtype)
+    _check_cuda(x, weight, cache, out, cache_out)
+    cfg = LaConfig(_dtype_code(x), 0, 0.0, _stream_handle(stream), None, None, None, 0)
+    rc = lib().la_causal_conv(_ptr(x), _ptr(weight), _ptr(cache), _ptr(out), _ptr(cache_out),
+                              B, H, N, d, w, ctypes.byref(cfg))
+    if rc != LA_OK:
+        raise LaError(rc, "la_causal_conv")
+    return out, cache_out
 
 
 def la_set_stage_events(events=None):

@@ -219,6 +219,40 @@ la_status la_gated_delta_decode_step(const void* q, const void* k, const void* v
     return la::from_cuda(la::launch_decode_gated_delta(a));
 }
 
+la_status la_causal_conv(const void* x, const float* weight, const void* cache, void* out, void* cache_out,
+                         int B, int H, int N, int d, int w, const la_config* cfg)
+{
+    if (!cfg) return LA_ERR_INVALID;
+    if (B < 0 || H < 0 || N < 0 || w < 1) return LA_ERR_INVALID;
+    if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
+    if (!la::head_ok(d) || w > 8) return LA_ERR_UNSUPPORTED;
+    const long long chains = (long long)B * H;
+    if (chains == 0) return LA_OK;
+    if (N > 0 && (!x || !weight || !out)) return LA_ERR_INVALID;
+    const size_t es = cfg->dtype == LA_BF16 ? 2 : 4;
+    const size_t cache_bytes = (size_t)chains * (w - 1) * d * es;
+    auto overlap = [](const void* a, size_t na, const void* b, size_t nb) {
+        if (!a || !b || na == 0 || nb == 0) return false;
+        const char* pa = static_cast<const char*>(a);
+        const char* pb = static_cast<const char*>(b);
+        return pa < pb + nb && pb < pa + na;
+    };
+    if (overlap(cache_out, cache_bytes, cache, cache_bytes) ||
+        overlap(cache_out, cache_bytes, x, (size_t)chains * N * d * es))
+        return LA_ERR_INVALID;
+    const void* ptrs[] = {x, weight, cache, out, cache_out};
+    for (const void* p : ptrs)
+        if (!la::aligned16(p)) return LA_ERR_ALIGN;
+    if (N == 0 && !cache_out) return LA_OK;
+    la::ConvArgs a{};
+    a.x = x; a.weight = weight; a.cache = cache; a.y = out; a.cache_out = w > 1 ? cache_out : nullptr;
+    a.B = B; a.H = H; a.N = N; a.d = d; a.w = w;
+    a.dtype = cfg->dtype;
+    a.stream = static_cast<cudaStream_t>(cfg->stream);
+    if (a.N == 0 && !a.cache_out) return LA_OK;
+    return la::from_cuda(la::launch_causal_conv(a));
+}
+
 la_status la_set_stage_events(void* const* events, int n)
 {
     if (n < 0 || n > la::kMaxStageEvents || (n > 0 && !events)) return LA_ERR_INVALID;

@@ -937,6 +937,9 @@ cudaError_t launch_gd(const PrefillArgs& a)
     const int s1 = PrepPlan<D>::BYTES;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e != cudaSuccess) return e;
+    // all of L1 as shared memory, so that two prep CTAs fit on an SM
+    e = cudaFuncSetAttribute(k1, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     const long long items = (long long)chains * nch;
     const int g1 = (int)std::min<long long>(items, 2LL * sms);
     k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mqb, mkt, mt, mp, a.alpha, a.g, a.N, chains);

@@ -46,7 +46,21 @@ struct DecodeArgs {
     cudaStream_t stream;
 };
 
+struct ConvArgs {
+    const void* x;
+    const float* weight;
+    const void* cache;   // may be null: zero history
+    void* y;
+    void* cache_out;     // may be null
+    int B, H, N, d, w;
+    la_dtype dtype;
+    cudaStream_t stream;
+};
+
 bool uses_tc_kernelized(la_dtype dt, la_mode m);
+
+// Short causal convolution with conv cache (memory-bound SIMT).
+cudaError_t launch_causal_conv(const ConvArgs& a);
 
 // SIMT prefill kernels (fp32 arithmetic; fp32 or bf16 inputs).
 cudaError_t launch_prefill_simt_kernelized(const PrefillArgs& a);

@@ -89,25 +89,17 @@ template <int D, int DV>
 struct SummaryPlan {
     static constexpr int STAGES = 4;
     static constexpr int KB = C * D * 2, VB = C * DV * 2;
-    static constexpr int STAGE = KB + VB;
-    static constexpr int OFF_ONES = STAGES * STAGE;
-    static constexpr int OFF_BAR = OFF_ONES + C * C * 2;           // full[S], empty[S], done
+    // stage: K tiles, V tiles, then a constant tile whose column 0 is ones:
+    // B = [V | 1] makes column dv of K~^T B the normaliser sum Delta z
+    static constexpr int LOAD_BYTES = KB + VB;
+    static constexpr int STAGE = KB + VB + TILE;
+    static constexpr int OFF_BAR = STAGES * STAGE;                // full[S], empty[S], done
     static constexpr int OFF_TMEM = OFF_BAR + (2 * STAGES + 1) * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
-    static constexpr uint32_t T_S = 0, T_Z = 128, T_COLS = 256;
+    static constexpr int NS = DV + 16;                            // accumulator columns
+    static constexpr uint32_t T_S = 0, T_COLS = 256;
 };
 
-
-// Constant A operand: a 64 x 64 bf16 tile whose row 0 is all ones.  One MMA
-// with it sums the rows of a B operand into accumulator row 0.
-__device__ __forceinline__ void init_ones_tile(unsigned char* tile, int tid, int nthreads)
-{
-    for (int e = tid; e < C * 8; e += nthreads) {
-        const int row = e / 8;
-        const uint32_t one2 = pack_bf16x2(1.f, 1.f);
-        reinterpret_cast<uint4*>(tile)[e] = row == 0 ? make_uint4(one2, one2, one2, one2) : make_uint4(0, 0, 0, 0);
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Kernel A: segment summaries  Delta S = sum_t gamma^(last-t) phi(k_t) v_t^T,
@@ -120,7 +112,6 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     using P = SummaryPlan<D, DV>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
-    unsigned char* ones = sm + P::OFF_ONES;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* empty = full + P::STAGES;
     uint64_t* done = empty + P::STAGES;
@@ -141,7 +132,14 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, P::T_COLS);
-    init_ones_tile(ones, tid, kThreads);
+    // the ones-column tile of every stage: element (t, 0) = 1, the rest 0
+    for (int s = 0; s < P::STAGES; ++s)
+        for (int e = tid; e < C * 8; e += kThreads) {
+            const int row = e / 8, chunk = e % 8;
+            // logical chunk 0 of row `row` sits at physical chunk row % 8
+            const uint32_t w = chunk == (row & 7) ? 0x3F80u : 0u;   // bf16 1.0 in the low half
+            reinterpret_cast<uint4*>(sm + s * P::STAGE + P::KB + P::VB)[e] = make_uint4(w, 0u, 0u, 0u);
+        }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -152,7 +150,7 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     auto issue = [&](int c) {
         const int s = c % P::STAGES;
         unsigned char* st = sm + s * P::STAGE;
-        mbar_expect_tx(&full[s], P::STAGE);
+        mbar_expect_tx(&full[s], P::LOAD_BYTES);
         for (int b = 0; b < D / 64; ++b) tma_load_3d(st + b * TILE, &tm_k, b * 64, t0 + c * C, chain, &full[s], pol);
         for (int b = 0; b < DV / 64; ++b)
             tma_load_3d(st + P::KB + b * TILE, &tm_v, b * 64, t0 + c * C, chain, &full[s], pol);
@@ -190,22 +188,20 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tc_fence_before();
         if (__syncthreads_or(bad)) { bad = true; break; }
         if (tid == 0) {
+            // [Delta S | Delta z] += K~^T [V | 1]   (M = d, N = dv + 16)
             tc_fence_after();
-            const uint32_t ka = smem_u32(kt), va = smem_u32(vt), oa = smem_u32(ones);
-            const uint32_t id_s = idesc_bf16_f32(D, DV, 1, 1);
-            const uint32_t id_z = idesc_bf16_f32(64, D, 0, 1);
+            const uint32_t ka = smem_u32(kt), va = smem_u32(vt);
+            const uint32_t id_s = idesc_bf16_f32(D, P::NS, 1, 1);
 #pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t bk = sdesc_sw128(ka + ks * 2048, TILE, 1024);
-                mma_bf16(tbase + P::T_S, bk, sdesc_sw128(va + ks * 2048, TILE, 1024), id_s, (c > 0 || ks > 0));
-                mma_bf16(tbase + P::T_Z, sdesc_sw128(oa + ks * 32, 16, 1024), bk, id_z, (c > 0 || ks > 0));
-            }
+            for (int ks = 0; ks < C / 16; ++ks)
+                mma_bf16(tbase + P::T_S, sdesc_sw128(ka + ks * 2048, TILE, 1024),
+                         sdesc_sw128(va + ks * 2048, TILE, 1024), id_s, (c > 0 || ks > 0));
             mma_commit(&empty[s]);
             if (c == nch - 1) mma_commit(done);
             commits = c + 1;
         }
-        // refill the stage chunk c-1 used: its MMA was issued a whole chunk ago
-        __syncthreads();
+        // refill the stage chunk c-1 used: its MMA was issued a whole chunk ago.
+        // The other threads go on to phi of the next chunk meanwhile.
         if (tid == 0 && c >= 1 && c - 1 + P::STAGES < nch) {
             const int sp = (c - 1) % P::STAGES;
             if (!mbar_wait(&empty[sp], ((c - 1) / P::STAGES) & 1, kErrMma)) bad = true;
@@ -229,21 +225,12 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                 for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
         }
-        // Delta z: row 0 of the ones-row product, in lane 0 of quadrant 0
-        if (quad == 0) {
-#pragma unroll
-            for (int gg = 0; gg < D / 64; ++gg) {
-                const int col0 = wg * (D / 4) + gg * 16;
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, 0, P::T_Z + col0), v);
-                tmem_ld_wait();
-                if (lane == 0) {
-                    float4* dst = reinterpret_cast<float4*>(slot + D * DV + col0);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                }
-            }
+        // Delta z: accumulator column dv, one row (feature) per lane
+        if (wg == 0) {
+            float v[16];
+            tmem_ld16(tmem_addr(tbase, quad, P::T_S + DV), v);
+            tmem_ld_wait();
+            if (f >= 0) slot[D * DV + f] = v[0];
         }
     }
     if (bad && tid == 0) {
@@ -443,8 +430,11 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 make_float4(qw * fq[u][0], qw * fq[u][1], qw * fq[u][2], qw * fq[u][3]);
             *reinterpret_cast<float4*>(qrow + sw128_offset(row, fb + 16)) =
                 make_float4(qw * fq[u][4], qw * fq[u][5], qw * fq[u][6], qw * fq[u][7]);
+            const float4 z0 = *reinterpret_cast<const float4*>(zc + f0);
+            const float4 z1 = *reinterpret_cast<const float4*>(zc + f0 + 4);
+            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
 #pragma unroll
-            for (int x = 0; x < 8; ++x) qz = fmaf(qw * fq[u][x], zc[f0 + x], qz);
+            for (int x = 0; x < 8; ++x) qz = fmaf(qw * fq[u][x], zz[x], qz);
             if (DECAY) {
                 const float kw = row < n ? __expf(-(float)(c0 + row + 1 - ref) * lam) : 0.f;
                 reinterpret_cast<uint4*>(khat + b * TILE)[rem] = pack8(fk[u], kw);
@@ -606,8 +596,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
                         const int j0 = wg * 16 + 2 * h;
-                        const float a = j0 <= i ? v[2 * h] * dtab[i - j0] : 0.f;
-                        const float b = j0 + 1 <= i ? v[2 * h + 1] * dtab[i - j0 - 1] : 0.f;
+                        const float a = j0 <= i ? (DECAY ? v[2 * h] * dtab[i - j0] : v[2 * h]) : 0.f;
+                        const float b = j0 + 1 <= i ? (DECAY ? v[2 * h + 1] * dtab[i - j0 - 1] : v[2 * h + 1]) : 0.f;
                         pk[h] = pack_bf16x2(a, b);
                         const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[h]));
                         rs += r.x + r.y;   // the row sum of exactly the values the MMA uses
@@ -759,6 +749,9 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     const int sa = SummaryPlan<D, DV>::BYTES;
     cudaError_t e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, sa);
     if (e != cudaSuccess) return e;
+    // all of L1 as shared memory, so that two CTAs fit on an SM where their plans allow
+    e = cudaFuncSetAttribute(ka, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     ka<<<units, kThreads, sa, a.stream>>>(mk, mv, a.gamma, ws, a.N, a.H, sg.G, sg.L);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(0, a.stream);
@@ -773,6 +766,8 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     auto kc = chunk_kernel<D, DV, DECAY>;
     const int sc = ChunkPlan<D, DV, DECAY>::BYTES;
     e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, sc);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kc, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     kc<<<units, kThreads + 32, sc, a.stream>>>(mq, mk, mv, mo, a.gamma, ws, a.N, a.H, sg.G, sg.L, a.eps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -186,12 +186,44 @@ LA_API la_status la_gated_delta_decode_step(const void* q, const void* k, const 
                                      int B, int H, int d, int dv, const la_config* cfg);
 
 /*
+ * la_causal_conv -- short causal convolution over the token axis with a conv
+ * cache ("What Is Linear Attention?" §5.4: a short convolution over the last
+ * w tokens beside the linear state; inference keeps the recent window as a
+ * conv cache).  One filter per (head, channel), no activation:
+ *
+ *   xh = [cache; x]  (the chain's previous w-1 inputs, then its N new ones)
+ *   out_t[c] = sum_{i=0}^{w-1} weight[h][c][i] * xh[t + i][c]
+ *
+ * i.e. weight i multiplies the input w-1-i tokens back (the last weight the
+ * current token); cache_out = the last w-1 rows of xh.
+ *
+ *   x          [B,H,N,d] input, element type cfg->dtype (bf16 or fp32).
+ *   weight     [H,d,w] fp32 filters.
+ *   cache      [B,H,w-1,d] (cfg->dtype) previous inputs, or NULL for zero history.
+ *   out        [B,H,N,d] (cfg->dtype); fp32 arithmetic, rounded once.
+ *   cache_out  [B,H,w-1,d] (cfg->dtype) or NULL; must not overlap cache or x
+ *              (continue a stream by alternating two cache buffers).
+ *   w          1..8.  d in {64, 128}.  N >= 0 (N = 0 only moves the cache).
+ *   cfg        dtype and stream are used; mode, eps, S0, z0, workspace ignored.
+ *
+ * Decoding is the N = 1 call.  Returns LA_OK once the work is enqueued;
+ * LA_ERR_INVALID for bad sizes, NULL x/weight/out (when N > 0) or an
+ * overlapping cache_out; LA_ERR_UNSUPPORTED for d or w out of range;
+ * LA_ERR_ALIGN for a pointer not 16-byte aligned.  Not part of the pages'
+ * attention method itself: the adjacent local operator the same layer runs.
+ */
+LA_API la_status la_causal_conv(const void* x, const float* weight, const void* cache,
+                                void* out, void* cache_out,
+                                int B, int H, int N, int d, int w, const la_config* cfg);
+
+/*
  * la_set_stage_events -- profiling hook, off by default.  With n > 0, every
- * later la_prefill / la_decode_step / la_gated_delta_decode_step records
+ * later la_prefill / la_decode_step / la_gated_delta_decode_step /
+ * la_causal_conv records
  * events[i] on its cfg->stream right after launching its i-th kernel
  * (i < n; a call launches 1 to 3 kernels: bf16 LA_PLAIN/LA_DECAY prefill =
  * segment summaries, scan, chunk loop; bf16 LA_GATED_DELTA prefill = chunk
- * prep, chain; every other path one kernel).  events are cudaEvent_t handles
+ * prep, chain; every other path, la_causal_conv included, one kernel).  events are cudaEvent_t handles
  * owned by the caller, who must keep them alive while the hook is set; n = 0
  * turns it off.  The setting is process-wide and not thread-safe: set it
  * only while no other thread launches through this library.  Returns

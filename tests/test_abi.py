@@ -21,6 +21,17 @@ def test_header_declares_the_binding_exports():
     assert declared() == set(la.EXPORTS)
 
 
+def test_binding_argument_counts_match_the_header():
+    # every declared function is bound in Python with as many argument types
+    # as the header gives it parameters
+    src = open(HEADER).read()
+    L = la.lib()
+    for name, params in re.findall(r"LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(([^)]*)\)", src):
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(getattr(L, name).argtypes) == n, name
+
+
 def test_library_exports_every_declared_symbol():
     L = la.lib()
     for name in sorted(declared()):
@@ -108,3 +119,21 @@ def test_stage_events_validation():
     assert L.la_set_stage_events(arr, 9) == la.LA_ERR_INVALID      # more than 8
     assert L.la_set_stage_events(None, -1) == la.LA_ERR_INVALID
     assert L.la_set_stage_events(None, 0) == la.LA_OK              # off
+
+
+def test_conv_validation_host_only():
+    # argument checks of la_causal_conv that return before any CUDA call
+    L = la.lib()
+    c = ctypes.c_void_p
+    cfg = LaConfig(la.LA_BF16, 0, 0.0, None, None, None, None, 0)
+    FAKE = c(1 << 20)   # never dereferenced: every call below fails validation first
+    assert L.la_causal_conv(FAKE, FAKE, None, FAKE, None, 1, 1, 8, 64, 0, ctypes.byref(cfg)) == la.LA_ERR_INVALID
+    assert L.la_causal_conv(FAKE, FAKE, None, FAKE, None, 1, 1, 8, 64, 9, ctypes.byref(cfg)) == la.LA_ERR_UNSUPPORTED
+    assert L.la_causal_conv(FAKE, FAKE, None, FAKE, None, 1, 1, 8, 32, 4, ctypes.byref(cfg)) == la.LA_ERR_UNSUPPORTED
+    assert L.la_causal_conv(None, FAKE, None, FAKE, None, 1, 1, 8, 64, 4, ctypes.byref(cfg)) == la.LA_ERR_INVALID
+    # cache_out overlapping the cache
+    assert L.la_causal_conv(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 4, ctypes.byref(cfg)) == la.LA_ERR_INVALID
+    # misaligned pointer
+    assert L.la_causal_conv(c((1 << 20) + 2), FAKE, None, FAKE, None, 1, 1, 8, 64, 4, ctypes.byref(cfg)) == la.LA_ERR_ALIGN
+    # nothing to do
+    assert L.la_causal_conv(None, None, None, None, None, 0, 4, 8, 64, 4, ctypes.byref(cfg)) == la.LA_OK
