@@ -16,6 +16,8 @@ return float64 arrays:
   ("Efficient attention variants" §7.4).
 * ``decode_step(q, k, v, S, z, eps)`` -> ``(o, S, z)``: one application of the
   kernelized loop body (gamma = 1) to a given state and one token.
+* ``gla(q, k, v, alpha, S0=None)`` -> ``(o, S)``: the per-key-channel gated
+  recurrence ("Efficient attention variants" §7.2).
 * ``causal_conv(x, w, cache=None)`` -> ``(y, cache_out)``: the short causal
   convolution with its conv cache ("What Is Linear Attention?" §5.4).
 
@@ -76,6 +78,8 @@ def _bind(lib):
     lib.la_oracle_kernelized.restype = None
     lib.la_oracle_gated_delta.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I]
     lib.la_oracle_gated_delta.restype = None
+    lib.la_oracle_gla.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I]
+    lib.la_oracle_gla.restype = None
     lib.la_oracle_causal_conv.argtypes = [P, P, P, P, P, I, I, I, I, I]
     lib.la_oracle_causal_conv.restype = None
     lib.la_oracle_threads.argtypes = []
@@ -146,6 +150,20 @@ def gated_delta_step(q, k, v, alpha, g, S):
                         np.asarray(v)[:, :, None, :], np.asarray(alpha)[:, :, None],
                         np.asarray(g)[:, :, None], S)
     return o[:, :, 0, :], S1
+
+
+def gla(q, k, v, alpha, S0=None):
+    """q,k,alpha [B,H,N,d], v [B,H,N,dv] -> o [B,H,N,dv], S [B,H,d,dv]."""
+    q, k, v, alpha, S0 = _f64(q), _f64(k), _f64(v), _f64(alpha), _f64(S0)
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, H, N, d) and alpha.shape == (B, H, N, d) and v.shape == (B, H, N, dv)
+    if S0 is not None:
+        assert S0.shape == (B, H, d, dv)
+    o = np.empty((B, H, N, dv))
+    S = np.empty((B, H, d, dv))
+    _load().la_oracle_gla(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(S0), _ptr(o), _ptr(S), B, H, N, d, dv)
+    return o, S
 
 
 def causal_conv(x, w, cache=None):

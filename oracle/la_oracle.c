@@ -152,6 +152,46 @@ void la_oracle_gated_delta(const double* q, const double* k, const double* v,
     }
 }
 
+/* GLA with a per-key-channel gate ("Efficient attention variants" §7.2): each
+ * entry of alpha_t says how much of the matching row of the state (one key
+ * channel) is kept, broadcast along the value dimension; then the usual write
+ * and read.  No feature map, no normaliser (the §7 recurrences leave both out).
+ *     S_t[i][:] = alpha_t[i] * S_{t-1}[i][:] + k_t[i] * v_t[:]
+ *     o_t = S_t^T q_t
+ * alpha [B,H,N,d]; S0 NULL means a zero start state. */
+void la_oracle_gla(const double* q, const double* k, const double* v, const double* alpha,
+                   const double* S0, double* o, double* S_out, int B, int H, int N, int d, int dv)
+{
+    const int chains = B * H;
+#pragma omp parallel
+    {
+        double* S = (double*)malloc(sizeof(double) * (size_t)d * dv);
+#pragma omp for schedule(dynamic, 1)
+        for (int c = 0; c < chains; ++c) {
+            const size_t qo = (size_t)c * N * d, vo = (size_t)c * N * dv, so = (size_t)c * d * dv;
+            for (size_t e = 0; e < (size_t)d * dv; ++e) S[e] = S0 ? S0[so + e] : 0.0;
+            for (int t = 0; t < N; ++t) {
+                const double* qt = q + qo + (size_t)t * d;
+                const double* kt = k + qo + (size_t)t * d;
+                const double* at = alpha + qo + (size_t)t * d;
+                const double* vt = v + vo + (size_t)t * dv;
+                for (int i = 0; i < d; ++i) {
+                    double* Si = S + (size_t)i * dv;
+                    for (int j = 0; j < dv; ++j) Si[j] = at[i] * Si[j] + kt[i] * vt[j];
+                }
+                double* ot = o + vo + (size_t)t * dv;
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < d; ++i) acc += qt[i] * S[(size_t)i * dv + j];
+                    ot[j] = acc;
+                }
+            }
+            if (S_out) memcpy(S_out + so, S, sizeof(double) * (size_t)d * dv);
+        }
+        free(S);
+    }
+}
+
 /* Short causal convolution ("What Is Linear Attention?" §5.4): a window of the
  * last w tokens, one filter per (head, channel), no activation.  With the
  * previous w-1 inputs of the chain as the window's history (cache; zero when

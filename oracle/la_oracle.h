@@ -46,6 +46,12 @@ void la_oracle_gated_delta(const double* q, const double* k, const double* v,
                            double* o, double* S_out,
                            int B, int H, int N, int d, int dv);
 
+/* GLA, per-key-channel gate ("Efficient attention variants" §7.2):
+ *     S_t = diag(alpha_t) S_{t-1} + k_t v_t^T,  o_t = S_t^T q_t
+ * alpha [B,H,N,d].  No feature map, no normaliser.  S0 NULL: zero start. */
+void la_oracle_gla(const double* q, const double* k, const double* v, const double* alpha,
+                   const double* S0, double* o, double* S_out, int B, int H, int N, int d, int dv);
+
 /* Short causal convolution ("What Is Linear Attention?" §5.4): x [B,H,N,d],
  * W [H,d,w], cache [B,H,w-1,d] or NULL (zero history) -> y [B,H,N,d] and, if
  * cache_out is not NULL, the last w-1 inputs [B,H,w-1,d].  Weight i multiplies

@@ -22,6 +22,10 @@ MUTANTS = {
     "delta_reads_with_key": ("for (int i = 0; i < d; ++i) s += S[(size_t)i * dv + j] * qt[i];",
                              "for (int i = 0; i < d; ++i) s += S[(size_t)i * dv + j] * kt[i];"),
     "delta_gate_dropped": ("gt * kt[i] * (vt[j]", "kt[i] * (vt[j]"),
+    "gla_gate_on_value_dim": ("Si[j] = at[i] * Si[j] + kt[i] * vt[j];", "Si[j] = at[j % d] * Si[j] + kt[i] * vt[j];"),
+    "gla_gate_after_write": ("Si[j] = at[i] * Si[j] + kt[i] * vt[j];", "Si[j] = at[i] * (Si[j] + kt[i] * vt[j]);"),
+    "gla_reads_with_key": ("for (int i = 0; i < d; ++i) acc += qt[i] * S[(size_t)i * dv + j];",
+                           "for (int i = 0; i < d; ++i) acc += kt[i] * S[(size_t)i * dv + j];"),
     "conv_reversed_taps": ("W[((size_t)h * d + c) * w + i] * XH(t + i, c)",
                            "W[((size_t)h * d + c) * w + (w - 1 - i)] * XH(t + i, c)"),
     "conv_window_off_by_one": ("acc += W[((size_t)h * d + c) * w + i] * XH(t + i, c);",

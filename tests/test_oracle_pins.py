@@ -373,3 +373,88 @@ def test_conv_width_one_is_a_channel_scale():
     w = rng.standard_normal((2, 4, 1))
     y, _ = oracle.causal_conv(x, w)
     np.testing.assert_allclose(y, x * w[None, :, None, :, 0], rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# GLA, per-key-channel gate ([B] §7.2): each entry of alpha_t scales the
+# matching row (key channel) of the state, broadcast along the value dimension.
+
+def gla_dense(q, k, v, alpha, S0=None):
+    """Unrolled form for one chain: row i of S_t is
+    prod_{m<=t} a_m[i] S0[i] + sum_{j<=t} (prod_{j<m<=t} a_m[i]) k_j[i] v_j,
+    so o_t = sum_j (q_t * decay_{t,j}) . k_j v_j + (q_t * prod_{m<=t} a_m) S0,
+    with the per-channel decay products taken as exp of log-cumsum differences."""
+    N, d = q.shape
+    L = np.cumsum(np.log(alpha), axis=0)                    # L_t[i] = sum_{m<=t} log a_m[i]
+    o = np.zeros((N, v.shape[1]))
+    for t in range(N):
+        dec = np.exp(L[t][None, :] - L[: t + 1])            # [j, i] = prod_{j<m<=t} a_m[i]
+        w = (dec * k[: t + 1]) @ q[t]                       # sum_i q_t[i] dec[j,i] k_j[i]
+        o[t] = w @ v[: t + 1]
+        if S0 is not None:
+            o[t] += (q[t] * np.exp(L[t])) @ S0
+    S = (np.exp(L[-1][None, :] - L) * k).T @ v
+    if S0 is not None:
+        S += np.exp(L[-1])[:, None] * S0
+    return o, S
+
+
+def _gla_inputs(rng, B, H, N, d, dv):
+    q = rng.standard_normal((B, H, N, d))
+    k = rng.standard_normal((B, H, N, d)) / np.sqrt(d)
+    v = rng.standard_normal((B, H, N, dv))
+    alpha = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, H, N, d)) - 2.0))   # in (0, 1)
+    return q, k, v, alpha
+
+
+@pytest.mark.parametrize("with_S0", [False, True])
+def test_gla_equals_unrolled_form(with_S0):
+    rng = np.random.default_rng(11)
+    q, k, v, alpha = _gla_inputs(rng, 2, 2, 23, 5, 3)
+    S0 = rng.standard_normal((2, 2, 5, 3)) if with_S0 else None
+    o, S = oracle.gla(q, k, v, alpha, S0)
+    for b in range(2):
+        for h in range(2):
+            od, Sd = gla_dense(q[b, h], k[b, h], v[b, h], alpha[b, h], None if S0 is None else S0[b, h])
+            np.testing.assert_allclose(o[b, h], od, rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(S[b, h], Sd, rtol=1e-10, atol=1e-12)
+
+
+def test_gla_without_forgetting_is_a_running_sum():
+    # alpha = 1: S_t = S0 + sum_{j<=t} k_j v_j^T and o_t = S_t^T q_t.
+    rng = np.random.default_rng(12)
+    q, k, v, _ = _gla_inputs(rng, 1, 1, 17, 4, 6)
+    S0 = rng.standard_normal((1, 1, 4, 6))
+    o, S = oracle.gla(q, k, v, np.ones_like(q), S0)
+    run = S0[0, 0] + np.cumsum(k[0, 0][:, :, None] * v[0, 0][:, None, :], axis=0)
+    np.testing.assert_allclose(o[0, 0], np.einsum("ti,tij->tj", q[0, 0], run), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S[0, 0], run[-1], rtol=1e-12, atol=1e-12)
+
+
+def test_gla_closed_gate_resets_only_its_channel():
+    # a zero gate entry at token t erases key channel i of the state and
+    # nothing else: afterwards row i holds exactly k_t[i] v_t, the other rows
+    # are those of the run with that entry set to one.
+    rng = np.random.default_rng(13)
+    q, k, v, alpha = _gla_inputs(rng, 1, 1, 9, 4, 3)
+    t, i = 5, 2
+    a0 = alpha.copy(); a0[0, 0, t, i] = 0.0
+    a1 = alpha.copy(); a1[0, 0, t, i] = 1.0
+    _, S0 = oracle.gla(q[:, :, : t + 1], k[:, :, : t + 1], v[:, :, : t + 1], a0[:, :, : t + 1])
+    _, S1 = oracle.gla(q[:, :, : t + 1], k[:, :, : t + 1], v[:, :, : t + 1], a1[:, :, : t + 1])
+    np.testing.assert_array_equal(S0[0, 0, i], k[0, 0, t, i] * v[0, 0, t])
+    rows = [r for r in range(4) if r != i]
+    np.testing.assert_array_equal(S0[0, 0, rows], S1[0, 0, rows])
+
+
+def test_gla_constant_gate_is_the_scalar_decay_form():
+    # alpha_t = gamma in every channel: the [B] §7.1 decay recurrence without
+    # a normaliser, o_t = sum_{j<=t} gamma^(t-j) (q_t . k_j) v_j.
+    rng = np.random.default_rng(14)
+    q, k, v, _ = _gla_inputs(rng, 1, 1, 20, 4, 3)
+    gamma = 0.9
+    o, _ = oracle.gla(q, k, v, np.full_like(q, gamma))
+    idx = np.arange(20)
+    Gam = np.where(idx[:, None] >= idx[None, :], gamma ** (idx[:, None] - idx[None, :]).clip(min=0), 0.0)
+    ref = ((q[0, 0] @ k[0, 0].T) * Gam) @ v[0, 0]
+    np.testing.assert_allclose(o[0, 0], ref, rtol=1e-11, atol=1e-12)
