@@ -50,6 +50,9 @@ def prefill_units(p) -> dict:
     if p.mode == "gated_delta":
         byts += th * 8  # alpha, g fp32
         flops = th * 6 * p.d * p.dv
+    elif p.mode == "gla":
+        byts += th * p.d * 4  # the per-channel gate, fp32
+        flops = th * 5 * p.d * p.dv
     else:
         byts += chains * p.d * 4
         flops = th * (4 * p.d * p.dv + 4 * p.d)
@@ -67,7 +70,8 @@ def workload_desc(name: str) -> str:
     if w["kind"] == "decode":
         return f"{name}: decode step, {w['S']} sequences x {w['H']} heads, d=dv={w['d']}, fp32 state, bf16 tokens"
     what = {"plain": "plain causal prefill with normaliser", "decay": "per-head decay prefill with decayed normaliser",
-            "gated_delta": "gated delta rule prefill"}[w.get("mode", "gated_delta")]
+            "gated_delta": "gated delta rule prefill", "gla": "per-key-channel gated (GLA) prefill"}[
+        w.get("mode", w["kind"])]
     return (f"{name}: B={w['B']} H={w['H']} N={w['N']} d=dv={w['d']} {w['dtype']} inputs, {what}")
 
 
@@ -194,6 +198,8 @@ def _prefill_device_args(p, torch):
         kw["gamma"] = _to_dev(p.gamma, torch)
     if p.mode == "gated_delta":
         kw["alpha"], kw["g"] = _to_dev(p.alpha, torch), _to_dev(p.g, torch)
+    if p.mode == "gla":
+        kw["alpha"] = _to_dev(p.alpha, torch)
     return q, k, v, kw
 
 
@@ -205,7 +211,7 @@ def time_prefill(p, steps, warmup, torch, la, flush):
     dv = v.shape[-1]
     out = torch.empty((B, H, N, dv), device="cuda", dtype=q.dtype)
     S_out = torch.empty((B, H, d, dv), device="cuda", dtype=torch.float32)
-    z_out = None if p.mode == "gated_delta" else torch.empty((B, H, d), device="cuda", dtype=torch.float32)
+    z_out = None if p.mode in ("gated_delta", "gla") else torch.empty((B, H, d), device="cuda", dtype=torch.float32)
     ws_bytes = la.la_prefill_workspace_bytes(B, H, N, d, dv, p.dtype, p.mode)
     ws = torch.empty(max(ws_bytes, 16), device="cuda", dtype=torch.uint8)
     stream = torch.cuda.current_stream()
@@ -244,6 +250,8 @@ def time_prefill_e2e(p, steps, warmup, torch, la):
         hextra["gamma"] = pin(p.gamma)
     if p.mode == "gated_delta":
         hextra["alpha"], hextra["g"] = pin(p.alpha), pin(p.g)
+    if p.mode == "gla":
+        hextra["alpha"] = pin(p.alpha)
     dq = torch.empty(hq.shape, dtype=hq.dtype, device="cuda")
     dk = torch.empty_like(dq)
     dvv = torch.empty(hv.shape, dtype=hv.dtype, device="cuda")
@@ -393,6 +401,8 @@ def path_dtype(p) -> str:
 def call_kernels(p) -> list:
     """The kernels one la_prefill call launches for this workload, in launch
     order (the dispatch documented with la_set_stage_events in include/la.h)."""
+    if p.mode == "gla":
+        return ["gla_token_simt"]
     if p.dtype == "bf16" and p.mode in ("plain", "decay"):
         return ["summary_kernel", "scan_kernel", "chunk_kernel"]
     if p.dtype == "bf16":
@@ -442,7 +452,7 @@ def time_kernels(p, steps, torch, la, flush):
     dv = v.shape[-1]
     out = torch.empty((B, H, N, dv), device="cuda", dtype=q.dtype)
     S_out = torch.empty((B, H, d, dv), device="cuda", dtype=torch.float32)
-    z_out = None if p.mode == "gated_delta" else torch.empty((B, H, d), device="cuda", dtype=torch.float32)
+    z_out = None if p.mode in ("gated_delta", "gla") else torch.empty((B, H, d), device="cuda", dtype=torch.float32)
     ws_bytes = la.la_prefill_workspace_bytes(B, H, N, d, dv, p.dtype, p.mode)
     ws = torch.empty(max(ws_bytes, 16), device="cuda", dtype=torch.uint8)
     stream = torch.cuda.current_stream()
@@ -503,11 +513,11 @@ def run_extra(args, torch, la, rank, flush):
     """Device-timed numbers for the other workloads (not the headline line)."""
     res = {}
     hbm_peak, _, _ = _measured_peaks()
-    for name in ("decay_bf16", "gdelta_bf16", "plain_f32"):
+    for name in ("decay_bf16", "gdelta_bf16", "plain_f32", "gla_bf16"):
         spec = inputs.WORKLOADS[name]
         p = inputs.make_workload(name, seed=rank_seed(spec["seed"], rank))
         u = prefill_units(p)
-        steps = 5 if name != "plain_f32" else 50
+        steps = {"plain_f32": 50, "gla_bf16": 3}.get(name, 5)
         ms = statistics.median(time_prefill(p, steps, 3, torch, la, flush))
         res[name] = {"tokens_per_s": u["tokens"] / (ms / 1e3), "ms": ms,
                      "hbm_frac": u["bytes"] / (ms / 1e3) / 1e9 / hbm_peak, "dtype": path_dtype(p)}
@@ -540,6 +550,8 @@ def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
         hs = slice(0, per_call)
         if p.mode == "gated_delta":
             oracle.gated_delta(p.q[:, hs], p.k[:, hs], p.v[:, hs], p.alpha[:, hs], p.g[:, hs])
+        elif p.mode == "gla":
+            oracle.gla(p.q[:, hs], p.k[:, hs], p.v[:, hs], p.alpha[:, hs])
         else:
             oracle.kernelized(p.q[:, hs], p.k[:, hs], p.v[:, hs],
                               None if p.gamma is None else p.gamma[hs], eps=p.eps)

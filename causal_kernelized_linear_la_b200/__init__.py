@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libla.so")
 
 LA_OK, LA_ERR_INVALID, LA_ERR_UNSUPPORTED, LA_ERR_ALIGN, LA_ERR_CUDA, LA_ERR_TIMEOUT, LA_ERR_WORKSPACE = range(7)
 LA_F32, LA_BF16 = 0, 1
-MODES = {"plain": 0, "decay": 1, "gated_delta": 2}
+MODES = {"plain": 0, "decay": 1, "gated_delta": 2, "gla": 3}
 
 # Symbols the library exports; the header include/la.h declares exactly these.
 EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
@@ -129,8 +129,9 @@ def la_prefill(q, k, v, mode="plain", gamma=None, alpha=None, g=None, S0=None, z
                out=None, S_out=None, z_out=None, workspace=None, stream=None):
     """Causal prefill over [B,H,N,*] tensors; returns ``(o, S_N, z_N)``.
 
-    mode "plain" (gamma = 1), "decay" (gamma [H] fp32), or "gated_delta"
-    (alpha, g [B,H,N] fp32; k L2-normalised; returns z_N = None)."""
+    mode "plain" (gamma = 1), "decay" (gamma [H] fp32), "gated_delta"
+    (alpha, g [B,H,N] fp32; k L2-normalised; returns z_N = None), or "gla"
+    (alpha [B,H,N,d] fp32, the per-key-channel gate; returns z_N = None)."""
     torch = _torch()
     if mode not in MODES:
         raise ValueError(f"mode must be one of {list(MODES)}")
@@ -138,7 +139,7 @@ def la_prefill(q, k, v, mode="plain", gamma=None, alpha=None, g=None, S0=None, z
     dv = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, N) or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k must be [B,H,N,d] and v [B,H,N,dv], all of one dtype")
-    delta = mode == "gated_delta"
+    delta = mode in ("gated_delta", "gla")   # the modes without a normaliser
     dev = q.device
     if out is None:
         out = torch.empty((B, H, N, dv), device=dev, dtype=q.dtype)

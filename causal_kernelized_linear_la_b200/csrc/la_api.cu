@@ -87,18 +87,22 @@ la_status la_prefill(const void* q, const void* k, const void* v,
     if (!cfg) return LA_ERR_INVALID;
     if (B < 0 || H < 0 || N < 0) return LA_ERR_INVALID;
     if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
-    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA) return LA_ERR_INVALID;
+    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA && cfg->mode != LA_GLA)
+        return LA_ERR_INVALID;
     if (!la::head_ok(d) || !la::head_ok(dv)) return LA_ERR_UNSUPPORTED;
     const bool delta = cfg->mode == LA_GATED_DELTA;
+    const bool gla = cfg->mode == LA_GLA;
+    const bool no_norm = delta || gla;   // modes without the z normaliser
     const bool work = (long long)B * H > 0;
     if (work) {
         if (!S_out) return LA_ERR_INVALID;
-        if (!delta && !z_out) return LA_ERR_INVALID;
-        if (delta && z_out) return LA_ERR_INVALID;
+        if (!no_norm && !z_out) return LA_ERR_INVALID;
+        if (no_norm && z_out) return LA_ERR_INVALID;
         if (N > 0 && (!q || !k || !v || !out)) return LA_ERR_INVALID;
         if (cfg->mode == LA_PLAIN && (gamma_or_alpha || g)) return LA_ERR_INVALID;
         if (cfg->mode == LA_DECAY && (!gamma_or_alpha || g)) return LA_ERR_INVALID;
         if (delta && N > 0 && (!gamma_or_alpha || !g)) return LA_ERR_INVALID;
+        if (gla && (g || (N > 0 && !gamma_or_alpha))) return LA_ERR_INVALID;
     }
     if (!(cfg->eps >= 0.f)) return LA_ERR_INVALID;
     if (work && ((cfg->S0 && cfg->S0 == S_out) || (cfg->z0 && cfg->z0 == z_out))) return LA_ERR_INVALID;
@@ -111,16 +115,17 @@ la_status la_prefill(const void* q, const void* k, const void* v,
     PrefillArgs a{};
     a.q = q; a.k = k; a.v = v;
     a.gamma = cfg->mode == LA_DECAY ? gamma_or_alpha : nullptr;
-    a.alpha = delta ? gamma_or_alpha : nullptr;
+    a.alpha = no_norm ? gamma_or_alpha : nullptr;
     a.g = delta ? g : nullptr;
-    a.out = out; a.S_out = S_out; a.z_out = delta ? nullptr : z_out;
-    a.S0 = cfg->S0; a.z0 = delta ? nullptr : cfg->z0;
+    a.out = out; a.S_out = S_out; a.z_out = no_norm ? nullptr : z_out;
+    a.S0 = cfg->S0; a.z0 = no_norm ? nullptr : cfg->z0;
     a.B = B; a.H = H; a.N = N; a.d = d; a.dv = dv;
     a.eps = cfg->eps; a.dtype = cfg->dtype; a.mode = cfg->mode;
     a.stream = static_cast<cudaStream_t>(cfg->stream);
     a.workspace = cfg->workspace; a.workspace_bytes = cfg->workspace_bytes;
 
     if (N == 0) return la::write_start_state(a);
+    if (gla) return la::from_cuda(la::launch_prefill_simt_gla(a));
     if (delta) {
         if (a.dtype == LA_BF16) return la::from_cuda(la::launch_prefill_tc_gated_delta(a));
         return la::from_cuda(la::launch_prefill_simt_gated_delta(a));
@@ -137,7 +142,8 @@ la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
     if (!cfg) return LA_ERR_INVALID;
     if (B < 0 || H < 0 || N < 0) return LA_ERR_INVALID;
     if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
-    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA) return LA_ERR_INVALID;
+    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA && cfg->mode != LA_GLA)
+        return LA_ERR_INVALID;
     if (!la::head_ok(d) || !la::head_ok(dv)) return LA_ERR_UNSUPPORTED;
     if (!la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return LA_ERR_UNSUPPORTED;
     const bool work = (long long)B * H > 0;

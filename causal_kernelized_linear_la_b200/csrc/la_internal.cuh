@@ -65,6 +65,7 @@ cudaError_t launch_causal_conv(const ConvArgs& a);
 // SIMT prefill kernels (fp32 arithmetic; fp32 or bf16 inputs).
 cudaError_t launch_prefill_simt_kernelized(const PrefillArgs& a);
 cudaError_t launch_prefill_simt_gated_delta(const PrefillArgs& a);
+cudaError_t launch_prefill_simt_gla(const PrefillArgs& a);
 
 // Decode kernels (HBM-streaming SIMT).
 cudaError_t launch_decode_kernelized(const DecodeArgs& a);

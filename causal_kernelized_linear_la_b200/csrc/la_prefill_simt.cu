@@ -250,7 +250,91 @@ cudaError_t launch_gdelta_t(const PrefillArgs& a)
     return e;
 }
 
+// ---------------------------------------------------------------------------
+// GLA, per-key-channel gate ("Efficient attention variants" §7.2), token
+// recurrence, one thread per column of S:
+//     S_t[i][j] = alpha_t[i] S_{t-1}[i][j] + k_t[i] v_t[j],  o_t[j] = sum_i q_t[i] S_t[i][j]
+
+constexpr int kGlaTile = 16;  // tokens staged in shared memory at a time
+
+template <typename T, int D>
+__global__ void __launch_bounds__(64)
+gla_token_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+               const float* __restrict__ alpha, const float* __restrict__ S0, T* __restrict__ out,
+               float* __restrict__ S_out, int N, int dv)
+{
+    __shared__ __align__(16) float kqa[3][kGlaTile][D];   // k, q, alpha of the staged tokens
+    const int j = blockIdx.y * blockDim.x + threadIdx.x;  // state column
+    const long long chain = blockIdx.x;
+    const bool active = j < dv;
+    const T* qc = q + chain * (long long)N * D;
+    const T* kc = k + chain * (long long)N * D;
+    const float* ac = alpha + chain * (long long)N * D;
+    const T* vc = v + chain * (long long)N * dv;
+    T* oc = out + chain * (long long)N * dv;
+
+    float s[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i)
+        s[i] = (S0 && active) ? S0[chain * (long long)D * dv + (long long)i * dv + j] : 0.f;
+
+    for (int t0 = 0; t0 < N; t0 += kGlaTile) {
+        const int n = min(kGlaTile, N - t0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < kGlaTile * D; e += blockDim.x) {
+            const int t = e / D, f = e % D;
+            const long long off = (long long)(t0 + t) * D + f;
+            kqa[0][t][f] = t < n ? to_f32(kc[off]) : 0.f;
+            kqa[1][t][f] = t < n ? to_f32(qc[off]) : 0.f;
+            kqa[2][t][f] = t < n ? ac[off] : 1.f;
+        }
+        __syncthreads();
+        for (int t = 0; t < n; ++t) {
+            const float vt = active ? to_f32(vc[(long long)(t0 + t) * dv + j]) : 0.f;
+            float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+#pragma unroll
+            for (int i = 0; i < D; i += 4) {
+                s[i + 0] = fmaf(kqa[2][t][i + 0], s[i + 0], kqa[0][t][i + 0] * vt);
+                s[i + 1] = fmaf(kqa[2][t][i + 1], s[i + 1], kqa[0][t][i + 1] * vt);
+                s[i + 2] = fmaf(kqa[2][t][i + 2], s[i + 2], kqa[0][t][i + 2] * vt);
+                s[i + 3] = fmaf(kqa[2][t][i + 3], s[i + 3], kqa[0][t][i + 3] * vt);
+                o0 = fmaf(s[i + 0], kqa[1][t][i + 0], o0);
+                o1 = fmaf(s[i + 1], kqa[1][t][i + 1], o1);
+                o2 = fmaf(s[i + 2], kqa[1][t][i + 2], o2);
+                o3 = fmaf(s[i + 3], kqa[1][t][i + 3], o3);
+            }
+            if (active) oc[(long long)(t0 + t) * dv + j] = from_f32<T>((o0 + o1) + (o2 + o3));
+        }
+    }
+    if (active) {
+#pragma unroll
+        for (int i = 0; i < D; ++i) S_out[chain * (long long)D * dv + (long long)i * dv + j] = s[i];
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_gla_t(const PrefillArgs& a)
+{
+    const int threads = 64;
+    dim3 grid(a.B * a.H, (a.dv + threads - 1) / threads);
+    gla_token_simt<T, D><<<grid, threads, 0, a.stream>>>(
+        (const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.S0, (T*)a.out, a.S_out, a.N, a.dv);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) stage_mark(0, a.stream);
+    return e;
+}
+
 }  // namespace
+
+cudaError_t launch_prefill_simt_gla(const PrefillArgs& a)
+{
+    if (a.dtype == LA_F32) {
+        if (a.d == 64) return launch_gla_t<float, 64>(a);
+        return launch_gla_t<float, 128>(a);
+    }
+    if (a.d == 64) return launch_gla_t<__nv_bfloat16, 64>(a);
+    return launch_gla_t<__nv_bfloat16, 128>(a);
+}
 
 cudaError_t launch_prefill_simt_kernelized(const PrefillArgs& a)
 {

@@ -61,10 +61,11 @@ class PrefillInputs:
     ``q``/``k``: [B,H,N,d]; ``v``: [B,H,N,dv].  ``dtype`` is "f32" or "bf16".
     For bf16, ``*_bits`` hold the uint16 patterns the device receives and the
     float32 arrays hold the same (exactly representable) numbers.
-    ``gamma`` [H] (decay mode), ``alpha``/``g`` [B,H,N] (gated delta) are fp32.
+    ``gamma`` [H] (decay mode), ``alpha``/``g`` [B,H,N] (gated delta) and
+    ``alpha`` [B,H,N,d] (gla) are fp32.
     """
     name: str
-    mode: str  # "plain" | "decay" | "gated_delta"
+    mode: str  # "plain" | "decay" | "gated_delta" | "gla"
     dtype: str  # "f32" | "bf16"
     B: int
     H: int
@@ -137,13 +138,29 @@ def make_gated_delta(B, H, N, d, dv, *, dtype="bf16", seed=BASE_SEED, name="cust
     return _finish(PrefillInputs(name, "gated_delta", dtype, B, H, N, d, dv, q, k, v, alpha=alpha, g=g))
 
 
-# The five named workloads, each with its own seed (base seed + index).
+def make_gla(B, H, N, d, dv, *, dtype="bf16", seed=BASE_SEED, name="custom") -> PrefillInputs:
+    """q,v ~ N(0,1); k ~ N(0,1)/sqrt(d); per-key-channel gate
+    alpha = exp(-0.1*softplus(y)) with y ~ N(0,1) per (b,h,t,channel),
+    evaluated in float64 and rounded to float32 once."""
+    rng = np.random.default_rng(seed)
+    q = _normal(rng, (B, H, N, d))
+    k = _normal(rng, (B, H, N, d), 1.0 / np.sqrt(d))
+    v = _normal(rng, (B, H, N, dv))
+    y = rng.standard_normal((B, H, N, d)).astype(np.float64)
+    softplus = np.log1p(np.exp(-np.abs(y))) + np.maximum(y, 0.0)
+    alpha = np.exp(-0.1 * softplus).astype(np.float32)
+    return _finish(PrefillInputs(name, "gla", dtype, B, H, N, d, dv, q, k, v, alpha=alpha))
+
+
+# The five named workloads, each with its own seed (base seed + index), and a
+# sixth for the per-key-channel gate (not one of the five benchmark configs).
 WORKLOADS = {
     "plain_f32": dict(kind="kernelized", B=1, H=1, N=256, d=64, dv=64, dtype="f32", mode="plain", seed=BASE_SEED + 1),
     "plain_bf16": dict(kind="kernelized", B=4, H=8, N=4096, d=64, dv=64, dtype="bf16", mode="plain", seed=BASE_SEED + 2),
     "decay_bf16": dict(kind="kernelized", B=2, H=16, N=32768, d=128, dv=128, dtype="bf16", mode="decay", seed=BASE_SEED + 3),
     "decode": dict(kind="decode", S=256, H=32, d=128, dv=128, steps=1000, seed=BASE_SEED + 4),
     "gdelta_bf16": dict(kind="gated_delta", B=1, H=32, N=65536, d=128, dv=128, dtype="bf16", seed=BASE_SEED + 5),
+    "gla_bf16": dict(kind="gla", B=1, H=32, N=8192, d=128, dv=128, dtype="bf16", seed=BASE_SEED + 6),
 }
 
 
@@ -159,6 +176,9 @@ def make_workload(name: str, **override) -> PrefillInputs:
     if kind == "gated_delta":
         return make_gated_delta(spec["B"], spec["H"], spec["N"], spec["d"], spec["dv"], dtype=spec["dtype"],
                                 seed=spec["seed"], name=name)
+    if kind == "gla":
+        return make_gla(spec["B"], spec["H"], spec["N"], spec["d"], spec["dv"], dtype=spec["dtype"],
+                        seed=spec["seed"], name=name)
     raise ValueError(f"{name} is not a prefill workload")
 
 

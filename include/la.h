@@ -68,7 +68,7 @@ typedef enum {
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
 
-typedef enum { LA_PLAIN = 0, LA_DECAY = 1, LA_GATED_DELTA = 2 } la_mode;
+typedef enum { LA_PLAIN = 0, LA_DECAY = 1, LA_GATED_DELTA = 2, LA_GLA = 3 } la_mode;
 
 typedef struct {
     la_dtype dtype;          /* element type of q, k, v, out */
@@ -91,15 +91,21 @@ typedef struct {
  *   q, k, v          inputs, layouts above, element type cfg->dtype.
  *   gamma_or_alpha   LA_PLAIN: must be NULL.  LA_DECAY: gamma [H], each in (0,1].
  *                    LA_GATED_DELTA: alpha [B,H,N], each in (0,1].
+ *                    LA_GLA: alpha [B,H,N,d], each in (0,1]: the per-key-channel
+ *                    gate ("Efficient attention variants" §7.2),
+ *                    S_t = diag(alpha_t) S_{t-1} + k_t v_t^T, o_t = S_t^T q_t.
  *   g                LA_GATED_DELTA: write strength g [B,H,N]; otherwise NULL.
  *   out              o [B,H,N,dv], element type cfg->dtype.
  *   S_out            final state S_N [B,H,d,dv] fp32 (required).
  *   z_out            final normaliser z_N [B,H,d] fp32 (kernelized modes, required);
- *                    must be NULL in LA_GATED_DELTA.
+ *                    must be NULL in LA_GATED_DELTA and LA_GLA.
  *   cfg              dtype, mode, eps, stream, optional start state and workspace.
  *
  * In LA_GATED_DELTA no feature map is applied; k is expected to be
  * L2-normalised by the caller (the rule is stable for ||k|| = 1, 0 < g <= 1).
+ * LA_GLA applies no feature map and no normaliser either (eps is unused); it
+ * runs a token-serial SIMT kernel (one thread per state column) for both
+ * dtypes.
  * S_out and z_out must not overlap cfg->S0 and cfg->z0 (blocks of one call
  * read the start state while others write the final state); continue a
  * sequence by alternating two state buffers.  LA_ERR_INVALID if they alias.

@@ -36,6 +36,8 @@ def run_library(p, S0=None, z0=None):
         kw["gamma"] = dev(p.gamma, torch)
     if p.mode == "gated_delta":
         kw["alpha"], kw["g"] = dev(p.alpha, torch), dev(p.g, torch)
+    if p.mode == "gla":
+        kw["alpha"] = dev(p.alpha, torch)
     o, S, z = la.la_prefill(q, k, v, mode=p.mode, eps=p.eps, S0=None if S0 is None else dev(S0, torch),
                             z0=None if z0 is None else dev(z0, torch), **kw)
     la.la_prefill_check()
@@ -55,6 +57,9 @@ def run_oracle(p, chains=None, S0=None, z0=None):
         s0 = None if S0 is None else S0[sl]
         if p.mode == "gated_delta":
             o, S = oracle.gated_delta(p.q[sl], p.k[sl], p.v[sl], p.alpha[sl], p.g[sl], s0)
+            z = None
+        elif p.mode == "gla":
+            o, S = oracle.gla(p.q[sl], p.k[sl], p.v[sl], p.alpha[sl], s0)
             z = None
         else:
             gam = None if p.gamma is None else p.gamma[h:h + 1]
