@@ -421,8 +421,17 @@ def la_launches_per_step(p) -> int:
 # benchmark reports null when the file differs now.
 TRAFFIC_CAPTURES = {
     ("plain_bf16", "chunk_kernel"): {
-        "bytes": 54647552 + 809216, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": None, "profile": "profiles/ncu_chunk_kernel_plain_bf16_4x8x4096_d64.md"},
+        "bytes": 54647040 + 551424, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "34f5c4a8f2ffe1865f945ede2552bb63546c329501eaa949cb564f1216d96c1b",
+        "profile": "profiles/traffic_dominant_kernels.md"},
+    ("decay_bf16", "chunk_kernel"): {
+        "bytes": 824409344 + 209686016, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "34f5c4a8f2ffe1865f945ede2552bb63546c329501eaa949cb564f1216d96c1b",
+        "profile": "profiles/traffic_dominant_kernels.md"},
+    ("gdelta_bf16", "gd_chain_kernel"): {
+        "bytes": 2709321216 + 526033152, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
+        "sha256": "a11a19c2736a087b8550876636f2490e5c1fad33aa74e7a29469470bc239091a",
+        "profile": "profiles/traffic_dominant_kernels.md"},
 }
 
 

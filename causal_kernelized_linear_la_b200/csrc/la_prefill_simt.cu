@@ -252,74 +252,138 @@ cudaError_t launch_gdelta_t(const PrefillArgs& a)
 
 // ---------------------------------------------------------------------------
 // GLA, per-key-channel gate ("Efficient attention variants" §7.2), token
-// recurrence, one thread per column of S:
+// recurrence:
 //     S_t[i][j] = alpha_t[i] S_{t-1}[i][j] + k_t[i] v_t[j],  o_t[j] = sum_i q_t[i] S_t[i][j]
+// Four threads share a state column (every fourth row each, in registers,
+// so that the four read neighbouring words of the staged vectors) and add
+// their parts of o_t with two shuffles.  k, q, alpha and
+// the block's v columns of kGlaTile tokens are staged in shared memory by
+// cp.async, double-buffered, so the next tile streams in while this one is
+// consumed.
 
-constexpr int kGlaTile = 16;  // tokens staged in shared memory at a time
+constexpr int kGlaTile = 16;   // tokens per staged tile
+constexpr int kGlaCols = 32;   // state columns per block (x 4 threads)
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes)
+{
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int Nleft>
+__device__ __forceinline__ void cp_async_wait_groups() { asm volatile("cp.async.wait_group %0;" ::"n"(Nleft) : "memory"); }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(64)
+struct GlaSmem {
+    T k[2][kGlaTile][D];
+    T q[2][kGlaTile][D];
+    float a[2][kGlaTile][D];
+    T v[2][kGlaTile][kGlaCols];
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(4 * kGlaCols)
 gla_token_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                const float* __restrict__ alpha, const float* __restrict__ S0, T* __restrict__ out,
                float* __restrict__ S_out, int N, int dv)
 {
-    __shared__ __align__(16) float kqa[3][kGlaTile][D];   // k, q, alpha of the staged tokens
-    const int j = blockIdx.y * blockDim.x + threadIdx.x;  // state column
+    constexpr int R = D / 4;                          // rows per thread
+    extern __shared__ __align__(16) unsigned char gla_smem[];
+    GlaSmem<T, D>& sh = *reinterpret_cast<GlaSmem<T, D>*>(gla_smem);
+    const int tid = threadIdx.x;
+    const int rg = tid & 3, jl = tid >> 2;            // row group, local column
+    const int j = blockIdx.y * kGlaCols + jl;         // state column
+    // this thread's rows: rg, rg + 4, rg + 8, ...
     const long long chain = blockIdx.x;
     const bool active = j < dv;
     const T* qc = q + chain * (long long)N * D;
     const T* kc = k + chain * (long long)N * D;
     const float* ac = alpha + chain * (long long)N * D;
-    const T* vc = v + chain * (long long)N * dv;
+    const T* vc = v + chain * (long long)N * dv + blockIdx.y * kGlaCols;
     T* oc = out + chain * (long long)N * dv;
+    const int vcols = min(kGlaCols, dv - (int)blockIdx.y * kGlaCols);
 
-    float s[D];
+    float s[R];
 #pragma unroll
-    for (int i = 0; i < D; ++i)
-        s[i] = (S0 && active) ? S0[chain * (long long)D * dv + (long long)i * dv + j] : 0.f;
+    for (int i = 0; i < R; ++i)
+        s[i] = (S0 && active) ? S0[chain * (long long)D * dv + (long long)(4 * i + rg) * dv + j] : 0.f;
 
-    for (int t0 = 0; t0 < N; t0 += kGlaTile) {
-        const int n = min(kGlaTile, N - t0);
-        __syncthreads();
-        for (int e = threadIdx.x; e < kGlaTile * D; e += blockDim.x) {
-            const int t = e / D, f = e % D;
-            const long long off = (long long)(t0 + t) * D + f;
-            kqa[0][t][f] = t < n ? to_f32(kc[off]) : 0.f;
-            kqa[1][t][f] = t < n ? to_f32(qc[off]) : 0.f;
-            kqa[2][t][f] = t < n ? ac[off] : 1.f;
-        }
-        __syncthreads();
-        for (int t = 0; t < n; ++t) {
-            const float vt = active ? to_f32(vc[(long long)(t0 + t) * dv + j]) : 0.f;
-            float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-#pragma unroll
-            for (int i = 0; i < D; i += 4) {
-                s[i + 0] = fmaf(kqa[2][t][i + 0], s[i + 0], kqa[0][t][i + 0] * vt);
-                s[i + 1] = fmaf(kqa[2][t][i + 1], s[i + 1], kqa[0][t][i + 1] * vt);
-                s[i + 2] = fmaf(kqa[2][t][i + 2], s[i + 2], kqa[0][t][i + 2] * vt);
-                s[i + 3] = fmaf(kqa[2][t][i + 3], s[i + 3], kqa[0][t][i + 3] * vt);
-                o0 = fmaf(s[i + 0], kqa[1][t][i + 0], o0);
-                o1 = fmaf(s[i + 1], kqa[1][t][i + 1], o1);
-                o2 = fmaf(s[i + 2], kqa[1][t][i + 2], o2);
-                o3 = fmaf(s[i + 3], kqa[1][t][i + 3], o3);
+    // stage tile `tile` into buffer `b`: 16-byte pieces, zero past the end
+    auto stage = [&](int tile, int b) {
+        const int t0 = tile * kGlaTile;
+        constexpr int KQ = kGlaTile * D * (int)sizeof(T) / 16;   // pieces of k (and of q)
+        constexpr int AP = kGlaTile * D * 4 / 16;                 // pieces of alpha
+        constexpr int VP = kGlaTile * kGlaCols * (int)sizeof(T) / 16;
+        constexpr int PR = D * (int)sizeof(T) / 16;               // pieces per k/q row
+        constexpr int PA = D * 4 / 16;
+        constexpr int PV = kGlaCols * (int)sizeof(T) / 16;
+        for (int e = tid; e < 2 * KQ + AP + VP; e += blockDim.x) {
+            if (e < 2 * KQ) {
+                const int which = e / KQ, r = (e % KQ) / PR, c = (e % KQ) % PR;
+                const int t = t0 + r;
+                const T* src = (which ? qc : kc) + (long long)min(t, N - 1) * D + c * (16 / (int)sizeof(T));
+                T* dst = (which ? &sh.q[b][r][0] : &sh.k[b][r][0]) + c * (16 / (int)sizeof(T));
+                cp_async16(dst, src, t < N ? 16u : 0u);
+            } else if (e < 2 * KQ + AP) {
+                const int f = e - 2 * KQ, r = f / PA, c = f % PA, t = t0 + r;
+                cp_async16(&sh.a[b][r][c * 4], ac + (long long)min(t, N - 1) * D + c * 4, t < N ? 16u : 0u);
+            } else {
+                const int f = e - 2 * KQ - AP, r = f / PV, c = f % PV, t = t0 + r;
+                const int col = c * (16 / (int)sizeof(T));
+                const bool ok = t < N && col < vcols;
+                cp_async16(&sh.v[b][r][col], vc + (long long)min(t, N - 1) * dv + (ok ? col : 0), ok ? 16u : 0u);
             }
-            if (active) oc[(long long)(t0 + t) * dv + j] = from_f32<T>((o0 + o1) + (o2 + o3));
         }
+        cp_async_commit_group();
+    };
+
+    const int tiles = (N + kGlaTile - 1) / kGlaTile;
+    stage(0, 0);
+    for (int tile = 0; tile < tiles; ++tile) {
+        const int b = tile & 1;
+        if (tile + 1 < tiles) {
+            stage(tile + 1, b ^ 1);
+            cp_async_wait_groups<1>();
+        } else {
+            cp_async_wait_groups<0>();
+        }
+        __syncthreads();
+        const int n = min(kGlaTile, N - tile * kGlaTile);
+        for (int t = 0; t < n; ++t) {
+            const float vt = to_f32(sh.v[b][t][jl]);
+            float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < R; i += 2) {
+                const int ra = 4 * i + rg, rb = 4 * (i + 1) + rg;
+                s[i] = fmaf(sh.a[b][t][ra], s[i], to_f32(sh.k[b][t][ra]) * vt);
+                s[i + 1] = fmaf(sh.a[b][t][rb], s[i + 1], to_f32(sh.k[b][t][rb]) * vt);
+                o0 = fmaf(s[i], to_f32(sh.q[b][t][ra]), o0);
+                o1 = fmaf(s[i + 1], to_f32(sh.q[b][t][rb]), o1);
+            }
+            float o = o0 + o1;
+            o += __shfl_xor_sync(0xffffffffu, o, 1);
+            o += __shfl_xor_sync(0xffffffffu, o, 2);
+            if (active && rg == 0) oc[(long long)(tile * kGlaTile + t) * dv + j] = from_f32<T>(o);
+        }
+        __syncthreads();   // buffer b is restaged two tiles from now
     }
     if (active) {
 #pragma unroll
-        for (int i = 0; i < D; ++i) S_out[chain * (long long)D * dv + (long long)i * dv + j] = s[i];
+        for (int i = 0; i < R; ++i) S_out[chain * (long long)D * dv + (long long)(4 * i + rg) * dv + j] = s[i];
     }
 }
 
 template <typename T, int D>
 cudaError_t launch_gla_t(const PrefillArgs& a)
 {
-    const int threads = 64;
-    dim3 grid(a.B * a.H, (a.dv + threads - 1) / threads);
-    gla_token_simt<T, D><<<grid, threads, 0, a.stream>>>(
-        (const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.S0, (T*)a.out, a.S_out, a.N, a.dv);
-    const cudaError_t e = cudaGetLastError();
+    auto kern = gla_token_simt<T, D>;
+    const int smem = (int)sizeof(GlaSmem<T, D>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.B * a.H, (a.dv + kGlaCols - 1) / kGlaCols);
+    kern<<<grid, 4 * kGlaCols, smem, a.stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.S0,
+                                                 (T*)a.out, a.S_out, a.N, a.dv);
+    e = cudaGetLastError();
     if (e == cudaSuccess) stage_mark(0, a.stream);
     return e;
 }
