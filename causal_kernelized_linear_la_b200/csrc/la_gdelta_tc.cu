@@ -133,6 +133,7 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 {
     using P = PrepPlan<D>;
     constexpr int NB = P::NB;
+    grid_launch_dependents();   // the chain kernel may launch; it waits for this grid's results
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
     unsigned char* kbt = sm + P::OFF_KB;
@@ -602,6 +603,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    grid_dependency_wait();   // the prep pass's operands are complete
 
     if (warp == 9) {
         // ---------------- TMA: stage loads and output stores ----------------
@@ -951,8 +953,21 @@ cudaError_t launch_gd(const PrefillArgs& a)
     const int s2 = ChainPlan<D>::BYTES;
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
     if (e != cudaSuccess) return e;
-    k2<<<chains * (a.dv / DVT), kChainThreads, s2, a.stream>>>(mqb, mkt, mv, mw, mt, mp, mo, a.alpha, a.S0, a.S_out,
-                                                           a.N, a.dv);
+    // programmatic serialization: the chain kernel sets up while the prep pass
+    // finishes, and waits (griddepcontrol.wait) before reading its operands
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(chains * (a.dv / DVT));
+    lc.blockDim = dim3(kChainThreads);
+    lc.dynamicSmemBytes = s2;
+    lc.stream = a.stream;
+    lc.attrs = pdl;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, k2, mqb, mkt, mv, mw, mt, mp, mo, (const float*)a.alpha, (const float*)a.S0,
+                           a.S_out, a.N, a.dv);
+    if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(1, a.stream);
     return cudaSuccess;

@@ -110,6 +110,7 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                const float* __restrict__ gamma, float* __restrict__ ws, int N, int H, int G, int L)
 {
     using P = SummaryPlan<D, DV>;
+    grid_launch_dependents();   // the scan may launch now; it waits for this grid's results
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
@@ -255,6 +256,8 @@ scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float
             int G, int L)
 {
     constexpr int SLOT = D * DV + D;
+    grid_launch_dependents();   // the chunk kernel may set up and load q, k, v meanwhile
+    grid_dependency_wait();     // the segment summaries are complete
     const int chain = blockIdx.x;
     const int e = blockIdx.y * 256 + threadIdx.x;
     if (e >= SLOT) return;
@@ -494,6 +497,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // Start state, transposed into TMEM: S^T[j][f] = S[f][j]; z as row 0 of
     // the normaliser accumulator (other rows zero).
     if (worker) {
+        grid_dependency_wait();   // start states from the scan
         const float* slot = ws + (size_t)unit * (D * DV + D);
         const int j = acc_row<DV>(quad, lane);
 #pragma unroll
@@ -757,9 +761,21 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     stage_mark(0, a.stream);
 
     constexpr int SLOT = D * DV + D;
-    dim3 gs(chains, (SLOT + 255) / 256);
-    scan_kernel<D, DV, DECAY><<<gs, 256, 0, a.stream>>>(ws, a.gamma, a.S0, a.z0, a.S_out, a.z_out, a.N, a.H,
-                                                        sg.G, sg.L);
+    // the scan and the chunk kernel start with programmatic serialization: each
+    // sets up while its predecessor finishes and waits only before reading
+    // what the predecessor wrote (griddepcontrol.wait)
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(chains, (SLOT + 255) / 256);
+    lc.blockDim = dim3(256);
+    lc.stream = a.stream;
+    lc.attrs = pdl;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, scan_kernel<D, DV, DECAY>, ws, a.gamma, a.S0, a.z0, a.S_out, a.z_out, a.N, a.H,
+                           sg.G, sg.L);
+    if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(1, a.stream);
 
@@ -769,7 +785,11 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kc, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    kc<<<units, kThreads + 32, sc, a.stream>>>(mq, mk, mv, mo, a.gamma, ws, a.N, a.H, sg.G, sg.L, a.eps);
+    lc.gridDim = dim3(units);
+    lc.blockDim = dim3(kThreads + 32);
+    lc.dynamicSmemBytes = sc;
+    e = cudaLaunchKernelEx(&lc, kc, mq, mk, mv, mo, a.gamma, (const float*)ws, a.N, a.H, sg.G, sg.L, a.eps);
+    if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(2, a.stream);
     return cudaSuccess;

@@ -331,6 +331,15 @@ __device__ __forceinline__ float2 phi2_fast(float x0, float x1)
     return make_float2(fmaxf(x0, 0.f) + e.x, fmaxf(x1, 0.f) + e.y);
 }
 
+// ---- programmatic dependent launch ---------------------------------------------
+
+// Wait until the grids this one depends on (launched before it on the stream
+// with programmatic serialization) have completed and their memory is visible.
+// A no-op in a grid launched without that attribute.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the grid launched after this one on the stream start its launch now.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- cp.async (4-byte global -> shared) ---------------------------------------
 
 // Asynchronous 4-byte copy; src_bytes = 0 stores zero and reads nothing.
