@@ -421,16 +421,16 @@ def la_launches_per_step(p) -> int:
 # benchmark reports null when the file differs now.
 TRAFFIC_CAPTURES = {
     ("plain_bf16", "chunk_kernel"): {
-        "bytes": 54647040 + 551424, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "34f5c4a8f2ffe1865f945ede2552bb63546c329501eaa949cb564f1216d96c1b",
+        "bytes": 54647296 + 322048, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "20ec1a93c4c04b4bd8f3d421111ea1c3b0220730efd2007ba93836df6fcc318f",
         "profile": "profiles/traffic_dominant_kernels.md"},
     ("decay_bf16", "chunk_kernel"): {
-        "bytes": 824409344 + 209686016, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "34f5c4a8f2ffe1865f945ede2552bb63546c329501eaa949cb564f1216d96c1b",
+        "bytes": 824594432 + 209871872, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "20ec1a93c4c04b4bd8f3d421111ea1c3b0220730efd2007ba93836df6fcc318f",
         "profile": "profiles/traffic_dominant_kernels.md"},
     ("gdelta_bf16", "gd_chain_kernel"): {
-        "bytes": 2709321216 + 526033152, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
-        "sha256": "a11a19c2736a087b8550876636f2490e5c1fad33aa74e7a29469470bc239091a",
+        "bytes": 2715619840 + 523374848, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
+        "sha256": "283d1c0683d294064029524eee119bea1750d755576060dc8bac89eedd94e1f0",
         "profile": "profiles/traffic_dominant_kernels.md"},
 }
 
