@@ -518,6 +518,39 @@ def time_conv(torch, la, rank, flush, hbm_peak, B=4, H=8, N=4096, d=64, w=4, ste
             "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak}
 
 
+def time_varlen(torch, la, rank, flush, hbm_peak, H=8, N=4096, d=64, steps=20):
+    """A right-padded batch of eight plain bf16 sequences of mixed lengths
+    (head size and padded length of the headline workload) through
+    la_prefill_varlen: device time per call, L2 flushed before each."""
+    g = torch.Generator(device="cpu").manual_seed(rank_seed(91, rank))
+    lens = [4096, 3000, 2048, 1500, 1000, 700, 300, 65]
+    B = len(lens)
+    q, k, v = ((torch.randn((B, H, N, d), generator=g) / 8).to(torch.bfloat16).cuda() for _ in range(3))
+    out = torch.empty_like(v)
+    S = torch.empty((B, H, d, d), device="cuda")
+    z = torch.empty((B, H, d), device="cuda")
+    ws = torch.empty(max(la.la_prefill_varlen_workspace_bytes(lens, H, d, d), 16), device="cuda",
+                     dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+    call = lambda: la.la_prefill_varlen(q, k, v, lens, out=out, S_out=S, z_out=z, workspace=ws)
+    for _ in range(3):
+        flush.fill_(1)
+        call()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        flush.fill_(1)
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    tokens = sum(lens)
+    nbytes = tokens * H * 4 * d * 2 + B * H * (d * d + d) * 4
+    return {"shape": f"B={B} H={H} padded N={N} d=dv={d} bf16 plain, lengths {lens}", "ms": ms,
+            "tokens_per_s": tokens / (ms / 1e3), "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+            "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak, "launches": 3 * B}
+
+
 def run_extra(args, torch, la, rank, flush):
     """Device-timed numbers for the other workloads (not the headline line)."""
     res = {}
@@ -532,6 +565,7 @@ def run_extra(args, torch, la, rank, flush):
                      "hbm_frac": u["bytes"] / (ms / 1e3) / 1e9 / hbm_peak, "dtype": path_dtype(p)}
         del p
     res["conv"] = time_conv(torch, la, rank, flush, hbm_peak)
+    res["varlen_bf16"] = time_varlen(torch, la, rank, flush, hbm_peak)
     dspec = inputs.WORKLOADS["decode"]
     dms = time_decode(1000, 20, torch, la, rank_seed(dspec["seed"], rank))
     du = decode_units(dspec["S"], dspec["H"], dspec["d"], dspec["dv"])

@@ -12,9 +12,12 @@ Entry points (same names as the C ABI):
 
 * ``la_prefill(q, k, v, mode=..., gamma=..., alpha=..., g=..., S0=..., z0=..., eps=...)``
   -> ``(o, S, z)`` (``z`` is None in gated-delta mode)
+* ``la_prefill_varlen(q, k, v, seq_lens, mode=..., ...)`` -> ``(o, S, z)`` for a
+  right-padded batch of sequences of different lengths
 * ``la_decode_step(q, k, v, S, z, eps=...)`` -> ``o``; S and z updated in place
 * ``la_gated_delta_decode_step(q, k, v, alpha, g, S)`` -> ``o``; S updated in place
-* ``la_prefill_workspace_bytes(...)``, ``la_status_string(code)``, ``lib()``
+* ``la_prefill_workspace_bytes(...)``, ``la_prefill_varlen_workspace_bytes(...)``,
+  ``la_status_string(code)``, ``lib()``
 """
 from __future__ import annotations
 
@@ -29,7 +32,8 @@ LA_F32, LA_BF16 = 0, 1
 MODES = {"plain": 0, "decay": 1, "gated_delta": 2, "gla": 3}
 
 # Symbols the library exports; the header include/la.h declares exactly these.
-EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
+EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_prefill_varlen",
+           "la_prefill_varlen_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
            "la_set_stage_events", "la_causal_conv",
            "la_prefill_check", "la_status_string", "la_version")
 
@@ -64,6 +68,11 @@ def lib() -> ctypes.CDLL:
         L.la_prefill_noalloc.restype = i
         L.la_prefill_workspace_bytes.argtypes = [i] * 5 + [cfgp]
         L.la_prefill_workspace_bytes.restype = ctypes.c_size_t
+        ip = ctypes.POINTER(ctypes.c_int)
+        L.la_prefill_varlen.argtypes = [vp] * 8 + [ip] + [i] * 5 + [cfgp]
+        L.la_prefill_varlen.restype = i
+        L.la_prefill_varlen_workspace_bytes.argtypes = [ip] + [i] * 4 + [cfgp]
+        L.la_prefill_varlen_workspace_bytes.restype = ctypes.c_size_t
         L.la_decode_step.argtypes = [vp] * 6 + [i] * 4 + [cfgp]
         L.la_decode_step.restype = i
         L.la_gated_delta_decode_step.argtypes = [vp] * 7 + [i] * 4 + [cfgp]
@@ -164,6 +173,63 @@ def la_prefill(q, k, v, mode="plain", gamma=None, alpha=None, g=None, S0=None, z
                           B, H, N, d, dv, ctypes.byref(cfg))
     if rc != LA_OK:
         raise LaError(rc, "la_prefill")
+    return out, S_out, z_out
+
+
+def _host_lens(seq_lens):
+    """The sequence lengths as a C int array (host memory)."""
+    lens = [int(n) for n in (seq_lens.tolist() if hasattr(seq_lens, "tolist") else seq_lens)]
+    return (ctypes.c_int * max(len(lens), 1))(*lens), len(lens)
+
+
+def la_prefill_varlen_workspace_bytes(seq_lens, H, d, dv, dtype="bf16", mode="plain") -> int:
+    arr, B = _host_lens(seq_lens)
+    cfg = LaConfig(LA_BF16 if dtype == "bf16" else LA_F32, MODES[mode], 0.0, None, None, None, None, 0)
+    return int(lib().la_prefill_varlen_workspace_bytes(arr, B, H, d, dv, ctypes.byref(cfg)))
+
+
+def la_prefill_varlen(q, k, v, seq_lens, mode="plain", gamma=None, alpha=None, g=None, S0=None, z0=None,
+                      eps=1e-6, out=None, S_out=None, z_out=None, workspace=None, stream=None):
+    """Prefill of a right-padded batch: q, k [B,H,N,d], v [B,H,N,dv] with
+    sequence b in rows 0..seq_lens[b]-1 (seq_lens: host ints).  Returns
+    ``(o, S, z)`` with each sequence's final state; rows of o past a
+    sequence's length are not written (uninitialised when o is allocated
+    here).  Other arguments as in ``la_prefill``."""
+    torch = _torch()
+    if mode not in MODES:
+        raise ValueError(f"mode must be one of {list(MODES)}")
+    B, H, N, d = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, N) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k must be [B,H,N,d] and v [B,H,N,dv], all of one dtype")
+    arr, nl = _host_lens(seq_lens)
+    if nl != B:
+        raise ValueError(f"seq_lens has {nl} entries for a batch of {B}")
+    delta = mode in ("gated_delta", "gla")   # the modes without a normaliser
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, H, N, dv), device=dev, dtype=q.dtype)
+    if S_out is None:
+        S_out = torch.empty((B, H, d, dv), device=dev, dtype=torch.float32)
+    if not delta and z_out is None:
+        z_out = torch.empty((B, H, d), device=dev, dtype=torch.float32)
+    if delta:
+        z_out = None
+    first = alpha if delta else gamma
+    for t in (first, g, S0, z0, S_out, z_out):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError("gamma/alpha/g/S0/z0/S_out/z_out must be float32")
+    _check_cuda(q, k, v, first, g, S0, z0, out, S_out, z_out, workspace)
+    cfg = LaConfig(_dtype_code(q), MODES[mode], float(eps), _stream_handle(stream), _ptr(S0), _ptr(z0), None, 0)
+    need = int(lib().la_prefill_varlen_workspace_bytes(arr, B, H, d, dv, ctypes.byref(cfg)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    cfg.workspace = _ptr(workspace)
+    cfg.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().la_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(first), _ptr(g), _ptr(out), _ptr(S_out),
+                                 _ptr(z_out), arr, B, H, N, d, dv, ctypes.byref(cfg))
+    if rc != LA_OK:
+        raise LaError(rc, "la_prefill_varlen")
     return out, S_out, z_out
 
 

@@ -47,6 +47,73 @@ la_status write_start_state(const PrefillArgs& a)
     return from_cuda(e);
 }
 
+// Argument checks of a prefill over a [B,H,N,.] batch (all but the workspace size).
+la_status check_prefill(const void* q, const void* k, const void* v, const float* gamma_or_alpha, const float* g,
+                        const void* out, const float* S_out, const float* z_out, int B, int H, int N, int d, int dv,
+                        const la_config* cfg)
+{
+    if (!cfg) return LA_ERR_INVALID;
+    if (B < 0 || H < 0 || N < 0) return LA_ERR_INVALID;
+    if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
+    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA && cfg->mode != LA_GLA)
+        return LA_ERR_INVALID;
+    if (!head_ok(d) || !head_ok(dv)) return LA_ERR_UNSUPPORTED;
+    const bool delta = cfg->mode == LA_GATED_DELTA;
+    const bool gla = cfg->mode == LA_GLA;
+    const bool no_norm = delta || gla;   // modes without the z normaliser
+    const bool work = (long long)B * H > 0;
+    if (work) {
+        if (!S_out) return LA_ERR_INVALID;
+        if (!no_norm && !z_out) return LA_ERR_INVALID;
+        if (no_norm && z_out) return LA_ERR_INVALID;
+        if (N > 0 && (!q || !k || !v || !out)) return LA_ERR_INVALID;
+        if (cfg->mode == LA_PLAIN && (gamma_or_alpha || g)) return LA_ERR_INVALID;
+        if (cfg->mode == LA_DECAY && (!gamma_or_alpha || g)) return LA_ERR_INVALID;
+        if (delta && N > 0 && (!gamma_or_alpha || !g)) return LA_ERR_INVALID;
+        if (gla && (g || (N > 0 && !gamma_or_alpha))) return LA_ERR_INVALID;
+    }
+    if (!(cfg->eps >= 0.f)) return LA_ERR_INVALID;
+    if (work && ((cfg->S0 && cfg->S0 == S_out) || (cfg->z0 && cfg->z0 == z_out))) return LA_ERR_INVALID;
+    const void* ptrs[] = {q, k, v, gamma_or_alpha, g, out, S_out, z_out, cfg->S0, cfg->z0, cfg->workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return LA_ERR_ALIGN;
+    return LA_OK;
+}
+
+PrefillArgs prefill_args(const void* q, const void* k, const void* v, const float* gamma_or_alpha, const float* g,
+                         void* out, float* S_out, float* z_out, int B, int H, int N, int d, int dv,
+                         const la_config* cfg)
+{
+    const bool delta = cfg->mode == LA_GATED_DELTA;
+    const bool no_norm = delta || cfg->mode == LA_GLA;
+    PrefillArgs a{};
+    a.q = q; a.k = k; a.v = v;
+    a.gamma = cfg->mode == LA_DECAY ? gamma_or_alpha : nullptr;
+    a.alpha = no_norm ? gamma_or_alpha : nullptr;
+    a.g = delta ? g : nullptr;
+    a.out = out; a.S_out = S_out; a.z_out = no_norm ? nullptr : z_out;
+    a.S0 = cfg->S0; a.z0 = no_norm ? nullptr : cfg->z0;
+    a.B = B; a.H = H; a.N = N; a.d = d; a.dv = dv;
+    a.ld = N;
+    a.eps = cfg->eps; a.dtype = cfg->dtype; a.mode = cfg->mode;
+    a.stream = static_cast<cudaStream_t>(cfg->stream);
+    a.workspace = cfg->workspace; a.workspace_bytes = cfg->workspace_bytes;
+    return a;
+}
+
+// One checked prefill to the kernels of its dtype and mode.
+la_status run_prefill(const PrefillArgs& a)
+{
+    if (a.N == 0) return write_start_state(a);
+    if (a.mode == LA_GLA) return from_cuda(launch_prefill_simt_gla(a));
+    if (a.mode == LA_GATED_DELTA) {
+        if (a.dtype == LA_BF16) return from_cuda(launch_prefill_tc_gated_delta(a));
+        return from_cuda(launch_prefill_simt_gated_delta(a));
+    }
+    if (uses_tc_kernelized(a.dtype, a.mode)) return from_cuda(launch_prefill_tc_kernelized(a));
+    return from_cuda(launch_prefill_simt_kernelized(a));
+}
+
 }  // namespace
 }  // namespace la
 
@@ -84,54 +151,66 @@ la_status la_prefill(const void* q, const void* k, const void* v,
                      void* out, float* S_out, float* z_out,
                      int B, int H, int N, int d, int dv, const la_config* cfg)
 {
-    if (!cfg) return LA_ERR_INVALID;
-    if (B < 0 || H < 0 || N < 0) return LA_ERR_INVALID;
-    if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
-    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA && cfg->mode != LA_GLA)
-        return LA_ERR_INVALID;
-    if (!la::head_ok(d) || !la::head_ok(dv)) return LA_ERR_UNSUPPORTED;
-    const bool delta = cfg->mode == LA_GATED_DELTA;
-    const bool gla = cfg->mode == LA_GLA;
-    const bool no_norm = delta || gla;   // modes without the z normaliser
-    const bool work = (long long)B * H > 0;
-    if (work) {
-        if (!S_out) return LA_ERR_INVALID;
-        if (!no_norm && !z_out) return LA_ERR_INVALID;
-        if (no_norm && z_out) return LA_ERR_INVALID;
-        if (N > 0 && (!q || !k || !v || !out)) return LA_ERR_INVALID;
-        if (cfg->mode == LA_PLAIN && (gamma_or_alpha || g)) return LA_ERR_INVALID;
-        if (cfg->mode == LA_DECAY && (!gamma_or_alpha || g)) return LA_ERR_INVALID;
-        if (delta && N > 0 && (!gamma_or_alpha || !g)) return LA_ERR_INVALID;
-        if (gla && (g || (N > 0 && !gamma_or_alpha))) return LA_ERR_INVALID;
-    }
-    if (!(cfg->eps >= 0.f)) return LA_ERR_INVALID;
-    if (work && ((cfg->S0 && cfg->S0 == S_out) || (cfg->z0 && cfg->z0 == z_out))) return LA_ERR_INVALID;
-    const void* ptrs[] = {q, k, v, gamma_or_alpha, g, out, S_out, z_out, cfg->S0, cfg->z0, cfg->workspace};
-    for (const void* p : ptrs)
-        if (!la::aligned16(p)) return LA_ERR_ALIGN;
+    const la_status st = la::check_prefill(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, cfg);
+    if (st != LA_OK) return st;
     if (cfg->workspace_bytes < la_prefill_workspace_bytes(B, H, N, d, dv, cfg)) return LA_ERR_WORKSPACE;
-    if (!work) return LA_OK;
+    if ((long long)B * H == 0) return LA_OK;
+    return la::run_prefill(la::prefill_args(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, cfg));
+}
 
-    PrefillArgs a{};
-    a.q = q; a.k = k; a.v = v;
-    a.gamma = cfg->mode == LA_DECAY ? gamma_or_alpha : nullptr;
-    a.alpha = no_norm ? gamma_or_alpha : nullptr;
-    a.g = delta ? g : nullptr;
-    a.out = out; a.S_out = S_out; a.z_out = no_norm ? nullptr : z_out;
-    a.S0 = cfg->S0; a.z0 = no_norm ? nullptr : cfg->z0;
-    a.B = B; a.H = H; a.N = N; a.d = d; a.dv = dv;
-    a.eps = cfg->eps; a.dtype = cfg->dtype; a.mode = cfg->mode;
-    a.stream = static_cast<cudaStream_t>(cfg->stream);
-    a.workspace = cfg->workspace; a.workspace_bytes = cfg->workspace_bytes;
-
-    if (N == 0) return la::write_start_state(a);
-    if (gla) return la::from_cuda(la::launch_prefill_simt_gla(a));
-    if (delta) {
-        if (a.dtype == LA_BF16) return la::from_cuda(la::launch_prefill_tc_gated_delta(a));
-        return la::from_cuda(la::launch_prefill_simt_gated_delta(a));
+size_t la_prefill_varlen_workspace_bytes(const int* seq_lens, int B, int H, int d, int dv, const la_config* cfg)
+{
+    if (!seq_lens || B <= 0) return 0;
+    size_t most = 0;
+    for (int b = 0; b < B; ++b) {
+        const size_t n = la_prefill_workspace_bytes(1, H, seq_lens[b], d, dv, cfg);
+        if (n > most) most = n;
     }
-    if (la::uses_tc_kernelized(a.dtype, a.mode)) return la::from_cuda(la::launch_prefill_tc_kernelized(a));
-    return la::from_cuda(la::launch_prefill_simt_kernelized(a));
+    return most;
+}
+
+la_status la_prefill_varlen(const void* q, const void* k, const void* v,
+                            const float* gamma_or_alpha, const float* g,
+                            void* out, float* S_out, float* z_out, const int* seq_lens,
+                            int B, int H, int N, int d, int dv, const la_config* cfg)
+{
+    const la_status st = la::check_prefill(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, cfg);
+    if (st != LA_OK) return st;
+    if ((long long)B * H == 0) return LA_OK;
+    if (!seq_lens) return LA_ERR_INVALID;
+    for (int b = 0; b < B; ++b)
+        if (seq_lens[b] < 0 || seq_lens[b] > N) return LA_ERR_INVALID;
+    if (cfg->workspace_bytes < la_prefill_varlen_workspace_bytes(seq_lens, B, H, d, dv, cfg))
+        return LA_ERR_WORKSPACE;
+
+    // Sequence b is the B = 1 batch of its H chains over its own length; its
+    // chains keep the batch's row stride N, so the padding rows are neither
+    // read (the TMA maps and the SIMT loops end at the length) nor written.
+    // The calls share the workspace: each one's first kernel is launched in
+    // full stream order, after the previous call's kernels.
+    const PrefillArgs base = la::prefill_args(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, cfg);
+    const size_t esz = cfg->dtype == LA_BF16 ? 2 : 4;
+    for (int b = 0; b < B; ++b) {
+        PrefillArgs a = base;
+        const size_t row0 = (size_t)b * H * N;   // first row of sequence b
+        const size_t st_s = (size_t)b * H * d * dv, st_z = (size_t)b * H * d;
+        a.q = static_cast<const char*>(q) + row0 * d * esz;
+        a.k = static_cast<const char*>(k) + row0 * d * esz;
+        a.v = static_cast<const char*>(v) + row0 * dv * esz;
+        a.out = static_cast<char*>(out) + row0 * dv * esz;
+        if (a.alpha) a.alpha += cfg->mode == LA_GLA ? row0 * d : row0;
+        if (a.g) a.g += row0;
+        a.S_out += st_s;
+        if (a.z_out) a.z_out += st_z;
+        if (a.S0) a.S0 += st_s;
+        if (a.z0) a.z0 += st_z;
+        a.B = 1;
+        a.N = seq_lens[b];
+        a.ld = N;
+        const la_status r = la::run_prefill(a);
+        if (r != LA_OK) return r;
+    }
+    return LA_OK;
 }
 
 la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
@@ -167,6 +246,7 @@ la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
     a.out = out; a.S_out = S_out; a.z_out = z_out;
     a.S0 = cfg->S0; a.z0 = cfg->z0;
     a.B = B; a.H = H; a.N = N; a.d = d; a.dv = dv;
+    a.ld = N;
     a.eps = cfg->eps; a.dtype = cfg->dtype; a.mode = cfg->mode;
     a.stream = static_cast<cudaStream_t>(cfg->stream);
     if (N == 0) return la::write_start_state(a);

@@ -129,7 +129,7 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qb,
                const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_t,
                const __grid_constant__ CUtensorMap tm_p, const float* __restrict__ alpha,
-               const float* __restrict__ gate, int N, int chains)
+               const float* __restrict__ gate, int N, int chains, int ld)
 {
     using P = PrepPlan<D>;
     constexpr int NB = P::NB;
@@ -187,8 +187,8 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // warp 1: alpha, g of a work item into staging buffer `buf` (lane: tokens 2 lane, 2 lane + 1)
     auto stage_vectors = [&](int item, int buf) {
         const int ch = item / nch, t0 = (item % nch) * C;
-        const float* al = alpha + (size_t)ch * N;
-        const float* gl = gate + (size_t)ch * N;
+        const float* al = alpha + (size_t)ch * ld;
+        const float* gl = gate + (size_t)ch * ld;
         float* dst = avec + buf * 2 * C;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -546,7 +546,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                 const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_p,
                 const __grid_constant__ CUtensorMap tm_o, const float* __restrict__ alpha,
-                const float* __restrict__ S0, float* __restrict__ S_out, int N, int dv)
+                const float* __restrict__ S0, float* __restrict__ S_out, int N, int dv, int ld)
 {
     using P = ChainPlan<D>;
     constexpr int NB = P::NB;
@@ -745,7 +745,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
         __syncwarp();
     } else {
         // ---------------- converters (warps 0-7) ----------------
-        const float* al = alpha + (size_t)chain * N;
+        const float* al = alpha + (size_t)chain * ld;
         // warp 1: alpha of chunk c into staging buffer c & 1
         auto stage_alpha = [&](int c) {
             float* dst = abuf + (c & 1) * C;
@@ -926,11 +926,11 @@ cudaError_t launch_gd(const PrefillArgs& a)
     unsigned char* tp = kt + (size_t)chains * npad * D * 2;
     unsigned char* pp = tp + (size_t)chains * npad * C * 2;
     CUtensorMap mq, mk, mv, mo, mw, mqb, mkt, mt, mp;
-    if (!make_map(&mq, a.q, D, a.N, chains) || !make_map(&mk, a.k, D, a.N, chains) ||
-        !make_map(&mv, a.v, a.dv, a.N, chains) || !make_map(&mo, a.out, a.dv, a.N, chains) ||
-        !make_map(&mw, wneg, D, npad, chains) || !make_map(&mqb, qb, D, npad, chains) ||
-        !make_map(&mkt, kt, D, npad, chains) ||
-        !make_map(&mt, tp, C, npad, chains) || !make_map(&mp, pp, C, npad, chains))
+    if (!make_map(&mq, a.q, D, a.N, chains, a.ld) || !make_map(&mk, a.k, D, a.N, chains, a.ld) ||
+        !make_map(&mv, a.v, a.dv, a.N, chains, a.ld) || !make_map(&mo, a.out, a.dv, a.N, chains, a.ld) ||
+        !make_map(&mw, wneg, D, npad, chains, npad) || !make_map(&mqb, qb, D, npad, chains, npad) ||
+        !make_map(&mkt, kt, D, npad, chains, npad) ||
+        !make_map(&mt, tp, C, npad, chains, npad) || !make_map(&mp, pp, C, npad, chains, npad))
         return cudaErrorInvalidValue;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
@@ -944,7 +944,7 @@ cudaError_t launch_gd(const PrefillArgs& a)
     if (e != cudaSuccess) return e;
     const long long items = (long long)chains * nch;
     const int g1 = (int)std::min<long long>(items, 2LL * sms);
-    k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mqb, mkt, mt, mp, a.alpha, a.g, a.N, chains);
+    k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mqb, mkt, mt, mp, a.alpha, a.g, a.N, chains, a.ld);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     stage_mark(0, a.stream);
@@ -966,7 +966,7 @@ cudaError_t launch_gd(const PrefillArgs& a)
     lc.attrs = pdl;
     lc.numAttrs = 1;
     e = cudaLaunchKernelEx(&lc, k2, mqb, mkt, mv, mw, mt, mp, mo, (const float*)a.alpha, (const float*)a.S0,
-                           a.S_out, a.N, a.dv);
+                           a.S_out, a.N, a.dv, a.ld);
     if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(1, a.stream);

@@ -23,6 +23,10 @@ struct PrefillArgs {
     const float* S0;
     const float* z0;
     int B, H, N, d, dv;
+    // tokens between the first rows of consecutive (b, h) chains of q, k, v,
+    // out, alpha and g: N for a dense [B,H,N,.] batch, the padded length when
+    // one sequence of a right-padded batch is run over its own length
+    int ld;
     float eps;
     la_dtype dtype;
     la_mode mode;

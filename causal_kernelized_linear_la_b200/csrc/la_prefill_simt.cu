@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kThreads)
 kernelized_chunk_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       const float* __restrict__ gamma, const float* __restrict__ S0,
                       const float* __restrict__ z0, T* __restrict__ out, float* __restrict__ S_out,
-                      float* __restrict__ z_out, int H, int N, int dv, float eps)
+                      float* __restrict__ z_out, int H, int N, int dv, float eps, int ld)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto& sm = *reinterpret_cast<KernelizedSmem<D, DVT>*>(smem_raw);
@@ -57,10 +57,10 @@ kernelized_chunk_simt(const T* __restrict__ q, const T* __restrict__ k, const T*
     const int h = (int)(chain % H);
     const float lam = gamma ? logf(gamma[h]) : 0.f;
 
-    const T* qc = q + chain * (long long)N * D;
-    const T* kc = k + chain * (long long)N * D;
-    const T* vc = v + chain * (long long)N * dv;
-    T* oc = out + chain * (long long)N * dv;
+    const T* qc = q + chain * (long long)ld * D;
+    const T* kc = k + chain * (long long)ld * D;
+    const T* vc = v + chain * (long long)ld * dv;
+    T* oc = out + chain * (long long)ld * dv;
 
     for (int e = tid; e < D * DVT; e += kThreads) {
         const int f = e / DVT, j = e % DVT;
@@ -155,7 +155,7 @@ cudaError_t launch_kernelized_t(const PrefillArgs& a)
     if (e != cudaSuccess) return e;
     dim3 grid(a.B * a.H, a.dv / DVT);
     kern<<<grid, kThreads, smem, a.stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.gamma, a.S0, a.z0,
-                                             (T*)a.out, a.S_out, a.z_out, a.H, a.N, a.dv, a.eps);
+                                             (T*)a.out, a.S_out, a.z_out, a.H, a.N, a.dv, a.eps, a.ld);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(0, a.stream);
     return cudaSuccess;
@@ -171,19 +171,19 @@ __global__ void __launch_bounds__(128)
 gated_delta_token_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                        const float* __restrict__ alpha, const float* __restrict__ g,
                        const float* __restrict__ S0, T* __restrict__ out, float* __restrict__ S_out,
-                       int N, int dv)
+                       int N, int dv, int ld)
 {
     __shared__ __align__(16) float kq[2][kDeltaTile][D];
     __shared__ float ag[2][kDeltaTile];
     const int j = blockIdx.y * blockDim.x + threadIdx.x;  // state column
     const long long chain = blockIdx.x;
     const bool active = j < dv;
-    const T* qc = q + chain * (long long)N * D;
-    const T* kc = k + chain * (long long)N * D;
-    const T* vc = v + chain * (long long)N * dv;
-    const float* al = alpha + chain * (long long)N;
-    const float* gl = g + chain * (long long)N;
-    T* oc = out + chain * (long long)N * dv;
+    const T* qc = q + chain * (long long)ld * D;
+    const T* kc = k + chain * (long long)ld * D;
+    const T* vc = v + chain * (long long)ld * dv;
+    const float* al = alpha + chain * (long long)ld;
+    const float* gl = g + chain * (long long)ld;
+    T* oc = out + chain * (long long)ld * dv;
 
     float s[D];
 #pragma unroll
@@ -244,7 +244,7 @@ cudaError_t launch_gdelta_t(const PrefillArgs& a)
     const int threads = 64;
     dim3 grid(a.B * a.H, (a.dv + threads - 1) / threads);
     gated_delta_token_simt<T, D><<<grid, threads, 0, a.stream>>>(
-        (const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.g, a.S0, (T*)a.out, a.S_out, a.N, a.dv);
+        (const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.g, a.S0, (T*)a.out, a.S_out, a.N, a.dv, a.ld);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) stage_mark(0, a.stream);
     return e;
@@ -285,7 +285,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(4 * kGlaCols)
 gla_token_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                const float* __restrict__ alpha, const float* __restrict__ S0, T* __restrict__ out,
-               float* __restrict__ S_out, int N, int dv)
+               float* __restrict__ S_out, int N, int dv, int ld)
 {
     constexpr int R = D / 4;                          // rows per thread
     extern __shared__ __align__(16) unsigned char gla_smem[];
@@ -296,11 +296,11 @@ gla_token_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __rest
     // this thread's rows: rg, rg + 4, rg + 8, ...
     const long long chain = blockIdx.x;
     const bool active = j < dv;
-    const T* qc = q + chain * (long long)N * D;
-    const T* kc = k + chain * (long long)N * D;
-    const float* ac = alpha + chain * (long long)N * D;
-    const T* vc = v + chain * (long long)N * dv + blockIdx.y * kGlaCols;
-    T* oc = out + chain * (long long)N * dv;
+    const T* qc = q + chain * (long long)ld * D;
+    const T* kc = k + chain * (long long)ld * D;
+    const float* ac = alpha + chain * (long long)ld * D;
+    const T* vc = v + chain * (long long)ld * dv + blockIdx.y * kGlaCols;
+    T* oc = out + chain * (long long)ld * dv;
     const int vcols = min(kGlaCols, dv - (int)blockIdx.y * kGlaCols);
 
     float s[R];
@@ -382,7 +382,7 @@ cudaError_t launch_gla_t(const PrefillArgs& a)
     if (e != cudaSuccess) return e;
     dim3 grid(a.B * a.H, (a.dv + kGlaCols - 1) / kGlaCols);
     kern<<<grid, 4 * kGlaCols, smem, a.stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.S0,
-                                                 (T*)a.out, a.S_out, a.N, a.dv);
+                                                 (T*)a.out, a.S_out, a.N, a.dv, a.ld);
     e = cudaGetLastError();
     if (e == cudaSuccess) stage_mark(0, a.stream);
     return e;

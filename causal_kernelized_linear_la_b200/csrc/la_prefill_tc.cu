@@ -721,14 +721,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 }  // namespace
 
-// 3-D map over a bf16 [chains][N][inner] tensor; box = 64 elements x 64 rows,
-// 128-byte swizzle; rows past N read as zero and are not written.
-bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains)
+// 3-D map over the first N rows of each chain of a bf16 [chains][ld][inner]
+// tensor; box = 64 elements x 64 rows, 128-byte swizzle; rows past N read as
+// zero and are not written.
+bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains, int ld)
 {
     auto fn = encode_fn();
-    if (!fn) return false;
+    if (!fn || ld < N) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)N, (cuuint64_t)chains};
-    cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)N * inner * 2};
+    cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)ld * inner * 2};
     cuuint32_t box[3] = {64, 64, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
@@ -743,8 +744,8 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
 {
     const int chains = a.B * a.H;
     CUtensorMap mq, mk, mv, mo;
-    if (!make_map(&mq, a.q, D, a.N, chains) || !make_map(&mk, a.k, D, a.N, chains) ||
-        !make_map(&mv, a.v, DV, a.N, chains) || !make_map(&mo, a.out, DV, a.N, chains))
+    if (!make_map(&mq, a.q, D, a.N, chains, a.ld) || !make_map(&mk, a.k, D, a.N, chains, a.ld) ||
+        !make_map(&mv, a.v, DV, a.N, chains, a.ld) || !make_map(&mo, a.out, DV, a.N, chains, a.ld))
         return cudaErrorInvalidValue;
     float* ws = static_cast<float*>(a.workspace);
     const int units = chains * sg.G;

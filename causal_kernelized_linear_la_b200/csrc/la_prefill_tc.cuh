@@ -23,9 +23,10 @@ constexpr size_t kNoAllocScratchBytes = 16u << 20;
 TcSegments tc_segments_noalloc(int B, int H, int N, int d, int dv);
 cudaError_t launch_prefill_tc_kernelized_noalloc(const PrefillArgs& a);
 
-// 3-D TMA map over a bf16 [chains][N][inner] tensor (box 64 x 64 rows,
-// 128-byte swizzle, zero fill past N).
-bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains);
+// 3-D TMA map over the first N rows of each chain of a bf16 tensor whose
+// chains start ld rows apart ([chains][ld][inner], ld >= N); box 64 x 64
+// rows, 128-byte swizzle, zero fill past N, stores clipped at N.
+bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains, int ld);
 
 // Gated-delta prefill on the tensor cores (bf16 inputs).  The workspace holds
 // the per-chunk operands the parallel pass hands to the sequential pass.

@@ -160,6 +160,46 @@ LA_API la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
 LA_API size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_config* cfg);
 
 /*
+ * la_prefill_varlen -- la_prefill over a right-padded batch of sequences of
+ * different lengths: sequence b holds seq_lens[b] tokens in rows
+ * 0 .. seq_lens[b]-1 of its [H, N, .] block.  Real batches carry padding and
+ * chunk boundaries that the pages' single-sequence examples leave out
+ * ("Efficient attention variants" §10, closing remarks); with a start state
+ * per sequence this is chunked-prefill continuation of a mixed batch.
+ *
+ *   q, k, v, out, gamma_or_alpha, g, S_out, z_out, cfg
+ *                    as in la_prefill, laid out for the padded length N:
+ *                    q, k [B,H,N,d]; v, out [B,H,N,dv]; alpha [B,H,N]
+ *                    (LA_GATED_DELTA) or [B,H,N,d] (LA_GLA); g [B,H,N];
+ *                    S_out, cfg->S0 [B,H,d,dv]; z_out, cfg->z0 [B,H,d].
+ *   seq_lens         HOST array of B lengths, each 0 <= seq_lens[b] <= N
+ *                    (LA_ERR_INVALID otherwise, or if NULL while B*H > 0).
+ *
+ * Sequence b's results equal those of la_prefill on that sequence alone
+ * (B = 1, N = seq_lens[b]) from its start state: out[b, :, t] for
+ * t < seq_lens[b], and S_out[b], z_out[b] after its last token (its start
+ * state when seq_lens[b] == 0).  Padding rows of q, k, v, alpha, g are never
+ * read and padding rows of out are never written.  The sequences run one
+ * after another on cfg->stream, each through the kernels la_prefill uses,
+ * and share cfg->workspace, which must hold
+ * la_prefill_varlen_workspace_bytes() bytes.  Returns LA_OK once all the
+ * work is enqueued; on an error from sequence b, sequences before b are
+ * enqueued and the rest are not.
+ */
+LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v,
+                                   const float* gamma_or_alpha, const float* g,
+                                   void* out, float* S_out, float* z_out, const int* seq_lens,
+                                   int B, int H, int N, int d, int dv, const la_config* cfg);
+
+/*
+ * la_prefill_varlen_workspace_bytes -- the workspace la_prefill_varlen needs:
+ * the largest la_prefill_workspace_bytes(1, H, seq_lens[b], d, dv, cfg) over
+ * the batch (seq_lens: host array of B lengths).  0 means none is needed.
+ */
+LA_API size_t la_prefill_varlen_workspace_bytes(const int* seq_lens, int B, int H, int d, int dv,
+                                                const la_config* cfg);
+
+/*
  * la_decode_step -- one decode step for B sequences x H heads, kernelized
  * recurrence with gamma = 1 (the state cache of "What Is Linear Attention?"
  * §6; update order of §4: write, then read):

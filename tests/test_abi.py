@@ -137,3 +137,31 @@ def test_conv_validation_host_only():
     assert L.la_causal_conv(c((1 << 20) + 2), FAKE, None, FAKE, None, 1, 1, 8, 64, 4, ctypes.byref(cfg)) == la.LA_ERR_ALIGN
     # nothing to do
     assert L.la_causal_conv(None, None, None, None, None, 0, 4, 8, 64, 4, ctypes.byref(cfg)) == la.LA_OK
+
+
+def _varlen(cfg, lens, B=2, H=1, N=8, d=64, dv=64, q=FAKE, out=FAKE, S=FAKE, z=FAKE):
+    c = ctypes.c_void_p
+    arr = None if lens is None else (ctypes.c_int * len(lens))(*lens)
+    return la.lib().la_prefill_varlen(c(q), c(q), c(q), None, None, c(out), c(S), c(z), arr, B, H, N, d, dv,
+                                      ctypes.byref(cfg))
+
+
+def test_varlen_validation():
+    # every call fails validation before anything is launched
+    assert _varlen(_cfg(), [3, 9]) == la.LA_ERR_INVALID        # a length past the padded N
+    assert _varlen(_cfg(), [-1, 2]) == la.LA_ERR_INVALID       # negative length
+    assert _varlen(_cfg(), None) == la.LA_ERR_INVALID          # lengths missing
+    assert _varlen(_cfg(), [3, 8], q=FAKE + 4) == la.LA_ERR_ALIGN
+    assert _varlen(_cfg(), [3, 8], d=48) == la.LA_ERR_UNSUPPORTED
+    assert _varlen(_cfg(), [3, 8], z=0) == la.LA_ERR_INVALID   # kernelized modes need z_out
+    assert _varlen(_cfg(), None, B=0) == la.LA_OK              # nothing to do
+    # bf16 kernelized needs a workspace for its segment summaries
+    assert _varlen(_cfg(), [3, 8]) == la.LA_ERR_WORKSPACE
+
+
+def test_varlen_workspace_is_the_largest_sequence():
+    lens = [0, 100, 5000, 64, 4096]
+    for dtype, mode in (("bf16", "plain"), ("bf16", "decay"), ("bf16", "gated_delta"), ("f32", "plain")):
+        want = max(la.la_prefill_workspace_bytes(1, 8, n, 128, 128, dtype, mode) if n > 0 else 0 for n in lens)
+        assert la.la_prefill_varlen_workspace_bytes(lens, 8, 128, 128, dtype, mode) == want
+    assert la.la_prefill_varlen_workspace_bytes([], 8, 128, 128) == 0
