@@ -421,16 +421,16 @@ def la_launches_per_step(p) -> int:
 # benchmark reports null when the file differs now.
 TRAFFIC_CAPTURES = {
     ("plain_bf16", "chunk_kernel"): {
-        "bytes": 54647296 + 322048, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "20ec1a93c4c04b4bd8f3d421111ea1c3b0220730efd2007ba93836df6fcc318f",
+        "bytes": 54647552 + 468736, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "3fc18696f316c1acb3926cfd21d665af34c10a99ecbf2df02eb163e17cf77fea",
         "profile": "profiles/traffic_dominant_kernels.md"},
     ("decay_bf16", "chunk_kernel"): {
-        "bytes": 824594432 + 209871872, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "20ec1a93c4c04b4bd8f3d421111ea1c3b0220730efd2007ba93836df6fcc318f",
+        "bytes": 824411136 + 209652992, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "3fc18696f316c1acb3926cfd21d665af34c10a99ecbf2df02eb163e17cf77fea",
         "profile": "profiles/traffic_dominant_kernels.md"},
     ("gdelta_bf16", "gd_chain_kernel"): {
-        "bytes": 2715619840 + 523374848, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
-        "sha256": "283d1c0683d294064029524eee119bea1750d755576060dc8bac89eedd94e1f0",
+        "bytes": 2693713152 + 525609728, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
+        "sha256": "9d9a2aa7ac6d580ccfa6de2fcbe335fd978cc0ba89cf113edd80e5009ae2f37b",
         "profile": "profiles/traffic_dominant_kernels.md"},
 }
 

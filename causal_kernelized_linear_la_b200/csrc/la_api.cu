@@ -101,6 +101,9 @@ PrefillArgs prefill_args(const void* q, const void* k, const void* v, const floa
     return a;
 }
 
+// Workspace slice of one sequence of la_prefill_varlen: 256-byte aligned.
+size_t varlen_slice(size_t bytes) { return (bytes + 255) / 256 * 256; }
+
 // One checked prefill to the kernels of its dtype and mode.
 la_status run_prefill(const PrefillArgs& a)
 {
@@ -161,12 +164,9 @@ la_status la_prefill(const void* q, const void* k, const void* v,
 size_t la_prefill_varlen_workspace_bytes(const int* seq_lens, int B, int H, int d, int dv, const la_config* cfg)
 {
     if (!seq_lens || B <= 0) return 0;
-    size_t most = 0;
-    for (int b = 0; b < B; ++b) {
-        const size_t n = la_prefill_workspace_bytes(1, H, seq_lens[b], d, dv, cfg);
-        if (n > most) most = n;
-    }
-    return most;
+    size_t total = 0;
+    for (int b = 0; b < B; ++b) total += la::varlen_slice(la_prefill_workspace_bytes(1, H, seq_lens[b], d, dv, cfg));
+    return total;
 }
 
 la_status la_prefill_varlen(const void* q, const void* k, const void* v,
@@ -186,12 +186,19 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v,
     // Sequence b is the B = 1 batch of its H chains over its own length; its
     // chains keep the batch's row stride N, so the padding rows are neither
     // read (the TMA maps and the SIMT loops end at the length) nor written.
-    // The calls share the workspace: each one's first kernel is launched in
-    // full stream order, after the previous call's kernels.
+    // Each sequence has a slice of the workspace of its own, so the first
+    // kernel of sequence b > 0 may start while sequence b-1's kernels drain
+    // (programmatic serialization); it finishes after them.
     const PrefillArgs base = la::prefill_args(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, cfg);
     const size_t esz = cfg->dtype == LA_BF16 ? 2 : 4;
+    size_t ws_off = 0;
     for (int b = 0; b < B; ++b) {
         PrefillArgs a = base;
+        const size_t ws_b = la_prefill_workspace_bytes(1, H, seq_lens[b], d, dv, cfg);
+        a.workspace = ws_b ? static_cast<char*>(cfg->workspace) + ws_off : nullptr;
+        a.workspace_bytes = ws_b;
+        ws_off += la::varlen_slice(ws_b);
+        a.pdl_first = b > 0 && seq_lens[b - 1] > 0;   // behind a kernel of sequence b-1
         const size_t row0 = (size_t)b * H * N;   // first row of sequence b
         const size_t st_s = (size_t)b * H * d * dv, st_z = (size_t)b * H * d;
         a.q = static_cast<const char*>(q) + row0 * d * esz;

@@ -504,6 +504,10 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, P::T_COLS);
+    // Launched early behind the previous call's kernels (one sequence after
+    // another), this grid reads none of their results, but it completes only
+    // after them, so the stream still finishes the calls in order.
+    grid_dependency_wait();
 }
 
 // ===========================================================================
@@ -550,6 +554,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
 {
     using P = ChainPlan<D>;
     constexpr int NB = P::NB;
+    grid_launch_dependents();   // a following call's prep pass may start on the idle SMs
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
     unsigned char* sbt = sm + P::OFF_SB;
@@ -944,7 +949,20 @@ cudaError_t launch_gd(const PrefillArgs& a)
     if (e != cudaSuccess) return e;
     const long long items = (long long)chains * nch;
     const int g1 = (int)std::min<long long>(items, 2LL * sms);
-    k1<<<g1, kThreads, s1, a.stream>>>(mq, mk, mw, mqb, mkt, mt, mp, a.alpha, a.g, a.N, chains, a.ld);
+    // behind an earlier call of the same batch (disjoint workspace), the prep
+    // pass starts with programmatic serialization too
+    cudaLaunchAttribute pdl1[1];
+    pdl1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl1[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t l1 = {};
+    l1.gridDim = dim3(g1);
+    l1.blockDim = dim3(kThreads);
+    l1.dynamicSmemBytes = s1;
+    l1.stream = a.stream;
+    l1.attrs = pdl1;
+    l1.numAttrs = a.pdl_first ? 1 : 0;
+    e = cudaLaunchKernelEx(&l1, k1, mq, mk, mw, mqb, mkt, mt, mp, a.alpha, a.g, a.N, chains, a.ld);
+    if (e != cudaSuccess) return e;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     stage_mark(0, a.stream);

@@ -27,6 +27,11 @@ struct PrefillArgs {
     // out, alpha and g: N for a dense [B,H,N,.] batch, the padded length when
     // one sequence of a right-padded batch is run over its own length
     int ld;
+    // launch the call's first kernel with programmatic serialization: it may
+    // start while the stream's previous kernels drain (it reads none of their
+    // results and finishes after them); only for back-to-back calls of one
+    // batch whose workspaces are disjoint
+    bool pdl_first;
     float eps;
     la_dtype dtype;
     la_mode mode;

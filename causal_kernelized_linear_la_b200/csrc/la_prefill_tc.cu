@@ -244,6 +244,10 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, P::T_COLS);
+    // Launched early behind the previous call's kernels (one sequence after
+    // another), this grid reads none of their results, but it completes only
+    // after them, so the stream still finishes the calls in order.
+    grid_dependency_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -322,6 +326,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     using P = ChunkPlan<D, DV, DECAY>;
     constexpr int NCHK = (D / 8) * C / kThreads;  // 16-byte chunks of a Q (or K) tile per worker thread
     static_assert(NCHK >= 1 && (D / 8) * C % kThreads == 0, "tile split");
+    grid_launch_dependents();   // a following call's summary pass may start as this grid drains
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
     unsigned char* khat = sm + P::OFF_KH;
@@ -757,22 +762,29 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     // all of L1 as shared memory, so that two CTAs fit on an SM where their plans allow
     e = cudaFuncSetAttribute(ka, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    ka<<<units, kThreads, sa, a.stream>>>(mk, mv, a.gamma, ws, a.N, a.H, sg.G, sg.L);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    stage_mark(0, a.stream);
-
-    constexpr int SLOT = D * DV + D;
-    // the scan and the chunk kernel start with programmatic serialization: each
+    // the scan and the chunk kernel (and, behind an earlier call of the same
+    // batch, the summary pass) start with programmatic serialization: each
     // sets up while its predecessor finishes and waits only before reading
     // what the predecessor wrote (griddepcontrol.wait)
     cudaLaunchAttribute pdl[1];
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(chains, (SLOT + 255) / 256);
-    lc.blockDim = dim3(256);
+    lc.gridDim = dim3(units);
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = sa;
     lc.stream = a.stream;
     lc.attrs = pdl;
+    lc.numAttrs = a.pdl_first ? 1 : 0;
+    e = cudaLaunchKernelEx(&lc, ka, mk, mv, a.gamma, ws, a.N, a.H, sg.G, sg.L);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stage_mark(0, a.stream);
+
+    constexpr int SLOT = D * DV + D;
+    lc.gridDim = dim3(chains, (SLOT + 255) / 256);
+    lc.blockDim = dim3(256);
+    lc.dynamicSmemBytes = 0;
     lc.numAttrs = 1;
     e = cudaLaunchKernelEx(&lc, scan_kernel<D, DV, DECAY>, ws, a.gamma, a.S0, a.z0, a.S_out, a.z_out, a.N, a.H,
                            sg.G, sg.L);

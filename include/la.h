@@ -180,11 +180,12 @@ LA_API size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, con
  * t < seq_lens[b], and S_out[b], z_out[b] after its last token (its start
  * state when seq_lens[b] == 0).  Padding rows of q, k, v, alpha, g are never
  * read and padding rows of out are never written.  The sequences run one
- * after another on cfg->stream, each through the kernels la_prefill uses,
- * and share cfg->workspace, which must hold
- * la_prefill_varlen_workspace_bytes() bytes.  Returns LA_OK once all the
- * work is enqueued; on an error from sequence b, sequences before b are
- * enqueued and the rest are not.
+ * after another on cfg->stream, each through the kernels la_prefill uses;
+ * each has a slice of cfg->workspace (which must hold
+ * la_prefill_varlen_workspace_bytes() bytes), so a sequence's first kernel
+ * may start while the previous sequence's last kernel drains.  Returns
+ * LA_OK once all the work is enqueued; on an error from sequence b,
+ * sequences before b are enqueued and the rest are not.
  */
 LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v,
                                    const float* gamma_or_alpha, const float* g,
@@ -193,8 +194,9 @@ LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v,
 
 /*
  * la_prefill_varlen_workspace_bytes -- the workspace la_prefill_varlen needs:
- * the largest la_prefill_workspace_bytes(1, H, seq_lens[b], d, dv, cfg) over
- * the batch (seq_lens: host array of B lengths).  0 means none is needed.
+ * the sum over the batch of la_prefill_workspace_bytes(1, H, seq_lens[b], d,
+ * dv, cfg), each rounded up to a multiple of 256 bytes (seq_lens: host array
+ * of B lengths).  0 means none is needed.
  */
 LA_API size_t la_prefill_varlen_workspace_bytes(const int* seq_lens, int B, int H, int d, int dv,
                                                 const la_config* cfg);

@@ -159,9 +159,10 @@ def test_varlen_validation():
     assert _varlen(_cfg(), [3, 8]) == la.LA_ERR_WORKSPACE
 
 
-def test_varlen_workspace_is_the_largest_sequence():
+def test_varlen_workspace_is_one_slice_per_sequence():
     lens = [0, 100, 5000, 64, 4096]
     for dtype, mode in (("bf16", "plain"), ("bf16", "decay"), ("bf16", "gated_delta"), ("f32", "plain")):
-        want = max(la.la_prefill_workspace_bytes(1, 8, n, 128, 128, dtype, mode) if n > 0 else 0 for n in lens)
+        each = [la.la_prefill_workspace_bytes(1, 8, n, 128, 128, dtype, mode) if n > 0 else 0 for n in lens]
+        want = sum((n + 255) // 256 * 256 for n in each)
         assert la.la_prefill_varlen_workspace_bytes(lens, 8, 128, 128, dtype, mode) == want
     assert la.la_prefill_varlen_workspace_bytes([], 8, 128, 128) == 0
