@@ -254,15 +254,20 @@ cudaError_t launch_gdelta_t(const PrefillArgs& a)
 // GLA, per-key-channel gate ("Efficient attention variants" §7.2), token
 // recurrence:
 //     S_t[i][j] = alpha_t[i] S_{t-1}[i][j] + k_t[i] v_t[j],  o_t[j] = sum_i q_t[i] S_t[i][j]
-// Four threads share a state column (every fourth row each, in registers,
-// so that the four read neighbouring words of the staged vectors) and add
-// their parts of o_t with two shuffles.  k, q, alpha and
-// the block's v columns of kGlaTile tokens are staged in shared memory by
-// cp.async, double-buffered, so the next tile streams in while this one is
-// consumed.
+// Eight threads share a state column, each holding a contiguous block of
+// R = d/8 rows in registers, and add their parts of o_t with three shuffles.
+// Per tile of kGlaTile tokens, k, q, alpha and the block's v columns stream
+// into shared memory by cp.async (double-buffered); k and q are converted to
+// fp32 once per tile, so the token loop reads every operand with 128-bit
+// loads.  The fp32 rows are stored as 8 blocks of R values with a 16-byte
+// skew between blocks (block stride an odd number of 16-byte units), so the
+// eight row blocks a warp reads at once fall in distinct banks.  Outputs of a
+// tile are collected in shared memory and written as 16-byte pieces.
 
 constexpr int kGlaTile = 16;   // tokens per staged tile
-constexpr int kGlaCols = 32;   // state columns per block (x 4 threads)
+constexpr int kGlaCols = 32;   // state columns per block
+constexpr int kGlaTpc = 8;     // threads per state column
+constexpr int kGlaThreads = kGlaCols * kGlaTpc;
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes)
 {
@@ -275,61 +280,86 @@ __device__ __forceinline__ void cp_async_wait_groups() { asm volatile("cp.async.
 
 template <typename T, int D>
 struct GlaSmem {
-    T k[2][kGlaTile][D];
-    T q[2][kGlaTile][D];
-    float a[2][kGlaTile][D];
+    static constexpr int R = D / kGlaTpc;     // rows per thread
+    static constexpr int BS = R + 4;          // fp32 row-block stride (R/4 + 1 16-byte units: odd)
+    static constexpr int RS = kGlaTpc * BS;   // fp32 row stride
+    T kr[2][kGlaTile][D];                     // k, q as loaded
+    T qr[2][kGlaTile][D];
+    float a[2][kGlaTile][RS];                 // alpha, skewed row blocks
     T v[2][kGlaTile][kGlaCols];
+    float kf[kGlaTile][RS];                   // k, q in fp32, skewed row blocks
+    float qf[kGlaTile][RS];
+    float o[kGlaTile][kGlaCols];
 };
 
+template <typename T> __device__ __forceinline__ void unpack16(const uint4& u, float* f);
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float* f)
+{
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+template <> __device__ __forceinline__ void unpack16<float>(const uint4& u, float* f)
+{
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(4 * kGlaCols)
+__global__ void __launch_bounds__(kGlaThreads)
 gla_token_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                const float* __restrict__ alpha, const float* __restrict__ S0, T* __restrict__ out,
                float* __restrict__ S_out, int N, int dv, int ld)
 {
-    constexpr int R = D / 4;                          // rows per thread
+    using SM = GlaSmem<T, D>;
+    constexpr int R = SM::R, BS = SM::BS;
+    constexpr int EP = 16 / (int)sizeof(T);           // elements per 16-byte piece
     extern __shared__ __align__(16) unsigned char gla_smem[];
-    GlaSmem<T, D>& sh = *reinterpret_cast<GlaSmem<T, D>*>(gla_smem);
+    SM& sh = *reinterpret_cast<SM*>(gla_smem);
     const int tid = threadIdx.x;
-    const int rg = tid & 3, jl = tid >> 2;            // row group, local column
-    const int j = blockIdx.y * kGlaCols + jl;         // state column
-    // this thread's rows: rg, rg + 4, rg + 8, ...
+    const int rg = tid & (kGlaTpc - 1), jl = tid / kGlaTpc;   // row block, local column
+    const int j = blockIdx.y * kGlaCols + jl;                 // state column
     const long long chain = blockIdx.x;
     const bool active = j < dv;
     const T* qc = q + chain * (long long)ld * D;
     const T* kc = k + chain * (long long)ld * D;
     const float* ac = alpha + chain * (long long)ld * D;
     const T* vc = v + chain * (long long)ld * dv + blockIdx.y * kGlaCols;
-    T* oc = out + chain * (long long)ld * dv;
+    T* oc = out + chain * (long long)ld * dv + blockIdx.y * kGlaCols;
     const int vcols = min(kGlaCols, dv - (int)blockIdx.y * kGlaCols);
 
+    // this thread's rows: rg*R .. rg*R + R-1
     float s[R];
 #pragma unroll
     for (int i = 0; i < R; ++i)
-        s[i] = (S0 && active) ? S0[chain * (long long)D * dv + (long long)(4 * i + rg) * dv + j] : 0.f;
+        s[i] = (S0 && active) ? S0[chain * (long long)D * dv + (long long)(rg * R + i) * dv + j] : 0.f;
 
     // stage tile `tile` into buffer `b`: 16-byte pieces, zero past the end
     auto stage = [&](int tile, int b) {
         const int t0 = tile * kGlaTile;
-        constexpr int KQ = kGlaTile * D * (int)sizeof(T) / 16;   // pieces of k (and of q)
-        constexpr int AP = kGlaTile * D * 4 / 16;                 // pieces of alpha
-        constexpr int VP = kGlaTile * kGlaCols * (int)sizeof(T) / 16;
-        constexpr int PR = D * (int)sizeof(T) / 16;               // pieces per k/q row
-        constexpr int PA = D * 4 / 16;
-        constexpr int PV = kGlaCols * (int)sizeof(T) / 16;
-        for (int e = tid; e < 2 * KQ + AP + VP; e += blockDim.x) {
+        constexpr int PR = D / EP;                              // pieces per k/q row
+        constexpr int KQ = kGlaTile * PR;                       // pieces of k (and of q)
+        constexpr int PA = D / 4;                               // pieces per alpha row
+        constexpr int AP = kGlaTile * PA;
+        constexpr int PV = kGlaCols / EP;                       // pieces per v row
+        constexpr int VP = kGlaTile * PV;
+        for (int e = tid; e < 2 * KQ + AP + VP; e += kGlaThreads) {
             if (e < 2 * KQ) {
                 const int which = e / KQ, r = (e % KQ) / PR, c = (e % KQ) % PR;
                 const int t = t0 + r;
-                const T* src = (which ? qc : kc) + (long long)min(t, N - 1) * D + c * (16 / (int)sizeof(T));
-                T* dst = (which ? &sh.q[b][r][0] : &sh.k[b][r][0]) + c * (16 / (int)sizeof(T));
+                const T* src = (which ? qc : kc) + (long long)min(t, N - 1) * D + c * EP;
+                T* dst = (which ? &sh.qr[b][r][0] : &sh.kr[b][r][0]) + c * EP;
                 cp_async16(dst, src, t < N ? 16u : 0u);
             } else if (e < 2 * KQ + AP) {
-                const int f = e - 2 * KQ, r = f / PA, c = f % PA, t = t0 + r;
-                cp_async16(&sh.a[b][r][c * 4], ac + (long long)min(t, N - 1) * D + c * 4, t < N ? 16u : 0u);
+                const int f = e - 2 * KQ, r = f / PA, f0 = (f % PA) * 4, t = t0 + r;
+                cp_async16(&sh.a[b][r][(f0 / R) * BS + f0 % R], ac + (long long)min(t, N - 1) * D + f0,
+                           t < N ? 16u : 0u);
             } else {
-                const int f = e - 2 * KQ - AP, r = f / PV, c = f % PV, t = t0 + r;
-                const int col = c * (16 / (int)sizeof(T));
+                const int f = e - 2 * KQ - AP, r = f / PV, col = (f % PV) * EP, t = t0 + r;
                 const bool ok = t < N && col < vcols;
                 cp_async16(&sh.v[b][r][col], vc + (long long)min(t, N - 1) * dv + (ok ? col : 0), ok ? 16u : 0u);
             }
@@ -348,28 +378,72 @@ gla_token_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __rest
             cp_async_wait_groups<0>();
         }
         __syncthreads();
+        // k, q of this tile to fp32 (8 consecutive features stay in one row block)
+        for (int e = tid; e < 2 * kGlaTile * (D / 8); e += kGlaThreads) {
+            const int which = e / (kGlaTile * (D / 8)), rem = e % (kGlaTile * (D / 8));
+            const int r = rem / (D / 8), f0 = (rem % (D / 8)) * 8;
+            const T* src = (which ? &sh.qr[b][r][0] : &sh.kr[b][r][0]) + f0;
+            float f[8];
+            unpack16<T>(*reinterpret_cast<const uint4*>(src), f);
+            if (EP == 4) unpack16<T>(*reinterpret_cast<const uint4*>(src + 4), f + 4);
+            float* dst = (which ? &sh.qf[r][0] : &sh.kf[r][0]) + (f0 / R) * BS + f0 % R;
+            reinterpret_cast<float4*>(dst)[0] = make_float4(f[0], f[1], f[2], f[3]);
+            reinterpret_cast<float4*>(dst)[1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+        __syncthreads();
         const int n = min(kGlaTile, N - tile * kGlaTile);
         for (int t = 0; t < n; ++t) {
             const float vt = to_f32(sh.v[b][t][jl]);
+            const float4* ap = reinterpret_cast<const float4*>(&sh.a[b][t][rg * BS]);
+            const float4* kp = reinterpret_cast<const float4*>(&sh.kf[t][rg * BS]);
+            const float4* qp = reinterpret_cast<const float4*>(&sh.qf[t][rg * BS]);
             float o0 = 0.f, o1 = 0.f;
 #pragma unroll
-            for (int i = 0; i < R; i += 2) {
-                const int ra = 4 * i + rg, rb = 4 * (i + 1) + rg;
-                s[i] = fmaf(sh.a[b][t][ra], s[i], to_f32(sh.k[b][t][ra]) * vt);
-                s[i + 1] = fmaf(sh.a[b][t][rb], s[i + 1], to_f32(sh.k[b][t][rb]) * vt);
-                o0 = fmaf(s[i], to_f32(sh.q[b][t][ra]), o0);
-                o1 = fmaf(s[i + 1], to_f32(sh.q[b][t][rb]), o1);
+            for (int i4 = 0; i4 < R / 4; ++i4) {
+                const float4 a4 = ap[i4], k4 = kp[i4], q4 = qp[i4];
+                float* si = s + 4 * i4;
+                si[0] = fmaf(a4.x, si[0], k4.x * vt);
+                si[1] = fmaf(a4.y, si[1], k4.y * vt);
+                si[2] = fmaf(a4.z, si[2], k4.z * vt);
+                si[3] = fmaf(a4.w, si[3], k4.w * vt);
+                o0 = fmaf(si[0], q4.x, o0);
+                o1 = fmaf(si[1], q4.y, o1);
+                o0 = fmaf(si[2], q4.z, o0);
+                o1 = fmaf(si[3], q4.w, o1);
             }
             float o = o0 + o1;
             o += __shfl_xor_sync(0xffffffffu, o, 1);
             o += __shfl_xor_sync(0xffffffffu, o, 2);
-            if (active && rg == 0) oc[(long long)(tile * kGlaTile + t) * dv + j] = from_f32<T>(o);
+            o += __shfl_xor_sync(0xffffffffu, o, 4);
+            if (rg == 0) sh.o[t][jl] = o;
         }
-        __syncthreads();   // buffer b is restaged two tiles from now
+        __syncthreads();
+        // this tile's outputs: n rows of the block's columns, 16-byte pieces
+        {
+            constexpr int PO = kGlaCols / EP;   // pieces per output row
+            for (int e = tid; e < n * PO; e += kGlaThreads) {
+                const int r = e / PO, col = (e % PO) * EP;
+                if (col < vcols) {
+                    const float* src = &sh.o[r][col];
+                    T* dst = oc + (long long)(tile * kGlaTile + r) * dv + col;
+                    if (EP == 8) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(src[2 * x], src[2 * x + 1]);
+                            w[x] = *reinterpret_cast<const uint32_t*>(&h);
+                        }
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                    } else {
+                        *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(src);
+                    }
+                }
+            }
+        }
     }
     if (active) {
 #pragma unroll
-        for (int i = 0; i < R; ++i) S_out[chain * (long long)D * dv + (long long)(4 * i + rg) * dv + j] = s[i];
+        for (int i = 0; i < R; ++i) S_out[chain * (long long)D * dv + (long long)(rg * R + i) * dv + j] = s[i];
     }
 }
 
@@ -381,7 +455,7 @@ cudaError_t launch_gla_t(const PrefillArgs& a)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.B * a.H, (a.dv + kGlaCols - 1) / kGlaCols);
-    kern<<<grid, 4 * kGlaCols, smem, a.stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.S0,
+    kern<<<grid, kGlaThreads, smem, a.stream>>>((const T*)a.q, (const T*)a.k, (const T*)a.v, a.alpha, a.S0,
                                                  (T*)a.out, a.S_out, a.N, a.dv, a.ld);
     e = cudaGetLastError();
     if (e == cudaSuccess) stage_mark(0, a.stream);
