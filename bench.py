@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -39,7 +40,8 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 # ----------------------------------------------------------------------------
-# work accounting (algorithmic bytes / flops per step)
+# work accounting (algorithmic bytes / flops per step: what the recurrence itself
+# must read, write and compute, not the chunk form's extra work)
 
 def prefill_units(p) -> dict:
     """Tokens, token-heads and the method's own bytes/flops for one prefill."""
@@ -329,8 +331,12 @@ def run_gpu(args, world, rank, local):
         if world > 1:
             torch.distributed.barrier()
 
-    clocks_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if os.path.isdir(
-        os.path.join(ROOT, "gpurun_out")) else None
+    # the SM clock record of the timed region: kept under --clocks-dir, else
+    # in a temporary file that is removed once read
+    if args.clocks_dir:
+        clocks_path = os.path.join(args.clocks_dir, f"clocks_rank{rank}.csv")
+    else:
+        clocks_path = os.path.join(tempfile.gettempdir(), f"la_bench_clocks_{os.getpid()}_rank{rank}.csv")
     with ClockSampler(local, clocks_path) as clk:
         barrier()
         ms = time_prefill(p, args.steps, args.warmup, torch, la, flush)
@@ -347,6 +353,11 @@ def run_gpu(args, world, rank, local):
     e2e_ms = max_over_ranks(e2e_ms, world, device="cuda")
     e2e_value = aggregate_throughput(u["tokens"], world, e2e_ms / 1e3)
     clk_sum = clk.summary()
+    if not args.clocks_dir:
+        try:
+            os.remove(clocks_path)
+        except OSError:
+            pass
 
     avg_launch_ms = local_total_ms / args.steps
     call_gbs = u["bytes"] / (avg_launch_ms / 1e3) / 1e9
@@ -367,7 +378,7 @@ def run_gpu(args, world, rank, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": path_dtype(p),
-        "data": "synthetic (seeded numpy normal draws; see DESIGN.md input recipe)",
+        "data": "synthetic (seeded numpy normal draws of the workload's shape and scale)",
         "config": {"workload": workload_desc(args.workload), "global_batch": p.B * world, "seq_len": p.N,
                    "heads": p.H, "d": p.d, "dv": p.dv, "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed before every timed step (256 MiB write outside the timed events)"},
@@ -642,6 +653,8 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--clocks-dir", default=None,
+                    help="keep the nvidia-smi clock samples of the timed region here (clocks_rank<r>.csv)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="profiling aid: the workload with this many tokens per chain instead of its own "
                          "(the line's config says so); not a benchmark configuration")
