@@ -95,6 +95,17 @@ def test_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 8, 64)
     with pytest.raises(ValueError):
         la.la_prefill(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        la.la_prefill_varlen(q, q, q, [5])
+
+
+def test_varlen_binding_checks_the_lengths_list():
+    import torch
+    q = torch.zeros(2, 1, 8, 64)
+    with pytest.raises(ValueError, match="seq_lens"):
+        la.la_prefill_varlen(q, q, q, [5])            # one length for a batch of two
+    with pytest.raises(ValueError, match="mode"):
+        la.la_prefill_varlen(q, q, q, [5, 8], mode="softmax")
 
 
 def test_workspace_query_is_host_only():
