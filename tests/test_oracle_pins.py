@@ -458,3 +458,25 @@ def test_gla_constant_gate_is_the_scalar_decay_form():
     Gam = np.where(idx[:, None] >= idx[None, :], gamma ** (idx[:, None] - idx[None, :]).clip(min=0), 0.0)
     ref = ((q[0, 0] @ k[0, 0].T) * Gam) @ v[0, 0]
     np.testing.assert_allclose(o[0, 0], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_empty_sequence_returns_the_start_state():
+    """A chain of no tokens has no update to apply: every mode returns its
+    start state unchanged (zero without one), which is what a zero-length
+    sequence of a padded batch must report."""
+    rng = np.random.default_rng(23)
+    B, H, d, dv = 2, 3, 4, 5
+    e = lambda *s: np.zeros(s)
+    S0 = rng.normal(size=(B, H, d, dv))
+    z0 = rng.uniform(1, 2, size=(B, H, d))
+    gam = np.array([0.9, 0.95, 1.0])
+    o, S, z = oracle.kernelized(e(B, H, 0, d), e(B, H, 0, d), e(B, H, 0, dv), gam, S0, z0)
+    assert o.shape == (B, H, 0, dv)
+    np.testing.assert_array_equal(S, S0)
+    np.testing.assert_array_equal(z, z0)
+    o, S, z = oracle.kernelized(e(B, H, 0, d), e(B, H, 0, d), e(B, H, 0, dv))
+    assert not S.any() and not z.any()
+    _, S = oracle.gated_delta(e(B, H, 0, d), e(B, H, 0, d), e(B, H, 0, dv), e(B, H, 0), e(B, H, 0), S0)
+    np.testing.assert_array_equal(S, S0)
+    _, S = oracle.gla(e(B, H, 0, d), e(B, H, 0, d), e(B, H, 0, dv), e(B, H, 0, d), S0)
+    np.testing.assert_array_equal(S, S0)
