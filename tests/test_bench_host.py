@@ -1,5 +1,6 @@
-"""Host logic of bench.py's clock record: the nvidia-smi sample parser and
-the sampler's behaviour where nvidia-smi cannot run (no GPU needed)."""
+"""Host logic of bench.py: the nvidia-smi clock-sample parser, the sampler
+where nvidia-smi cannot run, and the traffic record keyed to a source file
+(no GPU needed)."""
 import os
 import tempfile
 
@@ -34,3 +35,21 @@ def test_clock_sampler_without_samples():
     assert s["samples"] >= 0 and isinstance(s["reasons"], list)
     if os.path.exists(path):
         os.remove(path)
+
+
+def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from an ncu capture of a kernel's source file;
+    once the file differs from the captured one it must read as unknown."""
+    import hashlib
+    src = tmp_path / "kernel.cu"
+    src.write_text("// captured version\n")
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "TRAFFIC_CAPTURES", {("w", "k"): {"bytes": 123, "source": "kernel.cu",
+                                                                 "sha256": digest, "profile": "p.md"}})
+    assert bench.captured_traffic("w", "k") == 123
+    assert bench.captured_traffic("w", "other") is None
+    src.write_text("// changed since the capture\n")
+    assert bench.captured_traffic("w", "k") is None
+    src.unlink()
+    assert bench.captured_traffic("w", "k") is None
