@@ -138,9 +138,10 @@ LA_API la_status la_prefill(const void* q, const void* k, const void* v,
  * All calls in one process share the array and it keeps the last call's
  * contents: calls whose work can overlap on the GPU (enqueued on different
  * streams, or from different host threads) race on it and must be
- * serialised by the caller.  Separate processes each have their own copy.  The first call on each device looks up the array's device
- * address with that device current; make that first call before any stream
- * capture on that device.
+ * serialised by the caller.  Separate processes each have their own copy.
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture on
+ * that device.
  */
 LA_API la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
                                     const float* gamma_or_alpha, const float* g,
