@@ -34,7 +34,7 @@ MODES = {"plain": 0, "decay": 1, "gated_delta": 2, "gla": 3}
 # Symbols the library exports; the header include/la.h declares exactly these.
 EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_prefill_varlen",
            "la_prefill_varlen_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
-           "la_set_stage_events", "la_causal_conv",
+           "la_set_stage_events", "la_causal_conv", "la_selftest_wait_timeout",
            "la_prefill_check", "la_status_string", "la_version")
 
 
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.la_gated_delta_decode_step.restype = i
         L.la_prefill_check.argtypes = [vp, vp]
         L.la_prefill_check.restype = i
+        L.la_selftest_wait_timeout.argtypes = [vp]
+        L.la_selftest_wait_timeout.restype = i
         L.la_causal_conv.argtypes = [vp] * 5 + [i] * 5 + [cfgp]
         L.la_causal_conv.restype = i
         L.la_set_stage_events.argtypes = [ctypes.POINTER(vp), i]
@@ -300,6 +302,14 @@ def la_set_stage_events(events=None):
     rc = lib().la_set_stage_events(arr, len(events))
     if rc != LA_OK:
         raise LaError(rc, "la_set_stage_events")
+
+
+def la_selftest_wait_timeout(stream=None):
+    """Enqueue the bounded-wait failure self-test; the next la_prefill_check
+    on the stream raises LaError with code LA_ERR_TIMEOUT."""
+    rc = lib().la_selftest_wait_timeout(_stream_handle(stream))
+    if rc != LA_OK:
+        raise LaError(rc, "la_selftest_wait_timeout")
 
 
 def la_prefill_check(workspace=None, stream=None):

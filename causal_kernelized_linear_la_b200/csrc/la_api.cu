@@ -356,6 +356,11 @@ la_status la_set_stage_events(void* const* events, int n)
     return LA_OK;
 }
 
+la_status la_selftest_wait_timeout(void* stream)
+{
+    return la::from_cuda(la::launch_wait_timeout_selftest(static_cast<cudaStream_t>(stream)));
+}
+
 la_status la_prefill_check(const void* workspace, void* stream)
 {
     (void)workspace;
@@ -363,8 +368,9 @@ la_status la_prefill_check(const void* workspace, void* stream)
     if (cudaStreamSynchronize(s) != cudaSuccess) return LA_ERR_CUDA;
     const unsigned int e1 = la::read_and_clear_device_error(s);
     const unsigned int e2 = la::read_and_clear_device_error_gdelta(s);
+    const unsigned int e3 = la::read_and_clear_device_error_selftest(s);
     if (e1 == 4u || e2 == 4u) return LA_ERR_UNSUPPORTED;
-    if (e1 != 0 || e2 != 0) return LA_ERR_TIMEOUT;
+    if (e1 != 0 || e2 != 0 || e3 != 0) return LA_ERR_TIMEOUT;
     return LA_OK;
 }
 

@@ -103,4 +103,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // `stream` right after a call's i-th kernel launch, if one is set.
 void stage_mark(int i, cudaStream_t stream);
 
+// Failure-path self-test of the bounded waits (la_selftest.cu): one kernel
+// whose mbarrier wait runs out, and the reader of that unit's error word.
+cudaError_t launch_wait_timeout_selftest(cudaStream_t stream);
+unsigned int read_and_clear_device_error_selftest(cudaStream_t stream);
+
 }  // namespace la

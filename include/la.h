@@ -289,6 +289,17 @@ LA_API la_status la_set_stage_events(void* const* events, int n);
  */
 LA_API la_status la_prefill_check(const void* workspace, void* stream);
 
+/*
+ * la_selftest_wait_timeout -- exercise the failure path of the bounded
+ * device-side waits.  Enqueues on `stream` one kernel of 32 threads whose
+ * single mbarrier wait has nothing to wait for: the wait gives up after its
+ * bound (about a second), records the timeout in the device error word and
+ * returns, leaving the context usable.  The next la_prefill_check on that
+ * stream returns LA_ERR_TIMEOUT and clears the word.  For tests of error
+ * reporting; it issues no copy and no MMA.  Returns LA_OK once enqueued.
+ */
+LA_API la_status la_selftest_wait_timeout(void* stream);
+
 /* Human-readable name of a status code (static storage). */
 LA_API const char* la_status_string(la_status s);
 
