@@ -1,4 +1,6 @@
-"""Failure detection without a GPU fault: a bounded device-side wait that
+"""(Runs last: it is the one test that drives a device error path.)
+
+Failure detection without a GPU fault: a bounded device-side wait that
 runs out is reported to the host, and the context stays usable.
 
 la_selftest_wait_timeout enqueues one kernel whose mbarrier wait has nothing
