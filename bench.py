@@ -1,16 +1,24 @@
 """Benchmark: causal kernelized linear attention on B200.
 
 One step = one pass of the hot path over one batch of synthetic input:
-``la_prefill`` over the headline workload (``plain_bf16``: B=4, H=8, N=4096,
-d=dv=64, bf16 inputs, plain causal prefill with normaliser).  The metric is
-prefill tokens/s (tokens = B*N per step; each token carries H heads).
+``la_prefill`` over the headline workload ``gdelta_bf16`` (the largest
+single-GPU configuration: gated delta rule, B=1, H=32, N=65536,
+d=dv=128, bf16 inputs, fp32 state).  The metric is prefill tokens/s
+(tokens = B*N per step; each token carries H heads) and the roofline
+fraction of the call's dominant kernel.
 
 Timing: W untimed warm-up steps, then K timed steps.  Inputs stay resident in
 HBM; L2 is flushed (a 256 MiB write, outside the timed events) before every
-timed step because the headline inputs (~50 MB) fit in L2.  Each step is
-timed with CUDA events on the stream the kernels run on; for N GPUs every
-rank processes its own full batch (independent problems: weak scaling, no
-data-path collective) and the time is the max over ranks.
+timed step.  Each step is timed with CUDA events on the stream the kernels
+run on; for N GPUs every rank processes its own full batch (independent
+problems: weak scaling, no data-path collective) and the time is the max
+over ranks.  ``--gpus N`` starts the N ranks itself (one process per GPU)
+unless it runs under torchrun, whose WORLD_SIZE must then equal N.
+
+``other_workloads`` carries the other configurations, each with its own
+roofline and end-to-end numbers: plain and decay kernelized prefill, the
+fp32 prefill, the decode steps (kernelized and gated delta, 1000 chained
+steps), GLA, the short causal convolution and a variable-length batch.
 
 Printed: one JSON line (rank 0).  ``--impl reference`` times the float64 CPU
 oracle (the only reference this method has) on a bounded sample instead.
@@ -34,7 +42,7 @@ sys.path.insert(0, ROOT)
 
 from causal_kernelized_linear_la_b200 import inputs  # noqa: E402
 
-HEADLINE = "plain_bf16"
+HEADLINE = "gdelta_bf16"
 METRIC = "prefill tokens/s and decode state-updates/s on 1 B200; % of roofline"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -61,9 +69,13 @@ def prefill_units(p) -> dict:
     return {"tokens": p.B * p.N, "token_heads": th, "bytes": byts, "flops": flops}
 
 
-def decode_units(Bs, Hh, d, dv, eb=2) -> dict:
+def decode_units(Bs, Hh, d, dv, eb=2, gated=False) -> dict:
+    """Bytes one decode step must move: the fp32 state read and written, the
+    token in and the output out (kernelized: z read and written too; gated
+    delta: alpha and g in)."""
     states = Bs * Hh
-    byts = states * (2 * d * dv * 4 + 2 * d * 4 + (2 * d + 2 * dv) * eb)
+    side = 8 if gated else 2 * d * 4
+    byts = states * (2 * d * dv * 4 + side + (2 * d + 2 * dv) * eb)
     return {"state_updates": states, "tokens": Bs, "bytes": byts, "flops": states * 4 * d * dv}
 
 
@@ -71,6 +83,9 @@ def workload_desc(name: str) -> str:
     w = inputs.WORKLOADS[name]
     if w["kind"] == "decode":
         return f"{name}: decode step, {w['S']} sequences x {w['H']} heads, d=dv={w['d']}, fp32 state, bf16 tokens"
+    if w["kind"] == "decode_gated_delta":
+        return (f"{name}: gated delta decode step, {w['S']} sequences x {w['H']} heads, d=dv={w['d']}, "
+                f"fp32 state, bf16 tokens, alpha and g per step")
     what = {"plain": "plain causal prefill with normaliser", "decay": "per-head decay prefill with decayed normaliser",
             "gated_delta": "gated delta rule prefill", "gla": "per-key-channel gated (GLA) prefill"}[
         w.get("mode", w["kind"])]
@@ -236,78 +251,198 @@ def time_prefill(p, steps, warmup, torch, la, flush):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-def time_prefill_e2e(p, steps, warmup, torch, la):
-    """End to end through the public API with host buffers: pinned host inputs
-    copied in, la_prefill, output copied back, every step inside the events."""
-    pin = lambda x: None if x is None else torch.from_numpy(
-        np.ascontiguousarray(x).view(np.int16) if x.dtype == np.uint16 else np.ascontiguousarray(x)).pin_memory()
-    if p.dtype == "bf16":
-        hq, hk, hv = pin(p.q_bits), pin(p.k_bits), pin(p.v_bits)
-        tdt = torch.bfloat16
-    else:
-        hq, hk, hv = pin(p.q), pin(p.k), pin(p.v)
-        tdt = torch.float32
-    hextra = {}
-    if p.mode == "decay":
-        hextra["gamma"] = pin(p.gamma)
-    if p.mode == "gated_delta":
-        hextra["alpha"], hextra["g"] = pin(p.alpha), pin(p.g)
-    if p.mode == "gla":
-        hextra["alpha"] = pin(p.alpha)
-    dq = torch.empty(hq.shape, dtype=hq.dtype, device="cuda")
-    dk = torch.empty_like(dq)
-    dvv = torch.empty(hv.shape, dtype=hv.dtype, device="cuda")
-    dextra = {n: torch.empty_like(t, device="cuda") for n, t in hextra.items()}
-    B, H, N, d = p.q.shape
-    dv = p.v.shape[-1]
-    h_out = torch.empty((B, H, N, dv), dtype=tdt).pin_memory()
-    stream = torch.cuda.current_stream()
-    h2d = sum(t.numel() * t.element_size() for t in [hq, hk, hv] + list(hextra.values()))
-    d2h = h_out.numel() * h_out.element_size()
+def _pinned(x, torch):
+    """A pinned host tensor holding numpy array x (bf16 bit patterns as int16)."""
+    if x is None:
+        return None
+    a = np.ascontiguousarray(x)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).pin_memory()
+
+
+def time_e2e(host, call, steps, warmup, torch):
+    """End to end through the public API with host buffers: every step copies
+    the pinned host tensors ``host`` (name -> tensor) into their device twins,
+    runs ``call(device_tensors)`` (which returns the device results) and copies
+    the results back into pinned host buffers, all inside the CUDA events.
+    Returns (ms per step, H2D bytes per step, D2H bytes per step)."""
+    dev = {n: torch.empty(t.shape, dtype=t.dtype, device="cuda") for n, t in host.items()}
+    outs_h = []
 
     def step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dvv.copy_(hv, non_blocking=True)
-        for n in hextra:
-            dextra[n].copy_(hextra[n], non_blocking=True)
-        o, _, _ = la.la_prefill(dq.view(tdt), dk.view(tdt), dvv.view(tdt), mode=p.mode, eps=p.eps, **dextra)
-        h_out.copy_(o, non_blocking=True)
+        for n, t in host.items():
+            dev[n].copy_(t, non_blocking=True)
+        outs = call(dev)
+        if not outs_h:
+            outs_h.extend(torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs)
+        for h, o in zip(outs_h, outs):
+            h.copy_(o, non_blocking=True)
 
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(steps):
         step()
     b.record(stream)
     torch.cuda.synchronize()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
     return a.elapsed_time(b) / steps, h2d, d2h
 
 
-def time_decode(steps, warmup, torch, la, seed, Bs=256, Hh=32, d=128, dv=128, pool=8):
-    """Device time per decode step (ms) over `steps` chained steps; tokens come
-    from a pool of `pool` pre-generated steps (identical cost per step)."""
+def time_prefill_e2e(p, steps, warmup, torch, la):
+    """la_prefill end to end: q, k, v (and gamma / alpha / g) from pinned host
+    memory, the output o copied back, every step inside the events."""
+    host = {"q": _pinned(p.q_bits if p.dtype == "bf16" else p.q, torch),
+            "k": _pinned(p.k_bits if p.dtype == "bf16" else p.k, torch),
+            "v": _pinned(p.v_bits if p.dtype == "bf16" else p.v, torch)}
+    if p.mode == "decay":
+        host["gamma"] = _pinned(p.gamma, torch)
+    if p.mode in ("gated_delta", "gla"):
+        host["alpha"] = _pinned(p.alpha, torch)
+    if p.mode == "gated_delta":
+        host["g"] = _pinned(p.g, torch)
+    tdt = torch.bfloat16 if p.dtype == "bf16" else torch.float32
+
+    def call(d):
+        kw = {n: d[n] for n in ("gamma", "alpha", "g") if n in d}
+        o, _, _ = la.la_prefill(d["q"].view(tdt), d["k"].view(tdt), d["v"].view(tdt), mode=p.mode, eps=p.eps, **kw)
+        return [o]
+
+    return time_e2e(host, call, steps, warmup, torch)
+
+
+def time_decode(steps, warmup, torch, la, seed, gated=False, Bs=256, Hh=32, d=128, dv=128, pool=8):
+    """Device time per decode step (ms) over `steps` chained steps on the
+    resident state; tokens come from a pool of `pool` pre-generated steps
+    (identical cost per step).  Returns (ms per step, end-to-end record)."""
     st = inputs.make_decode_state(Bs, Hh, d, dv, seed=seed)
     S = torch.from_numpy(st.S).cuda()
     z = torch.from_numpy(st.z).cuda()
     toks = []
     for s in range(pool):
-        t = inputs.make_decode_token(s, Bs, Hh, d, dv, seed=seed)
-        toks.append(tuple(_to_dev(x, torch) for x in (t.q_bits, t.k_bits, t.v_bits)))
+        if gated:
+            t = inputs.make_gated_delta_decode_token(s, Bs, Hh, d, dv, seed=seed)
+            arrs = (t.q_bits, t.k_bits, t.v_bits, t.alpha, t.g)
+        else:
+            t = inputs.make_decode_token(s, Bs, Hh, d, dv, seed=seed)
+            arrs = (t.q_bits, t.k_bits, t.v_bits)
+        toks.append(arrs)
+    dtoks = [tuple(_to_dev(x, torch) for x in a) for a in toks]
     out = torch.empty((Bs, Hh, dv), device="cuda", dtype=torch.bfloat16)
+
+    def run(tk, o):
+        if gated:
+            return la.la_gated_delta_decode_step(*tk, S, out=o)
+        return la.la_decode_step(*tk, S, z, out=o)
+
     for i in range(warmup):
-        la.la_decode_step(*toks[i % pool], S, z, out=out)
+        run(dtoks[i % pool], out)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for i in range(steps):
-        la.la_decode_step(*toks[i % pool], S, z, out=out)
+        run(dtoks[i % pool], out)
     b.record(stream)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps
+    ms = a.elapsed_time(b) / steps
+
+    # end to end: each step's token from pinned host memory, o back to the
+    # host; the state stays resident on the device (the decode cache)
+    names = ("q", "k", "v", "alpha", "g") if gated else ("q", "k", "v")
+    hosts = [dict(zip(names, (_pinned(x, torch) for x in a))) for a in toks]
+    cur = {"i": 0}
+    host = dict(hosts[0])
+
+    def call(dd):
+        cur["i"] += 1
+        for n in names:   # the next token's host buffers for the next step
+            host[n] = hosts[cur["i"] % pool][n]
+        tk = [dd["q"].view(torch.bfloat16), dd["k"].view(torch.bfloat16), dd["v"].view(torch.bfloat16)]
+        if gated:
+            tk += [dd["alpha"], dd["g"]]
+        return [run(tk, None)]
+
+    e_ms, h2d, d2h = time_e2e(host, call, 200, 5, torch)
+    return ms, (e_ms, h2d, d2h)
+
+
+def roofline_block(nbytes, kms, hbm_peak, peak_kind, workload, call_ms):
+    """The roofline object of one call: algorithmic bytes over the dominant
+    kernel's CUDA-event time, against the measured HBM copy bandwidth."""
+    dom = max(kms, key=kms.get)
+    achieved = nbytes / (kms[dom] / 1e3) / 1e9
+    call_gbs = nbytes / (call_ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+            "traffic": captured_traffic(workload, dom), "kernel": dom, "kernel_ms": kms[dom],
+            "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": nbytes,
+            "call_kernels_ms": kms, "whole_call": {"achieved": call_gbs, "frac": call_gbs / hbm_peak}}
+
+
+def measure_prefill(name, p, steps, warmup, torch, la, flush, e2e_steps=10):
+    """Device-timed throughput, per-kernel roofline and end-to-end numbers of
+    one prefill workload.  Returns (record, list of per-step ms)."""
+    hbm_peak, _, peak_kind = _measured_peaks()
+    u = prefill_units(p)
+    ms = time_prefill(p, steps, warmup, torch, la, flush)
+    med = statistics.median(ms)
+    kms = time_kernels(p, max(3, min(steps, 20)), torch, la, flush)
+    e_ms, h2d, d2h = time_prefill_e2e(p, e2e_steps, 2, torch, la)
+    rec = {"workload": workload_desc(name), "value": u["tokens"] / (med / 1e3), "unit": "tokens/s", "ms": med,
+           "dtype": path_dtype(p), "roofline": roofline_block(u["bytes"], kms, hbm_peak, peak_kind, name, med),
+           "e2e": {"value": u["tokens"] / (e_ms / 1e3), "unit": "tokens/s", "ms": e_ms,
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           "gpu_launches_per_call": la_launches_per_step(p)}
+    return rec, ms
+
+
+def measure_decode(name, torch, la, rank):
+    hbm_peak, _, peak_kind = _measured_peaks()
+    spec = inputs.WORKLOADS[name]
+    gated = spec["kind"] == "decode_gated_delta"
+    steps = spec["steps"]
+    ms, (e_ms, h2d, d2h) = time_decode(steps, 20, torch, la, rank_seed(spec["seed"], rank), gated=gated,
+                                       Bs=spec["S"], Hh=spec["H"], d=spec["d"], dv=spec["dv"])
+    du = decode_units(spec["S"], spec["H"], spec["d"], spec["dv"], gated=gated)
+    kernel = "decode_gated_delta" if gated else "decode_kernelized"
+    gbs = du["bytes"] / (ms / 1e3) / 1e9
+    return {"workload": workload_desc(name), "value": du["state_updates"] / (ms / 1e3), "unit": "state-updates/s",
+            "tokens_per_s": du["tokens"] / (ms / 1e3), "ms_per_step": ms, "chained_steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "traffic": captured_traffic(name, kernel), "kernel": kernel, "kernel_ms": ms,
+                         "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": du["bytes"]},
+            "e2e": {"value": du["state_updates"] / (e_ms / 1e3), "unit": "state-updates/s", "ms": e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "note": "token in from pinned host memory and o out every step; the state stays resident"},
+            "gpu_launches_per_call": 1}
+
+
+def init_dist(world, local):
+    """Process group of this rank (NCCL on GPUs, gloo where there are none)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return backend
+
+
+def finish_line(line, world):
+    """Close the rank's process group (after a last barrier) and print the
+    line on rank 0."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if int(os.environ.get("RANK", "0")) == 0:
+        print(json.dumps(line), flush=True)
 
 
 def run_gpu(args, world, rank, local):
@@ -316,9 +451,7 @@ def run_gpu(args, world, rank, local):
 
     torch.cuda.set_device(local)
     if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        init_dist(world, local)
     hbm_peak, tc_peak, peak_kind = _measured_peaks()
     spec = inputs.WORKLOADS[args.workload]
     over = {"N": args.seq_len} if args.seq_len else {}
@@ -341,7 +474,9 @@ def run_gpu(args, world, rank, local):
         barrier()
         ms = time_prefill(p, args.steps, args.warmup, torch, la, flush)
         barrier()
-        # keep the device busy a little longer so the clock sampler sees load
+        # the kernel split of the call, the other workloads: the device stays
+        # busy, so the clock sampler sees the load
+        kms = time_kernels(p, max(3, min(args.steps, 20)), torch, la, flush)
         extra = {}
         if not args.no_extra:
             extra = run_extra(args, torch, la, rank, flush)
@@ -360,12 +495,6 @@ def run_gpu(args, world, rank, local):
             pass
 
     avg_launch_ms = local_total_ms / args.steps
-    call_gbs = u["bytes"] / (avg_launch_ms / 1e3) / 1e9
-    launches_per_step = la_launches_per_step(p)
-    # the dominant kernel of the call, timed on its own with CUDA events
-    kms = time_kernels(p, max(3, min(args.steps, 20)), torch, la, flush)
-    dom = max(kms, key=kms.get)
-    achieved_gbs = u["bytes"] / (kms[dom] / 1e3) / 1e9
     line = {
         "metric": METRIC,
         "value": value,
@@ -381,15 +510,13 @@ def run_gpu(args, world, rank, local):
         "data": "synthetic (seeded numpy normal draws of the workload's shape and scale)",
         "config": {"workload": workload_desc(args.workload), "global_batch": p.B * world, "seq_len": p.N,
                    "heads": p.H, "d": p.d, "dv": p.dv, "parallelism": f"replicas x{world} (independent batches)",
-                   "l2": "flushed before every timed step (256 MiB write outside the timed events)"},
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm_peak, "traffic": captured_traffic(args.workload, dom),
-                     "kernel": dom, "kernel_ms": kms[dom], "peak_kind": f"{peak_kind} hbm_gbs",
-                     "algorithmic_bytes_per_launch": u["bytes"],
-                     "call_kernels_ms": kms, "whole_call": {"achieved": call_gbs, "frac": call_gbs / hbm_peak}},
+                   "l2": "flushed before every timed step (256 MiB write outside the timed events); "
+                         "the inputs also exceed L2"},
+        "roofline": roofline_block(u["bytes"], kms, hbm_peak, peak_kind, args.workload, avg_launch_ms),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": la_launches_per_step(p) * args.steps,
         "clocks": clk_sum,
+        "rank_seeds": [rank_seed(spec["seed"], r) for r in range(world)],
     }
     if args.seq_len:
         line["config"]["note"] = "seq_len overridden for profiling; not the benchmark configuration"
@@ -397,12 +524,7 @@ def run_gpu(args, world, rank, local):
         line["other_workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    finish_line(line, world)
 
 
 def path_dtype(p) -> str:
@@ -426,24 +548,13 @@ def la_launches_per_step(p) -> int:
     return len(call_kernels(p))
 
 
-# DRAM traffic of one launch of a kernel, from an ncu capture (profiles/ has the
-# summary and the command).  A capture holds only while the kernel's source is
-# unchanged: the entry records the source file's sha256 at capture time, and the
-# benchmark reports null when the file differs now.
-TRAFFIC_CAPTURES = {
-    ("plain_bf16", "chunk_kernel"): {
-        "bytes": 54647552 + 468736, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "3fc18696f316c1acb3926cfd21d665af34c10a99ecbf2df02eb163e17cf77fea",
-        "profile": "profiles/traffic_dominant_kernels.md"},
-    ("decay_bf16", "chunk_kernel"): {
-        "bytes": 824411136 + 209652992, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "3fc18696f316c1acb3926cfd21d665af34c10a99ecbf2df02eb163e17cf77fea",
-        "profile": "profiles/traffic_dominant_kernels.md"},
-    ("gdelta_bf16", "gd_chain_kernel"): {
-        "bytes": 2693713152 + 525609728, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
-        "sha256": "9d9a2aa7ac6d580ccfa6de2fcbe335fd978cc0ba89cf113edd80e5009ae2f37b",
-        "profile": "profiles/traffic_dominant_kernels.md"},
-}
+# DRAM traffic of one launch of a kernel, from a one-pass ncu capture of that
+# kernel alone (--metrics dram__bytes_read.sum,dram__bytes_write.sum
+# --clock-control none, one launch) in the workload's launch configuration.
+# A capture holds only while the kernel's source is unchanged: the entry
+# records the source file's sha256 at capture time, and the benchmark reports
+# null when the file differs now.
+TRAFFIC_CAPTURES = {}
 
 
 def _file_sha256(rel):
@@ -501,38 +612,61 @@ def time_kernels(p, steps, torch, la, flush):
     return {n: sum(t) / len(t) for n, t in zip(names, per)}
 
 
-def time_conv(torch, la, rank, flush, hbm_peak, B=4, H=8, N=4096, d=64, w=4, steps=20):
-    """The short causal convolution (with conv cache) over one q-shaped bf16
-    stream of the headline workload's size, filter width 4: device time per
-    call, L2 flushed before each, and its bytes against HBM."""
-    g = torch.Generator(device="cpu").manual_seed(rank_seed(77, rank))
-    x = (torch.randn((B, H, N, d), generator=g) / 8).to(torch.bfloat16).cuda()
-    wt = (torch.randn((H, d, w), generator=g) / 2).cuda()
-    c0 = torch.randn((B, H, w - 1, d), generator=g).to(torch.bfloat16).cuda()
-    out = torch.empty_like(x)
-    c1 = torch.empty_like(c0)
+def _timed_calls(call, steps, flush, torch):
+    """Median device time (ms) of `call`, L2 flushed before each, 3 warm-ups."""
     stream = torch.cuda.current_stream()
     for _ in range(3):
         flush.fill_(1)
-        la.la_causal_conv(x, wt, c0, out=out, cache_out=c1)
+        call()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in ev:
         flush.fill_(1)
         a.record(stream)
-        la.la_causal_conv(x, wt, c0, out=out, cache_out=c1)
+        call()
         b.record(stream)
     torch.cuda.synchronize()
-    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+
+def time_conv(torch, la, rank, flush, B=4, H=8, N=4096, d=64, w=4, steps=20):
+    """The short causal convolution (with conv cache) over one q-shaped bf16
+    stream of the plain workload's size, filter width 4: device time per
+    call, L2 flushed before each, its bytes against HBM, and end to end."""
+    hbm_peak, _, peak_kind = _measured_peaks()
+    g = torch.Generator(device="cpu").manual_seed(rank_seed(77, rank))
+    xh = (torch.randn((B, H, N, d), generator=g) / 8).to(torch.bfloat16)
+    wt = (torch.randn((H, d, w), generator=g) / 2).cuda()
+    c0h = torch.randn((B, H, w - 1, d), generator=g).to(torch.bfloat16)
+    x, c0 = xh.cuda(), c0h.cuda()
+    out = torch.empty_like(x)
+    c1 = torch.empty_like(c0)
+    ms = _timed_calls(lambda: la.la_causal_conv(x, wt, c0, out=out, cache_out=c1), steps, flush, torch)
     nbytes = 2 * x.numel() * 2 + wt.numel() * 4 + 2 * c0.numel() * 2
-    return {"shape": f"x [B={B},H={H},N={N},d={d}] bf16, w={w}", "ms": ms,
-            "tokens_per_s": B * N / (ms / 1e3), "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
-            "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak}
+    host = {"x": xh.view(torch.int16).pin_memory(), "c": c0h.view(torch.int16).pin_memory()}
+
+    def call(dd):
+        o = torch.empty_like(x)
+        c = torch.empty_like(c0)
+        la.la_causal_conv(dd["x"].view(torch.bfloat16), wt, dd["c"].view(torch.bfloat16), out=o, cache_out=c)
+        return [o, c]
+
+    e_ms, h2d, d2h = time_e2e(host, call, 20, 3, torch)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"short causal conv, x [B={B},H={H},N={N},d={d}] bf16, w={w}, conv cache in and out",
+            "value": B * N / (ms / 1e3), "unit": "tokens/s", "ms": ms,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "traffic": None, "kernel": "causal_conv_kernel", "kernel_ms": ms,
+                         "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": nbytes},
+            "e2e": {"value": B * N / (e_ms / 1e3), "unit": "tokens/s", "ms": e_ms, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches_per_call": 1}
 
 
-def time_varlen(torch, la, rank, flush, hbm_peak, H=8, N=4096, d=64, steps=20):
+def time_varlen(torch, la, rank, flush, H=8, N=4096, d=64, steps=20):
     """A right-padded batch of eight plain bf16 sequences of mixed lengths
-    (head size and padded length of the headline workload) through
+    (head size and padded length of the plain workload) through
     la_prefill_varlen: device time per call, L2 flushed before each."""
+    hbm_peak, _, peak_kind = _measured_peaks()
     g = torch.Generator(device="cpu").manual_seed(rank_seed(91, rank))
     lens = [4096, 3000, 2048, 1500, 1000, 700, 300, 65]
     B = len(lens)
@@ -542,79 +676,67 @@ def time_varlen(torch, la, rank, flush, hbm_peak, H=8, N=4096, d=64, steps=20):
     z = torch.empty((B, H, d), device="cuda")
     ws = torch.empty(max(la.la_prefill_varlen_workspace_bytes(lens, H, d, d), 16), device="cuda",
                      dtype=torch.uint8)
-    stream = torch.cuda.current_stream()
-    call = lambda: la.la_prefill_varlen(q, k, v, lens, out=out, S_out=S, z_out=z, workspace=ws)
-    for _ in range(3):
-        flush.fill_(1)
-        call()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for a, b in ev:
-        flush.fill_(1)
-        a.record(stream)
-        call()
-        b.record(stream)
-    torch.cuda.synchronize()
-    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    ms = _timed_calls(lambda: la.la_prefill_varlen(q, k, v, lens, out=out, S_out=S, z_out=z, workspace=ws),
+                      steps, flush, torch)
     tokens = sum(lens)
     nbytes = tokens * H * 4 * d * 2 + B * H * (d * d + d) * 4
-    return {"shape": f"B={B} H={H} padded N={N} d=dv={d} bf16 plain, lengths {lens}", "ms": ms,
-            "tokens_per_s": tokens / (ms / 1e3), "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
-            "hbm_frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak, "launches": 3 * B}
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"variable-length batch: B={B} H={H} padded N={N} d=dv={d} bf16 plain, lengths {lens}",
+            "value": tokens / (ms / 1e3), "unit": "tokens/s", "ms": ms,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "traffic": None, "kernel": "whole call", "kernel_ms": ms,
+                         "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": nbytes},
+            "gpu_launches_per_call": 3 * B}
 
 
 def run_extra(args, torch, la, rank, flush):
-    """Device-timed numbers for the other workloads (not the headline line)."""
+    """The other workloads, each with its own roofline and end-to-end numbers."""
     res = {}
-    hbm_peak, _, _ = _measured_peaks()
-    for name in ("decay_bf16", "gdelta_bf16", "plain_f32", "gla_bf16"):
+    names = [n for n in ("plain_bf16", "decay_bf16", "gdelta_bf16", "plain_f32", "gla_bf16") if n != args.workload]
+    for name in names:
         spec = inputs.WORKLOADS[name]
         p = inputs.make_workload(name, seed=rank_seed(spec["seed"], rank))
-        u = prefill_units(p)
-        steps = {"plain_f32": 50, "gla_bf16": 3}.get(name, 5)
-        ms = statistics.median(time_prefill(p, steps, 3, torch, la, flush))
-        res[name] = {"tokens_per_s": u["tokens"] / (ms / 1e3), "ms": ms,
-                     "hbm_frac": u["bytes"] / (ms / 1e3) / 1e9 / hbm_peak, "dtype": path_dtype(p)}
+        steps = {"plain_f32": 50, "gla_bf16": 3, "plain_bf16": 20}.get(name, 5)
+        res[name], _ = measure_prefill(name, p, steps, 3, torch, la, flush, e2e_steps=3 if name == "gla_bf16" else 10)
         del p
-    res["conv"] = time_conv(torch, la, rank, flush, hbm_peak)
-    res["varlen_bf16"] = time_varlen(torch, la, rank, flush, hbm_peak)
-    dspec = inputs.WORKLOADS["decode"]
-    dms = time_decode(1000, 20, torch, la, rank_seed(dspec["seed"], rank))
-    du = decode_units(dspec["S"], dspec["H"], dspec["d"], dspec["dv"])
-    res["decode"] = {"state_updates_per_s": du["state_updates"] / (dms / 1e3),
-                     "tokens_per_s": du["tokens"] / (dms / 1e3), "ms_per_step": dms, "chained_steps": 1000,
-                     "hbm_frac": du["bytes"] / (dms / 1e3) / 1e9 / hbm_peak}
+    res["decode"] = measure_decode("decode", torch, la, rank)
+    res["gdelta_decode"] = measure_decode("gdelta_decode", torch, la, rank)
+    res["conv"] = time_conv(torch, la, rank, flush)
+    res["varlen_bf16"] = time_varlen(torch, la, rank, flush)
     return res
 
 
 # ----------------------------------------------------------------------------
 # CPU arm: the float64 oracle
 
-def cpu_baseline(workload: str, budget_s: float = 15.0) -> dict:
+def cpu_baseline(workload: str, budget_s: float = 15.0, max_tokens: int | None = None) -> dict:
     """Time the oracle as it stands on a bounded sample of the workload: whole
-    chains (all N tokens of one (b,h)), as many as fit the budget."""
+    chains (or, with max_tokens, the first max_tokens tokens of each chain),
+    as many as fit the budget; at least one call of as many chains as there
+    are host threads (up to the workload's head count)."""
     import oracle
     spec = inputs.WORKLOADS[workload]
-    p = inputs.make_workload(workload, B=1, H=min(spec["H"], 8))
+    threads = oracle.threads()
+    H = max(1, min(spec["H"], threads))
+    N = spec["N"] if max_tokens is None else min(spec["N"], max_tokens)
+    p = inputs.make_workload(workload, B=1, H=H, N=N)
     chains = 0
     t0 = time.perf_counter()
     elapsed = 0.0
-    threads = oracle.threads()
-    per_call = max(1, min(p.H, threads))
-    while elapsed < budget_s:
-        hs = slice(0, per_call)
+    while elapsed < budget_s or chains == 0:
         if p.mode == "gated_delta":
-            oracle.gated_delta(p.q[:, hs], p.k[:, hs], p.v[:, hs], p.alpha[:, hs], p.g[:, hs])
+            oracle.gated_delta(p.q, p.k, p.v, p.alpha, p.g)
         elif p.mode == "gla":
-            oracle.gla(p.q[:, hs], p.k[:, hs], p.v[:, hs], p.alpha[:, hs])
+            oracle.gla(p.q, p.k, p.v, p.alpha)
         else:
-            oracle.kernelized(p.q[:, hs], p.k[:, hs], p.v[:, hs],
-                              None if p.gamma is None else p.gamma[hs], eps=p.eps)
-        chains += per_call
+            oracle.kernelized(p.q, p.k, p.v, p.gamma, eps=p.eps)
+        chains += H
         elapsed = time.perf_counter() - t0
     token_heads = chains * p.N
     value = token_heads / spec["H"] / elapsed  # tokens/s (a token carries H heads)
+    what = "whole chains" if N == spec["N"] else f"chains cut to their first {N} tokens"
     return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{chains} whole chains of N={p.N} tokens ({token_heads} token-heads) of {workload}, "
+            "sample": f"{chains} {what} of N={p.N} tokens ({token_heads} token-heads) of {workload}, "
                       f"{elapsed:.1f} s"}
 
 
@@ -622,12 +744,14 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     spec = inputs.WORKLOADS[args.workload]
-    per_step = []
+    # each step: one oracle call over as many chains as there are host
+    # threads, cut to a prefix so the whole run stays within minutes
+    prefix = 8192
     for _ in range(args.warmup):
-        cpu_baseline(args.workload, budget_s=args.cpu_seconds / max(1, args.steps + args.warmup))
-    samples = []
+        cpu_baseline(args.workload, budget_s=0.0, max_tokens=prefix)
+    samples, per_step = [], []
     for _ in range(args.steps):
-        cb = cpu_baseline(args.workload, budget_s=args.cpu_seconds / max(1, args.steps))
+        cb = cpu_baseline(args.workload, budget_s=0.0, max_tokens=prefix)
         samples.append(cb)
         per_step.append(spec["B"] * spec["N"] / cb["value"] * 1e3)
     value = statistics.median(s["value"] for s in samples)
@@ -642,14 +766,39 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def main(argv=None):
+# ----------------------------------------------------------------------------
+# entry point and rank launcher
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_entry(rank, n, port, fn, fn_args):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(n), LOCAL_WORLD_SIZE=str(n),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    fn(*fn_args)
+
+
+def spawn_ranks(n: int, fn, fn_args=()) -> None:
+    """Run fn(*fn_args) in n fresh processes, one per GPU, with the torchrun
+    environment (RANK = LOCAL_RANK = r, WORLD_SIZE = n, MASTER_ADDR =
+    127.0.0.1 and a free MASTER_PORT); raises if any rank fails."""
+    import torch.multiprocessing as mp
+    mp.start_processes(_rank_entry, args=(n, _free_port(), fn, tuple(fn_args)), nprocs=n, join=True,
+                       start_method="spawn")
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=HEADLINE, choices=[k for k, v in inputs.WORKLOADS.items()
-                                                              if v["kind"] != "decode"])
+                                                              if not v["kind"].startswith("decode")])
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -661,11 +810,30 @@ def main(argv=None):
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     args.steps = max(1, args.steps)
+    args.gpus = max(1, args.gpus)
+    return args
+
+
+def run_rank(argv):
+    """One rank of the benchmark (rank, world size from the environment)."""
+    args = parse_args(argv)
     world, rank, local = dist_env()
     if args.impl == "reference":
         run_reference(args, world, rank)
         return
     run_gpu(args, world, rank, local)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        # no launcher: start one process per GPU here
+        spawn_ranks(args.gpus, run_rank, (argv if argv is not None else sys.argv[1:],))
+        return
+    if env_world is not None and int(env_world) != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but the launcher started WORLD_SIZE={env_world} ranks")
+    run_rank(argv)
 
 
 if __name__ == "__main__":

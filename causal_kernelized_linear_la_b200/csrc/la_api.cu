@@ -11,6 +11,32 @@ namespace {
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool head_ok(int x) { return x == 64 || x == 128; }
 
+// Byte ranges [a, a + na) and [b, b + nb) share at least one byte.
+bool overlap(const void* a, size_t na, const void* b, size_t nb)
+{
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const char* pa = static_cast<const char*>(a);
+    const char* pb = static_cast<const char*>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+// The final-state outputs of a prefill share no byte with its start state:
+// blocks of one call read S0 / z0 while others write S_out / z_out.
+bool state_outputs_alias(const float* S_out, const float* z_out, const float* S0, const float* z0, int B, int H, int d,
+                         int dv)
+{
+    const size_t chains = (size_t)B * H;
+    const size_t sb = chains * d * dv * sizeof(float), zb = chains * d * sizeof(float);
+    const void* outs[2] = {S_out, z_out};
+    const size_t on[2] = {sb, zb};
+    const void* ins[2] = {S0, z0};
+    const size_t in_n[2] = {sb, zb};
+    for (int i = 0; i < 2; ++i)
+        for (int j = 0; j < 2; ++j)
+            if (overlap(outs[i], on[i], ins[j], in_n[j])) return true;
+    return false;
+}
+
 // Stage events of la_set_stage_events (process-wide; see la.h).
 constexpr int kMaxStageEvents = 8;
 cudaEvent_t g_stage_events[kMaxStageEvents];
@@ -73,7 +99,8 @@ la_status check_prefill(const void* q, const void* k, const void* v, const float
         if (gla && (g || (N > 0 && !gamma_or_alpha))) return LA_ERR_INVALID;
     }
     if (!(cfg->eps >= 0.f)) return LA_ERR_INVALID;
-    if (work && ((cfg->S0 && cfg->S0 == S_out) || (cfg->z0 && cfg->z0 == z_out))) return LA_ERR_INVALID;
+    if (work && state_outputs_alias(S_out, z_out, cfg->S0, no_norm ? nullptr : cfg->z0, B, H, d, dv))
+        return LA_ERR_INVALID;
     const void* ptrs[] = {q, k, v, gamma_or_alpha, g, out, S_out, z_out, cfg->S0, cfg->z0, cfg->workspace};
     for (const void* p : ptrs)
         if (!aligned16(p)) return LA_ERR_ALIGN;
@@ -226,37 +253,22 @@ la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
                              int B, int H, int N, int d, int dv, const la_config* cfg)
 {
     if (!cfg) return LA_ERR_INVALID;
-    if (B < 0 || H < 0 || N < 0) return LA_ERR_INVALID;
-    if (cfg->dtype != LA_F32 && cfg->dtype != LA_BF16) return LA_ERR_INVALID;
-    if (cfg->mode != LA_PLAIN && cfg->mode != LA_DECAY && cfg->mode != LA_GATED_DELTA && cfg->mode != LA_GLA)
-        return LA_ERR_INVALID;
-    if (!la::head_ok(d) || !la::head_ok(dv)) return LA_ERR_UNSUPPORTED;
-    if (!la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return LA_ERR_UNSUPPORTED;
-    const bool work = (long long)B * H > 0;
-    if (work) {
-        if (!S_out || !z_out) return LA_ERR_INVALID;
-        if (N > 0 && (!q || !k || !v || !out)) return LA_ERR_INVALID;
-        if (cfg->mode == LA_PLAIN && (gamma_or_alpha || g)) return LA_ERR_INVALID;
-        if (cfg->mode == LA_DECAY && (!gamma_or_alpha || g)) return LA_ERR_INVALID;
+    la_config c = *cfg;   // cfg->workspace is ignored
+    c.workspace = nullptr;
+    c.workspace_bytes = 0;
+    const la_status st = la::check_prefill(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, &c);
+    if (st != LA_OK) return st;
+    if ((long long)B * H == 0) return LA_OK;
+    const PrefillArgs a = la::prefill_args(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, &c);
+    if (!la::uses_tc_kernelized(c.dtype, c.mode)) {
+        // paths that need no workspace run as la_prefill does; the bf16
+        // gated delta rule's per-chunk operands grow with N and have no
+        // fixed-size form
+        if (la_prefill_workspace_bytes(B, H, N, d, dv, &c) != 0) return LA_ERR_UNSUPPORTED;
+        return la::run_prefill(a);
     }
-    if (!(cfg->eps >= 0.f)) return LA_ERR_INVALID;
-    if (work && ((cfg->S0 && cfg->S0 == S_out) || (cfg->z0 && cfg->z0 == z_out))) return LA_ERR_INVALID;
-    const void* ptrs[] = {q, k, v, gamma_or_alpha, out, S_out, z_out, cfg->S0, cfg->z0};
-    for (const void* p : ptrs)
-        if (!la::aligned16(p)) return LA_ERR_ALIGN;
-    if (!work) return LA_OK;
-    if (N > 0 && la::tc_segments_noalloc(B, H, N, d, dv).G == 0) return LA_ERR_WORKSPACE;
-
-    PrefillArgs a{};
-    a.q = q; a.k = k; a.v = v;
-    a.gamma = cfg->mode == LA_DECAY ? gamma_or_alpha : nullptr;
-    a.out = out; a.S_out = S_out; a.z_out = z_out;
-    a.S0 = cfg->S0; a.z0 = cfg->z0;
-    a.B = B; a.H = H; a.N = N; a.d = d; a.dv = dv;
-    a.ld = N;
-    a.eps = cfg->eps; a.dtype = cfg->dtype; a.mode = cfg->mode;
-    a.stream = static_cast<cudaStream_t>(cfg->stream);
     if (N == 0) return la::write_start_state(a);
+    if (la::tc_segments_noalloc(B, H, N, d, dv).G == 0) return LA_ERR_WORKSPACE;
     return la::from_cuda(la::launch_prefill_tc_kernelized_noalloc(a));
 }
 
@@ -324,14 +336,8 @@ la_status la_causal_conv(const void* x, const float* weight, const void* cache, 
     if (N > 0 && (!x || !weight || !out)) return LA_ERR_INVALID;
     const size_t es = cfg->dtype == LA_BF16 ? 2 : 4;
     const size_t cache_bytes = (size_t)chains * (w - 1) * d * es;
-    auto overlap = [](const void* a, size_t na, const void* b, size_t nb) {
-        if (!a || !b || na == 0 || nb == 0) return false;
-        const char* pa = static_cast<const char*>(a);
-        const char* pb = static_cast<const char*>(b);
-        return pa < pb + nb && pb < pa + na;
-    };
-    if (overlap(cache_out, cache_bytes, cache, cache_bytes) ||
-        overlap(cache_out, cache_bytes, x, (size_t)chains * N * d * es))
+    if (la::overlap(cache_out, cache_bytes, cache, cache_bytes) ||
+        la::overlap(cache_out, cache_bytes, x, (size_t)chains * N * d * es))
         return LA_ERR_INVALID;
     const void* ptrs[] = {x, weight, cache, out, cache_out};
     for (const void* p : ptrs)

@@ -21,11 +21,14 @@ namespace sm100 {
 // la_prefill_check).  Non-zero: which wait gave up first.
 static __device__ unsigned int g_device_error = 0;
 
-// Each try_wait suspends the thread until the phase completes or a hinted
-// time (kSuspendNs) passes; kSpinLimit such waits bound a wait to about a
-// second, far above any legitimate latency.
-constexpr uint32_t kSuspendNs = 100000;
-constexpr uint32_t kSpinLimit = 10000;
+// A bounded wait gives up once kWaitLimitNs of %globaltimer time have passed
+// since it started (far above any legitimate latency).  Each try_wait may
+// suspend the thread for at most the hinted kSuspendNs; the hint only bounds
+// one try, so the deadline, not a count of tries, sets the bound.  kSpinLimit
+// is a backstop on the number of tries in case the timer is not advancing.
+constexpr uint32_t kSuspendNs = 20000;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
+constexpr uint32_t kSpinLimit = 200000000u;
 
 enum WaitSite : unsigned int {
     kErrTmaLoad = 1,
@@ -75,11 +78,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int site)
 {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
     atomicCAS(&g_device_error, 0u, site);
     return false;
 }
@@ -317,18 +331,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// elu(x) + 1 for a pair of values, the exponential of the non-positive part
-// evaluated two at a time by ex2.approx.f16x2: the argument min(x,0)*log2(e)
-// carries an 11-bit mantissa in fp16, finer than the bf16 rounding applied to
-// the result.  Arguments below fp16 range give 0, i.e. phi ~ e^x < 2^-24.
+// elu(x) + 1 for a pair of values: x + 1 above zero, e^x at or below it.
+// The exponential takes the full fp32 argument min(x, 0) (SFU __expf, a
+// relative error of a few fp32 ulps, far below the bf16 rounding applied to
+// the result); large negative x gives e^x -> 0.
 __device__ __forceinline__ float2 phi2_fast(float x0, float x1)
 {
-    constexpr float kLog2e = 1.4426950408889634f;
-    const __half2 a = __floats2half2_rn(fminf(x0, 0.f) * kLog2e, fminf(x1, 0.f) * kLog2e);
-    uint32_t ai = *reinterpret_cast<const uint32_t*>(&a), ei;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(ei) : "r"(ai));
-    const float2 e = __half22float2(*reinterpret_cast<const __half2*>(&ei));
-    return make_float2(fmaxf(x0, 0.f) + e.x, fmaxf(x1, 0.f) + e.y);
+    return make_float2(fmaxf(x0, 0.f) + __expf(fminf(x0, 0.f)), fmaxf(x1, 0.f) + __expf(fminf(x1, 0.f)));
 }
 
 // ---- programmatic dependent launch ---------------------------------------------

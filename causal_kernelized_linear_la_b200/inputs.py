@@ -161,6 +161,7 @@ WORKLOADS = {
     "decode": dict(kind="decode", S=256, H=32, d=128, dv=128, steps=1000, seed=BASE_SEED + 4),
     "gdelta_bf16": dict(kind="gated_delta", B=1, H=32, N=65536, d=128, dv=128, dtype="bf16", seed=BASE_SEED + 5),
     "gla_bf16": dict(kind="gla", B=1, H=32, N=8192, d=128, dv=128, dtype="bf16", seed=BASE_SEED + 6),
+    "gdelta_decode": dict(kind="decode_gated_delta", S=256, H=32, d=128, dv=128, steps=1000, seed=BASE_SEED + 7),
 }
 
 
@@ -216,3 +217,38 @@ def make_decode_token(step: int, Bs=256, H=32, d=128, dv=128, seed=BASE_SEED + 4
     kb, k = bf16_round(_normal(rng, (Bs, H, d), s))
     vb, v = bf16_round(_normal(rng, (Bs, H, dv), s))
     return DecodeToken(q, k, v, qb, kb, vb)
+
+
+@dataclasses.dataclass
+class GatedDeltaDecodeToken:
+    """One gated-delta decode token per (sequence, head): q,k [Bs,H,d],
+    v [Bs,H,dv] in bf16 (k L2-normalised), alpha, g [Bs,H] fp32."""
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    q_bits: np.ndarray
+    k_bits: np.ndarray
+    v_bits: np.ndarray
+    alpha: np.ndarray
+    g: np.ndarray
+
+
+def make_gated_delta_decode_token(step: int, Bs=256, H=32, d=128, dv=128,
+                                  seed=BASE_SEED + 7) -> GatedDeltaDecodeToken:
+    """Token of gated-delta decode step ``step`` from ``default_rng([seed, step])``,
+    drawn like the gated-delta prefill workload's tokens: q, v ~ N(0,1), k ~ N(0,1)
+    L2-normalised in fp32, g = sigmoid(x), alpha = exp(-0.1*softplus(y))."""
+    rng = np.random.default_rng([seed, step])
+    q = _normal(rng, (Bs, H, d))
+    k = _normal(rng, (Bs, H, d))
+    v = _normal(rng, (Bs, H, dv))
+    k /= np.sqrt(np.sum(k.astype(np.float64) ** 2, axis=-1, keepdims=True)).astype(np.float32)
+    x = rng.standard_normal((Bs, H)).astype(np.float64)
+    y = rng.standard_normal((Bs, H)).astype(np.float64)
+    g = (1.0 / (1.0 + np.exp(-x))).astype(np.float32)
+    softplus = np.log1p(np.exp(-np.abs(y))) + np.maximum(y, 0.0)
+    alpha = np.exp(-0.1 * softplus).astype(np.float32)
+    qb, q = bf16_round(q)
+    kb, k = bf16_round(k)
+    vb, v = bf16_round(v)
+    return GatedDeltaDecodeToken(q, k, v, qb, kb, vb, alpha, g)

@@ -106,9 +106,10 @@ typedef struct {
  * LA_GLA applies no feature map and no normaliser either (eps is unused); it
  * runs a token-serial SIMT kernel (one thread per state column) for both
  * dtypes.
- * S_out and z_out must not overlap cfg->S0 and cfg->z0 (blocks of one call
- * read the start state while others write the final state); continue a
- * sequence by alternating two state buffers.  LA_ERR_INVALID if they alias.
+ * S_out and z_out must not share a byte with cfg->S0 or cfg->z0 (blocks of
+ * one call read the start state while others write the final state);
+ * continue a sequence by alternating two state buffers.  LA_ERR_INVALID if
+ * any of these ranges overlap, in whole or in part.
  * Returns LA_OK once the work is enqueued.
  */
 LA_API la_status la_prefill(const void* q, const void* k, const void* v,
@@ -117,23 +118,25 @@ LA_API la_status la_prefill(const void* q, const void* k, const void* v,
                      int B, int H, int N, int d, int dv, const la_config* cfg);
 
 /*
- * la_prefill_noalloc -- the bf16 tensor-core prefill of the kernelized modes
- * (LA_PLAIN, LA_DECAY) for callers that cannot allocate device memory on
- * their launch path: a server that plans all device memory before it starts,
- * a plugin host that offers no workspace, or code that must avoid the device
- * synchronisation an allocation may cause.  The pages have no counterpart;
- * this is a service of this library.
+ * la_prefill_noalloc -- la_prefill for callers that cannot allocate device
+ * memory on their launch path: a server that plans all device memory before
+ * it starts, a plugin host that offers no workspace, or code that must avoid
+ * the device synchronisation an allocation may cause.  The pages have no
+ * counterpart; this is a service of this library.
  *
  * Arguments, layouts and results are those of la_prefill; cfg->workspace is
- * ignored.  Instead of a caller workspace the call uses a fixed 16 MiB array
- * of device memory inside the library, which every GPU that loads the
- * library holds until the process exits.  The segment summaries of one call
- * must fit in it: (B*H) * ceil(N / L) * (d*dv + d) * 4 bytes for a segment
- * length L the call picks (at least 64); a problem that does not fit even
- * with one segment per chain, i.e. B*H*(d*dv + d)*4 > 16 MiB, is rejected with
- * LA_ERR_WORKSPACE before anything is launched.  Only cfg->dtype == LA_BF16
- * with LA_PLAIN or LA_DECAY is served (LA_ERR_UNSUPPORTED otherwise; the
- * f32 paths need no workspace, and the gated delta rule's grows with N).
+ * ignored.  The bf16 tensor-core prefill of the kernelized modes (LA_PLAIN,
+ * LA_DECAY) keeps its segment summaries in a fixed 16 MiB array of device
+ * memory inside the library instead of a caller workspace; every GPU that
+ * loads the library holds that array until the process exits.  The
+ * summaries of one call must fit in it: (B*H) * ceil(N / L) * (d*dv + d) * 4
+ * bytes for a segment length L the call picks (a multiple of 64, at least
+ * 128; the call lengthens segments until the summaries fit).  A problem that
+ * does not fit even with one segment per chain, i.e. B*H*(d*dv + d)*4 >
+ * 16 MiB, is rejected with LA_ERR_WORKSPACE before anything is launched.
+ * Configurations whose la_prefill needs no workspace (fp32 inputs in every
+ * mode, LA_GLA) run exactly as la_prefill does.  bf16 LA_GATED_DELTA, whose
+ * workspace grows with N, returns LA_ERR_UNSUPPORTED.
  *
  * All calls in one process share the array and it keeps the last call's
  * contents: calls whose work can overlap on the GPU (enqueued on different

@@ -72,6 +72,11 @@ def test_prefill_validation():
     assert _prefill(_cfg(mode=0), ga=FAKE) == la.LA_ERR_INVALID         # plain takes no gamma
     assert _prefill(_cfg(eps=-1.0)) == la.LA_ERR_INVALID
     assert _prefill(_cfg(S0=FAKE), S=FAKE) == la.LA_ERR_INVALID          # output aliases start state
+    # partial overlaps are rejected too (S0 spans 64*64*4 bytes from FAKE)
+    assert _prefill(_cfg(S0=FAKE), S=FAKE + 4096) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(S0=FAKE), S=FAKE - 4096) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(S0=FAKE), S=FAKE + (1 << 20), z=FAKE + 256) == la.LA_ERR_INVALID
+    assert _prefill(_cfg(z0=FAKE + 16384 - 16), S=FAKE) == la.LA_ERR_INVALID
     # nothing to do: valid and launches nothing
     assert _prefill(_cfg(), B=0) == la.LA_OK
     assert _prefill(_cfg(), H=0, q=0, k=0, v=0, out=0, S=0, z=0) == la.LA_OK

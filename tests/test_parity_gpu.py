@@ -62,6 +62,13 @@ def test_gated_delta_bf16_heads(d, dv):
     _check(inputs.make_gated_delta(2, 2, 333, d, dv, dtype="bf16", seed=600 + d + dv))
 
 
+@pytest.mark.parametrize("mode", ["plain", "decay"])
+def test_kernelized_bf16_large_inputs(mode):
+    """q, k ~ 4 N(0,1): phi's exponential branch sees arguments down to about
+    -16, where e^x spans seven decades; every element against the oracle."""
+    _check(inputs.make_kernelized(1, 4, 700, 128, 128, dtype="bf16", mode=mode, scale=4.0, seed=1100))
+
+
 def test_gated_delta_f32_small():
     _check(inputs.make_gated_delta(1, 2, 190, 64, 64, dtype="f32", seed=700))
 

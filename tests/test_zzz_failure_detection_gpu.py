@@ -5,7 +5,8 @@ runs out is reported to the host, and the context stays usable.
 
 la_selftest_wait_timeout enqueues one kernel whose mbarrier wait has nothing
 to wait for; the wait gives up after its bound (about a second), records the
-timeout in the device error word and returns.  No copy or MMA is in flight,
+timeout in the device error word and returns.  The bound is a deadline
+of 1 s on the device's global timer.  No copy or MMA is in flight,
 nothing traps, nothing hangs.
 """
 import time
@@ -29,7 +30,10 @@ def test_bounded_wait_runs_out_and_is_reported():
         with pytest.raises(la.LaError) as ei:
             la.la_prefill_check()
         assert ei.value.code == la.LA_ERR_TIMEOUT
-        assert time.perf_counter() - t0 < 30.0, "the wait is bounded"
+        elapsed = time.perf_counter() - t0
+        # the wait gives up at a 1 s deadline of the device's global timer,
+        # not after a count of suspended tries whose length is only a hint
+        assert 0.5 <= elapsed < 5.0, f"wait gave up after {elapsed:.3f} s"
         la.la_prefill_check()   # reading the error cleared it
     finally:
         # never leave the error word set for later tests
