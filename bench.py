@@ -533,14 +533,20 @@ def path_dtype(p) -> str:
 
 def call_kernels(p) -> list:
     """The kernels one la_prefill call launches for this workload, in launch
-    order (the dispatch documented with la_set_stage_events in include/la.h)."""
+    order (the dispatch documented with la_set_stage_events in include/la.h;
+    the library reports how many)."""
+    import causal_kernelized_linear_la_b200 as la
+    n = la.la_prefill_kernel_count(p.B, p.H, p.N, p.d, p.dv, p.dtype, p.mode)
     if p.mode == "gla":
-        return ["gla_token_simt"]
-    if p.dtype == "bf16" and p.mode in ("plain", "decay"):
-        return ["summary_kernel", "scan_kernel", "chunk_kernel"]
-    if p.dtype == "bf16":
-        return ["gd_prep_kernel", "gd_chain_kernel"]
-    return ["gated_delta_token_simt" if p.mode == "gated_delta" else "kernelized_chunk_simt"]
+        names = ["gla_token_simt"]
+    elif p.dtype == "bf16" and p.mode in ("plain", "decay"):
+        names = ["summary_kernel", "scan_kernel", "chunk_kernel"]
+    elif p.dtype == "bf16":
+        names = ["gd_prep_kernel", "gd_chain_kernel"] * (n // 2)   # one pair per part of the sequence
+    else:
+        names = ["gated_delta_token_simt" if p.mode == "gated_delta" else "kernelized_chunk_simt"]
+    assert len(names) == n, (names, n)
+    return names
 
 
 def la_launches_per_step(p) -> int:
@@ -609,7 +615,13 @@ def time_kernels(p, steps, torch, la, flush):
             per[j].append(prev.elapsed_time(m))
             prev = m
     la.la_prefill_check(ws)
-    return {n: sum(t) / len(t) for n, t in zip(names, per)}
+    # kernels launched more than once per call (one per part of the sequence)
+    # are summed: the gaps between consecutive events are each kernel's share
+    # of the call
+    res = {}
+    for n, t in zip(names, per):
+        res[n] = res.get(n, 0.0) + sum(t) / len(t)
+    return res
 
 
 def _timed_calls(call, steps, flush, torch):

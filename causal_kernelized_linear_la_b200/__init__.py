@@ -16,7 +16,8 @@ Entry points (same names as the C ABI):
   right-padded batch of sequences of different lengths
 * ``la_decode_step(q, k, v, S, z, eps=...)`` -> ``o``; S and z updated in place
 * ``la_gated_delta_decode_step(q, k, v, alpha, g, S)`` -> ``o``; S updated in place
-* ``la_prefill_workspace_bytes(...)``, ``la_prefill_varlen_workspace_bytes(...)``,
+* ``la_prefill_workspace_bytes(...)``, ``la_prefill_kernel_count(...)``,
+  ``la_prefill_varlen_workspace_bytes(...)``,
   ``la_status_string(code)``, ``lib()``
 """
 from __future__ import annotations
@@ -32,7 +33,8 @@ LA_F32, LA_BF16 = 0, 1
 MODES = {"plain": 0, "decay": 1, "gated_delta": 2, "gla": 3}
 
 # Symbols the library exports; the header include/la.h declares exactly these.
-EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_prefill_varlen",
+EXPORTS = ("la_prefill", "la_prefill_noalloc", "la_prefill_workspace_bytes", "la_prefill_kernel_count",
+           "la_prefill_varlen",
            "la_prefill_varlen_workspace_bytes", "la_decode_step", "la_gated_delta_decode_step",
            "la_set_stage_events", "la_causal_conv", "la_selftest_wait_timeout",
            "la_prefill_check", "la_status_string", "la_version")
@@ -68,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.la_prefill_noalloc.restype = i
         L.la_prefill_workspace_bytes.argtypes = [i] * 5 + [cfgp]
         L.la_prefill_workspace_bytes.restype = ctypes.c_size_t
+        L.la_prefill_kernel_count.argtypes = [i] * 5 + [cfgp]
+        L.la_prefill_kernel_count.restype = i
         ip = ctypes.POINTER(ctypes.c_int)
         L.la_prefill_varlen.argtypes = [vp] * 8 + [ip] + [i] * 5 + [cfgp]
         L.la_prefill_varlen.restype = i
@@ -134,6 +138,12 @@ def _stream_handle(stream=None):
 def la_prefill_workspace_bytes(B, H, N, d, dv, dtype="bf16", mode="plain") -> int:
     cfg = LaConfig(LA_BF16 if dtype == "bf16" else LA_F32, MODES[mode], 0.0, None, None, None, None, 0)
     return int(lib().la_prefill_workspace_bytes(B, H, N, d, dv, ctypes.byref(cfg)))
+
+
+def la_prefill_kernel_count(B, H, N, d, dv, dtype="bf16", mode="plain") -> int:
+    """Kernels one la_prefill call with these sizes launches (host-only)."""
+    cfg = LaConfig(LA_BF16 if dtype == "bf16" else LA_F32, MODES[mode], 0.0, None, None, None, None, 0)
+    return int(lib().la_prefill_kernel_count(B, H, N, d, dv, ctypes.byref(cfg)))
 
 
 def la_prefill(q, k, v, mode="plain", gamma=None, alpha=None, g=None, S0=None, z0=None, eps=1e-6,

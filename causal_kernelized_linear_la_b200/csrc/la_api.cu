@@ -176,6 +176,14 @@ size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_c
     return 0;
 }
 
+int la_prefill_kernel_count(int B, int H, int N, int d, int dv, const la_config* cfg)
+{
+    if (!cfg || B <= 0 || H <= 0 || N <= 0 || !la::head_ok(d) || !la::head_ok(dv)) return 0;
+    if (la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return 3;
+    if (cfg->dtype == LA_BF16 && cfg->mode == LA_GATED_DELTA) return 2 * la::gd_parts(B, H, N, d, dv).P;
+    return 1;
+}
+
 la_status la_prefill(const void* q, const void* k, const void* v,
                      const float* gamma_or_alpha, const float* g,
                      void* out, float* S_out, float* z_out,

@@ -126,10 +126,9 @@ struct PrepPlan {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_qb,
-               const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_t,
+               const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_t,
                const __grid_constant__ CUtensorMap tm_p, const float* __restrict__ alpha,
-               const float* __restrict__ gate, int N, int chains, int ld)
+               const float* __restrict__ gate, float* __restrict__ vec, int N, int chains, int ld)
 {
     using P = PrepPlan<D>;
     constexpr int NB = P::NB;
@@ -149,7 +148,6 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float* avec = Lv + 3 * C;   // [2][2][C]: alpha, g of two work items
     float* ef = Lv + 7 * C;     // e^{L_t - L_m}, m the chunk's middle token
     float* eg = Lv + 8 * C;     // e^{L_m - L_t}
-    float* kr = Lv + 9 * C;     // b_C / b_t
     int* factored = reinterpret_cast<int*>(Lv + 10 * C);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* bar1 = full + 1;
@@ -250,13 +248,15 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
                 hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
             }
-            kr[2 * lane] = __expf(Lc - La);
-            kr[2 * lane + 1] = __expf(Lc - Lb);
             ef[2 * lane] = __expf(La - Lm);
             ef[2 * lane + 1] = __expf(Lb - Lm);
             eg[2 * lane] = __expf(Lm - La);
             eg[2 * lane + 1] = __expf(Lm - Lb);
             if (lane == 0) *factored = (hi - Lm <= 80.f && Lm - lo <= 80.f) ? 1 : 0;
+            // the chain pass's per-token factors: b_t, then b_C / b_t
+            float* vg = vec + (size_t)item * 2 * C;
+            reinterpret_cast<float2*>(vg)[lane] = make_float2(__expf(La), __expf(Lb));
+            reinterpret_cast<float2*>(vg + C)[lane] = make_float2(__expf(Lc - La), __expf(Lc - Lb));
             __syncwarp();
             if (next < items) stage_vectors(next, (it + 1) & 1);
         }
@@ -269,7 +269,6 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             unpack8(reinterpret_cast<const uint4*>(sm + (2 * b) * TILE)[rem], f);
             reinterpret_cast<uint4*>(kbt + b * TILE)[rem] = pack8(f, bv[row]);
         }
-        __syncthreads();   // raw K is rewritten in place below
 
         // score blocks -> A (fp32, strictly lower, gated and decayed) and P~ (bf16)
         if (!mbar_wait(bar1, ph, kErrMma)) bad = true;
@@ -322,43 +321,12 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     *reinterpret_cast<uint4*>(ptile + sw128_offset(i, wg * 64 + q * 16)) =
                         make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
             }
-            // diag(b) Q and diag(b_C / b) K in place (M1, their reader, is complete;
-            // Kb is built): the four threads that own row rq = r % 64 (both row
-            // halves, both column halves) take a quarter of its 16-byte chunks each.
-            // A row takes one factor, so any chunk order works: rotating it by the
-            // row keeps a warp's 32 rows on distinct banks.  Loads go first.
-            const int rq = r & 63, slot = (r >> 6) * 2 + wg;
-            const float bq = bv[rq], kq = kr[rq];
-            constexpr int PER = NB * 2;
-            uint4 xq[PER], xk[PER];
-#pragma unroll
-            for (int n = 0; n < PER; ++n) {
-                const int q = slot + 4 * n, chunk = ((q & 7) + rq) & 7;
-                const int off = rq * 128 + chunk * 16;
-                xq[n] = *reinterpret_cast<const uint4*>(sm + (2 * (q / 8) + 1) * TILE + off);
-                xk[n] = *reinterpret_cast<const uint4*>(sm + (2 * (q / 8)) * TILE + off);
-            }
-#pragma unroll
-            for (int n = 0; n < PER; ++n) {
-                const int q = slot + 4 * n, chunk = ((q & 7) + rq) & 7;
-                const int off = rq * 128 + chunk * 16;
-                float f[8];
-                unpack8(xq[n], f);
-                *reinterpret_cast<uint4*>(sm + (2 * (q / 8) + 1) * TILE + off) = pack8(f, bq);
-                unpack8(xk[n], f);
-                *reinterpret_cast<uint4*>(sm + (2 * (q / 8)) * TILE + off) = pack8(f, kq);
-            }
         }
         fence_async_smem();
         tc_fence_before();
         if (__syncthreads_or(bad)) { bad = true; break; }
-        if (tid == 0) {
-            for (int b = 0; b < NB; ++b) {
-                tma_store_3d(&tm_qb, sm + (2 * b + 1) * TILE, b * 64, c * C, chain);
-                tma_store_3d(&tm_kt, sm + (2 * b) * TILE, b * 64, c * C, chain);
-            }
-            tma_store_commit();
-        }
+        // M1 has read the K / Q tiles and Kb is built: they take the next item
+        if (tid == 0 && next < items) issue(next);
 
         // T = (I + A)^{-1}: diagonal 16 x 16 blocks (one thread per column) ...
         constexpr int TSt = P::TS;
@@ -417,11 +385,6 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 __syncthreads();
             }
-        }
-        // the diag(b) Q and K~ stores have long read their tiles: K/Q take the next item
-        if (tid == 0 && next < items) {
-            tma_store_wait_read();
-            issue(next);
         }
         // T' = T diag(g), bf16, K-major A operand of M2 (T is unit lower triangular)
         for (int e = tid; e < C * 8; e += kThreads) {
@@ -518,39 +481,50 @@ template <int D>
 struct ChainPlan {
     static constexpr int STAGES = 2;
     static constexpr int NB = D / 64;
-    // stage: K~[NB] | -W_0 Qb_0 -W_1 Qb_1 ... | T' Z P~ | V   (Z: a zero tile, never loaded)
-    // [-W_b; Qb_b], [T'; Z] and [Z; P~] are M = 128 K-major A operands.
+    // stage: K[NB] | -W_0 Q_0 -W_1 Q_1 ... | T' Z P~ | V | b[C] r[C]  (Z: a zero tile,
+    // never loaded; b_t = e^{L_t}, r_t = b_C / b_t from the prep pass)
+    // [-W_b; Q_b], [T'; Z] and [Z; P~] are M = 128 K-major A operands.
     static constexpr int O_K = 0, O_WQ = NB * TILE, O_T = 3 * NB * TILE;
     static constexpr int O_Z = O_T + TILE, O_P = O_Z + TILE, O_V = O_P + TILE;
-    static constexpr int STAGE = O_V + TILE;
-    static constexpr int LOAD_BYTES = STAGE - TILE;         // all but Z arrives by TMA
-    static constexpr int OFF_SB = STAGES * STAGE;           // S bf16 [D][64], MN-major B operand
-    static constexpr int OFF_U = OFF_SB + NB * TILE;        // U bf16 [C][64], MN-major B operand
-    static constexpr int OFF_O = OFF_U + TILE;              // output staging
-    static constexpr int OFF_VEC = OFF_O + TILE;            // staged alpha [2][C], b_C [3]
-    static constexpr int OFF_BAR = OFF_VEC + 2 * C * 4 + 16;
+    static constexpr int O_VEC = O_V + TILE;
+    static constexpr int VEC_BYTES = 2 * C * 4;
+    static constexpr int STAGE = O_VEC + 1024;                // stages stay 1024-byte aligned
+    static constexpr int LOAD_BYTES = (3 * NB + 3) * TILE + VEC_BYTES;
+    static constexpr int OFF_SB = STAGES * STAGE;             // S bf16 [D][64], MN-major B operand
+    static constexpr int OFF_U = OFF_SB + NB * TILE;          // U bf16 [C][64] (B of P~ U)
+    static constexpr int OFF_UH = OFF_U + TILE;               // diag(b_C / b) U bf16 (B of K^T U)
+    static constexpr int OFF_O = OFF_UH + TILE;               // output staging
+    static constexpr int OFF_BAR = OFF_O + TILE;
     // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready s_ready ostage_full ostage_empty
     // drain[2]
     static constexpr int NBAR = 17;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
-    // TMEM columns: the two issuers' partial [U; O] accumulators (two buffers each)
-    // and partial states; U, O and S are the sums of the pairs.
-    static constexpr uint32_t T_X1 = 0, T_X2 = 128, T_S1 = 256, T_S2 = 320, T_COLS = 512;
-    static constexpr int KS_HALF = D / 32;                   // K-steps of (-W) S per issuer
+    // TMEM columns: the two issuers' partial [U; Q S] accumulators X1, X2 and the
+    // P~ U accumulator X3 (two buffers each), and the two partial state updates
+    static constexpr uint32_t T_X1 = 0, T_X2 = 128, T_X3 = 256, T_S1 = 384, T_S2 = 448, T_COLS = 512;
+    static constexpr int KS_HALF = D / 32;                   // K-steps of [-W; Q] S per issuer
 };
 
 constexpr int kConv = 256;                   // converter threads (warps 0-7)
 constexpr int kChainThreads = kConv + 96;    // + issuer warps 8 and 10, TMA warp 9
 
+// The chain of one (chain, 64 value columns).  Per chunk c with start state S:
+//   issuers   X1 = [T'; 0] V (one chunk ahead) + [-W; Q]_1 S_1,  X2 = [-W; Q]_2 S_2
+//             (feature halves), so rows 0-63 of X1 + X2 are U and rows 64-127 are Q S;
+//             after U is in place: S1 = K_1^T U^, S2 = K_2^T U^ (token halves),
+//             U^ = diag(b_C / b) U; then X3 = [0; P~] U.
+//   converters  U, U^ to bf16;  S <- b_C S + S1 + S2 (fp32, held in registers), its
+//             bf16 copy for the next chunk;  o = diag(b) Q S + P~ U -> staging.
+// The converters signal with one arrival per warp.
 template <int D>
 __global__ void __launch_bounds__(kChainThreads, 1)
-gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant__ CUtensorMap tm_k,
+gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                 const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_p,
-                const __grid_constant__ CUtensorMap tm_o, const float* __restrict__ alpha,
-                const float* __restrict__ S0, float* __restrict__ S_out, int N, int dv, int ld)
+                const __grid_constant__ CUtensorMap tm_o, const float* __restrict__ vec,
+                const float* __restrict__ S0, float* __restrict__ S_out, int N, int dv)
 {
     using P = ChainPlan<D>;
     constexpr int NB = P::NB;
@@ -559,19 +533,18 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
     unsigned char* sm = align1024(smem_raw);
     unsigned char* sbt = sm + P::OFF_SB;
     unsigned char* utile = sm + P::OFF_U;
+    unsigned char* uhat = sm + P::OFF_UH;
     unsigned char* ostage = sm + P::OFF_O;
-    float* abuf = reinterpret_cast<float*>(sm + P::OFF_VEC);   // [2][C] staged alpha
-    float* vb_c = abuf + 2 * C;                                // [3] b_C
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
-    uint64_t* full = bars;          // TMA -> issuers, per stage
+    uint64_t* full = bars;          // TMA -> everyone, per stage
     uint64_t* empty = bars + 2;     // both issuers (commit) -> TMA, per stage
-    uint64_t* uo_full = bars + 4;   // both issuers: [U; Qb S] partials complete, per TMEM buffer
-    uint64_t* o_full = bars + 6;    // issuer B: output partial complete, per TMEM buffer
-    uint64_t* o_read = bars + 8;    // converters: output partials read, per TMEM buffer
+    uint64_t* uo_full = bars + 4;   // both issuers: [U; Q S] partials complete, per TMEM buffer
+    uint64_t* o_full = bars + 6;    // issuer B: P~ U complete, per TMEM buffer
+    uint64_t* o_read = bars + 8;    // output warps: the buffer's output rows read
     uint64_t* s_full = bars + 10;   // both issuers: state update partials complete
-    uint64_t* u_ready = bars + 11;  // converters: U in place, state rescaled
-    uint64_t* s_ready = bars + 12;  // converters: bf16 state written
-    uint64_t* os_full = bars + 13;  // converters: output staging written
+    uint64_t* u_ready = bars + 11;  // U warps: U and U^ in place
+    uint64_t* s_ready = bars + 12;  // every converter warp: bf16 state written
+    uint64_t* os_full = bars + 13;  // output warps: output staging written
     uint64_t* os_empty = bars + 14; // TMA: output staging read by its store
     uint64_t* drain = bars + 15;    // [2] issuers: every MMA each issued is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
@@ -588,13 +561,13 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
             mbar_init(&empty[s], 2);
             mbar_init(&uo_full[s], 2);
             mbar_init(&o_full[s], 1);
-            mbar_init(&o_read[s], 128);
+            mbar_init(&o_read[s], 4);
             mbar_init(&drain[s], 1);
         }
         mbar_init(s_full, 2);
-        mbar_init(u_ready, kConv);
-        mbar_init(s_ready, kConv);
-        mbar_init(os_full, 128);
+        mbar_init(u_ready, 4);
+        mbar_init(s_ready, 8);
+        mbar_init(os_full, 4);
         mbar_init(os_empty, 1);
         fence_mbar_init();
     }
@@ -615,6 +588,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
         if (lane == 0) {
             const uint64_t pol_once = policy_evict_first();
             const uint64_t pol_shared = ntile > 1 ? policy_evict_normal() : policy_evict_first();
+            const float* vchain = vec + (size_t)chain * nch * 2 * C;
             int loads = 0;
             auto issue = [&](int c) {
                 const int s = c % P::STAGES;
@@ -624,11 +598,12 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
                 for (int b = 0; b < NB; ++b) {
                     tma_load_3d(st + P::O_K + b * TILE, &tm_k, b * 64, y, chain, &full[s], pol_shared);
                     tma_load_3d(st + P::O_WQ + (2 * b) * TILE, &tm_w, b * 64, y, chain, &full[s], pol_shared);
-                    tma_load_3d(st + P::O_WQ + (2 * b + 1) * TILE, &tm_qb, b * 64, y, chain, &full[s], pol_shared);
+                    tma_load_3d(st + P::O_WQ + (2 * b + 1) * TILE, &tm_q, b * 64, y, chain, &full[s], pol_shared);
                 }
                 tma_load_3d(st + P::O_T, &tm_t, 0, y, chain, &full[s], pol_shared);
                 tma_load_3d(st + P::O_P, &tm_p, 0, y, chain, &full[s], pol_shared);
                 tma_load_3d(st + P::O_V, &tm_v, j0, y, chain, &full[s], pol_once);
+                bulk_load(st + P::O_VEC, vchain + (size_t)c * 2 * C, P::VEC_BYTES, &full[s]);
                 loads = c + 1;
             };
             // two stages give a load about one chunk of lead time; pulling the
@@ -638,7 +613,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
                 for (int b = 0; b < NB; ++b) {
                     tma_prefetch_3d(&tm_k, b * 64, y, chain);
                     tma_prefetch_3d(&tm_w, b * 64, y, chain);
-                    tma_prefetch_3d(&tm_qb, b * 64, y, chain);
+                    tma_prefetch_3d(&tm_q, b * 64, y, chain);
                 }
                 tma_prefetch_3d(&tm_t, 0, y, chain);
                 tma_prefetch_3d(&tm_p, 0, y, chain);
@@ -674,17 +649,13 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
         __syncwarp();
     } else if (warp == 8 || warp == 10) {
         // ---------------- MMA issuers ----------------
-        // Issuer A (warp 8): X1 = [T'; 0] V (one chunk ahead), X1 += [-W; Qb] S over
-        // the first half of the features, S1 += K~^T U over the first 32 tokens.
-        // Issuer B (warp 10): X2 = [-W; Qb] S over the second half, S2 = K~^T U
-        // over the last 32 tokens, X2 += [0; P~] U.  U = X1 + X2 (rows 0-63),
-        // O = X1 + X2 (rows 64-127), S = S1 + S2.
         if (lane == 0) {
             const bool A = warp == 8;
             const uint32_t id = idesc_bf16_f32(128, 64, 0, 1);
             const uint32_t ids = idesc_bf16_f32(D, 64, 1, 1);
             const uint64_t ds = sdesc_sw128(smem_u32(sbt), TILE, 1024);
             const uint64_t du = sdesc_sw128(smem_u32(utile), TILE, 1024);
+            const uint64_t duh = sdesc_sw128(smem_u32(uhat), TILE, 1024);
             const uint32_t tx = tbase + (A ? P::T_X1 : P::T_X2);
             const uint32_t tsp = tbase + (A ? P::T_S1 : P::T_S2);
             auto ready = [&](int c) {   // stage c loaded and TMEM buffer c & 1 read out
@@ -728,7 +699,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const int ks = t0 + kk;
-                    mma_bf16(tsp, dk + ((ks * 2048) >> 4), du + ((ks * 2048) >> 4), ids, (A || kk > 0) ? 1u : 0u);
+                    mma_bf16(tsp, dk + ((ks * 2048) >> 4), duh + ((ks * 2048) >> 4), ids, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full);
                 if (A) {
@@ -736,9 +707,10 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
                     if (c + 1 < nch) ok = m0(c + 1);
                 } else {
                     const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
+                    const uint32_t t3 = tbase + P::T_X3 + cp * 64;
 #pragma unroll
                     for (int ks = 0; ks < C / 16; ++ks)
-                        mma_bf16(txc, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, 1u);
+                        mma_bf16(t3, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, ks > 0 ? 1u : 0u);
                     mma_commit(&o_full[cp]);
                     mma_commit(&empty[s]);
                 }
@@ -750,159 +722,128 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_qb, const __grid_constant
         __syncwarp();
     } else {
         // ---------------- converters (warps 0-7) ----------------
-        const float* al = alpha + (size_t)chain * ld;
-        // warp 1: alpha of chunk c into staging buffer c & 1
-        auto stage_alpha = [&](int c) {
-            float* dst = abuf + (c & 1) * C;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int j = 2 * lane + h, t = c * C + j;
-                const bool ok = t < N;
-                cp_async4(dst + j, ok ? al + t : al, ok ? 4u : 0u);
-            }
-            cp_async_commit();
-        };
-        // warp 1: b_C of chunk c into vector buffer c % 3
-        auto chunk_vectors = [&](int c) {
-            cp_async_wait_all();
-            const float* a = abuf + (c & 1) * C;
-            const int t = c * C + 2 * lane;
-            float La, Lb, Lc;
-            chunk_logdecay(a[2 * lane], a[2 * lane + 1], t < N, t + 1 < N, lane, La, Lb, Lc);
-            if (lane == 0) vb_c[c % 3] = __expf(Lc);
-            __syncwarp();
-        };
+        // Thread (quad, lane) owns row r = 32 quad + lane of the M = 128
+        // accumulators, a token of U (quads 0, 1) or of the output (quads 2, 3),
+        // and row f of the M = D state accumulators (f = r for D = 128); warpgroup
+        // wg owns 32 of the tile's 64 value columns.
+        const int r = quad * 32 + lane;
+        const int f = acc_row<D>(quad, lane);   // state row (feature) of this thread, or -1
         bool bad = false;
-        // 32 columns of accumulator rows of this warp's quadrant: X1 + X2
-        auto ld_sum = [&](uint32_t col, float (&v)[32]) {
-            float w[32];
-            tmem_ld16(tmem_addr(tbase, quad, P::T_X1 + col), *reinterpret_cast<float(*)[16]>(v));
-            tmem_ld16(tmem_addr(tbase, quad, P::T_X1 + col + 16), *reinterpret_cast<float(*)[16]>(v + 16));
-            tmem_ld16(tmem_addr(tbase, quad, P::T_X2 + col), *reinterpret_cast<float(*)[16]>(w));
-            tmem_ld16(tmem_addr(tbase, quad, P::T_X2 + col + 16), *reinterpret_cast<float(*)[16]>(w + 16));
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] += w[x];
+        auto ld32 = [&](uint32_t col, float (&v)[32]) {
+            tmem_ld16(tmem_addr(tbase, quad, col), *reinterpret_cast<float(*)[16]>(v));
+            tmem_ld16(tmem_addr(tbase, quad, col + 16), *reinterpret_cast<float(*)[16]>(v + 16));
         };
-        // output rows of chunk cc (accumulator rows 64-127, quadrants 2 and 3) -> staging
-        auto output_tile = [&](int cc) {
-            if (quad < 2) return;
+        auto store_row = [&](unsigned char* tile, int row, const float (&v)[32], float w) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(tile + sw128_offset(row, wg * 64 + q * 16)) =
+                    make_uint4(pack_bf16x2(w * v[8 * q], w * v[8 * q + 1]), pack_bf16x2(w * v[8 * q + 2], w * v[8 * q + 3]),
+                               pack_bf16x2(w * v[8 * q + 4], w * v[8 * q + 5]),
+                               pack_bf16x2(w * v[8 * q + 6], w * v[8 * q + 7]));
+        };
+        // per-chunk factors of this thread, read from the stage before this warp's
+        // arrival that lets the stage be refilled: b_C, and b_t (output rows) or
+        // b_C / b_t (U rows) of token r % 64
+        float bc = 1.f, tokf = 1.f, tokf_prev = 1.f;
+        auto read_factors = [&](int c) {
+            if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) bad = true;
+            const float* vv = reinterpret_cast<const float*>(sm + (c % P::STAGES) * P::STAGE + P::O_VEC);
+            bc = vv[C - 1];
+            tokf = quad < 2 ? vv[C + r] : vv[r - 64];
+        };
+        // output rows of chunk cc (accumulator rows 64-127) -> staging
+        auto output_tile = [&](int cc, float bt) {
             if (!mbar_wait(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
             if (cc >= 1 && !mbar_wait(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
             tc_fence_after();
-            const int i = quad * 32 + lane - 64;
-            float o[32];
-            ld_sum((cc & 1) * 64 + wg * 32, o);
-            tc_fence_before();
-            mbar_arrive(&o_read[cc & 1]);
+            float o[32], w[32];
+            const uint32_t col = (cc & 1) * 64 + wg * 32;
+            ld32(P::T_X1 + col, o);
+            ld32(P::T_X2 + col, w);
+            tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4*>(ostage + sw128_offset(i, wg * 64 + q * 16)) =
-                    make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
-                               pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+            for (int x = 0; x < 32; ++x) o[x] += w[x];
+            ld32(P::T_X3 + col, w);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_read[cc & 1]);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = fmaf(bt, o[x], w[x]);
+            store_row(ostage, r - 64, o, 1.f);
             fence_async_smem();
-            mbar_arrive(os_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(os_full);
         };
 
-        if (warp == 1) {
-            stage_alpha(0);
-            chunk_vectors(0);
-            if (nch > 1) stage_alpha(1);
-        }
-        named_bar(1, kConv);
-        // start state slice S[:, j0:j0+64]: bf16 copy for the first read, b_C-scaled fp32 in S1
+        // start state slice S[:, j0:j0+64] in registers and, as bf16, in the B operand
+        float sreg[32];
         {
-            const int f = acc_row<D>(quad, lane);
-            const float bc = vb_c[0];
-            float v[32];
+            const float* src = (S0 && f >= 0) ? S0 + ((size_t)chain * D + f) * dv + j0 + wg * 32 : nullptr;
 #pragma unroll
-            for (int x = 0; x < 32; ++x)
-                v[x] = (f >= 0 && S0) ? S0[((size_t)chain * D + f) * dv + j0 + wg * 32 + x] : 0.f;
-            if (f >= 0) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4*>(sbt + sw128_offset(f, wg * 64 + q * 16)) =
-                        make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+            for (int q = 0; q < 8; ++q) {
+                const float4 t = src ? reinterpret_cast<const float4*>(src)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+                sreg[4 * q] = t.x; sreg[4 * q + 1] = t.y; sreg[4 * q + 2] = t.z; sreg[4 * q + 3] = t.w;
             }
+            if (f >= 0) store_row(sbt, f, sreg, 1.f);
+            read_factors(0);
             fence_async_smem();
-            mbar_arrive(s_ready);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] *= bc;
-            tmem_st16(tmem_addr(tbase, quad, P::T_S1 + wg * 32), *reinterpret_cast<float(*)[16]>(v));
-            tmem_st16(tmem_addr(tbase, quad, P::T_S1 + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
-            tmem_st_wait();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_ready);
         }
 
-        for (int c = 0; c < nch; ++c) {
+        for (int c = 0; c < nch && !bad; ++c) {
             const uint32_t cp = c & 1;
-            // off the chain, while [U; O] of this chunk is computed: the previous
-            // chunk's output and the next chunk's decay vector
-            if (c >= 1) output_tile(c - 1);
-            if (warp == 1 && c + 1 < nch) {
-                chunk_vectors(c + 1);
-                if (c + 2 < nch) stage_alpha(c + 2);
-            }
-            if (named_bar_or(1, kConv, bad)) { bad = true; break; }
-
-            // U (rows 0-63) -> bf16 (MN-major B operand)
-            if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
-            tc_fence_after();
             if (quad < 2) {
-                const int i = quad * 32 + lane;
-                float v[32];
-                ld_sum(cp * 64 + wg * 32, v);
+                // U (rows 0-63) -> bf16: U for P~ U, diag(b_C / b) U for the state update
+                if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
+                tc_fence_after();
+                float u[32], w[32];
+                ld32(P::T_X1 + cp * 64 + wg * 32, u);
+                ld32(P::T_X2 + cp * 64 + wg * 32, w);
+                tmem_ld_wait();
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4*>(utile + sw128_offset(i, wg * 64 + q * 16)) =
-                        make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                for (int x = 0; x < 32; ++x) u[x] += w[x];
+                store_row(utile, r, u, 1.f);
+                store_row(uhat, r, u, tokf);
                 fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(u_ready);
+            } else if (c >= 1) {
+                output_tile(c - 1, tokf_prev);
             }
-            tc_fence_before();
-            mbar_arrive(u_ready);
 
-            // state S = S1 + S2: bf16 copy for the next chunk, then S1 = b_C S
+            // state S <- b_C S + S1 + S2; its bf16 copy for the next chunk
             if (!mbar_wait(s_full, c & 1, kErrMma)) bad = true;
             tc_fence_after();
             {
-                const int f = acc_row<D>(quad, lane);
-                float v[32], w[32];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_S1 + wg * 32), *reinterpret_cast<float(*)[16]>(v));
-                tmem_ld16(tmem_addr(tbase, quad, P::T_S1 + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
-                tmem_ld16(tmem_addr(tbase, quad, P::T_S2 + wg * 32), *reinterpret_cast<float(*)[16]>(w));
-                tmem_ld16(tmem_addr(tbase, quad, P::T_S2 + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(w + 16));
+                float a[32], b[32];
+                ld32(P::T_S1 + wg * 32, a);
+                ld32(P::T_S2 + wg * 32, b);
                 tmem_ld_wait();
+                if (f >= 0) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) v[x] += w[x];
-                if (c + 1 < nch) {
-                    if (f >= 0) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            *reinterpret_cast<uint4*>(sbt + sw128_offset(f, wg * 64 + q * 16)) = make_uint4(
-                                pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-                    }
-                    fence_async_smem();
-                    tc_fence_before();
-                    mbar_arrive(s_ready);
-                    const float bc = vb_c[(c + 1) % 3];
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) v[x] *= bc;
-                    tmem_st16(tmem_addr(tbase, quad, P::T_S1 + wg * 32), *reinterpret_cast<float(*)[16]>(v));
-                    tmem_st16(tmem_addr(tbase, quad, P::T_S1 + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
-                    tmem_st_wait();
-                } else if (f >= 0 && !bad) {
-                    // final state slice
-                    float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)chain * D + f) * dv + j0 + wg * 32);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    for (int x = 0; x < 32; ++x) sreg[x] = fmaf(bc, sreg[x], a[x] + b[x]);
                 }
             }
+            if (c + 1 < nch) {
+                if (f >= 0) store_row(sbt, f, sreg, 1.f);
+                tokf_prev = tokf;
+                read_factors(c + 1);
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_ready);
+            } else if (f >= 0 && !bad) {
+                // final state slice
+                float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)chain * D + f) * dv + j0 + wg * 32);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    dst[q] = make_float4(sreg[4 * q], sreg[4 * q + 1], sreg[4 * q + 2], sreg[4 * q + 3]);
+            }
         }
-        if (!bad) output_tile(nch - 1);
-        if (warp == 1) cp_async_wait_all();
+        if (quad >= 2 && !bad) output_tile(nch - 1, tokf);
     }
     tc_fence_before();
     __syncthreads();
@@ -918,24 +859,22 @@ int sm_count()
 }
 
 template <int D>
-cudaError_t launch_gd(const PrefillArgs& a)
+cudaError_t launch_gd(const PrefillArgs& a, int prep_ctas, int mark)
 {
     const int chains = a.B * a.H;
     const int nch = (a.N + C - 1) / C;
     const int npad = nch * C;
-    // workspace: -W, diag(b) Q, diag(b_C / b) K [chains][npad][D], T' and P~
-    // [chains][npad][C], all bf16
+    // workspace: -W [chains][npad][D], T' and P~ [chains][npad][C] (bf16), then
+    // the per-token factors b, b_C / b [chains][nch][2][C] (fp32)
     unsigned char* wneg = static_cast<unsigned char*>(a.workspace);
-    unsigned char* qb = wneg + (size_t)chains * npad * D * 2;
-    unsigned char* kt = qb + (size_t)chains * npad * D * 2;
-    unsigned char* tp = kt + (size_t)chains * npad * D * 2;
+    unsigned char* tp = wneg + (size_t)chains * npad * D * 2;
     unsigned char* pp = tp + (size_t)chains * npad * C * 2;
-    CUtensorMap mq, mk, mv, mo, mw, mqb, mkt, mt, mp;
+    float* vec = reinterpret_cast<float*>(pp + (size_t)chains * npad * C * 2);
+    CUtensorMap mq, mk, mv, mo, mw, mt, mp;
     if (!make_map(&mq, a.q, D, a.N, chains, a.ld) || !make_map(&mk, a.k, D, a.N, chains, a.ld) ||
         !make_map(&mv, a.v, a.dv, a.N, chains, a.ld) || !make_map(&mo, a.out, a.dv, a.N, chains, a.ld) ||
-        !make_map(&mw, wneg, D, npad, chains, npad) || !make_map(&mqb, qb, D, npad, chains, npad) ||
-        !make_map(&mkt, kt, D, npad, chains, npad) ||
-        !make_map(&mt, tp, C, npad, chains, npad) || !make_map(&mp, pp, C, npad, chains, npad))
+        !make_map(&mw, wneg, D, npad, chains, npad) || !make_map(&mt, tp, C, npad, chains, npad) ||
+        !make_map(&mp, pp, C, npad, chains, npad))
         return cudaErrorInvalidValue;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
@@ -948,7 +887,7 @@ cudaError_t launch_gd(const PrefillArgs& a)
     e = cudaFuncSetAttribute(k1, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     const long long items = (long long)chains * nch;
-    const int g1 = (int)std::min<long long>(items, 2LL * sms);
+    const int g1 = (int)std::min<long long>(items, prep_ctas > 0 ? prep_ctas : 2LL * sms);
     // behind an earlier call of the same batch (disjoint workspace), the prep
     // pass starts with programmatic serialization too
     cudaLaunchAttribute pdl1[1];
@@ -961,11 +900,11 @@ cudaError_t launch_gd(const PrefillArgs& a)
     l1.stream = a.stream;
     l1.attrs = pdl1;
     l1.numAttrs = a.pdl_first ? 1 : 0;
-    e = cudaLaunchKernelEx(&l1, k1, mq, mk, mw, mqb, mkt, mt, mp, a.alpha, a.g, a.N, chains, a.ld);
+    e = cudaLaunchKernelEx(&l1, k1, mq, mk, mw, mt, mp, a.alpha, a.g, vec, a.N, chains, a.ld);
     if (e != cudaSuccess) return e;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    stage_mark(0, a.stream);
+    stage_mark(mark, a.stream);
 
     auto k2 = gd_chain_kernel<D>;
     const int s2 = ChainPlan<D>::BYTES;
@@ -983,29 +922,105 @@ cudaError_t launch_gd(const PrefillArgs& a)
     lc.stream = a.stream;
     lc.attrs = pdl;
     lc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&lc, k2, mqb, mkt, mv, mw, mt, mp, mo, (const float*)a.alpha, (const float*)a.S0,
-                           a.S_out, a.N, a.dv, a.ld);
+    e = cudaLaunchKernelEx(&lc, k2, mq, mk, mv, mw, mt, mp, mo, (const float*)vec, (const float*)a.S0, a.S_out,
+                           a.N, a.dv);
     if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    stage_mark(1, a.stream);
+    stage_mark(mark + 1, a.stream);
     return cudaSuccess;
+}
+
+}  // namespace
+
+// The sequence split of a gated-delta call.  The chain pass runs one CTA per
+// (chain, 64 value columns); when that leaves most SMs idle, the sequence is cut
+// into parts that run as a pipeline: the prep pass of part i + 1 runs on the
+// idle SMs while the chain pass of part i runs, and the chain of part i + 1
+// starts from the final state of part i.
+GdParts gd_parts(int B, int H, int N, int d, int dv)
+{
+    (void)d;
+    GdParts p;
+    p.P = 1;
+    p.len = N;
+    const long long nch = (N + C - 1) / C;
+    const long long ctas = (long long)B * H * (dv / DVT);
+    if (N >= 8192 && ctas <= 96) {
+        const long long P = std::min<long long>(kMaxGdParts, nch / 32);
+        const long long per = (nch + P - 1) / P;   // chunks per part
+        p.len = (int)(per * C);
+        p.P = (int)((N + p.len - 1) / p.len);
+    }
+    return p;
+}
+
+namespace {
+
+// Workspace of one part of n tokens: -W, T', P~ (bf16) and the per-token
+// factors (fp32), rounded up to 256 bytes.
+size_t gd_part_bytes(long long chains, int n, int d)
+{
+    const size_t nch = (size_t)((n + C - 1) / C);
+    const size_t npad = nch * C;
+    const size_t b = (size_t)chains * (npad * (size_t)(d + 2 * C) * 2 + nch * 2 * C * sizeof(float));
+    return (b + 255) / 256 * 256;
 }
 
 }  // namespace
 
 size_t gd_workspace_bytes(int B, int H, int N, int d, int dv)
 {
-    (void)dv;
-    const size_t npad = (size_t)((N + C - 1) / C) * C;
-    return (size_t)B * H * npad * (size_t)(3 * d + 2 * C) * 2;
+    const GdParts p = gd_parts(B, H, N, d, dv);
+    const long long chains = (long long)B * H;
+    size_t total = 0;
+    for (int i = 0; i < p.P; ++i) total += gd_part_bytes(chains, std::min(p.len, N - i * p.len), d);
+    // two fp32 states that carry the chain from one part to the next
+    if (p.P > 1) total += 2 * (size_t)chains * d * dv * sizeof(float);
+    return total;
 }
 
 cudaError_t launch_prefill_tc_gated_delta(const PrefillArgs& a)
 {
     if (!a.workspace || a.workspace_bytes < gd_workspace_bytes(a.B, a.H, a.N, a.d, a.dv))
         return cudaErrorInvalidValue;
-    if (a.d == 64) return launch_gd<64>(a);
-    return launch_gd<128>(a);
+    const GdParts parts = gd_parts(a.B, a.H, a.N, a.d, a.dv);
+    const long long chains = (long long)a.B * a.H;
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    // while a chain pass runs, the next part's prep pass gets the other SMs (two CTAs each)
+    const int busy = (int)(chains * (a.dv / DVT));
+    const int side_ctas = std::max(2, 2 * (sms - busy));
+    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+    size_t off = 0;
+    for (int i = 0; i < parts.P; ++i) off += gd_part_bytes(chains, std::min(parts.len, a.N - i * parts.len), a.d);
+    float* carry[2] = {reinterpret_cast<float*>(ws + off),
+                       reinterpret_cast<float*>(ws + off) + (size_t)chains * a.d * a.dv};
+    const size_t es = 2;   // bf16 elements
+    off = 0;
+    for (int i = 0; i < parts.P; ++i) {
+        const int t0 = i * parts.len;
+        const int n = std::min(parts.len, a.N - t0);
+        PrefillArgs pa = a;
+        pa.q = static_cast<const char*>(a.q) + (size_t)t0 * a.d * es;
+        pa.k = static_cast<const char*>(a.k) + (size_t)t0 * a.d * es;
+        pa.v = static_cast<const char*>(a.v) + (size_t)t0 * a.dv * es;
+        pa.out = static_cast<char*>(a.out) + (size_t)t0 * a.dv * es;
+        pa.alpha = a.alpha + t0;
+        pa.g = a.g + t0;
+        pa.N = n;
+        pa.S0 = i == 0 ? a.S0 : carry[(i - 1) & 1];
+        pa.S_out = i == parts.P - 1 ? a.S_out : carry[i & 1];
+        pa.workspace = ws + off;
+        pa.workspace_bytes = gd_part_bytes(chains, n, a.d);
+        off += pa.workspace_bytes;
+        // part 0 keeps the call's stream order; each later part's prep pass
+        // starts behind the previous chain pass and runs beside it
+        pa.pdl_first = i == 0 ? a.pdl_first : true;
+        const int prep_ctas = i == 0 ? 0 : side_ctas;
+        const cudaError_t e = a.d == 64 ? launch_gd<64>(pa, prep_ctas, 2 * i) : launch_gd<128>(pa, prep_ctas, 2 * i);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 unsigned int read_and_clear_device_error_gdelta(cudaStream_t stream)

@@ -29,7 +29,15 @@ cudaError_t launch_prefill_tc_kernelized_noalloc(const PrefillArgs& a);
 bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains, int ld);
 
 // Gated-delta prefill on the tensor cores (bf16 inputs).  The workspace holds
-// the per-chunk operands the parallel pass hands to the sequential pass.
+// the per-chunk operands the parallel pass hands to the sequential pass.  A
+// long sequence runs as up to kMaxGdParts parts of len tokens (a multiple of
+// the 64-token chunk) whose passes overlap; a call launches 2 P kernels.
+constexpr int kMaxGdParts = 4;
+struct GdParts {
+    int P = 1;
+    int len = 0;
+};
+GdParts gd_parts(int B, int H, int N, int d, int dv);
 size_t gd_workspace_bytes(int B, int H, int N, int d, int dv);
 cudaError_t launch_prefill_tc_gated_delta(const PrefillArgs& a);
 unsigned int read_and_clear_device_error_gdelta(cudaStream_t stream);

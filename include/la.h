@@ -156,12 +156,27 @@ LA_API la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
  * sizes and this cfg (dtype, mode).  0 means no workspace is needed.  The
  * workspace carries data between the kernels of one call: per-segment state
  * summaries for bf16 LA_PLAIN / LA_DECAY, and for bf16 LA_GATED_DELTA the
- * per-chunk operands (-W, diag(b) q, diag(b_C/b) k, T' and the masked score
- * block, bf16, ceil(N/64)*64 rows of 3d + 128 values per chain).  Its content need not be initialised and
+ * per-chunk operands of each part of the sequence (-W, T' and the masked
+ * score block, bf16, d + 128 values per token, and the per-token decay
+ * factors, two fp32 values per token) plus, for more than one part, two
+ * fp32 states that carry the chain between parts.  Its content need not be
+ * initialised and
  * is dead after the call's work completes.  Two calls in flight at once need
  * two workspaces.
  */
 LA_API size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_config* cfg);
+
+/*
+ * la_prefill_kernel_count -- how many kernels one la_prefill call with these
+ * sizes and this cfg (dtype, mode) launches, i.e. how many events
+ * la_set_stage_events records for it: 3 for bf16 LA_PLAIN / LA_DECAY (segment
+ * summaries, scan, chunk loop); 2 P for bf16 LA_GATED_DELTA, whose sequence
+ * runs as P <= 4 parts (each a chunk prep pass and a chain pass; the prep
+ * pass of part i + 1 overlaps the chain pass of part i); 1 otherwise; 0 when
+ * the call launches no kernel (N = 0, nothing to do, or unsupported sizes).
+ * Host-only.  Not from the pages: a service for profiling.
+ */
+LA_API int la_prefill_kernel_count(int B, int H, int N, int d, int dv, const la_config* cfg);
 
 /*
  * la_prefill_varlen -- la_prefill over a right-padded batch of sequences of
@@ -273,9 +288,10 @@ LA_API la_status la_causal_conv(const void* x, const float* weight, const void* 
  * later la_prefill / la_decode_step / la_gated_delta_decode_step /
  * la_causal_conv records
  * events[i] on its cfg->stream right after launching its i-th kernel
- * (i < n; a call launches 1 to 3 kernels: bf16 LA_PLAIN/LA_DECAY prefill =
- * segment summaries, scan, chunk loop; bf16 LA_GATED_DELTA prefill = chunk
- * prep, chain; every other path, la_causal_conv included, one kernel).  events are cudaEvent_t handles
+ * (i < n; a call launches 1 to 8 kernels, la_prefill_kernel_count gives the
+ * number for a prefill: bf16 LA_PLAIN/LA_DECAY prefill = segment summaries,
+ * scan, chunk loop; bf16 LA_GATED_DELTA prefill = chunk prep and chain per
+ * part; every other path, la_causal_conv included, one kernel).  events are cudaEvent_t handles
  * owned by the caller, who must keep them alive while the hook is set; n = 0
  * turns it off.  The setting is process-wide and not thread-safe: set it
  * only while no other thread launches through this library.  Returns

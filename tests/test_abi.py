@@ -119,10 +119,27 @@ def test_workspace_query_is_host_only():
 
 
 def test_gated_delta_workspace_size():
-    # bf16 gated delta: per chain ceil(N/64)*64 rows of 3d + 128 bf16 values; f32 needs none
+    # bf16 gated delta: per chain ceil(N/64)*64 rows of d + 128 bf16 values and
+    # two fp32 factors per token; f32 needs none
     n = la.la_prefill_workspace_bytes(1, 32, 1000, 128, 128, "bf16", "gated_delta")
-    assert n == 32 * 1024 * (3 * 128 + 128) * 2
+    assert n == 32 * (1024 * (128 + 128) * 2 + 1024 * 2 * 4)
     assert la.la_prefill_workspace_bytes(1, 32, 1000, 128, 128, "f32", "gated_delta") == 0
+    # the long workload runs as four parts of 16384 tokens, plus two carry states
+    part = 32 * (16384 * (128 + 128) * 2 + 16384 * 2 * 4)
+    n = la.la_prefill_workspace_bytes(1, 32, 65536, 128, 128, "bf16", "gated_delta")
+    assert n == 4 * part + 2 * 32 * 128 * 128 * 4
+
+
+def test_kernel_count():
+    kc = la.la_prefill_kernel_count
+    assert kc(4, 8, 4096, 64, 64, "bf16", "plain") == 3
+    assert kc(2, 16, 32768, 128, 128, "bf16", "decay") == 3
+    assert kc(1, 32, 65536, 128, 128, "bf16", "gated_delta") == 8     # four overlapped parts
+    assert kc(1, 3, 2100, 128, 128, "bf16", "gated_delta") == 2
+    assert kc(64, 32, 65536, 128, 128, "bf16", "gated_delta") == 2    # enough chains to fill the GPU
+    assert kc(1, 1, 256, 64, 64, "f32", "plain") == 1
+    assert kc(1, 32, 8192, 128, 128, "bf16", "gla") == 1
+    assert kc(1, 1, 0, 64, 64, "bf16", "plain") == 0
 
 
 def test_stage_events_validation():
