@@ -495,29 +495,32 @@ struct ChainPlan {
     static constexpr int OFF_UH = OFF_U + TILE;               // diag(b_C / b) U bf16 (B of K^T U)
     static constexpr int OFF_O = OFF_UH + TILE;               // output staging
     static constexpr int OFF_BAR = OFF_O + TILE;
-    // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready s_ready ostage_full ostage_empty
-    // drain[2]
+    // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready u2_ready s_ready
+    // ostage_full ostage_empty drain
     static constexpr int NBAR = 17;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
-    // TMEM columns: the two issuers' partial [U; Q S] accumulators X1, X2 and the
-    // P~ U accumulator X3 (two buffers each), and the two partial state updates
-    static constexpr uint32_t T_X1 = 0, T_X2 = 128, T_X3 = 256, T_S1 = 384, T_S2 = 448, T_COLS = 512;
-    static constexpr int KS_HALF = D / 32;                   // K-steps of [-W; Q] S per issuer
+    // TMEM columns: X = [U; Q S] and X3 = [0; P~ U] (two buffers each), the state update
+    static constexpr uint32_t T_X = 0, T_X3 = 128, T_S = 256, T_COLS = 512;
 };
 
-constexpr int kConv = 256;                   // converter threads (warps 0-7)
-constexpr int kChainThreads = kConv + 96;    // + issuer warps 8 and 10, TMA warp 9
+constexpr int kConvWarps = 16;                      // converter warps 0-15
+constexpr int kChainThreads = (kConvWarps + 2) * 32;  // + issuer warp 16, TMA warp 17
+constexpr int kIssuerWarp = kConvWarps, kTmaWarp = kConvWarps + 1;
 
-// The chain of one (chain, 64 value columns).  Per chunk c with start state S:
-//   issuers   X1 = [T'; 0] V (one chunk ahead) + [-W; Q]_1 S_1,  X2 = [-W; Q]_2 S_2
-//             (feature halves), so rows 0-63 of X1 + X2 are U and rows 64-127 are Q S;
-//             after U is in place: S1 = K_1^T U^, S2 = K_2^T U^ (token halves),
-//             U^ = diag(b_C / b) U; then X3 = [0; P~] U.
-//   converters  U, U^ to bf16;  S <- b_C S + S1 + S2 (fp32, held in registers), its
-//             bf16 copy for the next chunk;  o = diag(b) Q S + P~ U -> staging.
-// The converters signal with one arrival per warp.
+// The chain of one (chain, 64 value columns).  Per chunk c with start state S
+// (bf16 copy in shared memory, fp32 master in the converters' registers):
+//   issuer      X = [T'; 0] V (issued a chunk ahead) + [-W; Q] S, so rows 0-63 of X
+//               are U and rows 64-127 are Q S;  then, once U^ = diag(b_C / b) U is
+//               in place, dS = K^T U^;  then the next chunk's [T'; 0] V and, once U
+//               is in place, X3 = [0; P~] U.
+//   converters  U^ (first: the state update waits for it), U;  S <- b_C S + dS and
+//               its bf16 copy;  o = diag(b) Q S + P~ U -> staging.
+// One thread issues every MMA, in the order the chain needs them; the tensor
+// pipe runs them in that order.  Sixteen converter warps split each phase by
+// rows (TMEM lane quadrant = warp % 4) and 16-column groups (warp / 4), and
+// each warp arrives once on the barrier that ends its part of a phase.
 template <int D>
 __global__ void __launch_bounds__(kChainThreads, 1)
 gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -537,20 +540,20 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     unsigned char* ostage = sm + P::OFF_O;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* full = bars;          // TMA -> everyone, per stage
-    uint64_t* empty = bars + 2;     // both issuers (commit) -> TMA, per stage
-    uint64_t* uo_full = bars + 4;   // both issuers: [U; Q S] partials complete, per TMEM buffer
-    uint64_t* o_full = bars + 6;    // issuer B: P~ U complete, per TMEM buffer
+    uint64_t* empty = bars + 2;     // issuer (commit) -> TMA, per stage
+    uint64_t* uo_full = bars + 4;   // issuer: [U; Q S] complete, per TMEM buffer
+    uint64_t* o_full = bars + 6;    // issuer: P~ U complete, per TMEM buffer
     uint64_t* o_read = bars + 8;    // output warps: the buffer's output rows read
-    uint64_t* s_full = bars + 10;   // both issuers: state update partials complete
-    uint64_t* u_ready = bars + 11;  // U warps: U and U^ in place
-    uint64_t* s_ready = bars + 12;  // every converter warp: bf16 state written
-    uint64_t* os_full = bars + 13;  // output warps: output staging written
-    uint64_t* os_empty = bars + 14; // TMA: output staging read by its store
-    uint64_t* drain = bars + 15;    // [2] issuers: every MMA each issued is complete
+    uint64_t* s_full = bars + 10;   // issuer: state update complete
+    uint64_t* u_ready = bars + 11;  // U warps: U^ in place
+    uint64_t* u2_ready = bars + 12; // U warps: U in place
+    uint64_t* s_ready = bars + 13;  // every converter warp: bf16 state written
+    uint64_t* os_full = bars + 14;  // output warps: output staging written
+    uint64_t* os_empty = bars + 15; // TMA: output staging read by its store
+    uint64_t* drain = bars + 16;    // issuer: every MMA it issued is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, wg = (warp >> 2) & 1;
     const int ntile = dv / DVT;
     const int chain = blockIdx.x / ntile, j0 = (blockIdx.x % ntile) * DVT;
     const int nch = (N + C - 1) / C;
@@ -558,17 +561,18 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 2);
-            mbar_init(&uo_full[s], 2);
+            mbar_init(&empty[s], 1);
+            mbar_init(&uo_full[s], 1);
             mbar_init(&o_full[s], 1);
-            mbar_init(&o_read[s], 4);
-            mbar_init(&drain[s], 1);
+            mbar_init(&o_read[s], kConvWarps / 2);
         }
-        mbar_init(s_full, 2);
-        mbar_init(u_ready, 4);
-        mbar_init(s_ready, 8);
-        mbar_init(os_full, 4);
+        mbar_init(s_full, 1);
+        mbar_init(u_ready, kConvWarps / 2);
+        mbar_init(u2_ready, kConvWarps / 2);
+        mbar_init(s_ready, kConvWarps);
+        mbar_init(os_full, kConvWarps / 2);
         mbar_init(os_empty, 1);
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     // zero tiles of both stages (rows 64-127 of [T'; Z], rows 0-63 of [Z; P~])
@@ -583,7 +587,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tbase = *tmem_slot;
     grid_dependency_wait();   // the prep pass's operands are complete
 
-    if (warp == 9) {
+    if (warp == kTmaWarp) {
         // ---------------- TMA: stage loads and output stores ----------------
         if (lane == 0) {
             const uint64_t pol_once = policy_evict_first();
@@ -647,146 +651,127 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad);
         }
         __syncwarp();
-    } else if (warp == 8 || warp == 10) {
-        // ---------------- MMA issuers ----------------
+    } else if (warp == kIssuerWarp) {
+        // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            const bool A = warp == 8;
             const uint32_t id = idesc_bf16_f32(128, 64, 0, 1);
             const uint32_t ids = idesc_bf16_f32(D, 64, 1, 1);
             const uint64_t ds = sdesc_sw128(smem_u32(sbt), TILE, 1024);
             const uint64_t du = sdesc_sw128(smem_u32(utile), TILE, 1024);
             const uint64_t duh = sdesc_sw128(smem_u32(uhat), TILE, 1024);
-            const uint32_t tx = tbase + (A ? P::T_X1 : P::T_X2);
-            const uint32_t tsp = tbase + (A ? P::T_S1 : P::T_S2);
-            auto ready = [&](int c) {   // stage c loaded and TMEM buffer c & 1 read out
+            // X = [T'; 0] V of chunk c: stage c loaded, TMEM buffer c & 1 read out
+            auto tv = [&](int c) {
                 if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) return false;
                 if (c >= 2 && !mbar_wait(&o_read[c & 1], ((c - 2) / 2) & 1, kErrMma)) return false;
-                return true;
-            };
-            auto m0 = [&](int c) {
-                if (!ready(c)) return false;
                 tc_fence_after();
                 unsigned char* st = sm + (c % P::STAGES) * P::STAGE;
                 const uint64_t dt = sdesc_sw128(smem_u32(st + P::O_T), 16, 1024);
                 const uint64_t dvv = sdesc_sw128(smem_u32(st + P::O_V), TILE, 1024);
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tx + (c & 1) * 64, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id, ks > 0);
+                    mma_bf16(tbase + P::T_X + (c & 1) * 64, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id,
+                             ks > 0);
                 return true;
             };
-            bool ok = A ? m0(0) : true;
+            bool ok = tv(0);
             for (int c = 0; c < nch && ok; ++c) {
                 const int s = c % P::STAGES;
                 const uint32_t cp = c & 1;
                 unsigned char* st = sm + s * P::STAGE;
-                const uint32_t txc = tx + cp * 64;
-                if (!A && !(ok = ready(c))) break;
                 if (!(ok = mbar_wait(s_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
+                // X += [-W; Q] S
                 const uint64_t dwq = sdesc_sw128(smem_u32(st + P::O_WQ), 16, 1024);
-                const int k0 = A ? 0 : P::KS_HALF;
 #pragma unroll
-                for (int kk = 0; kk < P::KS_HALF; ++kk) {
-                    const int ks = k0 + kk;
-                    mma_bf16(txc, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4), ds + ((ks * 2048) >> 4), id,
-                             (A || kk > 0) ? 1u : 0u);
-                }
+                for (int ks = 0; ks < D / 16; ++ks)
+                    mma_bf16(tbase + P::T_X + cp * 64, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4),
+                             ds + ((ks * 2048) >> 4), id, 1u);
                 mma_commit(&uo_full[cp]);
+                // dS = K^T U^
                 if (!(ok = mbar_wait(u_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
                 const uint64_t dk = sdesc_sw128(smem_u32(st + P::O_K), TILE, 1024);
-                const int t0 = A ? 0 : 2;
 #pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                    const int ks = t0 + kk;
-                    mma_bf16(tsp, dk + ((ks * 2048) >> 4), duh + ((ks * 2048) >> 4), ids, kk > 0 ? 1u : 0u);
-                }
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tbase + P::T_S, dk + ((ks * 2048) >> 4), duh + ((ks * 2048) >> 4), ids, ks > 0);
                 mma_commit(s_full);
-                if (A) {
-                    mma_commit(&empty[s]);
-                    if (c + 1 < nch) ok = m0(c + 1);
-                } else {
-                    const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
-                    const uint32_t t3 = tbase + P::T_X3 + cp * 64;
+                // off the chain: the next chunk's [T'; 0] V, then this chunk's P~ U
+                if (c + 1 < nch && !(ok = tv(c + 1))) break;
+                if (!(ok = mbar_wait(u2_ready, c & 1, kErrMma))) break;
+                tc_fence_after();
+                const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
 #pragma unroll
-                    for (int ks = 0; ks < C / 16; ++ks)
-                        mma_bf16(t3, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, ks > 0 ? 1u : 0u);
-                    mma_commit(&o_full[cp]);
-                    mma_commit(&empty[s]);
-                }
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tbase + P::T_X3 + cp * 64, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, ks > 0);
+                mma_commit(&o_full[cp]);
+                mma_commit(&empty[s]);
             }
             // every MMA issued must complete before TMEM is released
-            mma_commit(&drain[A ? 0 : 1]);
-            mbar_wait(&drain[A ? 0 : 1], 0, kErrMma);
+            mma_commit(drain);
+            mbar_wait(drain, 0, kErrMma);
         }
         __syncwarp();
     } else {
-        // ---------------- converters (warps 0-7) ----------------
-        // Thread (quad, lane) owns row r = 32 quad + lane of the M = 128
-        // accumulators, a token of U (quads 0, 1) or of the output (quads 2, 3),
-        // and row f of the M = D state accumulators (f = r for D = 128); warpgroup
-        // wg owns 32 of the tile's 64 value columns.
+        // ---------------- converters (warps 0-15) ----------------
+        // Thread (quad, lane) of warp w (quad = w % 4, g = w / 4) owns row
+        // r = 32 quad + lane of the M = 128 accumulators, a token of U (quads 0,
+        // 1) or of the output (quads 2, 3), and row f of the M = D state
+        // accumulator (f = r for D = 128); g picks 16 of the tile's 64 columns.
+        const int quad = warp & 3, grp = warp >> 2;
         const int r = quad * 32 + lane;
-        const int f = acc_row<D>(quad, lane);   // state row (feature) of this thread, or -1
+        const int f = acc_row<D>(quad, lane);
+        const bool urow = quad < 2;
         bool bad = false;
-        auto ld32 = [&](uint32_t col, float (&v)[32]) {
-            tmem_ld16(tmem_addr(tbase, quad, col), *reinterpret_cast<float(*)[16]>(v));
-            tmem_ld16(tmem_addr(tbase, quad, col + 16), *reinterpret_cast<float(*)[16]>(v + 16));
+        auto ld16 = [&](uint32_t col, float (&v)[16]) { tmem_ld16(tmem_addr(tbase, quad, col), v); };
+        auto store16 = [&](unsigned char* tile, int row, const float (&v)[16], float w) {
+            const uint4 a = make_uint4(pack_bf16x2(w * v[0], w * v[1]), pack_bf16x2(w * v[2], w * v[3]),
+                                       pack_bf16x2(w * v[4], w * v[5]), pack_bf16x2(w * v[6], w * v[7]));
+            const uint4 b = make_uint4(pack_bf16x2(w * v[8], w * v[9]), pack_bf16x2(w * v[10], w * v[11]),
+                                       pack_bf16x2(w * v[12], w * v[13]), pack_bf16x2(w * v[14], w * v[15]));
+            *reinterpret_cast<uint4*>(tile + sw128_offset(row, grp * 32)) = a;
+            *reinterpret_cast<uint4*>(tile + sw128_offset(row, grp * 32 + 16)) = b;
         };
-        auto store_row = [&](unsigned char* tile, int row, const float (&v)[32], float w) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4*>(tile + sw128_offset(row, wg * 64 + q * 16)) =
-                    make_uint4(pack_bf16x2(w * v[8 * q], w * v[8 * q + 1]), pack_bf16x2(w * v[8 * q + 2], w * v[8 * q + 3]),
-                               pack_bf16x2(w * v[8 * q + 4], w * v[8 * q + 5]),
-                               pack_bf16x2(w * v[8 * q + 6], w * v[8 * q + 7]));
-        };
-        // per-chunk factors of this thread, read from the stage before this warp's
-        // arrival that lets the stage be refilled: b_C, and b_t (output rows) or
-        // b_C / b_t (U rows) of token r % 64
-        float bc = 1.f, tokf = 1.f, tokf_prev = 1.f;
-        auto read_factors = [&](int c) {
+        // per-chunk factors, read from the stage before this warp's arrival that
+        // lets the stage be refilled: b_C, and b_t (output rows) or b_C / b_t
+        // (U rows) of token r % 64
+        auto read_factors = [&](int c, float& bc, float& tf) {
             if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) bad = true;
             const float* vv = reinterpret_cast<const float*>(sm + (c % P::STAGES) * P::STAGE + P::O_VEC);
             bc = vv[C - 1];
-            tokf = quad < 2 ? vv[C + r] : vv[r - 64];
+            tf = urow ? vv[C + r] : vv[r - 64];
         };
         // output rows of chunk cc (accumulator rows 64-127) -> staging
         auto output_tile = [&](int cc, float bt) {
             if (!mbar_wait(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
             if (cc >= 1 && !mbar_wait(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
             tc_fence_after();
-            float o[32], w[32];
-            const uint32_t col = (cc & 1) * 64 + wg * 32;
-            ld32(P::T_X1 + col, o);
-            ld32(P::T_X2 + col, w);
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] += w[x];
-            ld32(P::T_X3 + col, w);
+            float o[16], w[16];
+            ld16(P::T_X + (cc & 1) * 64 + grp * 16, o);
+            ld16(P::T_X3 + (cc & 1) * 64 + grp * 16, w);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_read[cc & 1]);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = fmaf(bt, o[x], w[x]);
-            store_row(ostage, r - 64, o, 1.f);
+            for (int x = 0; x < 16; ++x) o[x] = fmaf(bt, o[x], w[x]);
+            store16(ostage, r - 64, o, 1.f);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(os_full);
         };
 
         // start state slice S[:, j0:j0+64] in registers and, as bf16, in the B operand
-        float sreg[32];
+        float sreg[16];
+        float bc, tokf, bc_next = 1.f, tokf_next = 1.f, bt_prev = 1.f;
         {
-            const float* src = (S0 && f >= 0) ? S0 + ((size_t)chain * D + f) * dv + j0 + wg * 32 : nullptr;
+            const float* src = (S0 && f >= 0) ? S0 + ((size_t)chain * D + f) * dv + j0 + grp * 16 : nullptr;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < 4; ++q) {
                 const float4 t = src ? reinterpret_cast<const float4*>(src)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
                 sreg[4 * q] = t.x; sreg[4 * q + 1] = t.y; sreg[4 * q + 2] = t.z; sreg[4 * q + 3] = t.w;
             }
-            if (f >= 0) store_row(sbt, f, sreg, 1.f);
-            read_factors(0);
+            if (f >= 0) store16(sbt, f, sreg, 1.f);
+            read_factors(0, bc, tokf);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_ready);
@@ -794,56 +779,55 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         for (int c = 0; c < nch && !bad; ++c) {
             const uint32_t cp = c & 1;
-            if (quad < 2) {
-                // U (rows 0-63) -> bf16: U for P~ U, diag(b_C / b) U for the state update
+            if (urow) {
+                // U (rows 0-63): U^ = diag(b_C / b) U first, the state update waits for it
                 if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
                 tc_fence_after();
-                float u[32], w[32];
-                ld32(P::T_X1 + cp * 64 + wg * 32, u);
-                ld32(P::T_X2 + cp * 64 + wg * 32, w);
+                float u[16];
+                ld16(P::T_X + cp * 64 + grp * 16, u);
                 tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < 32; ++x) u[x] += w[x];
-                store_row(utile, r, u, 1.f);
-                store_row(uhat, r, u, tokf);
+                store16(uhat, r, u, tokf);
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(u_ready);
+                store16(utile, r, u, 1.f);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(u2_ready);
             } else if (c >= 1) {
-                output_tile(c - 1, tokf_prev);
+                output_tile(c - 1, bt_prev);
             }
+            if (c + 1 < nch) read_factors(c + 1, bc_next, tokf_next);
 
-            // state S <- b_C S + S1 + S2; its bf16 copy for the next chunk
+            // state S <- b_C S + dS; its bf16 copy for the next chunk
             if (!mbar_wait(s_full, c & 1, kErrMma)) bad = true;
             tc_fence_after();
             {
-                float a[32], b[32];
-                ld32(P::T_S1 + wg * 32, a);
-                ld32(P::T_S2 + wg * 32, b);
+                float a[16];
+                ld16(P::T_S + grp * 16, a);
                 tmem_ld_wait();
-                if (f >= 0) {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) sreg[x] = fmaf(bc, sreg[x], a[x] + b[x]);
-                }
+                for (int x = 0; x < 16; ++x) sreg[x] = fmaf(bc, sreg[x], a[x]);
             }
             if (c + 1 < nch) {
-                if (f >= 0) store_row(sbt, f, sreg, 1.f);
-                tokf_prev = tokf;
-                read_factors(c + 1);
+                if (f >= 0) store16(sbt, f, sreg, 1.f);
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_ready);
+                bt_prev = tokf;
+                tokf = tokf_next;
+                bc = bc_next;
             } else if (f >= 0 && !bad) {
                 // final state slice
-                float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)chain * D + f) * dv + j0 + wg * 32);
+                float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)chain * D + f) * dv + j0 + grp * 16);
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
+                for (int q = 0; q < 4; ++q)
                     dst[q] = make_float4(sreg[4 * q], sreg[4 * q + 1], sreg[4 * q + 2], sreg[4 * q + 3]);
             }
         }
-        if (quad >= 2 && !bad) output_tile(nch - 1, tokf);
+        if (!urow && !bad) output_tile(nch - 1, tokf);
     }
     tc_fence_before();
     __syncthreads();
