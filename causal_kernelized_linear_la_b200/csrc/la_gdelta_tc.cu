@@ -496,31 +496,34 @@ struct ChainPlan {
     static constexpr int OFF_O = OFF_UH + TILE;               // output staging
     static constexpr int OFF_BAR = OFF_O + TILE;
     // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready u2_ready s_ready
-    // ostage_full ostage_empty drain
-    static constexpr int NBAR = 17;
+    // ostage_full ostage_empty drain[2]
+    static constexpr int NBAR = 18;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
-    // TMEM columns: X = [U; Q S] and X3 = [0; P~ U] (two buffers each), the state update
-    static constexpr uint32_t T_X = 0, T_X3 = 128, T_S = 256, T_COLS = 512;
+    // TMEM columns: the two issuers' partial [U; Q S] accumulators X1, X2 and the
+    // P~ U accumulator X3 (two buffers each), and the two partial state updates
+    static constexpr uint32_t T_X1 = 0, T_X2 = 128, T_X3 = 256, T_S1 = 384, T_S2 = 448, T_COLS = 512;
+    static constexpr int KS_HALF = D / 32;                   // K-steps of [-W; Q] S per issuer
 };
 
-constexpr int kConvWarps = 16;                      // converter warps 0-15
-constexpr int kChainThreads = (kConvWarps + 2) * 32;  // + issuer warp 16, TMA warp 17
-constexpr int kIssuerWarp = kConvWarps, kTmaWarp = kConvWarps + 1;
+constexpr int kConvWarps = 16;                        // converter warps 0-15
+constexpr int kChainThreads = (kConvWarps + 3) * 32;  // + issuer warps 16 and 18, TMA warp 17
+constexpr int kIssuerA = kConvWarps, kTmaWarp = kConvWarps + 1, kIssuerB = kConvWarps + 2;
 
 // The chain of one (chain, 64 value columns).  Per chunk c with start state S
 // (bf16 copy in shared memory, fp32 master in the converters' registers):
-//   issuer      X = [T'; 0] V (issued a chunk ahead) + [-W; Q] S, so rows 0-63 of X
-//               are U and rows 64-127 are Q S;  then, once U^ = diag(b_C / b) U is
-//               in place, dS = K^T U^;  then the next chunk's [T'; 0] V and, once U
-//               is in place, X3 = [0; P~] U.
+//   issuer A    X1 = [T'; 0] V (issued a chunk ahead) + [-W; Q]_1 S_1, then, once
+//               U^ = diag(b_C / b) U is in place, dS1 = K_1^T U^_1 (first 32 tokens)
+//   issuer B    X2 = [-W; Q]_2 S_2 (the other feature half), dS2 = K_2^T U^_2, then,
+//               once U is in place, X3 = [0; P~] U
+//   so rows 0-63 of X1 + X2 are U, rows 64-127 are Q S, and dS = dS1 + dS2.
 //   converters  U^ (first: the state update waits for it), U;  S <- b_C S + dS and
 //               its bf16 copy;  o = diag(b) Q S + P~ U -> staging.
-// One thread issues every MMA, in the order the chain needs them; the tensor
-// pipe runs them in that order.  Sixteen converter warps split each phase by
-// rows (TMEM lane quadrant = warp % 4) and 16-column groups (warp / 4), and
-// each warp arrives once on the barrier that ends its part of a phase.
+// A tcgen05.mma takes tens of cycles to issue, so the two contractions on the
+// chain are split between two issuing threads.  Sixteen converter warps split
+// each phase by rows (TMEM lane quadrant = warp % 4) and 16-column groups
+// (warp / 4), and each warp arrives once on the barrier that ends its part.
 template <int D>
 __global__ void __launch_bounds__(kChainThreads, 1)
 gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -540,17 +543,17 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     unsigned char* ostage = sm + P::OFF_O;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* full = bars;          // TMA -> everyone, per stage
-    uint64_t* empty = bars + 2;     // issuer (commit) -> TMA, per stage
-    uint64_t* uo_full = bars + 4;   // issuer: [U; Q S] complete, per TMEM buffer
-    uint64_t* o_full = bars + 6;    // issuer: P~ U complete, per TMEM buffer
+    uint64_t* empty = bars + 2;     // both issuers (commit) -> TMA, per stage
+    uint64_t* uo_full = bars + 4;   // both issuers: [U; Q S] partials complete, per TMEM buffer
+    uint64_t* o_full = bars + 6;    // issuer B: P~ U complete, per TMEM buffer
     uint64_t* o_read = bars + 8;    // output warps: the buffer's output rows read
-    uint64_t* s_full = bars + 10;   // issuer: state update complete
+    uint64_t* s_full = bars + 10;   // both issuers: state update partials complete
     uint64_t* u_ready = bars + 11;  // U warps: U^ in place
     uint64_t* u2_ready = bars + 12; // U warps: U in place
     uint64_t* s_ready = bars + 13;  // every converter warp: bf16 state written
     uint64_t* os_full = bars + 14;  // output warps: output staging written
     uint64_t* os_empty = bars + 15; // TMA: output staging read by its store
-    uint64_t* drain = bars + 16;    // issuer: every MMA it issued is complete
+    uint64_t* drain = bars + 16;    // [2] issuers: every MMA each issued is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -561,18 +564,18 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-            mbar_init(&uo_full[s], 1);
+            mbar_init(&empty[s], 2);
+            mbar_init(&uo_full[s], 2);
             mbar_init(&o_full[s], 1);
             mbar_init(&o_read[s], kConvWarps / 2);
+            mbar_init(&drain[s], 1);
         }
-        mbar_init(s_full, 1);
+        mbar_init(s_full, 2);
         mbar_init(u_ready, kConvWarps / 2);
         mbar_init(u2_ready, kConvWarps / 2);
         mbar_init(s_ready, kConvWarps);
         mbar_init(os_full, kConvWarps / 2);
         mbar_init(os_empty, 1);
-        mbar_init(drain, 1);
         fence_mbar_init();
     }
     // zero tiles of both stages (rows 64-127 of [T'; Z], rows 0-63 of [Z; P~])
@@ -651,64 +654,84 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad);
         }
         __syncwarp();
-    } else if (warp == kIssuerWarp) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == kIssuerA || warp == kIssuerB) {
+        // ---------------- MMA issuers ----------------
         if (lane == 0) {
+            const bool A = warp == kIssuerA;
             const uint32_t id = idesc_bf16_f32(128, 64, 0, 1);
             const uint32_t ids = idesc_bf16_f32(D, 64, 1, 1);
             const uint64_t ds = sdesc_sw128(smem_u32(sbt), TILE, 1024);
             const uint64_t du = sdesc_sw128(smem_u32(utile), TILE, 1024);
             const uint64_t duh = sdesc_sw128(smem_u32(uhat), TILE, 1024);
-            // X = [T'; 0] V of chunk c: stage c loaded, TMEM buffer c & 1 read out
-            auto tv = [&](int c) {
+            const uint32_t tx = tbase + (A ? P::T_X1 : P::T_X2);
+            const uint32_t tsp = tbase + (A ? P::T_S1 : P::T_S2);
+            // stage c loaded and TMEM buffer c & 1 read out
+            auto ready = [&](int c) {
                 if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) return false;
                 if (c >= 2 && !mbar_wait(&o_read[c & 1], ((c - 2) / 2) & 1, kErrMma)) return false;
+                return true;
+            };
+            // X1 = [T'; 0] V of chunk c
+            auto tv = [&](int c) {
+                if (!ready(c)) return false;
                 tc_fence_after();
                 unsigned char* st = sm + (c % P::STAGES) * P::STAGE;
                 const uint64_t dt = sdesc_sw128(smem_u32(st + P::O_T), 16, 1024);
                 const uint64_t dvv = sdesc_sw128(smem_u32(st + P::O_V), TILE, 1024);
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tbase + P::T_X + (c & 1) * 64, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id,
-                             ks > 0);
+                    mma_bf16(tx + (c & 1) * 64, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id, ks > 0);
                 return true;
             };
-            bool ok = tv(0);
+            bool ok = A ? tv(0) : true;
             for (int c = 0; c < nch && ok; ++c) {
                 const int s = c % P::STAGES;
                 const uint32_t cp = c & 1;
                 unsigned char* st = sm + s * P::STAGE;
+                if (!A && !(ok = ready(c))) break;
                 if (!(ok = mbar_wait(s_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
-                // X += [-W; Q] S
+                // X += [-W; Q] S over this issuer's half of the features
                 const uint64_t dwq = sdesc_sw128(smem_u32(st + P::O_WQ), 16, 1024);
+                const int k0 = A ? 0 : P::KS_HALF;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    mma_bf16(tbase + P::T_X + cp * 64, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4),
-                             ds + ((ks * 2048) >> 4), id, 1u);
+                for (int kk = 0; kk < P::KS_HALF; ++kk) {
+                    const int ks = k0 + kk;
+                    mma_bf16(tx + cp * 64, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4), ds + ((ks * 2048) >> 4),
+                             id, (A || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(&uo_full[cp]);
-                // dS = K^T U^
+                // dS = K^T U^ over this issuer's half of the tokens
                 if (!(ok = mbar_wait(u_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
                 const uint64_t dk = sdesc_sw128(smem_u32(st + P::O_K), TILE, 1024);
+                const int t0 = A ? 0 : 2;
 #pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tbase + P::T_S, dk + ((ks * 2048) >> 4), duh + ((ks * 2048) >> 4), ids, ks > 0);
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int ks = t0 + kk;
+                    mma_bf16(tsp, dk + ((ks * 2048) >> 4), duh + ((ks * 2048) >> 4), ids, kk > 0 ? 1u : 0u);
+                }
                 mma_commit(s_full);
-                // off the chain: the next chunk's [T'; 0] V, then this chunk's P~ U
-                if (c + 1 < nch && !(ok = tv(c + 1))) break;
-                if (!(ok = mbar_wait(u2_ready, c & 1, kErrMma))) break;
-                tc_fence_after();
-                const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
+                if (A) {
+                    // off the chain: the next chunk's [T'; 0] V
+                    mma_commit(&empty[s]);
+                    if (c + 1 < nch) ok = tv(c + 1);
+                } else {
+                    // off the chain: X3 = [0; P~] U once U is in place
+                    if (!(ok = mbar_wait(u2_ready, c & 1, kErrMma))) break;
+                    tc_fence_after();
+                    const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
 #pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tbase + P::T_X3 + cp * 64, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, ks > 0);
-                mma_commit(&o_full[cp]);
-                mma_commit(&empty[s]);
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_bf16(tbase + P::T_X3 + cp * 64, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id,
+                                 ks > 0);
+                    mma_commit(&o_full[cp]);
+                    mma_commit(&empty[s]);
+                }
             }
             // every MMA issued must complete before TMEM is released
-            mma_commit(drain);
-            mbar_wait(drain, 0, kErrMma);
+            mma_commit(&drain[A ? 0 : 1]);
+            mbar_wait(&drain[A ? 0 : 1], 0, kErrMma);
         }
         __syncwarp();
     } else {
@@ -745,15 +768,16 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!mbar_wait(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
             if (cc >= 1 && !mbar_wait(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
             tc_fence_after();
-            float o[16], w[16];
-            ld16(P::T_X + (cc & 1) * 64 + grp * 16, o);
-            ld16(P::T_X3 + (cc & 1) * 64 + grp * 16, w);
+            float o[16], w[16], y[16];
+            ld16(P::T_X1 + (cc & 1) * 64 + grp * 16, o);
+            ld16(P::T_X2 + (cc & 1) * 64 + grp * 16, w);
+            ld16(P::T_X3 + (cc & 1) * 64 + grp * 16, y);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_read[cc & 1]);
 #pragma unroll
-            for (int x = 0; x < 16; ++x) o[x] = fmaf(bt, o[x], w[x]);
+            for (int x = 0; x < 16; ++x) o[x] = fmaf(bt, o[x] + w[x], y[x]);
             store16(ostage, r - 64, o, 1.f);
             fence_async_smem();
             __syncwarp();
@@ -783,9 +807,12 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // U (rows 0-63): U^ = diag(b_C / b) U first, the state update waits for it
                 if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
                 tc_fence_after();
-                float u[16];
-                ld16(P::T_X + cp * 64 + grp * 16, u);
+                float u[16], w[16];
+                ld16(P::T_X1 + cp * 64 + grp * 16, u);
+                ld16(P::T_X2 + cp * 64 + grp * 16, w);
                 tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 16; ++x) u[x] += w[x];
                 store16(uhat, r, u, tokf);
                 fence_async_smem();
                 tc_fence_before();
@@ -804,11 +831,12 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!mbar_wait(s_full, c & 1, kErrMma)) bad = true;
             tc_fence_after();
             {
-                float a[16];
-                ld16(P::T_S + grp * 16, a);
+                float a[16], b[16];
+                ld16(P::T_S1 + grp * 16, a);
+                ld16(P::T_S2 + grp * 16, b);
                 tmem_ld_wait();
 #pragma unroll
-                for (int x = 0; x < 16; ++x) sreg[x] = fmaf(bc, sreg[x], a[x]);
+                for (int x = 0; x < 16; ++x) sreg[x] = fmaf(bc, sreg[x], a[x] + b[x]);
             }
             if (c + 1 < nch) {
                 if (f >= 0) store16(sbt, f, sreg, 1.f);
