@@ -507,8 +507,8 @@ struct ChainPlan {
     static constexpr int KS_HALF = D / 32;                   // K-steps of [-W; Q] S per issuer
 };
 
-constexpr int kConvWarps = 16;                        // converter warps 0-15
-constexpr int kChainThreads = (kConvWarps + 3) * 32;  // + issuer warps 16 and 18, TMA warp 17
+constexpr int kConvWarps = 8;                         // converter warps 0-7
+constexpr int kChainThreads = (kConvWarps + 3) * 32;  // + issuer warps 8 and 10, TMA warp 9
 constexpr int kIssuerA = kConvWarps, kTmaWarp = kConvWarps + 1, kIssuerB = kConvWarps + 2;
 
 // The chain of one (chain, 64 value columns).  Per chunk c with start state S
@@ -521,9 +521,9 @@ constexpr int kIssuerA = kConvWarps, kTmaWarp = kConvWarps + 1, kIssuerB = kConv
 //   converters  U^ (first: the state update waits for it), U;  S <- b_C S + dS and
 //               its bf16 copy;  o = diag(b) Q S + P~ U -> staging.
 // A tcgen05.mma takes tens of cycles to issue, so the two contractions on the
-// chain are split between two issuing threads.  Sixteen converter warps split
-// each phase by rows (TMEM lane quadrant = warp % 4) and 16-column groups
-// (warp / 4), and each warp arrives once on the barrier that ends its part.
+// chain are split between two issuing threads.  The converter warps split each
+// phase by rows (TMEM lane quadrant = warp % 4) and column groups (warp / 4),
+// and each warp arrives once on the barrier that ends its part.
 template <int D>
 __global__ void __launch_bounds__(kChainThreads, 1)
 gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -735,24 +735,35 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         __syncwarp();
     } else {
-        // ---------------- converters (warps 0-15) ----------------
+        // ---------------- converters ----------------
         // Thread (quad, lane) of warp w (quad = w % 4, g = w / 4) owns row
         // r = 32 quad + lane of the M = 128 accumulators, a token of U (quads 0,
         // 1) or of the output (quads 2, 3), and row f of the M = D state
-        // accumulator (f = r for D = 128); g picks 16 of the tile's 64 columns.
+        // accumulator (f = r for D = 128); g picks NG groups of 16 of the tile's
+        // 64 columns.
+        constexpr int NG = 64 / 16 / (kConvWarps / 4);
         const int quad = warp & 3, grp = warp >> 2;
+        const int col0 = grp * NG * 16;
         const int r = quad * 32 + lane;
         const int f = acc_row<D>(quad, lane);
         const bool urow = quad < 2;
         bool bad = false;
-        auto ld16 = [&](uint32_t col, float (&v)[16]) { tmem_ld16(tmem_addr(tbase, quad, col), v); };
-        auto store16 = [&](unsigned char* tile, int row, const float (&v)[16], float w) {
-            const uint4 a = make_uint4(pack_bf16x2(w * v[0], w * v[1]), pack_bf16x2(w * v[2], w * v[3]),
-                                       pack_bf16x2(w * v[4], w * v[5]), pack_bf16x2(w * v[6], w * v[7]));
-            const uint4 b = make_uint4(pack_bf16x2(w * v[8], w * v[9]), pack_bf16x2(w * v[10], w * v[11]),
-                                       pack_bf16x2(w * v[12], w * v[13]), pack_bf16x2(w * v[14], w * v[15]));
-            *reinterpret_cast<uint4*>(tile + sw128_offset(row, grp * 32)) = a;
-            *reinterpret_cast<uint4*>(tile + sw128_offset(row, grp * 32 + 16)) = b;
+        using Cols = float[NG][16];
+        auto ld = [&](uint32_t col, Cols& v) {
+#pragma unroll
+            for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(tbase, quad, col + col0 + 16 * g), v[g]);
+        };
+        auto store = [&](unsigned char* tile, int row, const Cols& v, float w) {
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                const uint4 a = make_uint4(pack_bf16x2(w * v[g][0], w * v[g][1]), pack_bf16x2(w * v[g][2], w * v[g][3]),
+                                           pack_bf16x2(w * v[g][4], w * v[g][5]), pack_bf16x2(w * v[g][6], w * v[g][7]));
+                const uint4 b = make_uint4(pack_bf16x2(w * v[g][8], w * v[g][9]), pack_bf16x2(w * v[g][10], w * v[g][11]),
+                                           pack_bf16x2(w * v[g][12], w * v[g][13]),
+                                           pack_bf16x2(w * v[g][14], w * v[g][15]));
+                *reinterpret_cast<uint4*>(tile + sw128_offset(row, (col0 + 16 * g) * 2)) = a;
+                *reinterpret_cast<uint4*>(tile + sw128_offset(row, (col0 + 16 * g) * 2 + 16)) = b;
+            }
         };
         // per-chunk factors, read from the stage before this warp's arrival that
         // lets the stage be refilled: b_C, and b_t (output rows) or b_C / b_t
@@ -768,33 +779,38 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!mbar_wait(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
             if (cc >= 1 && !mbar_wait(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
             tc_fence_after();
-            float o[16], w[16], y[16];
-            ld16(P::T_X1 + (cc & 1) * 64 + grp * 16, o);
-            ld16(P::T_X2 + (cc & 1) * 64 + grp * 16, w);
-            ld16(P::T_X3 + (cc & 1) * 64 + grp * 16, y);
+            Cols o, w, y;
+            ld(P::T_X1 + (cc & 1) * 64, o);
+            ld(P::T_X2 + (cc & 1) * 64, w);
+            ld(P::T_X3 + (cc & 1) * 64, y);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_read[cc & 1]);
 #pragma unroll
-            for (int x = 0; x < 16; ++x) o[x] = fmaf(bt, o[x] + w[x], y[x]);
-            store16(ostage, r - 64, o, 1.f);
+            for (int g = 0; g < NG; ++g)
+#pragma unroll
+                for (int x = 0; x < 16; ++x) o[g][x] = fmaf(bt, o[g][x] + w[g][x], y[g][x]);
+            store(ostage, r - 64, o, 1.f);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(os_full);
         };
 
         // start state slice S[:, j0:j0+64] in registers and, as bf16, in the B operand
-        float sreg[16];
+        Cols sreg;
         float bc, tokf, bc_next = 1.f, tokf_next = 1.f, bt_prev = 1.f;
         {
-            const float* src = (S0 && f >= 0) ? S0 + ((size_t)chain * D + f) * dv + j0 + grp * 16 : nullptr;
+            const float* src = (S0 && f >= 0) ? S0 + ((size_t)chain * D + f) * dv + j0 + col0 : nullptr;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 t = src ? reinterpret_cast<const float4*>(src)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-                sreg[4 * q] = t.x; sreg[4 * q + 1] = t.y; sreg[4 * q + 2] = t.z; sreg[4 * q + 3] = t.w;
-            }
-            if (f >= 0) store16(sbt, f, sreg, 1.f);
+            for (int g = 0; g < NG; ++g)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 t =
+                        src ? reinterpret_cast<const float4*>(src + 16 * g)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    sreg[g][4 * q] = t.x; sreg[g][4 * q + 1] = t.y; sreg[g][4 * q + 2] = t.z; sreg[g][4 * q + 3] = t.w;
+                }
+            if (f >= 0) store(sbt, f, sreg, 1.f);
             read_factors(0, bc, tokf);
             fence_async_smem();
             __syncwarp();
@@ -807,18 +823,20 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // U (rows 0-63): U^ = diag(b_C / b) U first, the state update waits for it
                 if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
                 tc_fence_after();
-                float u[16], w[16];
-                ld16(P::T_X1 + cp * 64 + grp * 16, u);
-                ld16(P::T_X2 + cp * 64 + grp * 16, w);
+                Cols u, w;
+                ld(P::T_X1 + cp * 64, u);
+                ld(P::T_X2 + cp * 64, w);
                 tmem_ld_wait();
 #pragma unroll
-                for (int x = 0; x < 16; ++x) u[x] += w[x];
-                store16(uhat, r, u, tokf);
+                for (int g = 0; g < NG; ++g)
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) u[g][x] += w[g][x];
+                store(uhat, r, u, tokf);
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(u_ready);
-                store16(utile, r, u, 1.f);
+                store(utile, r, u, 1.f);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(u2_ready);
@@ -831,15 +849,17 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!mbar_wait(s_full, c & 1, kErrMma)) bad = true;
             tc_fence_after();
             {
-                float a[16], b[16];
-                ld16(P::T_S1 + grp * 16, a);
-                ld16(P::T_S2 + grp * 16, b);
+                Cols a, b;
+                ld(P::T_S1, a);
+                ld(P::T_S2, b);
                 tmem_ld_wait();
 #pragma unroll
-                for (int x = 0; x < 16; ++x) sreg[x] = fmaf(bc, sreg[x], a[x] + b[x]);
+                for (int g = 0; g < NG; ++g)
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) sreg[g][x] = fmaf(bc, sreg[g][x], a[g][x] + b[g][x]);
             }
             if (c + 1 < nch) {
-                if (f >= 0) store16(sbt, f, sreg, 1.f);
+                if (f >= 0) store(sbt, f, sreg, 1.f);
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -849,10 +869,13 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 bc = bc_next;
             } else if (f >= 0 && !bad) {
                 // final state slice
-                float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)chain * D + f) * dv + j0 + grp * 16);
+                float* dst = S_out + ((size_t)chain * D + f) * dv + j0 + col0;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    dst[q] = make_float4(sreg[4 * q], sreg[4 * q + 1], sreg[4 * q + 2], sreg[4 * q + 3]);
+                for (int g = 0; g < NG; ++g)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        reinterpret_cast<float4*>(dst + 16 * g)[q] =
+                            make_float4(sreg[g][4 * q], sreg[g][4 * q + 1], sreg[g][4 * q + 2], sreg[g][4 * q + 3]);
             }
         }
         if (!urow && !bad) output_tile(nch - 1, tokf);
