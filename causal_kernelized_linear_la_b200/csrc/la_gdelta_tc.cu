@@ -637,21 +637,21 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             bool ok = true;
             for (int c = 0; c < nch && ok; ++c) {
                 if (c >= 1) {
-                    ok = mbar_wait(os_full, (c - 1) & 1, kErrMma);
+                    ok = mbar_wait_spin(os_full, (c - 1) & 1, kErrMma);
                     if (!ok) break;
                     store(c - 1);
                 }
                 if (c + P::STAGES < nch) {
-                    ok = mbar_wait(&empty[c % P::STAGES], (c / P::STAGES) & 1, kErrMma);
+                    ok = mbar_wait_spin(&empty[c % P::STAGES], (c / P::STAGES) & 1, kErrMma);
                     if (ok) issue(c + P::STAGES);
                     if (ok && c + 2 * P::STAGES < nch) prefetch(c + 2 * P::STAGES);
                 }
             }
-            if (ok && mbar_wait(os_full, (nch - 1) & 1, kErrMma)) store(nch - 1);
+            if (ok && mbar_wait_spin(os_full, (nch - 1) & 1, kErrMma)) store(nch - 1);
             tma_store_wait_all();
             // loads in flight must land before the block exits
             for (int c = max(0, loads - P::STAGES); c < loads; ++c)
-                mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad);
+                mbar_wait_spin(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad);
         }
         __syncwarp();
     } else if (warp == kIssuerA || warp == kIssuerB) {
@@ -667,8 +667,8 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t tsp = tbase + (A ? P::T_S1 : P::T_S2);
             // stage c loaded and TMEM buffer c & 1 read out
             auto ready = [&](int c) {
-                if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) return false;
-                if (c >= 2 && !mbar_wait(&o_read[c & 1], ((c - 2) / 2) & 1, kErrMma)) return false;
+                if (!mbar_wait_spin(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) return false;
+                if (c >= 2 && !mbar_wait_spin(&o_read[c & 1], ((c - 2) / 2) & 1, kErrMma)) return false;
                 return true;
             };
             // X1 = [T'; 0] V of chunk c
@@ -689,7 +689,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t cp = c & 1;
                 unsigned char* st = sm + s * P::STAGE;
                 if (!A && !(ok = ready(c))) break;
-                if (!(ok = mbar_wait(s_ready, c & 1, kErrMma))) break;
+                if (!(ok = mbar_wait_spin(s_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
                 // X += [-W; Q] S over this issuer's half of the features
                 const uint64_t dwq = sdesc_sw128(smem_u32(st + P::O_WQ), 16, 1024);
@@ -702,7 +702,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 mma_commit(&uo_full[cp]);
                 // dS = K^T U^ over this issuer's half of the tokens
-                if (!(ok = mbar_wait(u_ready, c & 1, kErrMma))) break;
+                if (!(ok = mbar_wait_spin(u_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
                 const uint64_t dk = sdesc_sw128(smem_u32(st + P::O_K), TILE, 1024);
                 const int t0 = A ? 0 : 2;
@@ -718,7 +718,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (c + 1 < nch) ok = tv(c + 1);
                 } else {
                     // off the chain: X3 = [0; P~] U once U is in place
-                    if (!(ok = mbar_wait(u2_ready, c & 1, kErrMma))) break;
+                    if (!(ok = mbar_wait_spin(u2_ready, c & 1, kErrMma))) break;
                     tc_fence_after();
                     const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
 #pragma unroll
@@ -731,7 +731,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             // every MMA issued must complete before TMEM is released
             mma_commit(&drain[A ? 0 : 1]);
-            mbar_wait(&drain[A ? 0 : 1], 0, kErrMma);
+            mbar_wait_spin(&drain[A ? 0 : 1], 0, kErrMma);
         }
         __syncwarp();
     } else {
@@ -769,15 +769,15 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // lets the stage be refilled: b_C, and b_t (output rows) or b_C / b_t
         // (U rows) of token r % 64
         auto read_factors = [&](int c, float& bc, float& tf) {
-            if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) bad = true;
+            if (!mbar_wait_spin(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) bad = true;
             const float* vv = reinterpret_cast<const float*>(sm + (c % P::STAGES) * P::STAGE + P::O_VEC);
             bc = vv[C - 1];
             tf = urow ? vv[C + r] : vv[r - 64];
         };
         // output rows of chunk cc (accumulator rows 64-127) -> staging
         auto output_tile = [&](int cc, float bt) {
-            if (!mbar_wait(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
-            if (cc >= 1 && !mbar_wait(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
+            if (!mbar_wait_spin(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
+            if (cc >= 1 && !mbar_wait_spin(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
             tc_fence_after();
             Cols o, w, y;
             ld(P::T_X1 + (cc & 1) * 64, o);
@@ -821,7 +821,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t cp = c & 1;
             if (urow) {
                 // U (rows 0-63): U^ = diag(b_C / b) U first, the state update waits for it
-                if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
+                if (!mbar_wait_spin(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
                 tc_fence_after();
                 Cols u, w;
                 ld(P::T_X1 + cp * 64, u);
@@ -846,7 +846,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (c + 1 < nch) read_factors(c + 1, bc_next, tokf_next);
 
             // state S <- b_C S + dS; its bf16 copy for the next chunk
-            if (!mbar_wait(s_full, c & 1, kErrMma)) bad = true;
+            if (!mbar_wait_spin(s_full, c & 1, kErrMma)) bad = true;
             tc_fence_after();
             {
                 Cols a, b;
