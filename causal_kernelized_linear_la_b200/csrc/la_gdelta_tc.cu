@@ -495,9 +495,9 @@ struct ChainPlan {
     static constexpr int OFF_UH = OFF_U + TILE;               // diag(b_C / b) U bf16 (B of K^T U)
     static constexpr int OFF_O = OFF_UH + TILE;               // output staging
     static constexpr int OFF_BAR = OFF_O + TILE;
-    // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready u2_ready s_ready
-    // ostage_full ostage_empty drain[2]
-    static constexpr int NBAR = 18;
+    // full[2] empty[2] uo_full[2] o_full[2] o_read[2] s_full u_ready s_ready ostage_full ostage_empty
+    // drain[2]
+    static constexpr int NBAR = 17;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
@@ -507,23 +507,17 @@ struct ChainPlan {
     static constexpr int KS_HALF = D / 32;                   // K-steps of [-W; Q] S per issuer
 };
 
-constexpr int kConvWarps = 8;                         // converter warps 0-7
-constexpr int kChainThreads = (kConvWarps + 3) * 32;  // + issuer warps 8 and 10, TMA warp 9
-constexpr int kIssuerA = kConvWarps, kTmaWarp = kConvWarps + 1, kIssuerB = kConvWarps + 2;
+constexpr int kConv = 256;                   // converter threads (warps 0-7)
+constexpr int kChainThreads = kConv + 96;    // + issuer warps 8 and 10, TMA warp 9
 
-// The chain of one (chain, 64 value columns).  Per chunk c with start state S
-// (bf16 copy in shared memory, fp32 master in the converters' registers):
-//   issuer A    X1 = [T'; 0] V (issued a chunk ahead) + [-W; Q]_1 S_1, then, once
-//               U^ = diag(b_C / b) U is in place, dS1 = K_1^T U^_1 (first 32 tokens)
-//   issuer B    X2 = [-W; Q]_2 S_2 (the other feature half), dS2 = K_2^T U^_2, then,
-//               once U is in place, X3 = [0; P~] U
-//   so rows 0-63 of X1 + X2 are U, rows 64-127 are Q S, and dS = dS1 + dS2.
-//   converters  U^ (first: the state update waits for it), U;  S <- b_C S + dS and
-//               its bf16 copy;  o = diag(b) Q S + P~ U -> staging.
-// A tcgen05.mma takes tens of cycles to issue, so the two contractions on the
-// chain are split between two issuing threads.  The converter warps split each
-// phase by rows (TMEM lane quadrant = warp % 4) and column groups (warp / 4),
-// and each warp arrives once on the barrier that ends its part.
+// The chain of one (chain, 64 value columns).  Per chunk c with start state S:
+//   issuers   X1 = [T'; 0] V (one chunk ahead) + [-W; Q]_1 S_1,  X2 = [-W; Q]_2 S_2
+//             (feature halves), so rows 0-63 of X1 + X2 are U and rows 64-127 are Q S;
+//             after U is in place: S1 = K_1^T U^, S2 = K_2^T U^ (token halves),
+//             U^ = diag(b_C / b) U; then X3 = [0; P~] U.
+//   converters  U, U^ to bf16;  S <- b_C S + S1 + S2 (fp32, held in registers), its
+//             bf16 copy for the next chunk;  o = diag(b) Q S + P~ U -> staging.
+// The converters signal with one arrival per warp.
 template <int D>
 __global__ void __launch_bounds__(kChainThreads, 1)
 gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -548,15 +542,15 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t* o_full = bars + 6;    // issuer B: P~ U complete, per TMEM buffer
     uint64_t* o_read = bars + 8;    // output warps: the buffer's output rows read
     uint64_t* s_full = bars + 10;   // both issuers: state update partials complete
-    uint64_t* u_ready = bars + 11;  // U warps: U^ in place
-    uint64_t* u2_ready = bars + 12; // U warps: U in place
-    uint64_t* s_ready = bars + 13;  // every converter warp: bf16 state written
-    uint64_t* os_full = bars + 14;  // output warps: output staging written
-    uint64_t* os_empty = bars + 15; // TMA: output staging read by its store
-    uint64_t* drain = bars + 16;    // [2] issuers: every MMA each issued is complete
+    uint64_t* u_ready = bars + 11;  // U warps: U and U^ in place
+    uint64_t* s_ready = bars + 12;  // every converter warp: bf16 state written
+    uint64_t* os_full = bars + 13;  // output warps: output staging written
+    uint64_t* os_empty = bars + 14; // TMA: output staging read by its store
+    uint64_t* drain = bars + 15;    // [2] issuers: every MMA each issued is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, wg = (warp >> 2) & 1;
     const int ntile = dv / DVT;
     const int chain = blockIdx.x / ntile, j0 = (blockIdx.x % ntile) * DVT;
     const int nch = (N + C - 1) / C;
@@ -567,14 +561,13 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&empty[s], 2);
             mbar_init(&uo_full[s], 2);
             mbar_init(&o_full[s], 1);
-            mbar_init(&o_read[s], kConvWarps / 2);
+            mbar_init(&o_read[s], 4);
             mbar_init(&drain[s], 1);
         }
         mbar_init(s_full, 2);
-        mbar_init(u_ready, kConvWarps / 2);
-        mbar_init(u2_ready, kConvWarps / 2);
-        mbar_init(s_ready, kConvWarps);
-        mbar_init(os_full, kConvWarps / 2);
+        mbar_init(u_ready, 4);
+        mbar_init(s_ready, 8);
+        mbar_init(os_full, 4);
         mbar_init(os_empty, 1);
         fence_mbar_init();
     }
@@ -590,7 +583,7 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tbase = *tmem_slot;
     grid_dependency_wait();   // the prep pass's operands are complete
 
-    if (warp == kTmaWarp) {
+    if (warp == 9) {
         // ---------------- TMA: stage loads and output stores ----------------
         if (lane == 0) {
             const uint64_t pol_once = policy_evict_first();
@@ -637,27 +630,27 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             bool ok = true;
             for (int c = 0; c < nch && ok; ++c) {
                 if (c >= 1) {
-                    ok = mbar_wait_spin(os_full, (c - 1) & 1, kErrMma);
+                    ok = mbar_wait(os_full, (c - 1) & 1, kErrMma);
                     if (!ok) break;
                     store(c - 1);
                 }
                 if (c + P::STAGES < nch) {
-                    ok = mbar_wait_spin(&empty[c % P::STAGES], (c / P::STAGES) & 1, kErrMma);
+                    ok = mbar_wait(&empty[c % P::STAGES], (c / P::STAGES) & 1, kErrMma);
                     if (ok) issue(c + P::STAGES);
                     if (ok && c + 2 * P::STAGES < nch) prefetch(c + 2 * P::STAGES);
                 }
             }
-            if (ok && mbar_wait_spin(os_full, (nch - 1) & 1, kErrMma)) store(nch - 1);
+            if (ok && mbar_wait(os_full, (nch - 1) & 1, kErrMma)) store(nch - 1);
             tma_store_wait_all();
             // loads in flight must land before the block exits
             for (int c = max(0, loads - P::STAGES); c < loads; ++c)
-                mbar_wait_spin(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad);
+                mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad);
         }
         __syncwarp();
-    } else if (warp == kIssuerA || warp == kIssuerB) {
+    } else if (warp == 8 || warp == 10) {
         // ---------------- MMA issuers ----------------
         if (lane == 0) {
-            const bool A = warp == kIssuerA;
+            const bool A = warp == 8;
             const uint32_t id = idesc_bf16_f32(128, 64, 0, 1);
             const uint32_t ids = idesc_bf16_f32(D, 64, 1, 1);
             const uint64_t ds = sdesc_sw128(smem_u32(sbt), TILE, 1024);
@@ -665,14 +658,12 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t duh = sdesc_sw128(smem_u32(uhat), TILE, 1024);
             const uint32_t tx = tbase + (A ? P::T_X1 : P::T_X2);
             const uint32_t tsp = tbase + (A ? P::T_S1 : P::T_S2);
-            // stage c loaded and TMEM buffer c & 1 read out
-            auto ready = [&](int c) {
-                if (!mbar_wait_spin(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) return false;
-                if (c >= 2 && !mbar_wait_spin(&o_read[c & 1], ((c - 2) / 2) & 1, kErrMma)) return false;
+            auto ready = [&](int c) {   // stage c loaded and TMEM buffer c & 1 read out
+                if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) return false;
+                if (c >= 2 && !mbar_wait(&o_read[c & 1], ((c - 2) / 2) & 1, kErrMma)) return false;
                 return true;
             };
-            // X1 = [T'; 0] V of chunk c
-            auto tv = [&](int c) {
+            auto m0 = [&](int c) {
                 if (!ready(c)) return false;
                 tc_fence_after();
                 unsigned char* st = sm + (c % P::STAGES) * P::STAGE;
@@ -683,26 +674,25 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_bf16(tx + (c & 1) * 64, dt + ((ks * 32) >> 4), dvv + ((ks * 2048) >> 4), id, ks > 0);
                 return true;
             };
-            bool ok = A ? tv(0) : true;
+            bool ok = A ? m0(0) : true;
             for (int c = 0; c < nch && ok; ++c) {
                 const int s = c % P::STAGES;
                 const uint32_t cp = c & 1;
                 unsigned char* st = sm + s * P::STAGE;
+                const uint32_t txc = tx + cp * 64;
                 if (!A && !(ok = ready(c))) break;
-                if (!(ok = mbar_wait_spin(s_ready, c & 1, kErrMma))) break;
+                if (!(ok = mbar_wait(s_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
-                // X += [-W; Q] S over this issuer's half of the features
                 const uint64_t dwq = sdesc_sw128(smem_u32(st + P::O_WQ), 16, 1024);
                 const int k0 = A ? 0 : P::KS_HALF;
 #pragma unroll
                 for (int kk = 0; kk < P::KS_HALF; ++kk) {
                     const int ks = k0 + kk;
-                    mma_bf16(tx + cp * 64, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4), ds + ((ks * 2048) >> 4),
-                             id, (A || kk > 0) ? 1u : 0u);
+                    mma_bf16(txc, dwq + (((ks / 4) * 2 * TILE + (ks % 4) * 32) >> 4), ds + ((ks * 2048) >> 4), id,
+                             (A || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&uo_full[cp]);
-                // dS = K^T U^ over this issuer's half of the tokens
-                if (!(ok = mbar_wait_spin(u_ready, c & 1, kErrMma))) break;
+                if (!(ok = mbar_wait(u_ready, c & 1, kErrMma))) break;
                 tc_fence_after();
                 const uint64_t dk = sdesc_sw128(smem_u32(st + P::O_K), TILE, 1024);
                 const int t0 = A ? 0 : 2;
@@ -713,105 +703,90 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 mma_commit(s_full);
                 if (A) {
-                    // off the chain: the next chunk's [T'; 0] V
                     mma_commit(&empty[s]);
-                    if (c + 1 < nch) ok = tv(c + 1);
+                    if (c + 1 < nch) ok = m0(c + 1);
                 } else {
-                    // off the chain: X3 = [0; P~] U once U is in place
-                    if (!(ok = mbar_wait_spin(u2_ready, c & 1, kErrMma))) break;
-                    tc_fence_after();
                     const uint64_t dzp = sdesc_sw128(smem_u32(st + P::O_Z), 16, 1024);
+                    const uint32_t t3 = tbase + P::T_X3 + cp * 64;
 #pragma unroll
                     for (int ks = 0; ks < C / 16; ++ks)
-                        mma_bf16(tbase + P::T_X3 + cp * 64, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id,
-                                 ks > 0);
+                        mma_bf16(t3, dzp + ((ks * 32) >> 4), du + ((ks * 2048) >> 4), id, ks > 0 ? 1u : 0u);
                     mma_commit(&o_full[cp]);
                     mma_commit(&empty[s]);
                 }
             }
             // every MMA issued must complete before TMEM is released
             mma_commit(&drain[A ? 0 : 1]);
-            mbar_wait_spin(&drain[A ? 0 : 1], 0, kErrMma);
+            mbar_wait(&drain[A ? 0 : 1], 0, kErrMma);
         }
         __syncwarp();
     } else {
-        // ---------------- converters ----------------
-        // Thread (quad, lane) of warp w (quad = w % 4, g = w / 4) owns row
-        // r = 32 quad + lane of the M = 128 accumulators, a token of U (quads 0,
-        // 1) or of the output (quads 2, 3), and row f of the M = D state
-        // accumulator (f = r for D = 128); g picks NG groups of 16 of the tile's
-        // 64 columns.
-        constexpr int NG = 64 / 16 / (kConvWarps / 4);
-        const int quad = warp & 3, grp = warp >> 2;
-        const int col0 = grp * NG * 16;
+        // ---------------- converters (warps 0-7) ----------------
+        // Thread (quad, lane) owns row r = 32 quad + lane of the M = 128
+        // accumulators, a token of U (quads 0, 1) or of the output (quads 2, 3),
+        // and row f of the M = D state accumulators (f = r for D = 128); warpgroup
+        // wg owns 32 of the tile's 64 value columns.
         const int r = quad * 32 + lane;
-        const int f = acc_row<D>(quad, lane);
-        const bool urow = quad < 2;
+        const int f = acc_row<D>(quad, lane);   // state row (feature) of this thread, or -1
         bool bad = false;
-        using Cols = float[NG][16];
-        auto ld = [&](uint32_t col, Cols& v) {
-#pragma unroll
-            for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(tbase, quad, col + col0 + 16 * g), v[g]);
+        auto ld32 = [&](uint32_t col, float (&v)[32]) {
+            tmem_ld16(tmem_addr(tbase, quad, col), *reinterpret_cast<float(*)[16]>(v));
+            tmem_ld16(tmem_addr(tbase, quad, col + 16), *reinterpret_cast<float(*)[16]>(v + 16));
         };
-        auto store = [&](unsigned char* tile, int row, const Cols& v, float w) {
+        auto store_row = [&](unsigned char* tile, int row, const float (&v)[32], float w) {
 #pragma unroll
-            for (int g = 0; g < NG; ++g) {
-                const uint4 a = make_uint4(pack_bf16x2(w * v[g][0], w * v[g][1]), pack_bf16x2(w * v[g][2], w * v[g][3]),
-                                           pack_bf16x2(w * v[g][4], w * v[g][5]), pack_bf16x2(w * v[g][6], w * v[g][7]));
-                const uint4 b = make_uint4(pack_bf16x2(w * v[g][8], w * v[g][9]), pack_bf16x2(w * v[g][10], w * v[g][11]),
-                                           pack_bf16x2(w * v[g][12], w * v[g][13]),
-                                           pack_bf16x2(w * v[g][14], w * v[g][15]));
-                *reinterpret_cast<uint4*>(tile + sw128_offset(row, (col0 + 16 * g) * 2)) = a;
-                *reinterpret_cast<uint4*>(tile + sw128_offset(row, (col0 + 16 * g) * 2 + 16)) = b;
-            }
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(tile + sw128_offset(row, wg * 64 + q * 16)) =
+                    make_uint4(pack_bf16x2(w * v[8 * q], w * v[8 * q + 1]), pack_bf16x2(w * v[8 * q + 2], w * v[8 * q + 3]),
+                               pack_bf16x2(w * v[8 * q + 4], w * v[8 * q + 5]),
+                               pack_bf16x2(w * v[8 * q + 6], w * v[8 * q + 7]));
         };
-        // per-chunk factors, read from the stage before this warp's arrival that
-        // lets the stage be refilled: b_C, and b_t (output rows) or b_C / b_t
-        // (U rows) of token r % 64
-        auto read_factors = [&](int c, float& bc, float& tf) {
-            if (!mbar_wait_spin(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) bad = true;
+        // per-chunk factors of this thread, read from the stage before this warp's
+        // arrival that lets the stage be refilled: b_C, and b_t (output rows) or
+        // b_C / b_t (U rows) of token r % 64
+        float bc = 1.f, tokf = 1.f, tokf_prev = 1.f;
+        auto read_factors = [&](int c) {
+            if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) bad = true;
             const float* vv = reinterpret_cast<const float*>(sm + (c % P::STAGES) * P::STAGE + P::O_VEC);
             bc = vv[C - 1];
-            tf = urow ? vv[C + r] : vv[r - 64];
+            tokf = quad < 2 ? vv[C + r] : vv[r - 64];
         };
         // output rows of chunk cc (accumulator rows 64-127) -> staging
         auto output_tile = [&](int cc, float bt) {
-            if (!mbar_wait_spin(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
-            if (cc >= 1 && !mbar_wait_spin(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
+            if (!mbar_wait(&o_full[cc & 1], (cc / 2) & 1, kErrMma)) bad = true;
+            if (cc >= 1 && !mbar_wait(os_empty, (cc - 1) & 1, kErrMma)) bad = true;
             tc_fence_after();
-            Cols o, w, y;
-            ld(P::T_X1 + (cc & 1) * 64, o);
-            ld(P::T_X2 + (cc & 1) * 64, w);
-            ld(P::T_X3 + (cc & 1) * 64, y);
+            float o[32], w[32];
+            const uint32_t col = (cc & 1) * 64 + wg * 32;
+            ld32(P::T_X1 + col, o);
+            ld32(P::T_X2 + col, w);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] += w[x];
+            ld32(P::T_X3 + col, w);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_read[cc & 1]);
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
-#pragma unroll
-                for (int x = 0; x < 16; ++x) o[g][x] = fmaf(bt, o[g][x] + w[g][x], y[g][x]);
-            store(ostage, r - 64, o, 1.f);
+            for (int x = 0; x < 32; ++x) o[x] = fmaf(bt, o[x], w[x]);
+            store_row(ostage, r - 64, o, 1.f);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(os_full);
         };
 
         // start state slice S[:, j0:j0+64] in registers and, as bf16, in the B operand
-        Cols sreg;
-        float bc, tokf, bc_next = 1.f, tokf_next = 1.f, bt_prev = 1.f;
+        float sreg[32];
         {
-            const float* src = (S0 && f >= 0) ? S0 + ((size_t)chain * D + f) * dv + j0 + col0 : nullptr;
+            const float* src = (S0 && f >= 0) ? S0 + ((size_t)chain * D + f) * dv + j0 + wg * 32 : nullptr;
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 t =
-                        src ? reinterpret_cast<const float4*>(src + 16 * g)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    sreg[g][4 * q] = t.x; sreg[g][4 * q + 1] = t.y; sreg[g][4 * q + 2] = t.z; sreg[g][4 * q + 3] = t.w;
-                }
-            if (f >= 0) store(sbt, f, sreg, 1.f);
-            read_factors(0, bc, tokf);
+            for (int q = 0; q < 8; ++q) {
+                const float4 t = src ? reinterpret_cast<const float4*>(src)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+                sreg[4 * q] = t.x; sreg[4 * q + 1] = t.y; sreg[4 * q + 2] = t.z; sreg[4 * q + 3] = t.w;
+            }
+            if (f >= 0) store_row(sbt, f, sreg, 1.f);
+            read_factors(0);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_ready);
@@ -819,66 +794,56 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         for (int c = 0; c < nch && !bad; ++c) {
             const uint32_t cp = c & 1;
-            if (urow) {
-                // U (rows 0-63): U^ = diag(b_C / b) U first, the state update waits for it
-                if (!mbar_wait_spin(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
+            if (quad < 2) {
+                // U (rows 0-63) -> bf16: U for P~ U, diag(b_C / b) U for the state update
+                if (!mbar_wait(&uo_full[cp], (c / 2) & 1, kErrMma)) bad = true;
                 tc_fence_after();
-                Cols u, w;
-                ld(P::T_X1 + cp * 64, u);
-                ld(P::T_X2 + cp * 64, w);
+                float u[32], w[32];
+                ld32(P::T_X1 + cp * 64 + wg * 32, u);
+                ld32(P::T_X2 + cp * 64 + wg * 32, w);
                 tmem_ld_wait();
 #pragma unroll
-                for (int g = 0; g < NG; ++g)
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) u[g][x] += w[g][x];
-                store(uhat, r, u, tokf);
+                for (int x = 0; x < 32; ++x) u[x] += w[x];
+                store_row(utile, r, u, 1.f);
+                store_row(uhat, r, u, tokf);
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(u_ready);
-                store(utile, r, u, 1.f);
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(u2_ready);
             } else if (c >= 1) {
-                output_tile(c - 1, bt_prev);
+                output_tile(c - 1, tokf_prev);
             }
-            if (c + 1 < nch) read_factors(c + 1, bc_next, tokf_next);
 
-            // state S <- b_C S + dS; its bf16 copy for the next chunk
-            if (!mbar_wait_spin(s_full, c & 1, kErrMma)) bad = true;
+            // state S <- b_C S + S1 + S2; its bf16 copy for the next chunk
+            if (!mbar_wait(s_full, c & 1, kErrMma)) bad = true;
             tc_fence_after();
             {
-                Cols a, b;
-                ld(P::T_S1, a);
-                ld(P::T_S2, b);
+                float a[32], b[32];
+                ld32(P::T_S1 + wg * 32, a);
+                ld32(P::T_S2 + wg * 32, b);
                 tmem_ld_wait();
+                if (f >= 0) {
 #pragma unroll
-                for (int g = 0; g < NG; ++g)
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) sreg[g][x] = fmaf(bc, sreg[g][x], a[g][x] + b[g][x]);
+                    for (int x = 0; x < 32; ++x) sreg[x] = fmaf(bc, sreg[x], a[x] + b[x]);
+                }
             }
             if (c + 1 < nch) {
-                if (f >= 0) store(sbt, f, sreg, 1.f);
+                if (f >= 0) store_row(sbt, f, sreg, 1.f);
+                tokf_prev = tokf;
+                read_factors(c + 1);
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_ready);
-                bt_prev = tokf;
-                tokf = tokf_next;
-                bc = bc_next;
             } else if (f >= 0 && !bad) {
                 // final state slice
-                float* dst = S_out + ((size_t)chain * D + f) * dv + j0 + col0;
+                float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)chain * D + f) * dv + j0 + wg * 32);
 #pragma unroll
-                for (int g = 0; g < NG; ++g)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        reinterpret_cast<float4*>(dst + 16 * g)[q] =
-                            make_float4(sreg[g][4 * q], sreg[g][4 * q + 1], sreg[g][4 * q + 2], sreg[g][4 * q + 3]);
+                for (int q = 0; q < 8; ++q)
+                    dst[q] = make_float4(sreg[4 * q], sreg[4 * q + 1], sreg[4 * q + 2], sreg[4 * q + 3]);
             }
         }
-        if (!urow && !bad) output_tile(nch - 1, tokf);
+        if (quad >= 2 && !bad) output_tile(nch - 1, tokf);
     }
     tc_fence_before();
     __syncthreads();

@@ -98,35 +98,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
     return false;
 }
 
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait that polls without suspending the thread, for the short
-// hand-offs of a latency-bound pipeline: a thread suspended in try_wait was
-// measured to resume several hundred cycles after the phase completed.  The
-// same deadline as mbar_wait applies.
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, unsigned int site)
-{
-    if (mbar_test(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1; i < kSpinLimit; ++i) {
-        if (mbar_test(bar, parity)) return true;
-        if ((i & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) break;
-    }
-    atomicCAS(&g_device_error, 0u, site);
-    return false;
-}
-
 // ---- proxy fences ------------------------------------------------------------
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
