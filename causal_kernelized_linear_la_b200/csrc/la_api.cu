@@ -38,7 +38,7 @@ bool state_outputs_alias(const float* S_out, const float* z_out, const float* S0
 }
 
 // Stage events of la_set_stage_events (process-wide; see la.h).
-constexpr int kMaxStageEvents = 8;
+constexpr int kMaxStageEvents = 16;
 cudaEvent_t g_stage_events[kMaxStageEvents];
 int g_stage_count = 0;
 

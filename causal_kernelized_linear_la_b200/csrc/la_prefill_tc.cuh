@@ -32,7 +32,7 @@ bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains, in
 // the per-chunk operands the parallel pass hands to the sequential pass.  A
 // long sequence runs as up to kMaxGdParts parts of len tokens (a multiple of
 // the 64-token chunk) whose passes overlap; a call launches 2 P kernels.
-constexpr int kMaxGdParts = 4;
+constexpr int kMaxGdParts = 8;
 struct GdParts {
     int P = 1;
     int len = 0;

@@ -171,7 +171,7 @@ LA_API size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, con
  * sizes and this cfg (dtype, mode) launches, i.e. how many events
  * la_set_stage_events records for it: 3 for bf16 LA_PLAIN / LA_DECAY (segment
  * summaries, scan, chunk loop); 2 P for bf16 LA_GATED_DELTA, whose sequence
- * runs as P <= 4 parts (each a chunk prep pass and a chain pass; the prep
+ * runs as P <= 8 parts (each a chunk prep pass and a chain pass; the prep
  * pass of part i + 1 overlaps the chain pass of part i); 1 otherwise; 0 when
  * the call launches no kernel (N = 0, nothing to do, or unsupported sizes).
  * Host-only.  Not from the pages: a service for profiling.
@@ -288,14 +288,14 @@ LA_API la_status la_causal_conv(const void* x, const float* weight, const void* 
  * later la_prefill / la_decode_step / la_gated_delta_decode_step /
  * la_causal_conv records
  * events[i] on its cfg->stream right after launching its i-th kernel
- * (i < n; a call launches 1 to 8 kernels, la_prefill_kernel_count gives the
+ * (i < n; a call launches 1 to 16 kernels, la_prefill_kernel_count gives the
  * number for a prefill: bf16 LA_PLAIN/LA_DECAY prefill = segment summaries,
  * scan, chunk loop; bf16 LA_GATED_DELTA prefill = chunk prep and chain per
  * part; every other path, la_causal_conv included, one kernel).  events are cudaEvent_t handles
  * owned by the caller, who must keep them alive while the hook is set; n = 0
  * turns it off.  The setting is process-wide and not thread-safe: set it
  * only while no other thread launches through this library.  Returns
- * LA_ERR_INVALID for n outside 0..8 or a NULL handle.  Not from the pages: a
+ * LA_ERR_INVALID for n outside 0..16 or a NULL handle.  Not from the pages: a
  * service for timing each kernel of a call with CUDA events.
  */
 LA_API la_status la_set_stage_events(void* const* events, int n);
