@@ -4,21 +4,25 @@
 // Method ("What Is Linear Attention?" §4/§5.1; "Efficient attention
 // variants" §5, §7.1 and §8 "chunkwise": parallel inside a chunk, state passed
 // between chunks).  For a chunk of C = 64 tokens with start state (S, z),
-// local positions i, j and lambda = log gamma_h:
-//   P~_ij = [j <= i] gamma^(i-j) phi(q_i).phi(k_j)         (bf16, fp32 products)
-//   o_i   = (sum_j P~_ij v_j + gamma^(i+1) S^T phi(q_i)) /
-//           (sum_j P~_ij     + gamma^(i+1) z.phi(q_i) + eps)
-//   S    <- gamma^n S + K~^T V,  z <- gamma^n z + sum_j K~_j,
-//   K~_j  = gamma^(n-1-j) phi(k_j)   (n valid tokens in the chunk)
-// The causal mask is multiplicative ("Transformers Are RNNs" notes).
+// local positions i, j, lambda = log gamma_h and the chunk's middle m = 32:
+//   Q~_i = gamma^(i-m) phi(q_i),   K~_j = gamma^(m-j) phi(k_j) [j < n]
+//   P~   = [j <= i] (Q~ K~^T)_ij = [j <= i] gamma^(i-j) phi(q_i).phi(k_j)
+//   o_i  = (P~ V + gamma^(i+1) phi(q_i)^T S)_i / (P~ 1 + gamma^(i+1) phi(q_i).z + eps)
+//   S   <- gamma^C S + sum_j gamma^(C-1-j) phi(k_j) v_j^T,  z likewise
+// (n valid tokens; the causal mask is multiplicative, "Transformers Are RNNs"
+// notes).  The state is carried in a scaled frame T = S / kappa, kappa =
+// gamma^(C-1-m), in which the carry reads T <- gamma^C T + K~^T V and the
+// start-state read is Q~ (gamma^C T): the same operands Q~, K~ serve all three
+// products, and no weight exceeds gamma^-32.
 //
-// The products are laid out so every contraction runs on the tensor cores:
-//   MMA1  P    = phi(Q) phi(K)^T      M=C,  N=C,  K=d    (TMEM, M=64 layout)
-//   MMA3  O^T  = S^T phi(Q)^T         M=dv, N=C,  K=d    (start-state read)
-//   MMA2  O^T += V^T P~^T             M=dv, N=C,  K=C    (intra-chunk)
-//   MMA4  S   += K~^T V               M=d,  N=dv, K=C    (state carry, fp32 in TMEM)
-// Putting dv (not the 64 tokens) on the M axis keeps the big products at
-// M = 128 and the output tile in TMEM with one value column per thread.
+// Every contraction runs on the tensor cores, with the normaliser carried as
+// a column of ones appended to V ([V | 1]) and to the state ([T | t_z]):
+//   MMA1  P      = Q~ K~^T                  M=64, N=64,    K=d
+//   MMA3  O      = Q~ [W | w_z],  W = gamma^C T (bf16 copy)   M=64, N=dv+16, K=d
+//   MMA2  O     += P~ [V | 1]               M=64, N=dv+16, K=64
+//   MMA4  [T|t_z] = [W|w_z] + K~^T [V | 1]   M=d,  N=dv+16, K=64  (fp32 in TMEM)
+// so column dv of O is the denominator, and each output row is divided and
+// stored as whole 16-byte pieces.
 //
 // Parallelism across the sequence ("Transformers Are RNNs" notes: the state
 // is a prefix sum, so it can be scanned): each (chain, segment) of L tokens
@@ -27,7 +31,7 @@
 // the final state; kernel C runs the chunk loop of every segment from its
 // true start state.
 //
-// Supported decay range on this path: gamma >= 0.3 (64 |log gamma| <= 80);
+// Supported decay range on this path: 32 |log gamma| <= 73 (gamma >= 0.1);
 // smaller gamma sets the device error word (la_prefill_check reports it).
 #include <cudaTypedefs.h>
 
@@ -45,44 +49,38 @@ using namespace sm100;
 constexpr int C = 64;             // tokens per chunk
 constexpr int kThreads = 512;     // four warpgroups; each phase is split by columns
 constexpr int TILE = C * 64 * 2;  // one 64-row x 128-byte swizzled tile (8 KB)
-// The scaled-frame exponents (decay) stay within +-kFrameLimit in natural-log
-// units, far from the fp32 / bf16 overflow at ~88.
-constexpr float kFrameLimit = 40.f;
 
 // ---------------------------------------------------------------------------
 // Shared-memory plan of the chunk kernel (all tiles 1024-byte aligned).
 template <int D, int DV, bool DECAY>
 struct ChunkPlan {
-    // d = dv = 64: two CTAs share an SM (three stages, 256 TMEM columns, at
-    // most 60 registers a thread), so one CTA's waits hide behind the other's work
+    // d = dv = 64: two CTAs share an SM, so one CTA's waits hide behind the other's work
     static constexpr bool TWO_PER_SM = D == 64 && DV == 64;
-    static constexpr int STAGES = TWO_PER_SM ? (DECAY ? 2 : 3) : (D + DV > 128) ? 3 : 4;
+    static constexpr int NW = TWO_PER_SM ? 8 : 16;        // worker warps
+    static constexpr int THREADS = (NW + 1) * 32;          // + the issuer warp
+    static constexpr int STAGES = 2;
+    static constexpr int NO = DV + 16;                     // accumulator columns of O and T
+    static constexpr int NBLK = DV / 64 + 1;               // 64-column blocks of [V | 1]
+    // stage: Q~ tiles | K~ tiles | V tiles | ones tile (column 0 = 1): [V | 1] is one
+    // MN-major B operand whose 64-column blocks are a tile apart
     static constexpr int QB = C * D * 2, KB = C * D * 2, VB = C * DV * 2;
-    static constexpr int STAGE = QB + KB + VB;
-    static constexpr int OFF_KH = STAGES * STAGE;                 // K^ (frame-weighted phi(K)), decay only
-    static constexpr int OFF_Q32 = OFF_KH + (DECAY ? KB : 0);     // Q^ fp32 [C][D], tf32 operand
-    static constexpr int OFF_P = OFF_Q32 + C * D * 4;             // P~ bf16 [C][C]
-    // The ones-row A operand of the normaliser MMA: only its row 0 (128
-    // bytes) must hold ones; rows 1..63 feed accumulator rows that are never
-    // read, so they overlap the small vectors below and the staging tile.
-    static constexpr int OFF_ONES = OFF_P + C * C * 2;
-    static constexpr int OFF_RDEN = OFF_ONES + 128;               // [C] 1 / denominator
-    static constexpr int OFF_DTAB = OFF_RDEN + C * 4;             // [C] gamma^k
-    static constexpr int OFF_O = OFF_ONES + 1024;                 // output staging bf16 [C][DV]
-    static constexpr int OFF_RSP = OFF_O + C * DV * 2;            // [4][C] row sums of P~ per warpgroup
-    static constexpr int OFF_DINT = OFF_RSP + 4 * C * 4;          // [2][C] Q^ . z per chunk parity
-    static constexpr int OFF_ZS = OFF_DINT + 2 * C * 4;           // [2][D] z at chunk start per parity
-    static constexpr int OFF_BAR = OFF_ZS + 2 * D * 4;
-    static constexpr int NBAR = STAGES + 5;                       // full[S], p, s, o, pt_full, o_free
+    static constexpr int LOAD_BYTES = QB + KB + VB;
+    static constexpr int STAGE = QB + KB + VB + TILE;
+    static constexpr int OFF_W = STAGES * STAGE;           // [W | w_z] bf16, NBLK blocks of D x 64
+    static constexpr int WBLK = D * 128;
+    static constexpr int OFF_P = OFF_W + NBLK * WBLK;      // P~ bf16 [C][C]
+    static constexpr int OFF_O = OFF_P + TILE;             // output staging bf16 [C][DV]
+    static constexpr int OFF_WT = OFF_O + C * DV * 2;      // [2][C] fp32 decay weights of Q~, K~
+    static constexpr int OFF_BAR = OFF_WT + 2 * C * 4;
+    // full[S] empty[S] phi w_ready t_done p_full ptil o_full o_read os_full os_empty drain
+    static constexpr int NBAR = 2 * STAGES + 10;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
-    static constexpr int BYTES = OFF_TMEM + 16 + 1024;            // + alignment slack
-    static_assert(OFF_DTAB + C * 4 <= OFF_O, "vectors overlap the staging tile");
-    static_assert(OFF_ONES + 8 * 1024 <= OFF_RSP, "ones operand must stay inside the plan");
+    static constexpr int BYTES = OFF_TMEM + 16 + 1024;     // + alignment slack
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
-    // TMEM columns: scores, output^T, state^T, normaliser row
-    static constexpr uint32_t T_P = 0, T_O = 64, T_S = 128;
-    static constexpr uint32_t T_Z = TWO_PER_SM ? 192 : 256, T_COLS = TWO_PER_SM ? 256 : 512;
     static_assert(!TWO_PER_SM || 2 * (BYTES + 1024) <= 233472, "two CTAs per SM");
+    // TMEM columns: scores, output (+ denominator), state (+ normaliser)
+    static constexpr uint32_t T_P = 0, T_O = 64, T_T = 64 + NO;
+    static constexpr uint32_t T_COLS = (T_T + NO <= 256) ? 256 : 512;
 };
 
 template <int D, int DV>
@@ -295,411 +293,326 @@ scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float
 // ---------------------------------------------------------------------------
 // Kernel C: the chunk loop of one (chain, segment) from its start state.
 //
-// The state is kept transposed in TMEM (S^T: lane = value index, column =
-// key feature), exactly the layout of the A operand of a tf32 MMA, so the
-// start-state read of every chunk is an MMA straight out of TMEM and the
-// state never passes through the CUDA cores.  The normaliser z is carried as
-// row 0 of a small accumulator fed by a constant "ones row" tile; the
-// denominators (row sums of P~ plus Q^.z) are formed on the CUDA cores.
-//
-// Decay uses a scaled frame: with r the frame's reference position, the
-// stored state is T = gamma^-(c0 - r) S(c0-1) at chunk start c0, key rows are
-// written as K^_t = gamma^-(t+1-r) phi(k_t) and query rows read as
-// Q^_t = gamma^(t+1-r) phi(q_t).  The frame moves (T is rescaled once) only
-// when |lambda| (t - r) would exceed kFrameLimit.
-//
-// Roles: warps 0..15 ("workers") run the epilogues and phi; lane 0 of warp 16
-// ("issuer") issues TMA and every MMA.  Chunk c, from barrier B1:
-//   issuer:  store o(c-1); MMA1 P = phi(Q)phi(K)^T; MMA3 O^T = S^T Q^^T
-//            (tf32, A in TMEM); MMA4 S^T += V^T K^ and MMA4d z += 1^T K^;
-//            prefetch; [wait P~] MMA2 O^T += V^T P~^T; release the staging tile
-//   workers: [P ready] mask/decay -> P~ and its row sums, signal;  phi(c+1)
-//            in place (overlaps the MMA batch);  [state carry done] frame
-//            move, z of c+1, Q^/K^ of c+1 and Q^.z;  [outputs ready] 1/den,
-//            o = O^T/den -> staging tile                              -> B1
+// Roles: worker warps 0..NW-1 do the CUDA-core steps; lane 0 of warp NW (the
+// issuer) issues every TMA copy and every MMA.  Per chunk c:
+//   workers  [t_done(c-1)] W = gamma^C T -> TMEM (decay) and bf16 -> smem;
+//            [p_full(c)]   P~ = causal mask of P -> bf16;
+//            [full(c+1)]   phi, weights of chunk c+1 in place;
+//            [o_full(c)]   o = O / (O[:, dv] + eps) -> staging
+//   issuer   [phi(c)] MMA1;  [w_ready(c), o_read(c-1)] MMA3, MMA4;
+//            [ptil(c)] MMA2;  TMA store of chunk c-1, loads of chunk c+2
+// The state chain of a CTA is t_done(c-1) -> W copy -> MMA3, MMA4 -> t_done(c);
+// everything else overlaps it (and the other CTA on the SM).
 template <int D, int DV, bool DECAY>
-__global__ void __launch_bounds__(kThreads + 32, ChunkPlan<D, DV, DECAY>::TWO_PER_SM ? 2 : 1)
+__global__ void __launch_bounds__(ChunkPlan<D, DV, DECAY>::THREADS, ChunkPlan<D, DV, DECAY>::TWO_PER_SM ? 2 : 1)
 chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
              const float* __restrict__ gamma, const float* __restrict__ ws, int N, int H, int G, int L, float eps)
 {
     using P = ChunkPlan<D, DV, DECAY>;
-    constexpr int NCHK = (D / 8) * C / kThreads;  // 16-byte chunks of a Q (or K) tile per worker thread
-    static_assert(NCHK >= 1 && (D / 8) * C % kThreads == 0, "tile split");
+    constexpr int NW = P::NW;
+    constexpr int NWT = NW * 32;                      // worker threads
+    constexpr int NQ = NW / 4;                        // worker warps per TMEM lane quadrant
     grid_launch_dependents();   // a following call's summary pass may start as this grid drains
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
-    unsigned char* khat = sm + P::OFF_KH;
-    unsigned char* q32 = sm + P::OFF_Q32;
+    unsigned char* wcp = sm + P::OFF_W;
     unsigned char* ptil = sm + P::OFF_P;
-    unsigned char* ones = sm + P::OFF_ONES;
     unsigned char* otil = sm + P::OFF_O;
-    float* rden = reinterpret_cast<float*>(sm + P::OFF_RDEN);
-    float* dtab = reinterpret_cast<float*>(sm + P::OFF_DTAB);
-    float* rsp = reinterpret_cast<float*>(sm + P::OFF_RSP);
-    float* dint = reinterpret_cast<float*>(sm + P::OFF_DINT);
-    float* zs = reinterpret_cast<float*>(sm + P::OFF_ZS);
+    float* wq = reinterpret_cast<float*>(sm + P::OFF_WT);
+    float* wk = wq + C;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
-    uint64_t* bar_p = full + P::STAGES;
-    uint64_t* bar_s = bar_p + 1;
-    uint64_t* bar_o = bar_p + 2;
-    uint64_t* pt_full = bar_p + 3;
-    uint64_t* o_free = bar_p + 4;
+    uint64_t* empty = full + P::STAGES;
+    uint64_t* phi_rdy = empty + P::STAGES;   // workers: Q~, K~ of the chunk in place
+    uint64_t* w_rdy = phi_rdy + 1;           // workers: W copy written (and T rescaled)
+    uint64_t* t_done = phi_rdy + 2;          // MMA3 + MMA4 complete
+    uint64_t* p_full = phi_rdy + 3;          // MMA1 complete
+    uint64_t* ptil_rdy = phi_rdy + 4;        // workers: P~ written
+    uint64_t* o_full = phi_rdy + 5;          // MMA2 complete
+    uint64_t* o_read = phi_rdy + 6;          // workers: O read out
+    uint64_t* os_full = phi_rdy + 7;         // workers: output staging written
+    uint64_t* os_empty = phi_rdy + 8;        // issuer: staging read by its store
+    uint64_t* drain = phi_rdy + 9;           // issuer: every MMA it issued is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, wg = warp >> 2;
-    const bool worker = tid < kThreads;        // warps 0..15: epilogues and phi
-    const bool issuer = tid == kThreads;       // lane 0 of warp 16: TMA and MMA issue
+    const bool worker = warp < NW;
+    const bool issuer = tid == NWT;
+    const int quad = warp & 3, qg = warp >> 2;        // TMEM lane quadrant, column group in it
     const int unit = blockIdx.x;
     const int chain = unit / G, seg = unit % G;
     const int t0 = seg * L, t1 = min(N, t0 + L);
     const int nch = (t1 - t0 + C - 1) / C;
     const float lam = DECAY ? logf(gamma[chain % H]) : 0.f;
     const uint64_t pol_in = policy_evict_first();
-    // One chunk's key weights reach gamma^-C; beyond e^80 they would overflow.
-    if (DECAY && tid == 0 && (float)C * fabsf(lam) > 80.f) atomicCAS(&g_device_error, 0u, (unsigned int)kErrRange);
+    // the scaled frame keeps every weight within gamma^-32
+    if (DECAY && tid == 0 && 32.f * fabsf(lam) > 73.f) atomicCAS(&g_device_error, 0u, (unsigned int)kErrRange);
 
     if (tid == 0) {
-        for (int s = 0; s < P::STAGES + 3; ++s) mbar_init(&full[s], 1);
-        mbar_init(pt_full, kThreads / 32);
-        mbar_init(o_free, 1);
+        for (int s = 0; s < P::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        mbar_init(phi_rdy, NW);
+        mbar_init(w_rdy, NW);
+        mbar_init(t_done, 1);
+        mbar_init(p_full, 1);
+        mbar_init(ptil_rdy, NW);
+        mbar_init(o_full, 1);
+        mbar_init(o_read, NW);
+        mbar_init(os_full, NW);
+        mbar_init(os_empty, 1);
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, P::T_COLS);
-    if (tid < C) dtab[tid] = DECAY ? __expf((float)tid * lam) : 1.f;   // gamma^(i-j)
-    if (tid < 8) {
-        const uint32_t one2 = pack_bf16x2(1.f, 1.f);
-        reinterpret_cast<uint4*>(ones)[tid] = make_uint4(one2, one2, one2, one2);   // row 0 only
+    if (tid < C) {
+        wq[tid] = DECAY ? __expf((float)(tid - C / 2) * lam) : 1.f;
+        wk[tid] = DECAY ? __expf((float)(C / 2 - tid) * lam) : 1.f;
     }
+    // the ones tile of every stage: element (t, 0) = 1, the rest 0
+    for (int s = 0; s < P::STAGES; ++s)
+        for (int e = tid; e < C * 8; e += P::THREADS) {
+            const int row = e / 8, chunk = e % 8;
+            const uint32_t one = chunk == (row & 7) ? 0x3F80u : 0u;   // bf16 1.0 in logical column 0
+            reinterpret_cast<uint4*>(sm + s * P::STAGE + P::QB + P::KB + P::VB)[e] = make_uint4(one, 0u, 0u, 0u);
+        }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    const float gC = DECAY ? __expf((float)C * lam) : 1.f;                 // gamma^C
+    const float rkappa = DECAY ? __expf(-(float)(C - 1 - C / 2) * lam) : 1.f;   // 1 / kappa
 
-    // bookkeeping for the error path (meaningful in the issuer)
-    int loads_issued = 0, commits = 0, commits_o = 0;
-    int ref = 0;  // frame reference position (segment-local)
     auto chunk_len = [&](int c) { return min(C, t1 - (t0 + c * C)); };
-    auto issue = [&](int c) {
-        const int s = c % P::STAGES;
-        unsigned char* st = sm + s * P::STAGE;
-        const int y = t0 + c * C;
-        loads_issued = c + 1;
-        mbar_expect_tx(&full[s], P::STAGE);
-        for (int b = 0; b < D / 64; ++b) tma_load_3d(st + b * TILE, &tm_q, b * 64, y, chain, &full[s], pol_in);
-        for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(st + P::QB + b * TILE, &tm_k, b * 64, y, chain, &full[s], pol_in);
-        for (int b = 0; b < DV / 64; ++b)
-            tma_load_3d(st + P::QB + P::KB + b * TILE, &tm_v, b * 64, y, chain, &full[s], pol_in);
-    };
-    // phi on load, part A: phi(q), phi(k) of chunk c into registers and, as
-    // bf16, back in place (the score MMA operands; K zeroed past the end).
-    float fq[NCHK][8], fk[NCHK][8];
-    auto phi_a = [&](int c) {
-        const int n = chunk_len(c);
-        unsigned char* qt = sm + (c % P::STAGES) * P::STAGE;
-        unsigned char* kt = qt + P::QB;
-#pragma unroll
-        for (int u = 0; u < NCHK; ++u) {
-            const int e = tid + u * kThreads;
-            const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
-            uint4* pq = reinterpret_cast<uint4*>(qt + b * TILE) + rem;
-            uint4* pk = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
-            unpack8(*pq, fq[u]);
-            unpack8(*pk, fk[u]);
-#pragma unroll
-            for (int x = 0; x < 8; x += 2) {
-                const float2 a = phi2_fast(fq[u][x], fq[u][x + 1]);
-                const float2 b = phi2_fast(fk[u][x], fk[u][x + 1]);
-                fq[u][x] = a.x; fq[u][x + 1] = a.y;
-                fk[u][x] = b.x; fk[u][x + 1] = b.y;
-            }
-            *pq = pack8(fq[u], 1.f);
-            *pk = pack8(fk[u], row < n ? 1.f : 0.f);
-        }
-    };
-    // part B: the frame-weighted operands Q^ (fp32, tf32 MMA) and K^ (bf16),
-    // and Q^ . z(c) for the denominators (8 consecutive threads share a row).
-    auto phi_b = [&](int c) {
-        const int n = chunk_len(c);
-        const int c0 = c * C;
-        const float* zc = zs + (c & 1) * D;
-        float qz = 0.f;
-#pragma unroll
-        for (int u = 0; u < NCHK; ++u) {
-            const int e = tid + u * kThreads;
-            const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
-            const int f0 = b * 64 + (((rem % 8) ^ (row & 7)) * 8);   // first feature of this 16-byte chunk
-            const float qw = DECAY ? __expf((float)(c0 + row + 1 - ref) * lam) : 1.f;
-            unsigned char* qrow = q32 + (f0 / 32) * TILE;
-            const int fb = (f0 % 32) * 4;
-            *reinterpret_cast<float4*>(qrow + sw128_offset(row, fb)) =
-                make_float4(qw * fq[u][0], qw * fq[u][1], qw * fq[u][2], qw * fq[u][3]);
-            *reinterpret_cast<float4*>(qrow + sw128_offset(row, fb + 16)) =
-                make_float4(qw * fq[u][4], qw * fq[u][5], qw * fq[u][6], qw * fq[u][7]);
-            const float4 z0 = *reinterpret_cast<const float4*>(zc + f0);
-            const float4 z1 = *reinterpret_cast<const float4*>(zc + f0 + 4);
-            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-#pragma unroll
-            for (int x = 0; x < 8; ++x) qz = fmaf(qw * fq[u][x], zz[x], qz);
-            if (DECAY) {
-                const float kw = row < n ? __expf(-(float)(c0 + row + 1 - ref) * lam) : 0.f;
-                reinterpret_cast<uint4*>(khat + b * TILE)[rem] = pack8(fk[u], kw);
-            }
-        }
-        qz += __shfl_xor_sync(0xffffffffu, qz, 1);
-        qz += __shfl_xor_sync(0xffffffffu, qz, 2);
-        qz += __shfl_xor_sync(0xffffffffu, qz, 4);
-        if ((tid & 7) == 0) dint[(c & 1) * C + tid / 8] = qz;   // row tid/8 for every u
-    };
-    // Move the frame to position c0 (decay): S^T and z row times gamma^(c0 - ref).
-    auto frame_move = [&](int c0) {
-        const float m = __expf((float)(c0 - ref) * lam);
-#pragma unroll
-        for (int gg = 0; gg < D / 64; ++gg) {
-            const int col0 = wg * (D / 4) + gg * 16;
-            float v[16];
-            tmem_ld16(tmem_addr(tbase, quad, P::T_S + col0), v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 16; ++x) v[x] *= m;
-            tmem_st16(tmem_addr(tbase, quad, P::T_S + col0), v);
-            tmem_ld16(tmem_addr(tbase, quad, P::T_Z + col0), v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 16; ++x) v[x] *= m;
-            tmem_st16(tmem_addr(tbase, quad, P::T_Z + col0), v);
-        }
-        tmem_st_wait();
-    };
-    // z at the start of chunk c (row 0 of the normaliser accumulator, lane 0
-    // of quadrant 0) into zs[c & 1]; the caller synchronises the workers.
-    auto z_to_smem = [&](int c) {
-        if (quad == 0) {
-#pragma unroll
-            for (int gg = 0; gg < D / 64; ++gg) {
-                const int col0 = wg * (D / 4) + gg * 16;
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, 0, P::T_Z + col0), v);
-                tmem_ld_wait();
-                if (lane == 0) {
-                    float4* dst = reinterpret_cast<float4*>(zs + (c & 1) * D + col0);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-                }
-            }
-        }
-    };
-    auto needs_move = [&](int c) {
-        if (!DECAY) return false;
-        return (float)(c * C + C - ref) * fabsf(lam) > kFrameLimit;
-    };
-
-    if (issuer)
-        for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
-
-    // Start state, transposed into TMEM: S^T[j][f] = S[f][j]; z as row 0 of
-    // the normaliser accumulator (other rows zero).
-    if (worker) {
-        grid_dependency_wait();   // start states from the scan
-        const float* slot = ws + (size_t)unit * (D * DV + D);
-        const int j = acc_row<DV>(quad, lane);
-#pragma unroll
-        for (int gg = 0; gg < D / 64; ++gg) {
-            const int col0 = wg * (D / 4) + gg * 16;
-            float v[16];
-#pragma unroll
-            for (int x = 0; x < 16; ++x) v[x] = j >= 0 ? slot[(size_t)(col0 + x) * DV + j] : 0.f;
-            tmem_st16(tmem_addr(tbase, quad, P::T_S + col0), v);
-#pragma unroll
-            for (int x = 0; x < 16; ++x) v[x] = (quad == 0 && lane == 0) ? slot[D * DV + col0 + x] : 0.f;
-            tmem_st16(tmem_addr(tbase, quad, P::T_Z + col0), v);
-        }
-        tmem_st_wait();
-        if (tid < D) zs[tid] = slot[D * DV + tid];
-        named_bar(5, kThreads);
-    }
     bool bad = false;
-    if (!mbar_wait(&full[0], 0, kErrTmaLoad)) bad = true;
-    if (!bad && worker) {
-        phi_a(0);
-        phi_b(0);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    if (__syncthreads_or(bad)) bad = true;
 
-    for (int c = 0; c < nch && !bad; ++c) {
-        const int s = c % P::STAGES;
-        const uint32_t cp = c & 1;
-        unsigned char* qt = sm + s * P::STAGE;
-        unsigned char* kt = qt + P::QB;
-        unsigned char* vt = kt + P::KB;
-        unsigned char* kh = DECAY ? khat : kt;
-
-        if (issuer) {
+    if (issuer) {
+        // ---------------- issuer: TMA and MMA ----------------
+        int loads = 0;
+        auto issue = [&](int c) {
+            const int s = c % P::STAGES;
+            unsigned char* st = sm + s * P::STAGE;
+            const int y = t0 + c * C;
+            mbar_expect_tx(&full[s], P::LOAD_BYTES);
+            for (int b = 0; b < D / 64; ++b) tma_load_3d(st + b * TILE, &tm_q, b * 64, y, chain, &full[s], pol_in);
+            for (int b = 0; b < D / 64; ++b)
+                tma_load_3d(st + P::QB + b * TILE, &tm_k, b * 64, y, chain, &full[s], pol_in);
+            for (int b = 0; b < DV / 64; ++b)
+                tma_load_3d(st + P::QB + P::KB + b * TILE, &tm_v, b * 64, y, chain, &full[s], pol_in);
+            loads = c + 1;
+        };
+        for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
+        const uint32_t id1 = idesc_bf16_f32(64, 64, 0, 0);
+        const uint32_t ido = idesc_bf16_f32(64, P::NO, 0, 1);
+        const uint32_t idt = idesc_bf16_f32(D, P::NO, 1, 1);
+        const uint64_t dw = sdesc_sw128(smem_u32(wcp), P::WBLK, 1024);
+        const uint64_t dp = sdesc_sw128(smem_u32(ptil), 16, 1024);
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % P::STAGES;
+            const uint32_t cp = c & 1;
+            unsigned char* st = sm + s * P::STAGE;
+            const uint64_t dq = sdesc_sw128(smem_u32(st), 16, 1024);                 // Q~, K-major
+            const uint64_t dk = sdesc_sw128(smem_u32(st + P::QB), 16, 1024);         // K~, K-major
+            const uint64_t dkm = sdesc_sw128(smem_u32(st + P::QB), TILE, 1024);      // K~^T, MN-major
+            const uint64_t dvb = sdesc_sw128(smem_u32(st + P::QB + P::KB), TILE, 1024);   // [V | 1]
+            // MMA1: P = Q~ K~^T (P of the previous chunk was read before its P~ was signalled)
+            if (!mbar_wait(phi_rdy, cp, kErrMma)) { bad = true; break; }
             tc_fence_after();
-            if (c >= 1) {
-                for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (c - 1) * C, chain);
-                tma_store_commit();
-            }
-            const uint64_t dq = sdesc_sw128(smem_u32(qt), 16, 1024);      // K-major tiles
-            const uint64_t dk = sdesc_sw128(smem_u32(kt), 16, 1024);
-            const uint64_t dq32 = sdesc_sw128(smem_u32(q32), 16, 1024);
-            const uint64_t dones = sdesc_sw128(smem_u32(ones), 16, 1024);
-            const uint64_t dp = sdesc_sw128(smem_u32(ptil), 16, 1024);
-            const uint64_t dv_mn = sdesc_sw128(smem_u32(vt), TILE, 1024);  // MN-major tiles
-            const uint64_t dkh_mn = sdesc_sw128(smem_u32(kh), TILE, 1024);
-            const uint32_t id1 = idesc_bf16_f32(64, 64, 0, 0);
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
                 const uint32_t off = ((ks / 4) * TILE + (ks % 4) * 32) >> 4;
                 mma_bf16(tbase + P::T_P, dq + off, dk + off, id1, ks > 0);
             }
-            mma_commit(bar_p);
-            // start-state read, tf32 with S^T from TMEM (before MMA4 updates it)
-            const uint32_t id3 = idesc_tf32_f32(DV, 64, 0, 0);
-#pragma unroll
-            for (int ks = 0; ks < D / 8; ++ks) {
-                const uint64_t b = dq32 + (((ks / 4) * TILE + (ks % 4) * 32) >> 4);
-                mma_tf32_ts(tbase + P::T_O, tbase + P::T_S + ks * 8, b, id3, ks > 0);
-            }
-            // state carry
-            const uint32_t id4 = idesc_bf16_f32(DV, D, 1, 1);
-            const uint32_t id4d = idesc_bf16_f32(64, D, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                const uint64_t bk = dkh_mn + ((ks * 2048) >> 4);
-                mma_bf16(tbase + P::T_S, dv_mn + ((ks * 2048) >> 4), bk, id4, 1u);
-                mma_bf16(tbase + P::T_Z, dones + ((ks * 32) >> 4), bk, id4d, 1u);
-            }
-            mma_commit(bar_s);
-            commits = c + 1;
-            if (c >= 1 && c - 1 + P::STAGES < nch) issue(c - 1 + P::STAGES);
-            // intra-chunk values once the workers have written P~
-            if (!mbar_wait(pt_full, cp, kErrMma)) bad = true;
+            mma_commit(p_full);
+            // MMA3: O = Q~ [W | w_z];  MMA4: T = [W | w_z] (already in TMEM) + K~^T [V | 1]
+            if (!mbar_wait(w_rdy, cp, kErrMma)) { bad = true; break; }
+            if (c >= 1 && !mbar_wait(o_read, (c - 1) & 1, kErrMma)) { bad = true; break; }
             tc_fence_after();
-            const uint32_t id2 = idesc_bf16_f32(DV, 64, 1, 0);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t off = ((ks / 4) * TILE + (ks % 4) * 32) >> 4;
+                mma_bf16(tbase + P::T_O, dq + off, dw + ((ks * 2048) >> 4), ido, ks > 0);
+            }
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks)
-                mma_bf16(tbase + P::T_O, dv_mn + ((ks * 2048) >> 4), dp + ((ks * 32) >> 4), id2, 1u);
-            mma_commit(bar_o);
-            commits_o = c + 1;
-            tma_store_wait_read();   // the staging tile may be rewritten
-            mbar_arrive(o_free);
-        }
-
-        if (worker) {
-            // scores -> P~: rows i (M=64 layout), columns split by warpgroup
-            if (!mbar_wait(bar_p, cp, kErrMma)) bad = true;
+                mma_bf16(tbase + P::T_T, dkm + ((ks * 2048) >> 4), dvb + ((ks * 2048) >> 4), idt, 1u);
+            mma_commit(t_done);
+            // MMA2: O += P~ [V | 1]
+            if (!mbar_wait(ptil_rdy, cp, kErrMma)) { bad = true; break; }
             tc_fence_after();
-            {
-                const int i = acc_row<64>(quad, lane);
+#pragma unroll
+            for (int ks = 0; ks < C / 16; ++ks)
+                mma_bf16(tbase + P::T_O, dp + ((ks * 32) >> 4), dvb + ((ks * 2048) >> 4), ido, 1u);
+            mma_commit(o_full);
+            mma_commit(&empty[s]);
+            // output of the previous chunk, then the loads of chunk c + STAGES
+            if (c >= 1) {
+                if (!mbar_wait(os_full, (c - 1) & 1, kErrMma)) { bad = true; break; }
+                fence_async_smem();
+                for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (c - 1) * C, chain);
+                tma_store_commit();
+                tma_store_wait_read();
+                mbar_arrive(os_empty);
+            }
+            if (c + P::STAGES < nch) {
+                if (!mbar_wait(&empty[s], (c / P::STAGES) & 1, kErrMma)) { bad = true; break; }
+                issue(c + P::STAGES);
+            }
+        }
+        if (!bad && nch > 0 && mbar_wait(os_full, (nch - 1) & 1, kErrMma)) {
+            for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (nch - 1) * C, chain);
+            tma_store_commit();
+        }
+        tma_store_wait_all();
+        // leave no copy or MMA in flight before TMEM is released
+        for (int cc = max(0, loads - P::STAGES); cc < loads; ++cc)
+            mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
+        mma_commit(drain);
+        mbar_wait(drain, 0, kErrMma);
+    } else if (worker) {
+        // ---------------- workers ----------------
+        // phi of chunk c in place: Q~ = w_q phi(q), K~ = w_k phi(k) [t < n]
+        auto phi = [&](int c) {
+            const int n = chunk_len(c);
+            unsigned char* qt = sm + (c % P::STAGES) * P::STAGE;
+            unsigned char* kt = qt + P::QB;
+            for (int e = tid; e < (D / 8) * C; e += NWT) {
+                const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
+                uint4* pq = reinterpret_cast<uint4*>(qt + b * TILE) + rem;
+                uint4* pk = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
+                float fq[8], fk[8];
+                unpack8(*pq, fq);
+                unpack8(*pk, fk);
+#pragma unroll
+                for (int x = 0; x < 8; x += 2) {
+                    const float2 a = phi2_fast(fq[x], fq[x + 1]);
+                    const float2 g = phi2_fast(fk[x], fk[x + 1]);
+                    fq[x] = a.x; fq[x + 1] = a.y;
+                    fk[x] = g.x; fk[x + 1] = g.y;
+                }
+                *pq = pack8(fq, wq[row]);
+                *pk = pack8(fk, row < n ? wk[row] : 0.f);
+            }
+        };
+        // T0 = S / kappa: the segment's start state (from the scan), normaliser as column dv
+        {
+            grid_dependency_wait();
+            const float* slot = ws + (size_t)unit * (D * DV + D);
+            const int f = acc_row<D>(quad, lane);
+            for (int g = qg; g < P::NO / 16; g += NQ) {
                 float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_P + wg * 16), v);
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    const int j = g * 16 + x;
+                    float t = 0.f;
+                    if (f >= 0) t = j < DV ? slot[(size_t)f * DV + j] : (j == DV ? slot[D * DV + f] : 0.f);
+                    v[x] = t * rkappa;
+                }
+                tmem_st16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
+            }
+            tmem_st_wait();
+        }
+        if (!mbar_wait(&full[0], 0, kErrTmaLoad)) bad = true;
+        if (!bad) phi(0);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(phi_rdy);
+
+        const int fr = acc_row<D>(quad, lane);      // state row of this thread (M = D accumulator)
+        const int ir = acc_row<64>(quad, lane);     // score / output row (M = 64 accumulators)
+        for (int c = 0; c < nch && !bad; ++c) {
+            const uint32_t cp = c & 1;
+            // W = gamma^C T: back into TMEM (the carry adds to it) and as the bf16 B operand
+            if (c >= 1 && !mbar_wait(t_done, (c - 1) & 1, kErrMma)) bad = true;
+            tc_fence_after();
+            for (int g = qg; g < P::NO / 16; g += NQ) {
+                float v[16];
+                tmem_ld16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
                 tmem_ld_wait();
-                if (i >= 0) {
+                if (DECAY) {
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) v[x] *= gC;
+                    tmem_st16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
+                }
+                if (fr >= 0) {
+                    unsigned char* blk = wcp + (g / 4) * P::WBLK;
+                    const int byte0 = (g % 4) * 32;
+                    *reinterpret_cast<uint4*>(blk + sw128_offset(fr, byte0)) =
+                        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                   pack_bf16x2(v[6], v[7]));
+                    *reinterpret_cast<uint4*>(blk + sw128_offset(fr, byte0 + 16)) =
+                        make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                                   pack_bf16x2(v[14], v[15]));
+                }
+            }
+            if (DECAY) tmem_st_wait();
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(w_rdy);
+
+            // P~ = causal mask of P (rows i, 64 / NQ columns per warp); the previous
+            // chunk's MMA2 has read P~ (its output was waited for)
+            if (!mbar_wait(p_full, cp, kErrMma)) bad = true;
+            tc_fence_after();
+            for (int g = qg; g < 4; g += NQ) {
+                float v[16];
+                tmem_ld16(tmem_addr(tbase, quad, P::T_P + g * 16), v);
+                tmem_ld_wait();
+                if (ir >= 0) {
                     uint32_t pk[8];
-                    float rs = 0.f;
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
-                        const int j0 = wg * 16 + 2 * h;
-                        const float a = j0 <= i ? (DECAY ? v[2 * h] * dtab[i - j0] : v[2 * h]) : 0.f;
-                        const float b = j0 + 1 <= i ? (DECAY ? v[2 * h + 1] * dtab[i - j0 - 1] : v[2 * h + 1]) : 0.f;
-                        pk[h] = pack_bf16x2(a, b);
-                        const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[h]));
-                        rs += r.x + r.y;   // the row sum of exactly the values the MMA uses
+                        const int j = g * 16 + 2 * h;
+                        pk[h] = pack_bf16x2(j <= ir ? v[2 * h] : 0.f, j + 1 <= ir ? v[2 * h + 1] : 0.f);
                     }
-                    rsp[wg * C + i] = rs;
-                    *reinterpret_cast<uint4*>(ptil + sw128_offset(i, wg * 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4*>(ptil + sw128_offset(i, wg * 32 + 16)) =
+                    *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32 + 16)) =
                         make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             }
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(pt_full);
+            if (lane == 0) mbar_arrive(ptil_rdy);
 
-            // phi of the next chunk, overlapping the MMA batch of this one
-            const bool more = c + 1 < nch;
-            const bool move = more && needs_move(c + 1);
-            if (more) {
+            // phi of the next chunk (its stage landed while this one computed)
+            if (c + 1 < nch) {
                 if (!mbar_wait(&full[(c + 1) % P::STAGES], ((c + 1) / P::STAGES) & 1, kErrTmaLoad)) bad = true;
-                else phi_a(c + 1);
-            }
-            // the state carry (and its reads of Q^ / K^) must be complete
-            if (!mbar_wait(bar_s, cp, kErrMma)) bad = true;
-            tc_fence_after();
-            if (move) {
-                frame_move((c + 1) * C);
-                ref = (c + 1) * C;
-            }
-            if (more) {
-                z_to_smem(c + 1);
-                named_bar(5, kThreads);   // z(c+1) and every row sum of P~(c) are in smem
-                phi_b(c + 1);
-            } else {
-                named_bar(5, kThreads);
+                else phi(c + 1);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(phi_rdy);
             }
 
-            // denominators: row 0 of the normaliser accumulator (lane 0, quadrant 0)
-            if (!mbar_wait(bar_o, cp, kErrMma)) bad = true;
+            // output rows: o = O[:, :dv] / (O[:, dv] + eps) -> staging
+            if (!mbar_wait(o_full, cp, kErrMma)) bad = true;
             tc_fence_after();
-            if (quad == 0 && lane < 16) {
-                const int i = wg * 16 + lane;
-                const float den = rsp[i] + rsp[C + i] + rsp[2 * C + i] + rsp[3 * C + i] + dint[cp * C + i];
-                rden[i] = __frcp_rn(den + eps);
-            }
-            named_bar(1 + wg, 128);   // this warpgroup's 16 denominators are in smem
-            if (!mbar_wait(o_free, cp, kErrMma)) bad = true;
-            // outputs o_i = O^T[:, i] / den_i -> staging tile (one value column per thread)
-            {
-                const int j = acc_row<DV>(quad, lane);
-                float v[16], r[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_O + wg * 16), v);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 t = reinterpret_cast<const float4*>(rden + wg * 16)[q4];
-                    r[4 * q4] = t.x; r[4 * q4 + 1] = t.y; r[4 * q4 + 2] = t.z; r[4 * q4 + 3] = t.w;
-                }
+            float den[16];
+            tmem_ld16(tmem_addr(tbase, quad, P::T_O + DV), den);
+            tmem_ld_wait();
+            const float rden = __frcp_rn(den[0] + eps);
+            if (c >= 1 && !mbar_wait(os_empty, (c - 1) & 1, kErrMma)) bad = true;
+            for (int g = qg; g < DV / 16; g += NQ) {
+                float v[16];
+                tmem_ld16(tmem_addr(tbase, quad, P::T_O + g * 16), v);
                 tmem_ld_wait();
-                if (j >= 0) {
-                    // element (i, j) of the swizzled staging tile: 16-byte chunk
-                    // (j % 64) / 8 of row i, XOR (i % 8); i % 8 == x % 8 here
-                    unsigned char* base = otil + (j / 64) * TILE + (j % 8) * 2;
-                    const int cj = (j % 64) >> 3;
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const int i = wg * 16 + x;
-                        *reinterpret_cast<__nv_bfloat16*>(base + i * 128 + ((cj ^ (x & 7)) << 4)) =
-                            __float2bfloat16_rn(v[x] * r[x]);
-                    }
+                if (ir >= 0) {
+                    unsigned char* blk = otil + (g / 4) * TILE;
+                    const int byte0 = (g % 4) * 32;
+                    *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0)) =
+                        make_uint4(pack_bf16x2(v[0] * rden, v[1] * rden), pack_bf16x2(v[2] * rden, v[3] * rden),
+                                   pack_bf16x2(v[4] * rden, v[5] * rden), pack_bf16x2(v[6] * rden, v[7] * rden));
+                    *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0 + 16)) =
+                        make_uint4(pack_bf16x2(v[8] * rden, v[9] * rden), pack_bf16x2(v[10] * rden, v[11] * rden),
+                                   pack_bf16x2(v[12] * rden, v[13] * rden), pack_bf16x2(v[14] * rden, v[15] * rden));
                 }
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(bad)) { bad = true; break; }                         // B1
-    }
-    if (issuer) {
-        if (!bad && nch > 0) {
-            tc_fence_after();
-            for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (nch - 1) * C, chain);
-            tma_store_commit();
-        }
-        tma_store_wait_all();
-        if (bad) {
-            // Leave no copy or MMA in flight before releasing TMEM and exiting:
-            // only the last STAGES loads can still be in flight.
-            for (int cc = max(0, loads_issued - P::STAGES); cc < loads_issued; ++cc)
-                mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
-            if (commits > 0) {
-                const uint32_t last = (commits - 1) & 1;
-                mbar_wait(bar_p, last, kErrMma);
-                mbar_wait(bar_s, last, kErrMma);
-                if (commits_o > 0) mbar_wait(bar_o, (commits_o - 1) & 1, kErrMma);
+            tc_fence_before();
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(o_read);
+                mbar_arrive(os_full);
             }
         }
     }
@@ -799,7 +712,7 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     e = cudaFuncSetAttribute(kc, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     lc.gridDim = dim3(units);
-    lc.blockDim = dim3(kThreads + 32);
+    lc.blockDim = dim3(ChunkPlan<D, DV, DECAY>::THREADS);
     lc.dynamicSmemBytes = sc;
     e = cudaLaunchKernelEx(&lc, kc, mq, mk, mv, mo, a.gamma, (const float*)ws, a.N, a.H, sg.G, sg.L, a.eps);
     if (e != cudaSuccess) return e;

@@ -89,7 +89,10 @@ typedef struct {
  * ("Efficient attention variants" §8).
  *
  *   q, k, v          inputs, layouts above, element type cfg->dtype.
- *   gamma_or_alpha   LA_PLAIN: must be NULL.  LA_DECAY: gamma [H], each in (0,1].
+ *   gamma_or_alpha   LA_PLAIN: must be NULL.  LA_DECAY: gamma [H], each in (0,1]
+ *                    (bf16 inputs: each >= 0.1, the range of the tensor-core
+ *                    path's scaled frame; a smaller gamma is reported as
+ *                    LA_ERR_UNSUPPORTED by la_prefill_check).
  *                    LA_GATED_DELTA: alpha [B,H,N], each in (0,1].
  *                    LA_GLA: alpha [B,H,N,d], each in (0,1]: the per-key-channel
  *                    gate ("Efficient attention variants" §7.2),

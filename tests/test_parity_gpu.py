@@ -69,6 +69,30 @@ def test_kernelized_bf16_large_inputs(mode):
     _check(inputs.make_kernelized(1, 4, 700, 128, 128, dtype="bf16", mode=mode, scale=4.0, seed=1100))
 
 
+@pytest.mark.parametrize("gam", [0.2, 0.1])
+def test_decay_bf16_small_gamma(gam):
+    """A fast decay (each token forgotten within a few steps) on the tensor-core
+    path: every element against the oracle."""
+    p = inputs.make_kernelized(1, 3, 300, 128, 128, dtype="bf16", mode="decay", seed=1200)
+    p.gamma = np.full(p.H, gam, np.float32)
+    _check(p)
+
+
+def test_decay_bf16_below_range_is_reported():
+    """gamma below 0.1 is outside the bf16 tensor-core path's range: the call
+    is reported as unsupported by la_prefill_check (no fault, no hang)."""
+    import causal_kernelized_linear_la_b200 as la
+    p = inputs.make_kernelized(1, 2, 200, 64, 64, dtype="bf16", mode="decay", seed=1201)
+    p.gamma = np.full(p.H, 0.05, np.float32)
+    import torch
+    q, k, v = H.device_inputs(p)
+    la.la_prefill(q, k, v, mode="decay", gamma=H.dev(p.gamma, torch))
+    with pytest.raises(la.LaError) as ei:
+        la.la_prefill_check()
+    assert ei.value.code == la.LA_ERR_UNSUPPORTED
+    la.la_prefill_check()   # reading the error cleared it
+
+
 def test_gated_delta_f32_small():
     _check(inputs.make_gated_delta(1, 2, 190, 64, 64, dtype="f32", seed=700))
 
