@@ -379,7 +379,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    const float gC = DECAY ? __expf((float)C * lam) : 1.f;                 // gamma^C
+    // gamma^C as two factors gamma^(C/2): gamma^C itself is below the fp32
+    // range for gamma < 0.25, while gamma^C T is not
+    const float gH = DECAY ? __expf((float)(C / 2) * lam) : 1.f;
     const float rkappa = DECAY ? __expf(-(float)(C - 1 - C / 2) * lam) : 1.f;   // 1 / kappa
 
     auto chunk_len = [&](int c) { return min(C, t1 - (t0 + c * C)); };
@@ -530,7 +532,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tmem_ld_wait();
                 if (DECAY) {
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) v[x] *= gC;
+                    for (int x = 0; x < 16; ++x) v[x] = (v[x] * gH) * gH;
                     tmem_st16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
                 }
                 if (fr >= 0) {
