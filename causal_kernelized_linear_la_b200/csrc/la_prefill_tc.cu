@@ -31,7 +31,7 @@
 // the final state; kernel C runs the chunk loop of every segment from its
 // true start state.
 //
-// Supported decay range on this path: 32 |log gamma| <= 73 (gamma >= 0.1);
+// Supported decay range on this path: 32 |log gamma| <= 73.7 (gamma >= 0.1);
 // smaller gamma sets the device error word (la_prefill_check reports it).
 #include <cudaTypedefs.h>
 
@@ -346,7 +346,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const float lam = DECAY ? logf(gamma[chain % H]) : 0.f;
     const uint64_t pol_in = policy_evict_first();
     // the scaled frame keeps every weight within gamma^-32
-    if (DECAY && tid == 0 && 32.f * fabsf(lam) > 73.f) atomicCAS(&g_device_error, 0u, (unsigned int)kErrRange);
+    if (DECAY && tid == 0 && 32.f * fabsf(lam) > 73.7f) atomicCAS(&g_device_error, 0u, (unsigned int)kErrRange);
 
     if (tid == 0) {
         for (int s = 0; s < P::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
