@@ -538,7 +538,7 @@ def call_kernels(p) -> list:
     import causal_kernelized_linear_la_b200 as la
     n = la.la_prefill_kernel_count(p.B, p.H, p.N, p.d, p.dv, p.dtype, p.mode)
     if p.mode == "gla":
-        names = ["gla_token_simt"]
+        names = ["gla_summary_kernel", "gla_scan_kernel", "gla_chunk_kernel"] if p.dtype == "bf16" else ["gla_token_simt"]
     elif p.dtype == "bf16" and p.mode in ("plain", "decay"):
         names = ["summary_kernel", "scan_kernel", "chunk_kernel"]
     elif p.dtype == "bf16":

@@ -135,7 +135,10 @@ size_t varlen_slice(size_t bytes) { return (bytes + 255) / 256 * 256; }
 la_status run_prefill(const PrefillArgs& a)
 {
     if (a.N == 0) return write_start_state(a);
-    if (a.mode == LA_GLA) return from_cuda(launch_prefill_simt_gla(a));
+    if (a.mode == LA_GLA) {
+        if (a.dtype == LA_BF16) return from_cuda(launch_prefill_tc_gla(a, tc_segments(a.B, a.H, a.N, a.d, a.dv)));
+        return from_cuda(launch_prefill_simt_gla(a));
+    }
     if (a.mode == LA_GATED_DELTA) {
         if (a.dtype == LA_BF16) return from_cuda(launch_prefill_tc_gated_delta(a));
         return from_cuda(launch_prefill_simt_gated_delta(a));
@@ -172,6 +175,7 @@ size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, const la_c
 {
     if (!cfg || B <= 0 || H <= 0 || N <= 0 || !la::head_ok(d) || !la::head_ok(dv)) return 0;
     if (la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return la::tc_workspace_bytes(B, H, N, d, dv);
+    if (cfg->dtype == LA_BF16 && cfg->mode == LA_GLA) return la::tc_workspace_bytes(B, H, N, d, dv);
     if (cfg->dtype == LA_BF16 && cfg->mode == LA_GATED_DELTA) return la::gd_workspace_bytes(B, H, N, d, dv);
     return 0;
 }
@@ -180,6 +184,7 @@ int la_prefill_kernel_count(int B, int H, int N, int d, int dv, const la_config*
 {
     if (!cfg || B <= 0 || H <= 0 || N <= 0 || !la::head_ok(d) || !la::head_ok(dv)) return 0;
     if (la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return 3;
+    if (cfg->dtype == LA_BF16 && cfg->mode == LA_GLA) return 3;
     if (cfg->dtype == LA_BF16 && cfg->mode == LA_GATED_DELTA) return 2 * la::gd_parts(B, H, N, d, dv).P;
     return 1;
 }
@@ -267,7 +272,18 @@ la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
     const la_status st = la::check_prefill(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, &c);
     if (st != LA_OK) return st;
     if ((long long)B * H == 0) return LA_OK;
-    const PrefillArgs a = la::prefill_args(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, &c);
+    PrefillArgs a = la::prefill_args(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, &c);
+    if (c.dtype == LA_BF16 && c.mode == LA_GLA) {
+        // the GLA segment summaries have the kernelized modes' slot size
+        if (N == 0) return la::write_start_state(a);
+        const la::TcSegments sg = la::tc_segments_noalloc(B, H, N, d, dv);
+        if (sg.G == 0) return LA_ERR_WORKSPACE;
+        cudaError_t e;
+        a.workspace = la::noalloc_scratch_address(&e);
+        if (!a.workspace) return la::from_cuda(e);
+        a.workspace_bytes = la::kNoAllocScratchBytes;
+        return la::from_cuda(la::launch_prefill_tc_gla(a, sg));
+    }
     if (!la::uses_tc_kernelized(c.dtype, c.mode)) {
         // paths that need no workspace run as la_prefill does; the bf16
         // gated delta rule's per-chunk operands grow with N and have no
@@ -383,8 +399,9 @@ la_status la_prefill_check(const void* workspace, void* stream)
     const unsigned int e1 = la::read_and_clear_device_error(s);
     const unsigned int e2 = la::read_and_clear_device_error_gdelta(s);
     const unsigned int e3 = la::read_and_clear_device_error_selftest(s);
-    if (e1 == 4u || e2 == 4u) return LA_ERR_UNSUPPORTED;
-    if (e1 != 0 || e2 != 0 || e3 != 0) return LA_ERR_TIMEOUT;
+    const unsigned int e4 = la::read_and_clear_device_error_gla(s);
+    if (e1 == 4u || e2 == 4u || e4 == 4u) return LA_ERR_UNSUPPORTED;
+    if (e1 != 0 || e2 != 0 || e3 != 0 || e4 != 0) return LA_ERR_TIMEOUT;
     return LA_OK;
 }
 

@@ -782,8 +782,6 @@ cudaError_t launch_prefill_tc_kernelized(const PrefillArgs& a)
 // kernels overwrite every byte they later read, so nothing needs clearing.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-namespace {
-
 // Device address of g_noalloc_scratch for the current device, looked up once
 // per device with that device current.  In host code the symbol itself is
 // only a host-side stand-in and must never be handed to a kernel.
@@ -807,8 +805,6 @@ void* noalloc_scratch_address(cudaError_t* err)
     }
     return addr[dev];
 }
-
-}  // namespace
 
 // Segment split that fits the fixed scratch: start from the usual split and
 // lengthen segments until chains * segments summaries fit.  G == 0 means the

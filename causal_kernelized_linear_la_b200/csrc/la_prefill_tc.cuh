@@ -22,6 +22,14 @@ cudaError_t launch_prefill_tc_kernelized(const PrefillArgs& a);
 constexpr size_t kNoAllocScratchBytes = 16u << 20;
 TcSegments tc_segments_noalloc(int B, int H, int N, int d, int dv);
 cudaError_t launch_prefill_tc_kernelized_noalloc(const PrefillArgs& a);
+// Device address of that scratch on the current device (looked up once per device).
+void* noalloc_scratch_address(cudaError_t* err);
+
+// GLA (per-key-channel gate) on the tensor cores, bf16 inputs: segment
+// summaries, scan, chunk loop; the workspace (or the fixed scratch) holds one
+// d x dv + d slot per (chain, segment), as for the kernelized modes.
+cudaError_t launch_prefill_tc_gla(const PrefillArgs& a, const TcSegments& sg);
+unsigned int read_and_clear_device_error_gla(cudaStream_t stream);
 
 // 3-D TMA map over the first N rows of each chain of a bf16 tensor whose
 // chains start ld rows apart ([chains][ld][inner], ld >= N); box 64 x 64

@@ -84,6 +84,30 @@ def test_noalloc_lengthened_segments_match_the_oracle():
 
 
 @pytest.mark.gpu
+def test_noalloc_gla_matches_la_prefill():
+    """bf16 GLA keeps its segment summaries in the fixed scratch too; two calls
+    in a row against la_prefill with a caller workspace."""
+    import torch
+    p = inputs.make_gla(2, 4, 1000, 128, 128, dtype="bf16", seed=34)
+    q, k, v = H.device_inputs(p)
+    al = H.dev(p.alpha, torch)
+    o_ref, S_ref, _ = la.la_prefill(q, k, v, mode="gla", alpha=al)
+    la.la_prefill_check()
+    s = torch.cuda.current_stream()
+    cfg = LaConfig(la.LA_BF16, la.MODES["gla"], 0.0, ctypes.c_void_p(s.cuda_stream), None, None, None, 0)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    for _ in range(2):
+        out = torch.full_like(v, float("nan"))
+        S_out = torch.full_like(S_ref, float("nan"))
+        rc = la.lib().la_prefill_noalloc(ptr(q), ptr(k), ptr(v), ptr(al), None, ptr(out), ptr(S_out), None,
+                                         p.B, p.H, p.N, p.d, p.dv, ctypes.byref(cfg))
+        assert rc == la.LA_OK, la.la_status_string(rc)
+        la.la_prefill_check()
+        assert H.rel_max(out.float().cpu().numpy(), o_ref.float().cpu().numpy()) <= H.TOL_O["bf16"]
+        assert H.rel_fro(S_out.cpu().numpy(), S_ref.cpu().numpy()) <= H.TOL_STATE
+
+
+@pytest.mark.gpu
 def test_noalloc_runs_workspace_free_paths_as_la_prefill():
     """fp32 inputs need no workspace: the no-allocation call runs them as
     la_prefill does, bit for bit."""
