@@ -59,7 +59,7 @@ __device__ __forceinline__ float log_gate(float a, bool valid)
 template <int D, int DV>
 struct GlaSummaryPlan {
     static constexpr int THREADS = 512;
-    static constexpr int STAGES = 2;
+    static constexpr int STAGES = (D + DV > 128) ? 3 : 4;
     static constexpr int KB = C * D * 2, VB = C * DV * 2, AB = C * D * 4;
     static constexpr int LOAD_BYTES = KB + VB;   // + the alpha block of the chunk (bulk copy)
     static constexpr int STAGE = KB + VB + AB;
