@@ -490,10 +490,16 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 unpack8(*pq, fq);
                 unpack8(*pk, fk);
                 const bool valid = row < n;
+                float Bv[8], bcv8[8], rv8[8];
+                *reinterpret_cast<float4*>(Bv) = *reinterpret_cast<const float4*>(at + row * D + f0);
+                *reinterpret_cast<float4*>(Bv + 4) = *reinterpret_cast<const float4*>(at + row * D + f0 + 4);
+                *reinterpret_cast<float4*>(bcv8) = *reinterpret_cast<const float4*>(bcv + f0);
+                *reinterpret_cast<float4*>(bcv8 + 4) = *reinterpret_cast<const float4*>(bcv + f0 + 4);
+                *reinterpret_cast<float4*>(rv8) = *reinterpret_cast<const float4*>(rv + f0);
+                *reinterpret_cast<float4*>(rv8 + 4) = *reinterpret_cast<const float4*>(rv + f0 + 4);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
-                    const float B = at[row * D + f0 + x];
-                    const float bcx = bcv[f0 + x], R = rv[f0 + x];
+                    const float B = Bv[x], bcx = bcv8[x], R = rv8[x];
                     fqt[x] = fq[x] * __expf(B - R);
                     fkt[x] = valid ? fk[x] * __expf(R - B) : 0.f;
                     fq[x] *= __expf(B);
