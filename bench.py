@@ -560,7 +560,21 @@ def la_launches_per_step(p) -> int:
 # A capture holds only while the kernel's source is unchanged: the entry
 # records the source file's sha256 at capture time, and the benchmark reports
 # null when the file differs now.
-TRAFFIC_CAPTURES = {}
+TRAFFIC_CAPTURES = {
+    # one call's eight chain launches (8 parts of 8192 tokens)
+    ("gdelta_bf16", "gd_chain_kernel"): {
+        "bytes": 2727170048 + 405584128, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
+        "sha256": "c7a8ade2fe0fc70fcf7996bdca15f82c27f81b22e80b1c05fae9fb5db6494d9f"},
+    ("plain_bf16", "chunk_kernel"): {
+        "bytes": 54631680 + 423168, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "31a166ca127dd08e294d19aaea425624b4bbfac4aba1b10a9d0bdcabaeb942cd"},
+    ("decay_bf16", "chunk_kernel"): {
+        "bytes": 824675072 + 209730816, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "31a166ca127dd08e294d19aaea425624b4bbfac4aba1b10a9d0bdcabaeb942cd"},
+    ("gla_bf16", "gla_chunk_kernel"): {
+        "bytes": 343997952 + 34664448, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
+        "sha256": "a34afc293737a363cd4e03694777a2e2a5a9bda1be0a2a250272c85d32aff1d6"},
+}
 
 
 def _file_sha256(rel):
