@@ -572,8 +572,8 @@ TRAFFIC_CAPTURES = {
         "bytes": 824675072 + 209730816, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
         "sha256": "31a166ca127dd08e294d19aaea425624b4bbfac4aba1b10a9d0bdcabaeb942cd"},
     ("gla_bf16", "gla_chunk_kernel"): {
-        "bytes": 343997952 + 34664448, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
-        "sha256": "a34afc293737a363cd4e03694777a2e2a5a9bda1be0a2a250272c85d32aff1d6"},
+        "bytes": 343998464 + 34603776, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
+        "sha256": "df531a0094a1c31add68b9a1e698af5ce866bdb8c811d3172ea2235d3476a473"},
 }
 
 
