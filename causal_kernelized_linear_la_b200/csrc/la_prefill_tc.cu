@@ -70,8 +70,8 @@ struct ChunkPlan {
     static constexpr int WBLK = D * 128;
     static constexpr int OFF_P = OFF_W + NBLK * WBLK;      // P~ bf16 [C][C]
     static constexpr int OFF_O = OFF_P + TILE;             // output staging bf16 [C][DV]
-    static constexpr int OFF_WT = OFF_O + C * DV * 2;      // [2][C] fp32 decay weights of Q~, K~
-    static constexpr int OFF_BAR = OFF_WT + 2 * C * 4;
+    static constexpr int OFF_WT = OFF_O + C * DV * 2;      // [4][C] fp32 decay weights of Q~, K~ and their log2
+    static constexpr int OFF_BAR = OFF_WT + 4 * C * 4;
     // full[S] empty[S] phi w_ready t_done p_full ptil o_full o_read os_full os_empty drain
     static constexpr int NBAR = 2 * STAGES + 10;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
@@ -321,6 +321,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     unsigned char* otil = sm + P::OFF_O;
     float* wq = reinterpret_cast<float*>(sm + P::OFF_WT);
     float* wk = wq + C;
+    float* lwq = wq + 2 * C;
+    float* lwk = wq + 3 * C;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* empty = full + P::STAGES;
     uint64_t* phi_rdy = empty + P::STAGES;   // workers: Q~, K~ of the chunk in place
@@ -364,8 +366,11 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     if (warp == 0) tmem_alloc(tmem_slot, P::T_COLS);
     if (tid < C) {
+        constexpr float kLog2e = 1.4426950408889634f;
         wq[tid] = DECAY ? __expf((float)(tid - C / 2) * lam) : 1.f;
         wk[tid] = DECAY ? __expf((float)(C / 2 - tid) * lam) : 1.f;
+        lwq[tid] = DECAY ? (float)(tid - C / 2) * lam * kLog2e : 0.f;   // log2 of the weights
+        lwk[tid] = DECAY ? (float)(C / 2 - tid) * lam * kLog2e : 0.f;
     }
     // the ones tile of every stage: element (t, 0) = 1, the rest 0
     for (int s = 0; s < P::STAGES; ++s)
@@ -382,6 +387,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // gamma^C as two factors gamma^(C/2): gamma^C itself is below the fp32
     // range for gamma < 0.25, while gamma^C T is not
     const float gH = DECAY ? __expf((float)(C / 2) * lam) : 1.f;
+    const bool one_factor = (float)C * fabsf(lam) < 80.f;   // gamma^C itself is a normal fp32
+    const float gC = gH * gH;
     const float rkappa = DECAY ? __expf(-(float)(C - 1 - C / 2) * lam) : 1.f;   // 1 / kappa
 
     auto chunk_len = [&](int c) { return min(C, t1 - (t0 + c * C)); };
@@ -473,26 +480,31 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     } else if (worker) {
         // ---------------- workers ----------------
         // phi of chunk c in place: Q~ = w_q phi(q), K~ = w_k phi(k) [t < n]
+        // w phi(x) = w max(x, 0) + 2^(min(x, 0) log2 e + log2 w): the operand weight rides in
+        // the exponent (w = 0, for key rows past the sequence's end, gives exactly 0)
         auto phi = [&](int c) {
             const int n = chunk_len(c);
             unsigned char* qt = sm + (c % P::STAGES) * P::STAGE;
             unsigned char* kt = qt + P::QB;
+            constexpr float kLog2e = 1.4426950408889634f;
             for (int e = tid; e < (D / 8) * C; e += NWT) {
                 const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
                 uint4* pq = reinterpret_cast<uint4*>(qt + b * TILE) + rem;
                 uint4* pk = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
+                const bool kv = row < n;
+                const float aq = DECAY ? wq[row] : 1.f, lq = DECAY ? lwq[row] : 0.f;
+                const float ak = kv ? (DECAY ? wk[row] : 1.f) : 0.f;
+                const float lk = kv ? (DECAY ? lwk[row] : 0.f) : -INFINITY;
                 float fq[8], fk[8];
                 unpack8(*pq, fq);
                 unpack8(*pk, fk);
 #pragma unroll
-                for (int x = 0; x < 8; x += 2) {
-                    const float2 a = phi2_fast(fq[x], fq[x + 1]);
-                    const float2 g = phi2_fast(fk[x], fk[x + 1]);
-                    fq[x] = a.x; fq[x + 1] = a.y;
-                    fk[x] = g.x; fk[x + 1] = g.y;
+                for (int x = 0; x < 8; ++x) {
+                    fq[x] = fmaf(fmaxf(fq[x], 0.f), aq, ex2_approx(fmaf(fminf(fq[x], 0.f), kLog2e, lq)));
+                    fk[x] = fmaf(fmaxf(fk[x], 0.f), ak, ex2_approx(fmaf(fminf(fk[x], 0.f), kLog2e, lk)));
                 }
-                *pq = pack8(fq, wq[row]);
-                *pk = pack8(fk, row < n ? wk[row] : 0.f);
+                *pq = pack8(fq, 1.f);
+                *pk = pack8(fk, 1.f);
             }
         };
         // T0 = S / kappa: the segment's start state (from the scan), normaliser as column dv
@@ -532,7 +544,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tmem_ld_wait();
                 if (DECAY) {
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) v[x] = (v[x] * gH) * gH;
+                    for (int x = 0; x < 16; ++x) v[x] = one_factor ? v[x] * gC : (v[x] * gH) * gH;
                     tmem_st16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
                 }
                 if (fr >= 0) {

@@ -341,6 +341,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// 2^x by the SFU (ex2.approx, flush-to-zero): relative error a few fp32 ulps,
+// 2^-inf = 0.
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // elu(x) + 1 for a pair of values: x + 1 above zero, e^x at or below it.
 // The exponential takes the full fp32 argument min(x, 0) (SFU __expf, a
 // relative error of a few fp32 ulps, far below the bf16 rounding applied to
