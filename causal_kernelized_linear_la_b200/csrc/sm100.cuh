@@ -85,20 +85,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
-// Bounded wait for the phase with the given parity to complete.  The timer is
-// read once every 64 tries (a read of %globaltimer is not free), so the bound
-// is the deadline plus at most 64 tries.
+// Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int site)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t t0 = 0;
-    for (uint32_t i = 1; i < kSpinLimit; ++i) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            const uint64_t t = globaltimer_ns();
-            if (t0 == 0) t0 = t;
-            else if (t - t0 > kWaitLimitNs) break;
-        }
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
     }
     atomicCAS(&g_device_error, 0u, site);
     return false;
