@@ -22,11 +22,9 @@ namespace sm100 {
 static __device__ unsigned int g_device_error = 0;
 
 // A bounded wait gives up once kWaitLimitNs of %globaltimer time have passed
-// since it started (far above any legitimate latency).  Each try_wait may
-// suspend the thread for at most the hinted kSuspendNs; the hint only bounds
-// one try, so the deadline, not a count of tries, sets the bound.  kSpinLimit
+// since it started (far above any legitimate latency); each try_wait without
+// a suspend-time hint returns after a short, system-dependent time.  kSpinLimit
 // is a backstop on the number of tries in case the timer is not advancing.
-constexpr uint32_t kSuspendNs = 20000;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
 constexpr uint32_t kSpinLimit = 200000000u;
 
@@ -70,10 +68,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
