@@ -691,7 +691,8 @@ def time_conv(torch, la, rank, flush, B=4, H=8, N=4096, d=64, w=4, steps=20):
 def time_varlen(torch, la, rank, flush, H=8, N=4096, d=64, steps=20):
     """A right-padded batch of eight plain bf16 sequences of mixed lengths
     (head size and padded length of the plain workload) through
-    la_prefill_varlen: device time per call, L2 flushed before each."""
+    la_prefill_varlen, which runs it as one launch set: device time per call,
+    L2 flushed before each."""
     hbm_peak, _, peak_kind = _measured_peaks()
     g = torch.Generator(device="cpu").manual_seed(rank_seed(91, rank))
     lens = [4096, 3000, 2048, 1500, 1000, 700, 300, 65]
@@ -712,7 +713,7 @@ def time_varlen(torch, la, rank, flush, H=8, N=4096, d=64, steps=20):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
                          "traffic": None, "kernel": "whole call", "kernel_ms": ms,
                          "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": nbytes},
-            "gpu_launches_per_call": 3 * B}
+            "gpu_launches_per_call": 3}   # one launch set (summaries, scan, chunk loop) for the batch
 
 
 def run_extra(args, torch, la, rank, flush):

@@ -128,6 +128,17 @@ PrefillArgs prefill_args(const void* q, const void* k, const void* v, const floa
     return a;
 }
 
+// A right-padded batch runs as one launch set (instead of one per sequence)
+// on the bf16 tensor-core path of the kernelized modes, up to kMaxVarlenSeqs
+// sequences.
+bool varlen_one_launch_set(const int* lens, int B, int H, int d, int dv, const la_config* cfg)
+{
+    if (!cfg || !lens || B <= 0 || B > kMaxVarlenSeqs || H <= 0 || !head_ok(d) || !head_ok(dv)) return false;
+    for (int b = 0; b < B; ++b)
+        if (lens[b] < 0) return false;
+    return uses_tc_kernelized(cfg->dtype, cfg->mode);
+}
+
 // Workspace slice of one sequence of la_prefill_varlen: 256-byte aligned.
 size_t varlen_slice(size_t bytes) { return (bytes + 255) / 256 * 256; }
 
@@ -204,6 +215,8 @@ la_status la_prefill(const void* q, const void* k, const void* v,
 size_t la_prefill_varlen_workspace_bytes(const int* seq_lens, int B, int H, int d, int dv, const la_config* cfg)
 {
     if (!seq_lens || B <= 0) return 0;
+    if (la::varlen_one_launch_set(seq_lens, B, H, d, dv, cfg))
+        return la::tc_varlen_workspace_bytes(seq_lens, B, H, d, dv);
     size_t total = 0;
     for (int b = 0; b < B; ++b) total += la::varlen_slice(la_prefill_workspace_bytes(1, H, seq_lens[b], d, dv, cfg));
     return total;
@@ -230,6 +243,13 @@ la_status la_prefill_varlen(const void* q, const void* k, const void* v,
     // kernel of sequence b > 0 may start while sequence b-1's kernels drain
     // (programmatic serialization); it finishes after them.
     const PrefillArgs base = la::prefill_args(q, k, v, gamma_or_alpha, g, out, S_out, z_out, B, H, N, d, dv, cfg);
+    if (la::varlen_one_launch_set(seq_lens, B, H, d, dv, cfg)) {
+        // one launch set over every sequence of the batch
+        bool any = false;
+        for (int b = 0; b < B; ++b) any = any || seq_lens[b] > 0;
+        if (!any) return la::write_start_state(base);
+        return la::from_cuda(la::launch_prefill_tc_kernelized_varlen(base, seq_lens));
+    }
     const size_t esz = cfg->dtype == LA_BF16 ? 2 : 4;
     size_t ws_off = 0;
     for (int b = 0; b < B; ++b) {

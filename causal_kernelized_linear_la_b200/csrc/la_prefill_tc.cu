@@ -100,12 +100,75 @@ struct SummaryPlan {
 
 
 // ---------------------------------------------------------------------------
+// Units of a segment map: one (chain, segment) each, with its token range.
+struct Unit {
+    int chain, t0, t1;
+    bool clip;   // a sequence of a padded batch: rows past t1 may hold padding
+};
+
+__device__ __forceinline__ Unit unit_of(const SegMap& m, int unit)
+{
+    Unit u;
+    if (m.B == 0) {
+        const int seg = unit % m.G;
+        u.chain = unit / m.G;
+        u.t0 = seg * m.L;
+        u.t1 = min(m.N, u.t0 + m.L);
+        u.clip = false;
+        return u;
+    }
+    int base = 0, b = 0;
+    for (; b < m.B; ++b) {
+        const int n = m.H * ((m.lens[b] + m.L - 1) / m.L);
+        if (unit < base + n) break;
+        base += n;
+    }
+    const int g = (m.lens[b] + m.L - 1) / m.L;
+    const int r = unit - base;
+    u.chain = b * m.H + r / g;
+    u.t0 = (r % g) * m.L;
+    u.t1 = min(m.lens[b], u.t0 + m.L);
+    u.clip = true;
+    return u;
+}
+
+__device__ __forceinline__ int chunk_len_of(int t0, int t1, int c) { return min(C, t1 - (t0 + c * C)); }
+
+// First slot, segment count and token count of chain c.
+__device__ __forceinline__ void chain_of(const SegMap& m, int c, int& slot0, int& g, int& n)
+{
+    if (m.B == 0) {
+        slot0 = c * m.G;
+        g = m.G;
+        n = m.N;
+        return;
+    }
+    const int b = c / m.H, h = c % m.H;
+    int base = 0;
+    for (int i = 0; i < b; ++i) base += m.H * ((m.lens[i] + m.L - 1) / m.L);
+    n = m.lens[b];
+    g = (n + m.L - 1) / m.L;
+    slot0 = base + h * g;
+}
+
+// Zero the value rows n..C-1 of a chunk's V tiles (a padded batch's padding may
+// hold anything, and a zero weight times a non-finite value is not zero).
+template <int DV>
+__device__ __forceinline__ void zero_tail_rows(unsigned char* vt, int n, int tid, int nthreads)
+{
+    for (int e = tid; e < (DV / 8) * C; e += nthreads) {
+        const int rem = e % (8 * C), row = rem / 8;
+        if (row >= n) reinterpret_cast<uint4*>(vt)[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Kernel A: segment summaries  Delta S = sum_t gamma^(last-t) phi(k_t) v_t^T,
 // Delta z = sum_t gamma^(last-t) phi(k_t), over the tokens of one segment.
 template <int D, int DV, bool DECAY>
 __global__ void __launch_bounds__(kThreads, 1)
 summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const float* __restrict__ gamma, float* __restrict__ ws, int N, int H, int G, int L)
+               const float* __restrict__ gamma, float* __restrict__ ws, const __grid_constant__ SegMap m)
 {
     using P = SummaryPlan<D, DV>;
     grid_launch_dependents();   // the scan may launch now; it waits for this grid's results
@@ -119,10 +182,10 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, wg = warp >> 2;
     const int unit = blockIdx.x;
-    const int chain = unit / G, seg = unit % G;
-    const int t0 = seg * L, t1 = min(N, t0 + L);
+    const Unit un = unit_of(m, unit);
+    const int chain = un.chain, t0 = un.t0, t1 = un.t1;
     const int nch = (t1 - t0 + C - 1) / C;
-    const float lam = DECAY ? logf(gamma[chain % H]) : 0.f;
+    const float lam = DECAY ? logf(gamma[chain % m.H]) : 0.f;
     const uint64_t pol = policy_evict_last();  // the chunk kernel reads k, v again
 
     if (tid == 0) {
@@ -167,6 +230,7 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         unsigned char* vt = kt + P::KB;
         if (!mbar_wait(&full[s], ph, kErrTmaLoad)) bad = true;
         else loads_waited = c + 1;
+        if (un.clip && t1 - (t0 + c * C) < C) zero_tail_rows<DV>(vt, t1 - (t0 + c * C), tid, kThreads);
         // K~_t = gamma^(last - t) phi(k_t), zero past the end of the sequence
         const int tc0 = t0 + c * C;
         for (int e = tid; e < (D / 8) * C; e += kThreads) {
@@ -181,7 +245,9 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                 const float2 y = phi2_fast(f[x], f[x + 1]);
                 f[x] = y.x; f[x + 1] = y.y;
             }
-            *p = pack8(f, w);
+            // rows past the end are stored as zeros: a padded batch's padding
+            // may hold anything, and a zero weight times inf is not zero
+            *p = t <= last ? pack8(f, w) : make_uint4(0u, 0u, 0u, 0u);
         }
         fence_async_smem();
         tc_fence_before();
@@ -254,8 +320,8 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 template <int D, int DV, bool DECAY>
 __global__ void __launch_bounds__(256)
 scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float* __restrict__ S0,
-            const float* __restrict__ z0, float* __restrict__ S_out, float* __restrict__ z_out, int N, int H,
-            int G, int L)
+            const float* __restrict__ z0, float* __restrict__ S_out, float* __restrict__ z_out,
+            const __grid_constant__ SegMap m)
 {
     constexpr int SLOT = D * DV + D;
     grid_launch_dependents();   // the chunk kernel may set up and load q, k, v meanwhile
@@ -263,12 +329,15 @@ scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float
     const int chain = blockIdx.x;
     const int e = blockIdx.y * 256 + threadIdx.x;
     if (e >= SLOT) return;
-    const float lam = DECAY ? logf(gamma[chain % H]) : 0.f;
+    int slot0, G, N;
+    chain_of(m, chain, slot0, G, N);
+    const int L = m.L;
+    const float lam = DECAY ? logf(gamma[chain % m.H]) : 0.f;
     const bool isz = e >= D * DV;
     float acc;
     if (!isz) acc = S0 ? S0[(size_t)chain * D * DV + e] : 0.f;
     else acc = z0 ? z0[(size_t)chain * D + (e - D * DV)] : 0.f;
-    float* base = ws + (size_t)chain * G * SLOT + e;
+    float* base = ws + (size_t)slot0 * SLOT + e;
     const float full_dec = DECAY ? expf((float)L * lam) : 1.f;
     constexpr int BATCH = 8;
     for (int s0 = 0; s0 < G; s0 += BATCH) {
@@ -307,7 +376,8 @@ template <int D, int DV, bool DECAY>
 __global__ void __launch_bounds__(ChunkPlan<D, DV, DECAY>::THREADS, ChunkPlan<D, DV, DECAY>::TWO_PER_SM ? 2 : 1)
 chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-             const float* __restrict__ gamma, const float* __restrict__ ws, int N, int H, int G, int L, float eps)
+             const float* __restrict__ gamma, const float* __restrict__ ws, const __grid_constant__ SegMap m,
+             float eps, __nv_bfloat16* __restrict__ out, int ld)
 {
     using P = ChunkPlan<D, DV, DECAY>;
     constexpr int NW = P::NW;
@@ -342,10 +412,13 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const bool issuer = tid == NWT;
     const int quad = warp & 3, qg = warp >> 2;        // TMEM lane quadrant, column group in it
     const int unit = blockIdx.x;
-    const int chain = unit / G, seg = unit % G;
-    const int t0 = seg * L, t1 = min(N, t0 + L);
+    const Unit un = unit_of(m, unit);
+    const int chain = un.chain, t0 = un.t0, t1 = un.t1;
     const int nch = (t1 - t0 + C - 1) / C;
-    const float lam = DECAY ? logf(gamma[chain % H]) : 0.f;
+    // a padded batch's last chunk of a sequence: its rows past the end hold
+    // padding, so V's are zeroed and the output rows are stored one by one
+    const bool clip_tail = un.clip && chunk_len_of(t0, t1, nch - 1) < C;
+    const float lam = DECAY ? logf(gamma[chain % m.H]) : 0.f;
     const uint64_t pol_in = policy_evict_first();
     // the scaled frame keeps every weight within gamma^-32
     if (DECAY && tid == 0 && 32.f * fabsf(lam) > 73.7f) atomicCAS(&g_device_error, 0u, (unsigned int)kErrRange);
@@ -467,7 +540,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 issue(c + P::STAGES);
             }
         }
-        if (!bad && nch > 0 && mbar_wait(os_full, (nch - 1) & 1, kErrMma)) {
+        if (!bad && nch > 0 && mbar_wait(os_full, (nch - 1) & 1, kErrMma) && !clip_tail) {
             for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (nch - 1) * C, chain);
             tma_store_commit();
         }
@@ -504,8 +577,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     fk[x] = fmaf(fmaxf(fk[x], 0.f), ak, ex2_approx(fmaf(fminf(fk[x], 0.f), kLog2e, lk)));
                 }
                 *pq = pack8(fq, 1.f);
-                *pk = pack8(fk, 1.f);
+                *pk = kv ? pack8(fk, 1.f) : make_uint4(0u, 0u, 0u, 0u);
             }
+            if (clip_tail && c == nch - 1) zero_tail_rows<DV>(kt + P::KB, n, tid, NWT);
         };
         // T0 = S / kappa: the segment's start state (from the scan), normaliser as column dv
         {
@@ -606,11 +680,24 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tmem_ld_wait();
             const float rden = __frcp_rn(den[0] + eps);
             if (c >= 1 && !mbar_wait(os_empty, (c - 1) & 1, kErrMma)) bad = true;
+            const bool direct = clip_tail && c == nch - 1;
+            const int nrow = chunk_len(c);
             for (int g = qg; g < DV / 16; g += NQ) {
                 float v[16];
                 tmem_ld16(tmem_addr(tbase, quad, P::T_O + g * 16), v);
                 tmem_ld_wait();
-                if (ir >= 0) {
+                if (direct) {
+                    // the padded batch's last rows of this sequence: only rows < n are written
+                    if (ir >= 0 && ir < nrow) {
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            out + ((size_t)chain * ld + t0 + c * C + ir) * DV + g * 16);
+                        dst[0] = make_uint4(pack_bf16x2(v[0] * rden, v[1] * rden), pack_bf16x2(v[2] * rden, v[3] * rden),
+                                            pack_bf16x2(v[4] * rden, v[5] * rden), pack_bf16x2(v[6] * rden, v[7] * rden));
+                        dst[1] = make_uint4(pack_bf16x2(v[8] * rden, v[9] * rden), pack_bf16x2(v[10] * rden, v[11] * rden),
+                                            pack_bf16x2(v[12] * rden, v[13] * rden),
+                                            pack_bf16x2(v[14] * rden, v[15] * rden));
+                    }
+                } else if (ir >= 0) {
                     unsigned char* blk = otil + (g / 4) * TILE;
                     const int byte0 = (g % 4) * 32;
                     *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0)) =
@@ -672,7 +759,7 @@ bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains, in
 namespace {
 
 template <int D, int DV, bool DECAY>
-cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
+cudaError_t launch_tc_map(const PrefillArgs& a, const SegMap& m, int units)
 {
     const int chains = a.B * a.H;
     CUtensorMap mq, mk, mv, mo;
@@ -680,7 +767,6 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
         !make_map(&mv, a.v, DV, a.N, chains, a.ld) || !make_map(&mo, a.out, DV, a.N, chains, a.ld))
         return cudaErrorInvalidValue;
     float* ws = static_cast<float*>(a.workspace);
-    const int units = chains * sg.G;
 
     auto ka = summary_kernel<D, DV, DECAY>;
     const int sa = SummaryPlan<D, DV>::BYTES;
@@ -703,7 +789,7 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     lc.stream = a.stream;
     lc.attrs = pdl;
     lc.numAttrs = a.pdl_first ? 1 : 0;
-    e = cudaLaunchKernelEx(&lc, ka, mk, mv, a.gamma, ws, a.N, a.H, sg.G, sg.L);
+    e = cudaLaunchKernelEx(&lc, ka, mk, mv, a.gamma, ws, m);
     if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(0, a.stream);
@@ -713,8 +799,7 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     lc.blockDim = dim3(256);
     lc.dynamicSmemBytes = 0;
     lc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&lc, scan_kernel<D, DV, DECAY>, ws, a.gamma, a.S0, a.z0, a.S_out, a.z_out, a.N, a.H,
-                           sg.G, sg.L);
+    e = cudaLaunchKernelEx(&lc, scan_kernel<D, DV, DECAY>, ws, a.gamma, a.S0, a.z0, a.S_out, a.z_out, m);
     if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(1, a.stream);
@@ -728,11 +813,24 @@ cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
     lc.gridDim = dim3(units);
     lc.blockDim = dim3(ChunkPlan<D, DV, DECAY>::THREADS);
     lc.dynamicSmemBytes = sc;
-    e = cudaLaunchKernelEx(&lc, kc, mq, mk, mv, mo, a.gamma, (const float*)ws, a.N, a.H, sg.G, sg.L, a.eps);
+    e = cudaLaunchKernelEx(&lc, kc, mq, mk, mv, mo, a.gamma, (const float*)ws, m, a.eps,
+                           static_cast<__nv_bfloat16*>(a.out), a.ld);
     if (e != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(2, a.stream);
     return cudaSuccess;
+}
+
+template <int D, int DV, bool DECAY>
+cudaError_t launch_tc(const PrefillArgs& a, const TcSegments& sg)
+{
+    SegMap m;
+    m.H = a.H;
+    m.L = sg.L;
+    m.B = 0;
+    m.N = a.N;
+    m.G = sg.G;
+    return launch_tc_map<D, DV, DECAY>(a, m, a.B * a.H * sg.G);
 }
 
 }  // namespace
@@ -774,6 +872,56 @@ cudaError_t launch_prefill_tc_kernelized(const PrefillArgs& a)
     const bool dec = a.mode == LA_DECAY;
 #define LA_TC(D, DV)                                                               \
     if (a.d == D && a.dv == DV) return dec ? launch_tc<D, DV, true>(a, sg) : launch_tc<D, DV, false>(a, sg);
+    LA_TC(64, 64)
+    LA_TC(64, 128)
+    LA_TC(128, 64)
+    LA_TC(128, 128)
+#undef LA_TC
+    return cudaErrorInvalidValue;
+}
+
+// A right-padded batch as one launch set: one segment length L for all
+// sequences, the smallest multiple of the chunk (at least two chunks) whose
+// units fit one wave of resident CTAs, at most 4096 tokens.
+namespace {
+long long varlen_units(const int* lens, int B, int H, int L)
+{
+    long long u = 0;
+    for (int b = 0; b < B; ++b) u += (long long)H * ((lens[b] + L - 1) / L);
+    return u;
+}
+}  // namespace
+
+int varlen_segment_length(const int* lens, int B, int H, int d, int dv)
+{
+    const long long slots = (d == 64 && dv == 64) ? 2 * 148 : 148;
+    int L = 2 * C;
+    while (L < 4096 && varlen_units(lens, B, H, L) > slots) L += C;
+    return L;
+}
+
+size_t tc_varlen_workspace_bytes(const int* lens, int B, int H, int d, int dv)
+{
+    const int L = varlen_segment_length(lens, B, H, d, dv);
+    return (size_t)varlen_units(lens, B, H, L) * ((size_t)d * dv + d) * sizeof(float);
+}
+
+cudaError_t launch_prefill_tc_kernelized_varlen(const PrefillArgs& a, const int* lens)
+{
+    if (a.B > kMaxVarlenSeqs) return cudaErrorInvalidValue;
+    SegMap m;
+    m.H = a.H;
+    m.L = varlen_segment_length(lens, a.B, a.H, a.d, a.dv);
+    m.B = a.B;
+    for (int b = 0; b < a.B; ++b) m.lens[b] = lens[b];
+    const long long units = varlen_units(lens, a.B, a.H, m.L);
+    if (!a.workspace || a.workspace_bytes < tc_varlen_workspace_bytes(lens, a.B, a.H, a.d, a.dv))
+        return cudaErrorInvalidValue;
+    if (units == 0 || units > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const bool dec = a.mode == LA_DECAY;
+#define LA_TC(D, DV)                                                                                   \
+    if (a.d == D && a.dv == DV)                                                                         \
+        return dec ? launch_tc_map<D, DV, true>(a, m, (int)units) : launch_tc_map<D, DV, false>(a, m, (int)units);
     LA_TC(64, 64)
     LA_TC(64, 128)
     LA_TC(128, 64)

@@ -15,8 +15,29 @@ struct TcSegments {
 };
 
 TcSegments tc_segments(int B, int H, int N, int d, int dv);
+
+// Segment map of one launch set of the kernelized tensor-core prefill: either a
+// uniform batch (every chain has N tokens in G segments of L) or a right-padded
+// batch of up to kMaxVarlenSeqs sequences of their own lengths (sequence b: H
+// chains of lens[b] tokens in ceil(lens[b] / L) segments; units are numbered
+// sequence by sequence, head by head, segment by segment).
+constexpr int kMaxVarlenSeqs = 64;
+struct SegMap {
+    int H = 0;
+    int L = 0;
+    int B = 0;   // 0: uniform batch
+    int N = 0;   // uniform: tokens per chain
+    int G = 0;   // uniform: segments per chain
+    int lens[kMaxVarlenSeqs] = {};
+};
 size_t tc_workspace_bytes(int B, int H, int N, int d, int dv);
 cudaError_t launch_prefill_tc_kernelized(const PrefillArgs& a);
+
+// One launch set over a right-padded batch (a.B <= kMaxVarlenSeqs sequences,
+// a.N = a.ld = the padded length): segment length and workspace slots.
+int varlen_segment_length(const int* lens, int B, int H, int d, int dv);
+size_t tc_varlen_workspace_bytes(const int* lens, int B, int H, int d, int dv);
+cudaError_t launch_prefill_tc_kernelized_varlen(const PrefillArgs& a, const int* lens);
 
 // Fixed scratch of the no-allocation entry point (la_prefill_noalloc).
 constexpr size_t kNoAllocScratchBytes = 16u << 20;

@@ -200,14 +200,23 @@ LA_API int la_prefill_kernel_count(int B, int H, int N, int d, int dv, const la_
  * Sequence b's results equal those of la_prefill on that sequence alone
  * (B = 1, N = seq_lens[b]) from its start state: out[b, :, t] for
  * t < seq_lens[b], and S_out[b], z_out[b] after its last token (its start
- * state when seq_lens[b] == 0).  Padding rows of q, k, v, alpha, g are never
- * read and padding rows of out are never written.  The sequences run one
- * after another on cfg->stream, each through the kernels la_prefill uses;
- * each has a slice of cfg->workspace (which must hold
- * la_prefill_varlen_workspace_bytes() bytes), so a sequence's first kernel
- * may start while the previous sequence's last kernel drains.  Returns
- * LA_OK once all the work is enqueued; on an error from sequence b,
- * sequences before b are enqueued and the rest are not.
+ * state when seq_lens[b] == 0), up to rounding: the bf16 LA_PLAIN / LA_DECAY
+ * path may cut a sequence into segments at other points than the solo call
+ * does.  Padding rows of out are never written.  Padding rows of q, k, v,
+ * alpha, g never affect a result, whatever they hold (NaN and inf included).
+ *
+ * bf16 LA_PLAIN / LA_DECAY with B <= 64: the whole batch runs as one set of
+ * three kernels (segment summaries, scan, chunk loop) whose segments are the
+ * (sequence, head, segment) triples of all sequences, with one segment length
+ * chosen so that they fill one wave of the GPU; these kernels may read
+ * padding rows of q, k, v inside a sequence's last 64-token chunk and discard
+ * them.  Otherwise the sequences run one after another on cfg->stream, each
+ * through the kernels la_prefill uses, and padding rows are not read; each
+ * has a slice of cfg->workspace, so a sequence's first kernel may start while
+ * the previous sequence's last kernel drains.  cfg->workspace must hold
+ * la_prefill_varlen_workspace_bytes() bytes.  Returns LA_OK once all the work
+ * is enqueued; on an error from sequence b of the one-by-one form, sequences
+ * before b are enqueued and the rest are not.
  */
 LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v,
                                    const float* gamma_or_alpha, const float* g,
@@ -215,10 +224,12 @@ LA_API la_status la_prefill_varlen(const void* q, const void* k, const void* v,
                                    int B, int H, int N, int d, int dv, const la_config* cfg);
 
 /*
- * la_prefill_varlen_workspace_bytes -- the workspace la_prefill_varlen needs:
- * the sum over the batch of la_prefill_workspace_bytes(1, H, seq_lens[b], d,
- * dv, cfg), each rounded up to a multiple of 256 bytes (seq_lens: host array
- * of B lengths).  0 means none is needed.
+ * la_prefill_varlen_workspace_bytes -- the workspace la_prefill_varlen needs
+ * (seq_lens: host array of B lengths).  For the one-launch-set form (bf16
+ * LA_PLAIN / LA_DECAY, B <= 64) one fp32 summary of d*dv + d values per
+ * segment of the batch; otherwise the sum over the batch of
+ * la_prefill_workspace_bytes(1, H, seq_lens[b], d, dv, cfg), each rounded up
+ * to a multiple of 256 bytes.  0 means none is needed.
  */
 LA_API size_t la_prefill_varlen_workspace_bytes(const int* seq_lens, int B, int H, int d, int dv,
                                                 const la_config* cfg);

@@ -195,9 +195,41 @@ def test_varlen_validation():
 
 
 def test_varlen_workspace_is_one_slice_per_sequence():
+    # paths that run one sequence at a time take one 256-byte aligned slice each
     lens = [0, 100, 5000, 64, 4096]
-    for dtype, mode in (("bf16", "plain"), ("bf16", "decay"), ("bf16", "gated_delta"), ("f32", "plain")):
+    for dtype, mode in (("bf16", "gated_delta"), ("f32", "plain"), ("bf16", "gla")):
         each = [la.la_prefill_workspace_bytes(1, 8, n, 128, 128, dtype, mode) if n > 0 else 0 for n in lens]
         want = sum((n + 255) // 256 * 256 for n in each)
         assert la.la_prefill_varlen_workspace_bytes(lens, 8, 128, 128, dtype, mode) == want
     assert la.la_prefill_varlen_workspace_bytes([], 8, 128, 128) == 0
+
+
+def _one_set_units(lens, H, d, dv):
+    """Segments of the one-launch-set padded batch: the smallest segment length
+    (a multiple of 64 tokens, at least 128, at most 4096) whose segment count
+    over all (sequence, head) chains fits one wave of resident CTAs."""
+    slots = 296 if (d, dv) == (64, 64) else 148
+    L = 128
+    while True:
+        units = sum(H * -(-n // L) for n in lens)
+        if units <= slots or L >= 4096:
+            return L, units
+        L += 64
+
+
+def test_varlen_workspace_of_the_one_launch_set():
+    # the bf16 kernelized modes run a padded batch as one launch set; its
+    # workspace holds one (d*dv + d) fp32 summary per segment
+    cases = [([0, 100, 5000, 64, 4096], 8, 128, 128), ([1] * 64, 32, 64, 64),
+             ([65536, 3, 0], 16, 128, 64), ([0, 0], 4, 64, 128)]
+    for lens, H, d, dv in cases:
+        L, units = _one_set_units(lens, H, d, dv)
+        assert L % 64 == 0 and 128 <= L <= 4096
+        for mode in ("plain", "decay"):
+            got = la.la_prefill_varlen_workspace_bytes(lens, H, d, dv, "bf16", mode)
+            assert got == units * (d * dv + d) * 4, (lens, H, d, dv, mode)
+    # more sequences than one launch set takes: one slice per sequence again
+    lens = [100] * 65
+    each = la.la_prefill_workspace_bytes(1, 8, 100, 64, 64, "bf16", "plain")
+    want = 65 * ((each + 255) // 256 * 256)
+    assert la.la_prefill_varlen_workspace_bytes(lens, 8, 64, 64, "bf16", "plain") == want

@@ -3,11 +3,14 @@ different lengths ("Efficient attention variants" §10, closing remarks: real
 batches carry padding and chunk boundaries that the single-sequence examples
 leave out).
 
-Every padding row of q, k, v (and alpha, g) is NaN, so a kernel that read one
-would spread NaN into that sequence's outputs or state; out is pre-filled
-with a sentinel, and its padding rows must still hold it afterwards.  Each
-sequence is checked against the oracle over its own length, and must be
-bit-identical to la_prefill on that sequence alone.
+Every padding row of q, k, v (and alpha, g) is NaN or inf, so a kernel that
+let one into a result would spread a non-finite value into that sequence's
+outputs or state; out is pre-filled with a sentinel, and its padding rows
+must still hold it afterwards.  Each sequence is checked against the oracle
+over its own length, and against la_prefill on that sequence alone: bit for
+bit where the batch runs one sequence at a time (the same kernels and segment
+plan), within the oracle tolerance where the bf16 kernelized batch runs as one
+launch set (its segment length is chosen for the whole batch).
 """
 import numpy as np
 import pytest
@@ -29,15 +32,21 @@ def _make(mode, dtype, B, H_, N, d, dv, seed):
 
 
 def _device(p, lens, torch):
-    """Device tensors with NaN in every padding row."""
+    """Device tensors with NaN, +inf or -inf in every padding row."""
     q, k, v = H.device_inputs(p)
     a = None if p.alpha is None else H.dev(p.alpha, torch)
     g = None if p.g is None else H.dev(p.g, torch)
+    junk = (float("nan"), float("inf"), float("-inf"))
     for b, n in enumerate(lens):
         for t in (q, k, v, a, g):
             if t is not None:
-                t[b, :, n:] = float("nan")
+                for r in range(n, t.shape[2]):
+                    t[b, :, r] = junk[(r + b) % 3]
     return q, k, v, a, g
+
+
+def _one_launch_set(mode, dtype, B):
+    return dtype == "bf16" and mode in ("plain", "decay") and B <= 64
 
 
 def _kw(p, a, g, torch):
@@ -96,11 +105,31 @@ CASES = [
 ]
 
 
+LARGE_CASES = [
+    # 16 heads: the batch's 1,184 segments of 128 tokens are too many for one
+    # wave, so the segment length grows to 1,408 tokens (not a power of two)
+    ("decay", "bf16", 128, 128, 4096, [4096, 3000, 1, 0, 2049], 16),
+    # 40 sequences of scattered lengths, two segments per SM
+    ("plain", "bf16", 64, 64, 640, [(37 * i * i + 11 * i) % 641 for i in range(40)], 4),
+    # 65 sequences: more than one launch set takes, one sequence at a time
+    ("plain", "bf16", 64, 64, 80, [(7 * i) % 81 for i in range(65)], 1),
+]
+
+
 @pytest.mark.parametrize("mode,dtype,d,dv,N,lens", CASES)
 def test_varlen_matches_oracle_and_solo_calls(mode, dtype, d, dv, N, lens):
+    _run_case(mode, dtype, d, dv, N, lens, 3)
+
+
+@pytest.mark.parametrize("mode,dtype,d,dv,N,lens,heads", LARGE_CASES)
+def test_varlen_large_batches(mode, dtype, d, dv, N, lens, heads):
+    _run_case(mode, dtype, d, dv, N, lens, heads)
+
+
+def _run_case(mode, dtype, d, dv, N, lens, H_):
     import torch
     import causal_kernelized_linear_la_b200 as la
-    B, H_ = len(lens), 3
+    B = len(lens)
     p = _make(mode, dtype, B, H_, N, d, dv, seed=1300 + N + d)
     q, k, v, a, g = _device(p, lens, torch)
     kw = _kw(p, a, g, torch)
@@ -114,8 +143,8 @@ def test_varlen_matches_oracle_and_solo_calls(mode, dtype, d, dv, N, lens):
         assert np.all(o_h[b, :, n:] == SENTINEL), f"padding rows of sequence {b} were written"
         assert np.all(np.isfinite(o_h[b, :, :n])) and np.all(np.isfinite(S_h[b])), f"sequence {b} read padding"
         _check_seq(p, (o_h, S_h, z_h), b, n)
-    # each sequence alone through la_prefill: the same kernels and segment
-    # plan, so the same bits
+    # each sequence alone through la_prefill
+    exact = not _one_launch_set(mode, dtype, B)
     for b, n in enumerate(lens):
         sub = lambda t: None if t is None else t[b:b + 1, :, :n].contiguous()
         kw1 = dict(kw)
@@ -124,10 +153,17 @@ def test_varlen_matches_oracle_and_solo_calls(mode, dtype, d, dv, N, lens):
         if "g" in kw1:
             kw1["g"] = sub(g)
         o1, S1, z1 = la.la_prefill(sub(q), sub(k), sub(v), **kw1)
-        assert torch.equal(o1[0], o[b, :, :n]), f"sequence {b}: o differs from the solo call"
-        assert torch.equal(S1[0], S[b]), f"sequence {b}: S differs from the solo call"
-        if z is not None:
-            assert torch.equal(z1[0], z[b]), f"sequence {b}: z differs from the solo call"
+        if exact:
+            assert torch.equal(o1[0], o[b, :, :n]), f"sequence {b}: o differs from the solo call"
+            assert torch.equal(S1[0], S[b]), f"sequence {b}: S differs from the solo call"
+            if z is not None:
+                assert torch.equal(z1[0], z[b]), f"sequence {b}: z differs from the solo call"
+            continue
+        if n > 0:
+            e = H.rel_max(o1[0].float().cpu().numpy(), o_h[b, :, :n])
+            assert e <= H.TOL_O[dtype], f"sequence {b}: o differs from the solo call by {e:.3e}"
+        es = H.rel_fro(S1[0].cpu().numpy(), S_h[b])
+        assert es <= H.TOL_STATE, f"sequence {b}: S differs from the solo call by {es:.3e}"
 
 
 @pytest.mark.parametrize("mode", ["plain", "decay", "gated_delta"])
