@@ -56,7 +56,11 @@ template <int D, int DV, bool DECAY>
 struct ChunkPlan {
     // d = dv = 64: two CTAs share an SM, so one CTA's waits hide behind the other's work
     static constexpr bool TWO_PER_SM = D == 64 && DV == 64;
-    static constexpr int NW = TWO_PER_SM ? 8 : 16;        // worker warps
+    // worker warps: a TMEM group of NT (every lane quadrant) and a phi group of
+    // NW - NT; with the issuer warp a CTA has 16 (two per SM: 8) warps, four
+    // (two) per SM sub-partition, which leaves 128 registers a thread
+    static constexpr int NW = TWO_PER_SM ? 7 : 15;
+    static constexpr int NT = TWO_PER_SM ? 4 : 8;
     static constexpr int THREADS = (NW + 1) * 32;          // + the issuer warp
     static constexpr int STAGES = 2;
     static constexpr int NO = DV + 16;                     // accumulator columns of O and T
@@ -72,8 +76,8 @@ struct ChunkPlan {
     static constexpr int OFF_O = OFF_P + TILE;             // output staging bf16 [C][DV]
     static constexpr int OFF_WT = OFF_O + C * DV * 2;      // [4][C] fp32 decay weights of Q~, K~ and their log2
     static constexpr int OFF_BAR = OFF_WT + 4 * C * 4;
-    // full[S] empty[S] phi w_ready t_done p_full ptil o_full o_read os_full os_empty drain
-    static constexpr int NBAR = 2 * STAGES + 10;
+    // full[S] empty[S] phi[S] w_ready t_done p_full ptil o_full o_read os_full os_empty drain
+    static constexpr int NBAR = 3 * STAGES + 9;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;     // + alignment slack
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
@@ -362,16 +366,20 @@ scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float
 // ---------------------------------------------------------------------------
 // Kernel C: the chunk loop of one (chain, segment) from its start state.
 //
-// Roles: worker warps 0..NW-1 do the CUDA-core steps; lane 0 of warp NW (the
-// issuer) issues every TMA copy and every MMA.  Per chunk c:
-//   workers  [t_done(c-1)] W = gamma^C T -> TMEM (decay) and bf16 -> smem;
+// Roles: worker warps 0..NW-1 do the CUDA-core steps in two groups that run
+// side by side; lane 0 of warp NW (the issuer) issues every TMA copy and every
+// MMA.  Per chunk c:
+//   TMEM group (warps 0..NT-1, every lane quadrant)
+//            [t_done(c-1)] W = gamma^C T -> TMEM (decay) and bf16 -> smem;
 //            [p_full(c)]   P~ = causal mask of P -> bf16;
-//            [full(c+1)]   phi, weights of chunk c+1 in place;
 //            [o_full(c)]   o = O / (O[:, dv] + eps) -> staging
+//   phi group (warps NT..NW-1)
+//            [full(c)]     phi, weights of chunk c in place (runs a chunk ahead)
 //   issuer   [phi(c)] MMA1;  [w_ready(c), o_read(c-1)] MMA3, MMA4;
-//            [ptil(c)] MMA2;  TMA store of chunk c-1, loads of chunk c+2
-// The state chain of a CTA is t_done(c-1) -> W copy -> MMA3, MMA4 -> t_done(c);
-// everything else overlaps it (and the other CTA on the SM).
+//            TMA store of chunk c-1;  [ptil(c)] MMA2;  loads of chunk c+2
+// The state chain of a CTA is t_done(c-1) -> W copy -> MMA3, MMA4 -> t_done(c).
+// phi is bound by the exponential unit and the TMEM steps by load latency, so
+// the two groups fill each other's gaps.
 template <int D, int DV, bool DECAY>
 __global__ void __launch_bounds__(ChunkPlan<D, DV, DECAY>::THREADS, ChunkPlan<D, DV, DECAY>::TWO_PER_SM ? 2 : 1)
 chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -382,7 +390,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     using P = ChunkPlan<D, DV, DECAY>;
     constexpr int NW = P::NW;
     constexpr int NWT = NW * 32;                      // worker threads
-    constexpr int NQ = NW / 4;                        // worker warps per TMEM lane quadrant
+    constexpr int NT = P::NT;                         // TMEM group: warps 0 .. NT-1
+    constexpr int NTQ = NT / 4;                       // TMEM group warps per lane quadrant
+    constexpr int NPT = (NW - NT) * 32;               // phi group threads (warps NT .. NW-1)
     grid_launch_dependents();   // a following call's summary pass may start as this grid drains
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = align1024(smem_raw);
@@ -395,22 +405,25 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     float* lwk = wq + 3 * C;
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* empty = full + P::STAGES;
-    uint64_t* phi_rdy = empty + P::STAGES;   // workers: Q~, K~ of the chunk in place
-    uint64_t* w_rdy = phi_rdy + 1;           // workers: W copy written (and T rescaled)
-    uint64_t* t_done = phi_rdy + 2;          // MMA3 + MMA4 complete
-    uint64_t* p_full = phi_rdy + 3;          // MMA1 complete
-    uint64_t* ptil_rdy = phi_rdy + 4;        // workers: P~ written
-    uint64_t* o_full = phi_rdy + 5;          // MMA2 complete
-    uint64_t* o_read = phi_rdy + 6;          // workers: O read out
-    uint64_t* os_full = phi_rdy + 7;         // workers: output staging written
-    uint64_t* os_empty = phi_rdy + 8;        // issuer: staging read by its store
-    uint64_t* drain = phi_rdy + 9;           // issuer: every MMA it issued is complete
+    // phi group: Q~, K~ of the stage's chunk in place.  One barrier per stage: the
+    // phi group's warps run independently, and a warp that finished chunk c may
+    // arrive for chunk c + 1 before the others arrived for chunk c.
+    uint64_t* phi_rdy = empty + P::STAGES;
+    uint64_t* w_rdy = phi_rdy + P::STAGES;   // TMEM group: W copy written (and T rescaled)
+    uint64_t* t_done = w_rdy + 1;            // MMA3 + MMA4 complete
+    uint64_t* p_full = w_rdy + 2;            // MMA1 complete
+    uint64_t* ptil_rdy = w_rdy + 3;          // TMEM group: P~ written
+    uint64_t* o_full = w_rdy + 4;            // MMA2 complete
+    uint64_t* o_read = w_rdy + 5;            // TMEM group: O read out
+    uint64_t* os_full = w_rdy + 6;           // TMEM group: output staging written
+    uint64_t* os_empty = w_rdy + 7;          // issuer: staging read by its store
+    uint64_t* drain = w_rdy + 8;             // issuer: every MMA it issued is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool worker = warp < NW;
     const bool issuer = tid == NWT;
-    const int quad = warp & 3, qg = warp >> 2;        // TMEM lane quadrant, column group in it
+    const int quad = warp & 3;                        // TMEM lane quadrant
     const int unit = blockIdx.x;
     const Unit un = unit_of(m, unit);
     const int chain = un.chain, t0 = un.t0, t1 = un.t1;
@@ -425,14 +438,14 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     if (tid == 0) {
         for (int s = 0; s < P::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        mbar_init(phi_rdy, NW);
-        mbar_init(w_rdy, NW);
+        for (int s = 0; s < P::STAGES; ++s) mbar_init(&phi_rdy[s], NW - NT);
+        mbar_init(w_rdy, NT);
         mbar_init(t_done, 1);
         mbar_init(p_full, 1);
-        mbar_init(ptil_rdy, NW);
+        mbar_init(ptil_rdy, NT);
         mbar_init(o_full, 1);
-        mbar_init(o_read, NW);
-        mbar_init(os_full, NW);
+        mbar_init(o_read, NT);
+        mbar_init(os_full, NT);
         mbar_init(os_empty, 1);
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -497,7 +510,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const uint64_t dkm = sdesc_sw128(smem_u32(st + P::QB), TILE, 1024);      // K~^T, MN-major
             const uint64_t dvb = sdesc_sw128(smem_u32(st + P::QB + P::KB), TILE, 1024);   // [V | 1]
             // MMA1: P = Q~ K~^T (P of the previous chunk was read before its P~ was signalled)
-            if (!mbar_wait(phi_rdy, cp, kErrMma)) { bad = true; break; }
+            if (!mbar_wait(&phi_rdy[s], (c / P::STAGES) & 1, kErrMma)) { bad = true; break; }
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
@@ -518,6 +531,14 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             for (int ks = 0; ks < C / 16; ++ks)
                 mma_bf16(tbase + P::T_T, dkm + ((ks * 2048) >> 4), dvb + ((ks * 2048) >> 4), idt, 1u);
             mma_commit(t_done);
+            // the output of the previous chunk: its staging was written before W of
+            // this chunk (the TMEM group's order), so the wait returns at once
+            if (c >= 1) {
+                if (!mbar_wait(os_full, (c - 1) & 1, kErrMma)) { bad = true; break; }
+                fence_async_smem();
+                for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (c - 1) * C, chain);
+                tma_store_commit();
+            }
             // MMA2: O += P~ [V | 1]
             if (!mbar_wait(ptil_rdy, cp, kErrMma)) { bad = true; break; }
             tc_fence_after();
@@ -526,12 +547,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mma_bf16(tbase + P::T_O, dp + ((ks * 32) >> 4), dvb + ((ks * 2048) >> 4), ido, 1u);
             mma_commit(o_full);
             mma_commit(&empty[s]);
-            // output of the previous chunk, then the loads of chunk c + STAGES
+            // the staging is free once the store has read it (long done by now);
+            // then the loads of chunk c + STAGES
             if (c >= 1) {
-                if (!mbar_wait(os_full, (c - 1) & 1, kErrMma)) { bad = true; break; }
-                fence_async_smem();
-                for (int b = 0; b < DV / 64; ++b) tma_store_3d(&tm_o, otil + b * TILE, b * 64, t0 + (c - 1) * C, chain);
-                tma_store_commit();
                 tma_store_wait_read();
                 mbar_arrive(os_empty);
             }
@@ -550,24 +568,25 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
         mma_commit(drain);
         mbar_wait(drain, 0, kErrMma);
-    } else if (worker) {
-        // ---------------- workers ----------------
-        // phi of chunk c in place: Q~ = w_q phi(q), K~ = w_k phi(k) [t < n]
+    } else if (warp >= NT && warp < NW) {
+        // ---------------- phi group: Q~, K~ of every chunk in place ----------------
         // w phi(x) = w max(x, 0) + 2^(min(x, 0) log2 e + log2 w): the operand weight rides in
         // the exponent (w = 0, for key rows past the sequence's end, gives exactly 0)
-        auto phi = [&](int c) {
+        const int ptid = tid - NT * 32;
+        for (int c = 0; c < nch && !bad; ++c) {
+            if (!mbar_wait(&full[c % P::STAGES], (c / P::STAGES) & 1, kErrTmaLoad)) { bad = true; break; }
             const int n = chunk_len(c);
             unsigned char* qt = sm + (c % P::STAGES) * P::STAGE;
             unsigned char* kt = qt + P::QB;
             constexpr float kLog2e = 1.4426950408889634f;
-            for (int e = tid; e < (D / 8) * C; e += NWT) {
+#pragma unroll 1
+            for (int e = ptid; e < (D / 8) * C; e += NPT) {
                 const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
                 uint4* pq = reinterpret_cast<uint4*>(qt + b * TILE) + rem;
                 uint4* pk = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
                 const bool kv = row < n;
                 const float aq = DECAY ? wq[row] : 1.f, lq = DECAY ? lwq[row] : 0.f;
-                const float ak = kv ? (DECAY ? wk[row] : 1.f) : 0.f;
-                const float lk = kv ? (DECAY ? lwk[row] : 0.f) : -INFINITY;
+                const float ak = DECAY ? wk[row] : 1.f, lk = DECAY ? lwk[row] : 0.f;
                 float fq[8], fk[8];
                 unpack8(*pq, fq);
                 unpack8(*pk, fk);
@@ -577,85 +596,127 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     fk[x] = fmaf(fmaxf(fk[x], 0.f), ak, ex2_approx(fmaf(fminf(fk[x], 0.f), kLog2e, lk)));
                 }
                 *pq = pack8(fq, 1.f);
+                // key rows past the end are stored as zeros: a padded batch's padding
+                // may hold anything, and a zero weight times inf is not zero
                 *pk = kv ? pack8(fk, 1.f) : make_uint4(0u, 0u, 0u, 0u);
             }
-            if (clip_tail && c == nch - 1) zero_tail_rows<DV>(kt + P::KB, n, tid, NWT);
-        };
-        // T0 = S / kappa: the segment's start state (from the scan), normaliser as column dv
-        {
-            grid_dependency_wait();
-            const float* slot = ws + (size_t)unit * (D * DV + D);
-            const int f = acc_row<D>(quad, lane);
-            for (int g = qg; g < P::NO / 16; g += NQ) {
-                float v[16];
-#pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const int j = g * 16 + x;
-                    float t = 0.f;
-                    if (f >= 0) t = j < DV ? slot[(size_t)f * DV + j] : (j == DV ? slot[D * DV + f] : 0.f);
-                    v[x] = t * rkappa;
-                }
-                tmem_st16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
-            }
-            tmem_st_wait();
+            if (clip_tail && c == nch - 1) zero_tail_rows<DV>(kt + P::KB, n, ptid, NPT);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&phi_rdy[c % P::STAGES]);
         }
-        if (!mbar_wait(&full[0], 0, kErrTmaLoad)) bad = true;
-        if (!bad) phi(0);
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(phi_rdy);
-
+    } else if (worker) {
+        // ---------------- TMEM group: state copy, P~, output ----------------
+        // NTQ warps per TMEM lane quadrant; warp `sub` of a quadrant takes the
+        // 16-column groups sub, sub + NTQ, ...  Each batch of TMEM loads waits once.
+        const int sub = warp >> 2;
+        constexpr int KB = 1;       // TMEM loads per wait
         const int fr = acc_row<D>(quad, lane);      // state row of this thread (M = D accumulator)
         const int ir = acc_row<64>(quad, lane);     // score / output row (M = 64 accumulators)
-        for (int c = 0; c < nch && !bad; ++c) {
-            const uint32_t cp = c & 1;
-            // W = gamma^C T: back into TMEM (the carry adds to it) and as the bf16 B operand
-            if (c >= 1 && !mbar_wait(t_done, (c - 1) & 1, kErrMma)) bad = true;
-            tc_fence_after();
-            for (int g = qg; g < P::NO / 16; g += NQ) {
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
-                tmem_ld_wait();
-                if (DECAY) {
+        // W = gamma^C T of one 16-column group: into TMEM (the carry adds to it) and
+        // as the bf16 B operand
+        auto put_w = [&](int g, float (&v)[16], bool to_tmem) {
+            if (DECAY) {
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) v[x] = one_factor ? v[x] * gC : (v[x] * gH) * gH;
-                    tmem_st16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
-                }
-                if (fr >= 0) {
-                    unsigned char* blk = wcp + (g / 4) * P::WBLK;
-                    const int byte0 = (g % 4) * 32;
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(fr, byte0)) =
-                        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                   pack_bf16x2(v[6], v[7]));
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(fr, byte0 + 16)) =
-                        make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                                   pack_bf16x2(v[14], v[15]));
-                }
+                for (int x = 0; x < 16; ++x) v[x] = one_factor ? v[x] * gC : (v[x] * gH) * gH;
             }
-            if (DECAY) tmem_st_wait();
+            if (to_tmem) tmem_st16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
+            if (fr >= 0) {
+                unsigned char* blk = wcp + (g / 4) * P::WBLK;
+                const int byte0 = (g % 4) * 32;
+                *reinterpret_cast<uint4*>(blk + sw128_offset(fr, byte0)) =
+                    make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                               pack_bf16x2(v[6], v[7]));
+                *reinterpret_cast<uint4*>(blk + sw128_offset(fr, byte0 + 16)) =
+                    make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                               pack_bf16x2(v[14], v[15]));
+            }
+        };
+        auto w_ready = [&]() {
+            tmem_st_wait();
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(w_rdy);
-
-            // P~ = causal mask of P (rows i, 64 / NQ columns per warp); the previous
-            // chunk's MMA2 has read P~ (its output was waited for)
-            if (!mbar_wait(p_full, cp, kErrMma)) bad = true;
-            tc_fence_after();
-            for (int g = qg; g < 4; g += NQ) {
+        };
+        // chunk 0: T0 = S / kappa, the segment's start state from the scan (normaliser
+        // as column dv), goes to TMEM and to W straight from the registers
+        {
+            grid_dependency_wait();
+            const float* slot = ws + (size_t)unit * (D * DV + D);
+#pragma unroll 1
+            for (int g = sub; g < P::NO / 16; g += NTQ) {
                 float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_P + g * 16), v);
-                tmem_ld_wait();
-                if (ir >= 0) {
-                    uint32_t pk[8];
+                if (g < DV / 16) {
+                    const float4* src = reinterpret_cast<const float4*>(slot + (size_t)(fr >= 0 ? fr : 0) * DV + g * 16);
 #pragma unroll
-                    for (int h = 0; h < 8; ++h) {
-                        const int j = g * 16 + 2 * h;
-                        pk[h] = pack_bf16x2(j <= ir ? v[2 * h] : 0.f, j + 1 <= ir ? v[2 * h + 1] : 0.f);
+                    for (int x = 0; x < 4; ++x) {
+                        const float4 t = fr >= 0 ? src[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+                        v[4 * x] = t.x * rkappa;
+                        v[4 * x + 1] = t.y * rkappa;
+                        v[4 * x + 2] = t.z * rkappa;
+                        v[4 * x + 3] = t.w * rkappa;
                     }
-                    *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32 + 16)) =
-                        make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) v[x] = 0.f;
+                    if (fr >= 0) v[0] = slot[D * DV + fr] * rkappa;
+                }
+                put_w(g, v, true);
+            }
+            w_ready();
+        }
+
+        for (int c = 0; c < nch && !bad; ++c) {
+            const uint32_t cp = c & 1;
+            if (c >= 1) {
+                // W = gamma^C T from the carried state
+                if (!mbar_wait(t_done, (c - 1) & 1, kErrMma)) { bad = true; break; }
+                tc_fence_after();
+                constexpr int NGT = P::NO / 16;
+#pragma unroll 1
+                for (int g0 = sub; g0 < NGT; g0 += KB * NTQ) {
+                    float v[KB][16];
+#pragma unroll
+                    for (int i = 0; i < KB; ++i)
+                        if (g0 + i * NTQ < NGT) tmem_ld16(tmem_addr(tbase, quad, P::T_T + (g0 + i * NTQ) * 16), v[i]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < KB; ++i) tmem_regs_after_wait(v[i]);
+#pragma unroll
+                    for (int i = 0; i < KB; ++i)
+                        if (g0 + i * NTQ < NGT) put_w(g0 + i * NTQ, v[i], DECAY);
+                }
+                w_ready();
+            }
+
+            // P~ = causal mask of P (rows i); the previous chunk's MMA2 has read P~
+            // (its output was waited for)
+            if (!mbar_wait(p_full, cp, kErrMma)) { bad = true; break; }
+            tc_fence_after();
+#pragma unroll 1
+            for (int g0 = sub; g0 < 4; g0 += KB * NTQ) {
+                float v[KB][16];
+#pragma unroll
+                for (int i = 0; i < KB; ++i) tmem_ld16(tmem_addr(tbase, quad, P::T_P + (g0 + i * NTQ) * 16), v[i]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < KB; ++i) tmem_regs_after_wait(v[i]);
+                if (ir >= 0) {
+#pragma unroll
+                    for (int i = 0; i < KB; ++i) {
+                        const int g = g0 + i * NTQ;
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            const int j = g * 16 + 2 * h;
+                            pk[h] = pack_bf16x2(j <= ir ? v[i][2 * h] : 0.f, j + 1 <= ir ? v[i][2 * h + 1] : 0.f);
+                        }
+                        *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32)) =
+                            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32 + 16)) =
+                            make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
                 }
             }
             fence_async_smem();
@@ -663,49 +724,49 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) mbar_arrive(ptil_rdy);
 
-            // phi of the next chunk (its stage landed while this one computed)
-            if (c + 1 < nch) {
-                if (!mbar_wait(&full[(c + 1) % P::STAGES], ((c + 1) / P::STAGES) & 1, kErrTmaLoad)) bad = true;
-                else phi(c + 1);
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(phi_rdy);
-            }
-
             // output rows: o = O[:, :dv] / (O[:, dv] + eps) -> staging
-            if (!mbar_wait(o_full, cp, kErrMma)) bad = true;
+            if (!mbar_wait(o_full, cp, kErrMma)) { bad = true; break; }
             tc_fence_after();
-            float den[16];
-            tmem_ld16(tmem_addr(tbase, quad, P::T_O + DV), den);
-            tmem_ld_wait();
-            const float rden = __frcp_rn(den[0] + eps);
+            float den = tmem_ld1(tmem_addr(tbase, quad, P::T_O + DV));
             if (c >= 1 && !mbar_wait(os_empty, (c - 1) & 1, kErrMma)) bad = true;
             const bool direct = clip_tail && c == nch - 1;
             const int nrow = chunk_len(c);
-            for (int g = qg; g < DV / 16; g += NQ) {
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_O + g * 16), v);
+            constexpr int NGO = DV / 16;
+#pragma unroll 1
+            for (int g0 = sub; g0 < NGO; g0 += KB * NTQ) {
+                float v[KB][16];
+#pragma unroll
+                for (int i = 0; i < KB; ++i)
+                    if (g0 + i * NTQ < NGO) tmem_ld16(tmem_addr(tbase, quad, P::T_O + (g0 + i * NTQ) * 16), v[i]);
                 tmem_ld_wait();
-                if (direct) {
-                    // the padded batch's last rows of this sequence: only rows < n are written
-                    if (ir >= 0 && ir < nrow) {
-                        uint4* dst = reinterpret_cast<uint4*>(
-                            out + ((size_t)chain * ld + t0 + c * C + ir) * DV + g * 16);
-                        dst[0] = make_uint4(pack_bf16x2(v[0] * rden, v[1] * rden), pack_bf16x2(v[2] * rden, v[3] * rden),
-                                            pack_bf16x2(v[4] * rden, v[5] * rden), pack_bf16x2(v[6] * rden, v[7] * rden));
-                        dst[1] = make_uint4(pack_bf16x2(v[8] * rden, v[9] * rden), pack_bf16x2(v[10] * rden, v[11] * rden),
-                                            pack_bf16x2(v[12] * rden, v[13] * rden),
-                                            pack_bf16x2(v[14] * rden, v[15] * rden));
+#pragma unroll
+                for (int i = 0; i < KB; ++i) tmem_regs_after_wait(v[i]);
+                tmem_regs_after_wait(den);
+                const float rden = __frcp_rn(den + eps);
+#pragma unroll
+                for (int i = 0; i < KB; ++i) {
+                    const int g = g0 + i * NTQ;
+                    if (g < NGO) {
+                    const float* o = v[i];
+                    const uint4 lo = make_uint4(pack_bf16x2(o[0] * rden, o[1] * rden), pack_bf16x2(o[2] * rden, o[3] * rden),
+                                                pack_bf16x2(o[4] * rden, o[5] * rden), pack_bf16x2(o[6] * rden, o[7] * rden));
+                    const uint4 hi = make_uint4(pack_bf16x2(o[8] * rden, o[9] * rden), pack_bf16x2(o[10] * rden, o[11] * rden),
+                                                pack_bf16x2(o[12] * rden, o[13] * rden),
+                                                pack_bf16x2(o[14] * rden, o[15] * rden));
+                    if (direct) {
+                        // the padded batch's last rows of this sequence: only rows < n are written
+                        if (ir >= 0 && ir < nrow) {
+                            uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)chain * ld + t0 + c * C + ir) * DV + g * 16);
+                            dst[0] = lo;
+                            dst[1] = hi;
+                        }
+                    } else if (ir >= 0) {
+                        unsigned char* blk = otil + (g / 4) * TILE;
+                        const int byte0 = (g % 4) * 32;
+                        *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0)) = lo;
+                        *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0 + 16)) = hi;
                     }
-                } else if (ir >= 0) {
-                    unsigned char* blk = otil + (g / 4) * TILE;
-                    const int byte0 = (g % 4) * 32;
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0)) =
-                        make_uint4(pack_bf16x2(v[0] * rden, v[1] * rden), pack_bf16x2(v[2] * rden, v[3] * rden),
-                                   pack_bf16x2(v[4] * rden, v[5] * rden), pack_bf16x2(v[6] * rden, v[7] * rden));
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0 + 16)) =
-                        make_uint4(pack_bf16x2(v[8] * rden, v[9] * rden), pack_bf16x2(v[10] * rden, v[11] * rden),
-                                   pack_bf16x2(v[12] * rden, v[13] * rden), pack_bf16x2(v[14] * rden, v[15] * rden));
+                    }
                 }
             }
             tc_fence_before();

@@ -285,7 +285,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// One column: thread t of the warp receives lane (warp quadrant base + t), column col.
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr)
+{
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return __uint_as_float(r);
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// tcgen05.ld fills its registers asynchronously, but the compiler sees them as
+// written by the load itself and may move a computation on them above the
+// wait (a loop-invariant one, say).  Passing the values through an empty
+// volatile statement after the wait ties every later use to the wait.
+__device__ __forceinline__ void tmem_regs_after_wait(float& x) { asm volatile("" : "+f"(x)); }
+template <int N>
+__device__ __forceinline__ void tmem_regs_after_wait(float (&v)[N])
+{
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
 {
