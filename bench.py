@@ -566,14 +566,14 @@ TRAFFIC_CAPTURES = {
         "bytes": 2727170048 + 405584128, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
         "sha256": "c7a8ade2fe0fc70fcf7996bdca15f82c27f81b22e80b1c05fae9fb5db6494d9f"},
     ("plain_bf16", "chunk_kernel"): {
-        "bytes": 54631680 + 423168, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "31a166ca127dd08e294d19aaea425624b4bbfac4aba1b10a9d0bdcabaeb942cd"},
+        "bytes": 54629376 + 315648, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "b237f56eec21ccb6550652fe15ed34583fd08837bbad5b2fdef8d9f28e12beed"},
     ("decay_bf16", "chunk_kernel"): {
-        "bytes": 824675072 + 209730816, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "31a166ca127dd08e294d19aaea425624b4bbfac4aba1b10a9d0bdcabaeb942cd"},
+        "bytes": 824387072 + 209595136, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "b237f56eec21ccb6550652fe15ed34583fd08837bbad5b2fdef8d9f28e12beed"},
     ("gla_bf16", "gla_chunk_kernel"): {
-        "bytes": 343998464 + 34603776, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
-        "sha256": "df531a0094a1c31add68b9a1e698af5ce866bdb8c811d3172ea2235d3476a473"},
+        "bytes": 344070912 + 34972672, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
+        "sha256": "a9a55bd527432b8b9b9242190501241d82556415c0a1a57f7858652060f5bad1"},
 }
 
 

@@ -524,19 +524,9 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (lane == 0) mbar_arrive(phi_rdy);
             return false;
         };
-        // T = S (the segment's start state, from the scan)
-        {
-            grid_dependency_wait();
-            const float* slot = ws + (size_t)unit * (D * DV + D);
-            const int f = acc_row<D>(quad, lane);
-            for (int g = qg; g < DV / 16; g += NQ) {
-                float v[16];
-#pragma unroll
-                for (int x = 0; x < 16; ++x) v[x] = f >= 0 ? slot[(size_t)f * DV + g * 16 + x] : 0.f;
-                tmem_st16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
-            }
-            tmem_st_wait();
-        }
+        // the segment's start state S (from the scan) is read in chunk 0's state step
+        grid_dependency_wait();
+        const float* slot = ws + (size_t)unit * (D * DV + D);
         bool stop = nch > 0 ? gates(0) : false;
 
         const int fr = acc_row<D>(quad, lane);
@@ -549,8 +539,22 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const float eb = fr >= 0 ? ebc[cp * D + fr] : 0.f;
             for (int g = qg; g < DV / 16; g += NQ) {
                 float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
-                tmem_ld_wait();
+                if (c == 0) {
+                    // chunk 0: S straight from the scan's slot (16-byte loads), not via TMEM
+                    const float4* src = reinterpret_cast<const float4*>(slot + (size_t)(fr >= 0 ? fr : 0) * DV + g * 16);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const float4 t = fr >= 0 ? src[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+                        v[4 * x] = t.x;
+                        v[4 * x + 1] = t.y;
+                        v[4 * x + 2] = t.z;
+                        v[4 * x + 3] = t.w;
+                    }
+                } else {
+                    tmem_ld16(tmem_addr(tbase, quad, P::T_T + g * 16), v);
+                    tmem_ld_wait();
+                    tmem_regs_after_wait(v);
+                }
                 if (fr >= 0) {
                     unsigned char* blk = scp + (g / 4) * P::SBLK;
                     const int byte0 = (g % 4) * 32;
