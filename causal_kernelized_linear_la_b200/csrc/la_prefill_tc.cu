@@ -95,8 +95,8 @@ struct SummaryPlan {
     // B = [V | 1] makes column dv of K~^T B the normaliser sum Delta z
     static constexpr int LOAD_BYTES = KB + VB;
     static constexpr int STAGE = KB + VB + TILE;
-    static constexpr int OFF_BAR = STAGES * STAGE;                // full[S], empty[S], done
-    static constexpr int OFF_TMEM = OFF_BAR + (2 * STAGES + 1) * 8;
+    static constexpr int OFF_BAR = STAGES * STAGE;                // full[S], empty[S], phi[S], done
+    static constexpr int OFF_TMEM = OFF_BAR + (3 * STAGES + 1) * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static constexpr int NS = DV + 16;                            // accumulator columns
     static constexpr uint32_t T_S = 0, T_COLS = 256;
@@ -169,8 +169,13 @@ __device__ __forceinline__ void zero_tail_rows(unsigned char* vt, int n, int tid
 // ---------------------------------------------------------------------------
 // Kernel A: segment summaries  Delta S = sum_t gamma^(last-t) phi(k_t) v_t^T,
 // Delta z = sum_t gamma^(last-t) phi(k_t), over the tokens of one segment.
+//
+// Roles: warps 0..15 apply phi (and the decay weight) to each stage's K in
+// place and signal its per-stage barrier; lane 0 of warp 16 issues the TMA
+// loads and the MMAs.  The phi warps run as far ahead as the loads allow, so
+// their exponentials overlap the copies and the contraction.
 template <int D, int DV, bool DECAY>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads + 32, 1)
 summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const float* __restrict__ gamma, float* __restrict__ ws, const __grid_constant__ SegMap m)
 {
@@ -180,11 +185,13 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     unsigned char* sm = align1024(smem_raw);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* empty = full + P::STAGES;
-    uint64_t* done = empty + P::STAGES;
+    uint64_t* phi_rdy = empty + P::STAGES;   // phi warps: K~ of the stage's chunk in place
+    uint64_t* done = phi_rdy + P::STAGES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, wg = warp >> 2;
+    const int quad = warp & 3, wg = (warp >> 2) & 3;
+    const bool issuer = tid == kThreads;
     const int unit = blockIdx.x;
     const Unit un = unit_of(m, unit);
     const int chain = un.chain, t0 = un.t0, t1 = un.t1;
@@ -193,14 +200,18 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     const uint64_t pol = policy_evict_last();  // the chunk kernel reads k, v again
 
     if (tid == 0) {
-        for (int s = 0; s < P::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < P::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&phi_rdy[s], kThreads / 32);
+        }
         mbar_init(done, 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, P::T_COLS);
     // the ones-column tile of every stage: element (t, 0) = 1, the rest 0
     for (int s = 0; s < P::STAGES; ++s)
-        for (int e = tid; e < C * 8; e += kThreads) {
+        for (int e = tid; e < C * 8; e += kThreads + 32) {
             const int row = e / 8, chunk = e % 8;
             // logical chunk 0 of row `row` sits at physical chunk row % 8
             const uint32_t w = chunk == (row & 7) ? 0x3F80u : 0u;   // bf16 1.0 in the low half
@@ -212,55 +223,26 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
-    int loads_issued = 0, loads_waited = 0, commits = 0;
-    auto issue = [&](int c) {
-        const int s = c % P::STAGES;
-        unsigned char* st = sm + s * P::STAGE;
-        mbar_expect_tx(&full[s], P::LOAD_BYTES);
-        for (int b = 0; b < D / 64; ++b) tma_load_3d(st + b * TILE, &tm_k, b * 64, t0 + c * C, chain, &full[s], pol);
-        for (int b = 0; b < DV / 64; ++b)
-            tma_load_3d(st + P::KB + b * TILE, &tm_v, b * 64, t0 + c * C, chain, &full[s], pol);
-        loads_issued = c + 1;
-    };
-    if (tid == 0)
-        for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
-
     bool bad = false;
-    const int last = t1 - 1;
-    for (int c = 0; c < nch; ++c) {
-        const int s = c % P::STAGES;
-        const uint32_t ph = (c / P::STAGES) & 1;
-        unsigned char* kt = sm + s * P::STAGE;
-        unsigned char* vt = kt + P::KB;
-        if (!mbar_wait(&full[s], ph, kErrTmaLoad)) bad = true;
-        else loads_waited = c + 1;
-        if (un.clip && t1 - (t0 + c * C) < C) zero_tail_rows<DV>(vt, t1 - (t0 + c * C), tid, kThreads);
-        // K~_t = gamma^(last - t) phi(k_t), zero past the end of the sequence
-        const int tc0 = t0 + c * C;
-        for (int e = tid; e < (D / 8) * C; e += kThreads) {
-            const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
-            uint4* p = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
-            const int t = tc0 + row;
-            const float w = t <= last ? (DECAY ? __expf((float)(last - t) * lam) : 1.f) : 0.f;
-            float f[8];
-            unpack8(*p, f);
-#pragma unroll
-            for (int x = 0; x < 8; x += 2) {
-                const float2 y = phi2_fast(f[x], f[x + 1]);
-                f[x] = y.x; f[x + 1] = y.y;
-            }
-            // rows past the end are stored as zeros: a padded batch's padding
-            // may hold anything, and a zero weight times inf is not zero
-            *p = t <= last ? pack8(f, w) : make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(bad)) { bad = true; break; }
-        if (tid == 0) {
-            // [Delta S | Delta z] += K~^T [V | 1]   (M = d, N = dv + 16)
+    if (issuer) {
+        int loads = 0, commits = 0;
+        auto issue = [&](int c) {
+            const int s = c % P::STAGES;
+            unsigned char* st = sm + s * P::STAGE;
+            mbar_expect_tx(&full[s], P::LOAD_BYTES);
+            for (int b = 0; b < D / 64; ++b) tma_load_3d(st + b * TILE, &tm_k, b * 64, t0 + c * C, chain, &full[s], pol);
+            for (int b = 0; b < DV / 64; ++b)
+                tma_load_3d(st + P::KB + b * TILE, &tm_v, b * 64, t0 + c * C, chain, &full[s], pol);
+            loads = c + 1;
+        };
+        for (int c = 0; c < min(nch, P::STAGES); ++c) issue(c);
+        const uint32_t id_s = idesc_bf16_f32(D, P::NS, 1, 1);
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % P::STAGES;
+            if (!mbar_wait(&phi_rdy[s], (c / P::STAGES) & 1, kErrMma)) { bad = true; break; }
             tc_fence_after();
-            const uint32_t ka = smem_u32(kt), va = smem_u32(vt);
-            const uint32_t id_s = idesc_bf16_f32(D, P::NS, 1, 1);
+            // [Delta S | Delta z] += K~^T [V | 1]   (M = d, N = dv + 16)
+            const uint32_t ka = smem_u32(sm + s * P::STAGE), va = ka + P::KB;
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks)
                 mma_bf16(tbase + P::T_S, sdesc_sw128(ka + ks * 2048, TILE, 1024),
@@ -268,19 +250,56 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             mma_commit(&empty[s]);
             if (c == nch - 1) mma_commit(done);
             commits = c + 1;
+            // refill the stage chunk c-1 used: its MMA was issued a chunk ago
+            if (c >= 1 && c - 1 + P::STAGES < nch) {
+                if (!mbar_wait(&empty[(c - 1) % P::STAGES], ((c - 1) / P::STAGES) & 1, kErrMma)) { bad = true; break; }
+                issue(c - 1 + P::STAGES);
+            }
         }
-        // refill the stage chunk c-1 used: its MMA was issued a whole chunk ago.
-        // The other threads go on to phi of the next chunk meanwhile.
-        if (tid == 0 && c >= 1 && c - 1 + P::STAGES < nch) {
-            const int sp = (c - 1) % P::STAGES;
-            if (!mbar_wait(&empty[sp], ((c - 1) / P::STAGES) & 1, kErrMma)) bad = true;
-            else issue(c - 1 + P::STAGES);
+        if (bad) {
+            // leave no copy or MMA in flight before TMEM is released
+            for (int cc = max(0, loads - P::STAGES); cc < loads; ++cc)
+                mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
+            if (commits > 0)
+                mbar_wait(&empty[(commits - 1) % P::STAGES], ((commits - 1) / P::STAGES) & 1, kErrMma);
         }
+    } else if (warp < kThreads / 32) {
+        const int last = t1 - 1;
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % P::STAGES;
+            unsigned char* kt = sm + s * P::STAGE;
+            unsigned char* vt = kt + P::KB;
+            if (!mbar_wait(&full[s], (c / P::STAGES) & 1, kErrTmaLoad)) { bad = true; break; }
+            if (un.clip && t1 - (t0 + c * C) < C) zero_tail_rows<DV>(vt, t1 - (t0 + c * C), tid, kThreads);
+            // K~_t = gamma^(last - t) phi(k_t), zero past the end of the sequence
+            const int tc0 = t0 + c * C;
+            for (int e = tid; e < (D / 8) * C; e += kThreads) {
+                const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
+                uint4* p = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
+                const int t = tc0 + row;
+                const float w = t <= last ? (DECAY ? __expf((float)(last - t) * lam) : 1.f) : 0.f;
+                float f[8];
+                unpack8(*p, f);
+#pragma unroll
+                for (int x = 0; x < 8; x += 2) {
+                    const float2 y = phi2_fast(f[x], f[x + 1]);
+                    f[x] = y.x; f[x + 1] = y.y;
+                }
+                // rows past the end are stored as zeros: a padded batch's padding
+                // may hold anything, and a zero weight times inf is not zero
+                *p = t <= last ? pack8(f, w) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&phi_rdy[s]);
+        }
+        if (!bad && !mbar_wait(done, 0, kErrMma)) bad = true;
     }
-    if (!bad && !mbar_wait(done, 0, kErrMma)) bad = true;
+    // every thread agrees whether the summary is complete before it is read out
+    const bool any_bad = __syncthreads_or(bad);
     tc_fence_after();
     float* slot = ws + (size_t)unit * (D * DV + D);
-    if (!bad) {
+    if (!any_bad && warp < kThreads / 32) {
         const int f = acc_row<D>(quad, lane);
 #pragma unroll
         for (int gg = 0; gg < DV / 64; ++gg) {
@@ -288,6 +307,7 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             float v[16];
             tmem_ld16(tmem_addr(tbase, quad, P::T_S + col0), v);
             tmem_ld_wait();
+            tmem_regs_after_wait(v);
             if (f >= 0) {
                 float4* dst = reinterpret_cast<float4*>(slot + (size_t)f * DV + col0);
 #pragma unroll
@@ -296,18 +316,11 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         }
         // Delta z: accumulator column dv, one row (feature) per lane
         if (wg == 0) {
-            float v[16];
-            tmem_ld16(tmem_addr(tbase, quad, P::T_S + DV), v);
+            float z = tmem_ld1(tmem_addr(tbase, quad, P::T_S + DV));
             tmem_ld_wait();
-            if (f >= 0) slot[D * DV + f] = v[0];
+            tmem_regs_after_wait(z);
+            if (f >= 0) slot[D * DV + f] = z;
         }
-    }
-    if (bad && tid == 0) {
-        // Leave no copy or MMA in flight before releasing TMEM and exiting.
-        for (int cc = loads_waited; cc < loads_issued; ++cc)
-            mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
-        if (commits > 0)
-            mbar_wait(&empty[(commits - 1) % P::STAGES], ((commits - 1) / P::STAGES) & 1, kErrMma);
     }
     tc_fence_before();
     __syncthreads();
@@ -845,7 +858,7 @@ cudaError_t launch_tc_map(const PrefillArgs& a, const SegMap& m, int units)
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(units);
-    lc.blockDim = dim3(kThreads);
+    lc.blockDim = dim3(kThreads + 32);   // + the issuing warp
     lc.dynamicSmemBytes = sa;
     lc.stream = a.stream;
     lc.attrs = pdl;
