@@ -16,13 +16,15 @@ def _dev(p):
     return b(p.q_bits), b(p.k_bits), b(p.v_bits)
 
 
-@pytest.mark.parametrize("name,nk", [("plain_bf16", 3), ("gdelta_bf16", 2)])
+@pytest.mark.parametrize("name,nk", [("plain_bf16", 3), ("gdelta_bf16", 2), ("gla_bf16", 3)])
 def test_stage_events_follow_the_kernels(name, nk):
     p = inputs.make_workload(name, B=1, H=2, N=512)
     q, k, v = _dev(p)
     kw = {}
     if p.mode == "gated_delta":
         kw = dict(alpha=torch.from_numpy(p.alpha).cuda(), g=torch.from_numpy(p.g).cuda())
+    elif p.mode == "gla":
+        kw = dict(alpha=torch.from_numpy(p.alpha).cuda())
     ref = la.la_prefill(q, k, v, mode=p.mode, **kw)
     torch.cuda.synchronize()
     s = torch.cuda.current_stream()
