@@ -271,23 +271,27 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             unsigned char* vt = kt + P::KB;
             if (!mbar_wait(&full[s], (c / P::STAGES) & 1, kErrTmaLoad)) { bad = true; break; }
             if (un.clip && t1 - (t0 + c * C) < C) zero_tail_rows<DV>(vt, t1 - (t0 + c * C), tid, kThreads);
-            // K~_t = gamma^(last - t) phi(k_t), zero past the end of the sequence
+            // K~_t = gamma^(last - t) phi(k_t), zero past the end of the sequence:
+            // w phi(x) = w max(x, 0) + 2^((x - max(x, 0)) log2 e + log2 w), the weight
+            // riding in the exponent
+            constexpr float kLog2e = 1.4426950408889634f;
             const int tc0 = t0 + c * C;
             for (int e = tid; e < (D / 8) * C; e += kThreads) {
                 const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
                 uint4* p = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
                 const int t = tc0 + row;
-                const float w = t <= last ? (DECAY ? __expf((float)(last - t) * lam) : 1.f) : 0.f;
+                const float lw = DECAY ? (float)(last - t) * lam * kLog2e : 0.f;
+                const float w = DECAY ? ex2_approx(lw) : 1.f;
                 float f[8];
                 unpack8(*p, f);
 #pragma unroll
-                for (int x = 0; x < 8; x += 2) {
-                    const float2 y = phi2_fast(f[x], f[x + 1]);
-                    f[x] = y.x; f[x + 1] = y.y;
+                for (int x = 0; x < 8; ++x) {
+                    const float mx = fmaxf(f[x], 0.f);
+                    f[x] = fmaf(mx, w, ex2_approx(fmaf(f[x] - mx, kLog2e, lw)));
                 }
                 // rows past the end are stored as zeros: a padded batch's padding
                 // may hold anything, and a zero weight times inf is not zero
-                *p = t <= last ? pack8(f, w) : make_uint4(0u, 0u, 0u, 0u);
+                *p = t <= last ? pack8(f, 1.f) : make_uint4(0u, 0u, 0u, 0u);
             }
             fence_async_smem();
             __syncwarp();
@@ -605,8 +609,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 unpack8(*pk, fk);
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
-                    fq[x] = fmaf(fmaxf(fq[x], 0.f), aq, ex2_approx(fmaf(fminf(fq[x], 0.f), kLog2e, lq)));
-                    fk[x] = fmaf(fmaxf(fk[x], 0.f), ak, ex2_approx(fmaf(fminf(fk[x], 0.f), kLog2e, lk)));
+                    // min(x, 0) = x - max(x, 0) exactly: an add instead of a second min
+                    const float mq = fmaxf(fq[x], 0.f), mk = fmaxf(fk[x], 0.f);
+                    fq[x] = fmaf(mq, aq, ex2_approx(fmaf(fq[x] - mq, kLog2e, lq)));
+                    fk[x] = fmaf(mk, ak, ex2_approx(fmaf(fk[x] - mk, kLog2e, lk)));
                 }
                 *pq = pack8(fq, 1.f);
                 // key rows past the end are stored as zeros: a padded batch's padding
@@ -707,29 +713,35 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             // (its output was waited for)
             if (!mbar_wait(p_full, cp, kErrMma)) { bad = true; break; }
             tc_fence_after();
+            // This warp's rows are quad*16 .. quad*16+15 (lanes 0-15), so its column
+            // groups below quad are kept whole, group quad is the diagonal block, and
+            // the groups above are zero (not loaded).
 #pragma unroll 1
-            for (int g0 = sub; g0 < 4; g0 += KB * NTQ) {
-                float v[KB][16];
+            for (int g = sub; g < 4; g += NTQ) {
+                uint32_t pk[8];
+                if (g > quad) {
 #pragma unroll
-                for (int i = 0; i < KB; ++i) tmem_ld16(tmem_addr(tbase, quad, P::T_P + (g0 + i * NTQ) * 16), v[i]);
-                tmem_ld_wait();
+                    for (int h = 0; h < 8; ++h) pk[h] = 0u;
+                } else {
+                    float v[16];
+                    tmem_ld16(tmem_addr(tbase, quad, P::T_P + g * 16), v);
+                    tmem_ld_wait();
+                    tmem_regs_after_wait(v);
+                    if (g < quad) {
 #pragma unroll
-                for (int i = 0; i < KB; ++i) tmem_regs_after_wait(v[i]);
-                if (ir >= 0) {
-#pragma unroll
-                    for (int i = 0; i < KB; ++i) {
-                        const int g = g0 + i * NTQ;
-                        uint32_t pk[8];
+                        for (int h = 0; h < 8; ++h) pk[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
+                    } else {
 #pragma unroll
                         for (int h = 0; h < 8; ++h) {
                             const int j = g * 16 + 2 * h;
-                            pk[h] = pack_bf16x2(j <= ir ? v[i][2 * h] : 0.f, j + 1 <= ir ? v[i][2 * h + 1] : 0.f);
+                            pk[h] = pack_bf16x2(j <= ir ? v[2 * h] : 0.f, j + 1 <= ir ? v[2 * h + 1] : 0.f);
                         }
-                        *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32)) =
-                            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32 + 16)) =
-                            make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
+                }
+                if (ir >= 0) {
+                    *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4*>(ptil + sw128_offset(ir, g * 32 + 16)) =
+                        make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             }
             fence_async_smem();

@@ -368,15 +368,6 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
-// elu(x) + 1 for a pair of values: x + 1 above zero, e^x at or below it.
-// The exponential takes the full fp32 argument min(x, 0) (SFU __expf, a
-// relative error of a few fp32 ulps, far below the bf16 rounding applied to
-// the result); large negative x gives e^x -> 0.
-__device__ __forceinline__ float2 phi2_fast(float x0, float x1)
-{
-    return make_float2(fmaxf(x0, 0.f) + __expf(fminf(x0, 0.f)), fmaxf(x1, 0.f) + __expf(fminf(x1, 0.f)));
-}
-
 // ---- programmatic dependent launch ---------------------------------------------
 
 // Wait until the grids this one depends on (launched before it on the stream
