@@ -578,10 +578,18 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // P~ = causal mask of P
             if (!bad && !mbar_wait(p_full, cp, kErrMma)) bad = true;
             tc_fence_after();
+            // this warp's rows are quad*16 .. quad*16+15: column groups above quad are
+            // zero (not loaded), the one at quad is the diagonal block
             for (int g = qg; g < 4; g += NQ) {
                 float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_P + g * 16), v);
-                tmem_ld_wait();
+                if (g <= quad) {
+                    tmem_ld16(tmem_addr(tbase, quad, P::T_P + g * 16), v);
+                    tmem_ld_wait();
+                    tmem_regs_after_wait(v);
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) v[x] = 0.f;
+                }
                 if (ir >= 0) {
                     uint32_t pk[8];
 #pragma unroll
@@ -606,19 +614,30 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (!bad && !mbar_wait(o_full, cp, kErrMma)) bad = true;
             tc_fence_after();
             if (!bad && c >= 1 && !mbar_wait(os_empty, (c - 1) & 1, kErrMma)) bad = true;
-            for (int g = qg; g < DV / 16; g += NQ) {
-                float v[16];
-                tmem_ld16(tmem_addr(tbase, quad, P::T_O + g * 16), v);
+            // all of this warp's column groups (at most two) per TMEM wait
+            {
+                constexpr int NGO = (DV / 16 + NQ - 1) / NQ;
+                float v[NGO][16];
+#pragma unroll
+                for (int i = 0; i < NGO; ++i)
+                    if (qg + i * NQ < DV / 16) tmem_ld16(tmem_addr(tbase, quad, P::T_O + (qg + i * NQ) * 16), v[i]);
                 tmem_ld_wait();
-                if (ir >= 0) {
-                    unsigned char* blk = otil + (g / 4) * TILE;
-                    const int byte0 = (g % 4) * 32;
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0)) =
-                        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                   pack_bf16x2(v[6], v[7]));
-                    *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0 + 16)) =
-                        make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                                   pack_bf16x2(v[14], v[15]));
+#pragma unroll
+                for (int i = 0; i < NGO; ++i) tmem_regs_after_wait(v[i]);
+#pragma unroll
+                for (int i = 0; i < NGO; ++i) {
+                    const int g = qg + i * NQ;
+                    if (g < DV / 16 && ir >= 0) {
+                        unsigned char* blk = otil + (g / 4) * TILE;
+                        const int byte0 = (g % 4) * 32;
+                        const float* o = v[i];
+                        *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0)) =
+                            make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                       pack_bf16x2(o[6], o[7]));
+                        *reinterpret_cast<uint4*>(blk + sw128_offset(ir, byte0 + 16)) =
+                            make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
+                                       pack_bf16x2(o[14], o[15]));
+                    }
                 }
             }
             tc_fence_before();
