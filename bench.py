@@ -566,14 +566,14 @@ TRAFFIC_CAPTURES = {
         "bytes": 2727170048 + 405584128, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
         "sha256": "c7a8ade2fe0fc70fcf7996bdca15f82c27f81b22e80b1c05fae9fb5db6494d9f"},
     ("plain_bf16", "chunk_kernel"): {
-        "bytes": 54629376 + 315648, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "b237f56eec21ccb6550652fe15ed34583fd08837bbad5b2fdef8d9f28e12beed"},
+        "bytes": 54631424 + 692992, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "822c104f7f6d87e47dd2fa8c295d1a553102378351f103b6d94235b580e6ef05"},
     ("decay_bf16", "chunk_kernel"): {
-        "bytes": 824387072 + 209595136, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "b237f56eec21ccb6550652fe15ed34583fd08837bbad5b2fdef8d9f28e12beed"},
+        "bytes": 824388608 + 209677568, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "822c104f7f6d87e47dd2fa8c295d1a553102378351f103b6d94235b580e6ef05"},
     ("gla_bf16", "gla_chunk_kernel"): {
-        "bytes": 344070912 + 34972672, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
-        "sha256": "a9a55bd527432b8b9b9242190501241d82556415c0a1a57f7858652060f5bad1"},
+        "bytes": 343999232 + 35813888, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
+        "sha256": "043d29032d7115c41591e917102f5998e9156c7252bd65a93f96edf7c3680c3d"},
 }
 
 
