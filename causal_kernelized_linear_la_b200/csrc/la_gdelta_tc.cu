@@ -279,6 +279,7 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tmem_ld16(tmem_addr(tbase, quad, P::T_KQ + wg * 32), *reinterpret_cast<float(*)[16]>(v));
             tmem_ld16(tmem_addr(tbase, quad, P::T_KQ + wg * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
             tmem_ld_wait();
+            tmem_regs_after_wait(v);
             const bool fact = *factored != 0;
             if (r < 64) {
                 const float gr = gv[r], Lr = Lv[r], sr = gr * ef[r];
@@ -433,6 +434,7 @@ gd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tmem_ld16(tmem_addr(tbase, quad, P::T_W + col0), *reinterpret_cast<float(*)[16]>(v));
                 tmem_ld16(tmem_addr(tbase, quad, P::T_W + col0 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
                 tmem_ld_wait();
+                tmem_regs_after_wait(v);
                 if (i >= 0) {
                     unsigned char* blk = wstage + (col0 / 64) * TILE;
                     const int byte0 = (col0 % 64) * 2;
@@ -761,10 +763,13 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ld32(P::T_X1 + col, o);
             ld32(P::T_X2 + col, w);
             tmem_ld_wait();
+            tmem_regs_after_wait(o);
+            tmem_regs_after_wait(w);
 #pragma unroll
             for (int x = 0; x < 32; ++x) o[x] += w[x];
             ld32(P::T_X3 + col, w);
             tmem_ld_wait();
+            tmem_regs_after_wait(w);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_read[cc & 1]);
@@ -802,6 +807,8 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ld32(P::T_X1 + cp * 64 + wg * 32, u);
                 ld32(P::T_X2 + cp * 64 + wg * 32, w);
                 tmem_ld_wait();
+                tmem_regs_after_wait(u);
+                tmem_regs_after_wait(w);
 #pragma unroll
                 for (int x = 0; x < 32; ++x) u[x] += w[x];
                 store_row(utile, r, u, 1.f);
@@ -822,6 +829,8 @@ gd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ld32(P::T_S1 + wg * 32, a);
                 ld32(P::T_S2 + wg * 32, b);
                 tmem_ld_wait();
+                tmem_regs_after_wait(a);
+                tmem_regs_after_wait(b);
                 if (f >= 0) {
 #pragma unroll
                     for (int x = 0; x < 32; ++x) sreg[x] = fmaf(bc, sreg[x], a[x] + b[x]);

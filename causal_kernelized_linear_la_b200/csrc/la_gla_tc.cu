@@ -208,6 +208,7 @@ gla_summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             float v[16];
             tmem_ld16(tmem_addr(tbase, quad, P::T_S + g * 16), v);
             tmem_ld_wait();
+            tmem_regs_after_wait(v);
             if (f >= 0) {
                 float4* dst = reinterpret_cast<float4*>(slot + (size_t)f * DV + g * 16);
 #pragma unroll
