@@ -563,8 +563,8 @@ def la_launches_per_step(p) -> int:
 TRAFFIC_CAPTURES = {
     # one call's eight chain launches (8 parts of 8192 tokens)
     ("gdelta_bf16", "gd_chain_kernel"): {
-        "bytes": 2727170048 + 405584128, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
-        "sha256": "c7a8ade2fe0fc70fcf7996bdca15f82c27f81b22e80b1c05fae9fb5db6494d9f"},
+        "bytes": 2721053696 + 405298688, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
+        "sha256": "6603babe911794e43ae63435e60faa7a51603d44a692bffe61c96349acd135fc"},
     ("plain_bf16", "chunk_kernel"): {
         "bytes": 54631424 + 692992, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
         "sha256": "822c104f7f6d87e47dd2fa8c295d1a553102378351f103b6d94235b580e6ef05"},
@@ -572,8 +572,8 @@ TRAFFIC_CAPTURES = {
         "bytes": 824388608 + 209677568, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
         "sha256": "822c104f7f6d87e47dd2fa8c295d1a553102378351f103b6d94235b580e6ef05"},
     ("gla_bf16", "gla_chunk_kernel"): {
-        "bytes": 343999232 + 35813888, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
-        "sha256": "043d29032d7115c41591e917102f5998e9156c7252bd65a93f96edf7c3680c3d"},
+        "bytes": 343999488 + 34967808, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
+        "sha256": "fe9b2686838a7a2713b4a95fecbfe3a5888b77d963b639eaaf06c87e4ed8d9ea"},
 }
 
 
