@@ -692,7 +692,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 // W = gamma^C T from the carried state
                 if (!mbar_wait(t_done, (c - 1) & 1, kErrMma)) { bad = true; break; }
                 tc_fence_after();
-                constexpr int NGT = P::NO / 16;
+                // the dv value columns in 16-column groups; the normaliser column
+                // (dv) alone after them: its group's other 15 columns stay zero
+                constexpr int NGT = DV / 16;
 #pragma unroll 1
                 for (int g0 = sub; g0 < NGT; g0 += KB * NTQ) {
                     float v[KB][16];
@@ -705,6 +707,18 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                     for (int i = 0; i < KB; ++i)
                         if (g0 + i * NTQ < NGT) put_w(g0 + i * NTQ, v[i], DECAY);
+                }
+                if (sub == (DV / 16) % NTQ) {
+                    float z = tmem_ld1(tmem_addr(tbase, quad, P::T_T + DV));
+                    tmem_ld_wait();
+                    tmem_regs_after_wait(z);
+                    if (DECAY) {
+                        z = one_factor ? z * gC : (z * gH) * gH;
+                        tmem_st1(tmem_addr(tbase, quad, P::T_T + DV), z);
+                    }
+                    if (fr >= 0)
+                        *reinterpret_cast<uint4*>(wcp + (DV / 64) * P::WBLK + sw128_offset(fr, 0)) =
+                            make_uint4(pack_bf16x2(z, 0.f), 0u, 0u, 0u);
                 }
                 w_ready();
             }

@@ -293,6 +293,12 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr)
     return __uint_as_float(r);
 }
 
+// One column: thread t of the warp writes lane (warp quadrant base + t), column col.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // tcgen05.ld fills its registers asynchronously, but the compiler sees them as
