@@ -46,6 +46,14 @@ def test_plain_bf16_small(N):
     _check(inputs.make_kernelized(2, 2, N, 64, 64, dtype="bf16", mode="plain", seed=300 + N))
 
 
+@pytest.mark.parametrize("d,dv", [(128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("N", [77, 1500])
+def test_plain_bf16_heads(d, dv, N):
+    """The plain mode at every head-size pair of the tensor-core path (the
+    chunk kernel's worker groups and column splits differ with d and dv)."""
+    _check(inputs.make_kernelized(1, 16, N, d, dv, dtype="bf16", mode="plain", seed=450 + d + dv + N))
+
+
 @pytest.mark.parametrize("d,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
 @pytest.mark.parametrize("N", [77, 1500])
 def test_decay_bf16_heads(d, dv, N):
