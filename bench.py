@@ -566,11 +566,11 @@ TRAFFIC_CAPTURES = {
         "bytes": 2721053696 + 405298688, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
         "sha256": "6603babe911794e43ae63435e60faa7a51603d44a692bffe61c96349acd135fc"},
     ("plain_bf16", "chunk_kernel"): {
-        "bytes": 54631424 + 692992, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "822c104f7f6d87e47dd2fa8c295d1a553102378351f103b6d94235b580e6ef05"},
+        "bytes": 54633216 + 431104, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "1210dc256f4e02ac5d869765fc94411e086bcd0679139979b221db85bd2dce5f"},
     ("decay_bf16", "chunk_kernel"): {
-        "bytes": 824388608 + 209677568, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "822c104f7f6d87e47dd2fa8c295d1a553102378351f103b6d94235b580e6ef05"},
+        "bytes": 824388608 + 209968896, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "1210dc256f4e02ac5d869765fc94411e086bcd0679139979b221db85bd2dce5f"},
     ("gla_bf16", "gla_chunk_kernel"): {
         "bytes": 343999488 + 34967808, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
         "sha256": "fe9b2686838a7a2713b4a95fecbfe3a5888b77d963b639eaaf06c87e4ed8d9ea"},
