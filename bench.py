@@ -263,31 +263,64 @@ def _pinned(x, torch):
 
 def time_e2e(host, call, steps, warmup, torch):
     """End to end through the public API with host buffers: every step copies
-    the pinned host tensors ``host`` (name -> tensor) into their device twins,
-    runs ``call(device_tensors)`` (which returns the device results) and copies
-    the results back into pinned host buffers, all inside the CUDA events.
+    the pinned host tensors ``host`` (name -> tensor) into device twins, runs
+    ``call(device_tensors)`` (which returns the device results) and copies the
+    results back into pinned host buffers, all inside the CUDA events.  Steps
+    run as a serving loop would run them: the inputs of step i + 1 go in on one
+    copy stream while step i computes and step i - 1's results come out on
+    another (the two directions of the bus run at once); two sets of device
+    input buffers alternate, and a step computes only after the previous
+    step's results are out (so ``call`` may reuse its output buffers).
     Returns (ms per step, H2D bytes per step, D2H bytes per step)."""
-    dev = {n: torch.empty(t.shape, dtype=t.dtype, device="cuda") for n, t in host.items()}
+    sets = [{n: torch.empty(t.shape, dtype=t.dtype, device="cuda") for n, t in host.items()} for _ in range(2)]
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = torch.cuda.Event()
     outs_h = []
+    state = {"i": 0}
 
     def step():
-        for n, t in host.items():
-            dev[n].copy_(t, non_blocking=True)
-        outs = call(dev)
+        i = state["i"]
+        state["i"] += 1
+        k = i % 2
+        dev = sets[k]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(comp_done[k])     # the set's previous step has computed
+            for n, t in host.items():
+                dev[n].copy_(t, non_blocking=True)
+            in_done[k].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(in_done[k])
+            if i >= 1:
+                s_comp.wait_event(out_done)       # the previous step's results are out
+            outs = call(dev)
+            comp_done[k].record(s_comp)
         if not outs_h:
             outs_h.extend(torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs)
-        for h, o in zip(outs_h, outs):
-            h.copy_(o, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[k])
+            for h, o in zip(outs_h, outs):
+                h.copy_(o, non_blocking=True)
+                o.record_stream(s_out)
+            out_done.record(s_out)
 
+    main = torch.cuda.current_stream()
+    for st in (s_in, s_comp, s_out):
+        st.wait_stream(main)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    a.record(main)
+    for st in (s_in, s_comp, s_out):
+        st.wait_event(a)
     for _ in range(steps):
         step()
-    b.record(stream)
+    for st in (s_in, s_comp, s_out):
+        main.wait_stream(st)
+    b.record(main)
     torch.cuda.synchronize()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in outs_h)
