@@ -576,8 +576,10 @@ def call_kernels(p) -> list:
         names = ["summary_kernel", "scan_kernel", "chunk_kernel"]
     elif p.dtype == "bf16":
         names = ["gd_prep_kernel", "gd_chain_kernel"] * (n // 2)   # one pair per part of the sequence
-    else:
-        names = ["gated_delta_token_simt" if p.mode == "gated_delta" else "kernelized_chunk_simt"]
+    elif p.mode == "gated_delta":
+        names = ["gated_delta_token_simt"]
+    else:   # fp32 kernelized: the parallel form for short sequences, else the chunk loop
+        names = ["kernelized_parallel_simt", "kernelized_state_simt"] if n == 2 else ["kernelized_chunk_simt"]
     assert len(names) == n, (names, n)
     return names
 

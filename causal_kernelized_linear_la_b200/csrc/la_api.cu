@@ -197,6 +197,7 @@ int la_prefill_kernel_count(int B, int H, int N, int d, int dv, const la_config*
     if (la::uses_tc_kernelized(cfg->dtype, cfg->mode)) return 3;
     if (cfg->dtype == LA_BF16 && cfg->mode == LA_GLA) return 3;
     if (cfg->dtype == LA_BF16 && cfg->mode == LA_GATED_DELTA) return 2 * la::gd_parts(B, H, N, d, dv).P;
+    if (cfg->mode == LA_PLAIN || cfg->mode == LA_DECAY) return la::simt_kernelized_kernel_count(N, cfg->dtype);
     return 1;
 }
 

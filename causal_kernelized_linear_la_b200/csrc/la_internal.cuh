@@ -73,6 +73,8 @@ cudaError_t launch_causal_conv(const ConvArgs& a);
 
 // SIMT prefill kernels (fp32 arithmetic; fp32 or bf16 inputs).
 cudaError_t launch_prefill_simt_kernelized(const PrefillArgs& a);
+// kernels one fp32 kernelized prefill of N tokens launches (the parallel form for short sequences)
+int simt_kernelized_kernel_count(int N, la_dtype dt);
 cudaError_t launch_prefill_simt_gated_delta(const PrefillArgs& a);
 cudaError_t launch_prefill_simt_gla(const PrefillArgs& a);
 

@@ -462,6 +462,236 @@ cudaError_t launch_gla_t(const PrefillArgs& a)
     return e;
 }
 
+// ---------------------------------------------------------------------------
+// Short sequences (N <= kParallelMaxN): the parallel form of the same
+// quantities, no chunk loop.  "What Is Linear Attention?" §3 and "Transformers
+// Are RNNs" (the masked-matrix form equals the recurrence): for every token i
+//   num_i = sum_{j <= i} gamma^(i-j) phi(q_i).phi(k_j) v_j + gamma^(i+1) phi(q_i)^T S0
+//   den_i = sum_{j <= i} gamma^(i-j) phi(q_i).phi(k_j)     + gamma^(i+1) phi(q_i)^T z0
+//   o_i   = num_i / (den_i + eps)
+// and the final state
+//   S_N = gamma^N S0 + sum_t gamma^(N-1-t) phi(k_t) v_t^T,   z_N likewise.
+// Every output row and every state element is an independent sum, so a
+// single short chain spreads over many CTAs instead of running its chunks
+// one after another on one.
+
+constexpr int kParallelMaxN = 1024;
+constexpr int kRows = 16;    // query rows per CTA
+constexpr int kKeys = 32;    // keys per staged block
+
+// Row blocks of fp32 [rows][W] in 16-byte pieces, in two halves so that the
+// loads of the next block are in flight while the current one is used: load()
+// issues a thread's loads into registers, store() writes them to shared memory
+// (row pitch P floats), phi applied when PHI, rows past nvalid as zeros.
+template <int ROWS, int W>
+struct RowBlock {
+    static constexpr int V = ROWS * W / 4;                  // float4 pieces
+    static constexpr int PER = (V + kThreads - 1) / kThreads;
+    float4 x[PER];
+    __device__ __forceinline__ void load(const float* __restrict__ src, int nvalid, int tid)
+    {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = tid + u * kThreads;
+            const int row = e / (W / 4), c4 = e % (W / 4);
+            x[u] = (e < V && row < nvalid) ? reinterpret_cast<const float4*>(src + (size_t)row * W)[c4]
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    template <int P, bool PHI>
+    __device__ __forceinline__ void store(float (*sm)[P], int nvalid, int tid) const
+    {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = tid + u * kThreads;
+            if (e >= V) break;
+            const int row = e / (W / 4), c = (e % (W / 4)) * 4;
+            const bool ph = PHI && row < nvalid;
+            sm[row][c] = ph ? phi(x[u].x) : x[u].x;
+            sm[row][c + 1] = ph ? phi(x[u].y) : x[u].y;
+            sm[row][c + 2] = ph ? phi(x[u].z) : x[u].z;
+            sm[row][c + 3] = ph ? phi(x[u].w) : x[u].w;
+        }
+    }
+};
+
+template <int D, int DV>
+struct ParallelSmem {
+    float fq[kRows][D + 1];
+    float fk[kKeys][D + 1];
+    float vv[kKeys][DV];
+    float P[kRows][kKeys + 1];
+};
+
+// grid (chains, ceil(N / kRows)), 256 threads: thread (r, c) accumulates row r,
+// columns c, c + 16, ... of the numerator; every thread of a row keeps its den.
+template <typename T, int D, int DV>
+__global__ void __launch_bounds__(kThreads)
+kernelized_parallel_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                         const float* __restrict__ gamma, const float* __restrict__ S0,
+                         const float* __restrict__ z0, T* __restrict__ out, int H, int N, float eps, int ld)
+{
+    static_assert(sizeof(T) == 4, "the parallel form stages fp32 rows");
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto& sm = *reinterpret_cast<ParallelSmem<D, DV>*>(smem_raw);
+    constexpr int CPT = DV / 16;    // numerator columns per thread
+    const int tid = threadIdx.x, r = tid / 16, cl = tid % 16;
+    const long long chain = blockIdx.x;
+    const int h = (int)(chain % H);
+    const float lam = gamma ? logf(gamma[h]) : 0.f;
+    const int i0 = blockIdx.y * kRows;
+    const int rows = min(kRows, N - i0);
+    const T* qc = q + chain * (long long)ld * D;
+    const T* kc = k + chain * (long long)ld * D;
+    const T* vc = v + chain * (long long)ld * DV;
+    T* oc = out + chain * (long long)ld * DV;
+
+    const float* kf = reinterpret_cast<const float*>(kc);
+    const float* vf = reinterpret_cast<const float*>(vc);
+    {
+        RowBlock<kRows, D> qb;
+        qb.load(reinterpret_cast<const float*>(qc) + (size_t)i0 * D, rows, tid);
+        qb.store<D + 1, true>(sm.fq, rows, tid);
+    }
+    float num[CPT];
+#pragma unroll
+    for (int m = 0; m < CPT; ++m) num[m] = 0.f;
+    float den = 0.f;
+    const int i = i0 + r;
+    const int jend = i0 + rows;    // keys 0 .. jend-1 reach some row of this CTA
+    RowBlock<kKeys, D> kb;
+    RowBlock<kKeys, DV> vb;
+    kb.load(kf, min(kKeys, jend), tid);
+    vb.load(vf, min(kKeys, jend), tid);
+    for (int j0 = 0; j0 < jend; j0 += kKeys) {
+        const int nk = min(kKeys, jend - j0);
+        __syncthreads();   // the previous block's P, fk, vv are consumed
+        kb.store<D + 1, true>(sm.fk, nk, tid);
+        vb.store<DV, false>(sm.vv, nk, tid);
+        __syncthreads();
+        if (j0 + kKeys < jend) {   // the next block's loads fly while this one is used
+            kb.load(kf + (size_t)(j0 + kKeys) * D, min(kKeys, jend - j0 - kKeys), tid);
+            vb.load(vf + (size_t)(j0 + kKeys) * DV, min(kKeys, jend - j0 - kKeys), tid);
+        }
+        // P[r][jj] = [j <= i] gamma^(i-j) phi(q_i).phi(k_j), two entries per thread
+        for (int e = tid; e < kRows * kKeys; e += kThreads) {
+            const int rr = e / kKeys, jj = e % kKeys;
+            const int ii = i0 + rr, j = j0 + jj;
+            float s = 0.f;
+            if (rr < rows && jj < nk && j <= ii) {
+#pragma unroll 8
+                for (int f = 0; f < D; ++f) s = fmaf(sm.fq[rr][f], sm.fk[jj][f], s);
+                s *= expf((float)(ii - j) * lam);
+            }
+            sm.P[rr][jj] = s;
+        }
+        __syncthreads();
+        for (int jj = 0; jj < nk; ++jj) {
+            const float pv = sm.P[r][jj];
+            den += pv;
+#pragma unroll
+            for (int m = 0; m < CPT; ++m) num[m] = fmaf(pv, sm.vv[jj][cl + 16 * m], num[m]);
+        }
+    }
+    if (r >= rows) return;
+    // the start state's share
+    const float w = expf((float)(i + 1) * lam);
+    if (S0) {
+        const float* s0 = S0 + chain * (long long)D * DV;
+#pragma unroll
+        for (int m = 0; m < CPT; ++m) {
+            float acc = 0.f;
+            for (int f = 0; f < D; ++f) acc = fmaf(sm.fq[r][f], s0[(long long)f * DV + cl + 16 * m], acc);
+            num[m] = fmaf(w, acc, num[m]);
+        }
+    }
+    if (z0) {
+        const float* zz = z0 + chain * (long long)D;
+        float acc = 0.f;
+        for (int f = 0; f < D; ++f) acc = fmaf(sm.fq[r][f], zz[f], acc);
+        den = fmaf(w, acc, den);
+    }
+    const float rden = 1.f / (den + eps);
+#pragma unroll
+    for (int m = 0; m < CPT; ++m) oc[(long long)i * DV + cl + 16 * m] = from_f32<T>(num[m] * rden);
+}
+
+// grid (chains, ceil((D*DV + D) / 256)): one state element per thread, the sum
+// over the chain's tokens in token order (keys staged through shared memory).
+template <typename T, int D, int DV>
+__global__ void __launch_bounds__(kThreads)
+kernelized_state_simt(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ gamma,
+                      const float* __restrict__ S0, const float* __restrict__ z0, float* __restrict__ S_out,
+                      float* __restrict__ z_out, int H, int N, int ld)
+{
+    static_assert(sizeof(T) == 4, "the parallel form stages fp32 rows");
+    __shared__ float kt[kKeys][D];
+    __shared__ float vt[kKeys][DV];
+    __shared__ float wt[kKeys];
+    const int tid = threadIdx.x;
+    const long long chain = blockIdx.x;
+    const int h = (int)(chain % H);
+    const float lam = gamma ? logf(gamma[h]) : 0.f;
+    const int e = blockIdx.y * kThreads + tid;
+    const bool isz = e >= D * DV && e < D * DV + D;
+    const bool active = e < D * DV + D;
+    const int f = isz ? e - D * DV : e / DV, c = isz ? 0 : e % DV;
+    const T* kc = k + chain * (long long)ld * D;
+    const T* vc = v + chain * (long long)ld * DV;
+    float acc = 0.f;
+    const float* kf = reinterpret_cast<const float*>(kc);
+    const float* vf = reinterpret_cast<const float*>(vc);
+    RowBlock<kKeys, D> kb;
+    RowBlock<kKeys, DV> vb;
+    kb.load(kf, min(kKeys, N), tid);
+    vb.load(vf, min(kKeys, N), tid);
+    for (int t0 = 0; t0 < N; t0 += kKeys) {
+        const int n = min(kKeys, N - t0);
+        __syncthreads();
+        kb.store<D, true>(kt, n, tid);
+        vb.store<DV, false>(vt, n, tid);
+        if (t0 + kKeys < N) {
+            kb.load(kf + (size_t)(t0 + kKeys) * D, min(kKeys, N - t0 - kKeys), tid);
+            vb.load(vf + (size_t)(t0 + kKeys) * DV, min(kKeys, N - t0 - kKeys), tid);
+        }
+        if (tid < kKeys) wt[tid] = tid < n ? expf((float)(N - 1 - (t0 + tid)) * lam) : 0.f;
+        __syncthreads();
+        if (active) {
+            if (isz)
+                for (int t = 0; t < n; ++t) acc = fmaf(wt[t], kt[t][f], acc);
+            else
+                for (int t = 0; t < n; ++t) acc = fmaf(wt[t] * kt[t][f], vt[t][c], acc);
+        }
+    }
+    if (!active) return;
+    const float wn = expf((float)N * lam);
+    if (isz) {
+        z_out[chain * D + f] = fmaf(wn, z0 ? z0[chain * D + f] : 0.f, acc);
+    } else {
+        const long long off = chain * (long long)D * DV + (long long)f * DV + c;
+        S_out[off] = fmaf(wn, S0 ? S0[off] : 0.f, acc);
+    }
+}
+
+template <typename T, int D, int DV>
+cudaError_t launch_parallel_t(const PrefillArgs& a)
+{
+    auto k1 = kernelized_parallel_simt<T, D, DV>;
+    const size_t smem = sizeof(ParallelSmem<D, DV>);
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int chains = a.B * a.H;
+    k1<<<dim3(chains, (a.N + kRows - 1) / kRows), kThreads, smem, a.stream>>>(
+        (const T*)a.q, (const T*)a.k, (const T*)a.v, a.gamma, a.S0, a.z0, (T*)a.out, a.H, a.N, a.eps, a.ld);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stage_mark(0, a.stream);
+    kernelized_state_simt<T, D, DV><<<dim3(chains, (D * DV + D + kThreads - 1) / kThreads), kThreads, 0, a.stream>>>(
+        (const T*)a.k, (const T*)a.v, a.gamma, a.S0, a.z0, a.S_out, a.z_out, a.H, a.N, a.ld);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    stage_mark(1, a.stream);
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_prefill_simt_gla(const PrefillArgs& a)
@@ -474,9 +704,19 @@ cudaError_t launch_prefill_simt_gla(const PrefillArgs& a)
     return launch_gla_t<__nv_bfloat16, 128>(a);
 }
 
+// Sequences of at most kParallelMaxN tokens in fp32 take the parallel form
+// (two kernels); longer ones the chunk loop (one kernel).
+int simt_kernelized_kernel_count(int N, la_dtype dt) { return dt == LA_F32 && N <= kParallelMaxN ? 2 : 1; }
+
 cudaError_t launch_prefill_simt_kernelized(const PrefillArgs& a)
 {
     if (a.dtype == LA_F32) {
+        if (a.N <= kParallelMaxN) {
+            if (a.d == 64 && a.dv == 64) return launch_parallel_t<float, 64, 64>(a);
+            if (a.d == 64 && a.dv == 128) return launch_parallel_t<float, 64, 128>(a);
+            if (a.d == 128 && a.dv == 64) return launch_parallel_t<float, 128, 64>(a);
+            return launch_parallel_t<float, 128, 128>(a);
+        }
         if (a.d == 64) return launch_kernelized_t<float, 64, 32>(a);
         return launch_kernelized_t<float, 128, 32>(a);
     }

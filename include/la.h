@@ -175,7 +175,9 @@ LA_API size_t la_prefill_workspace_bytes(int B, int H, int N, int d, int dv, con
  * la_set_stage_events records for it: 3 for bf16 LA_PLAIN / LA_DECAY (segment
  * summaries, scan, chunk loop); 2 P for bf16 LA_GATED_DELTA, whose sequence
  * runs as P <= 8 parts (each a chunk prep pass and a chain pass; the prep
- * pass of part i + 1 overlaps the chain pass of part i); 1 otherwise; 0 when
+ * pass of part i + 1 overlaps the chain pass of part i); 2 for fp32
+ * LA_PLAIN / LA_DECAY with N <= 1024 (the parallel form: outputs, then the
+ * final state); 1 otherwise; 0 when
  * the call launches no kernel (N = 0, nothing to do, or unsupported sizes).
  * Host-only.  Not from the pages: a service for profiling.
  */

@@ -138,7 +138,8 @@ def test_kernel_count():
     assert kc(1, 32, 8192, 128, 128, "bf16", "gated_delta") == 8      # four parts of 2048
     assert kc(1, 3, 2100, 128, 128, "bf16", "gated_delta") == 2
     assert kc(64, 32, 65536, 128, 128, "bf16", "gated_delta") == 2    # enough chains to fill the GPU
-    assert kc(1, 1, 256, 64, 64, "f32", "plain") == 1
+    assert kc(1, 1, 256, 64, 64, "f32", "plain") == 2        # parallel form: outputs, final state
+    assert kc(1, 1, 5000, 64, 64, "f32", "plain") == 1       # chunk loop
     assert kc(1, 32, 8192, 128, 128, "bf16", "gla") == 3      # summaries, scan, chunk loop
     assert kc(1, 32, 8192, 128, 128, "f32", "gla") == 1
     assert kc(1, 1, 0, 64, 64, "bf16", "plain") == 0

@@ -36,6 +36,13 @@ def test_plain_f32_small(N):
     _check(inputs.make_kernelized(2, 3, N, 64, 64, dtype="f32", mode="plain", seed=100 + N))
 
 
+@pytest.mark.parametrize("mode,N", [("plain", 1024), ("plain", 1025), ("decay", 2000)])
+def test_kernelized_f32_both_forms(mode, N):
+    """fp32 inputs: up to 1024 tokens take the parallel form, longer sequences
+    the chunk loop; both against the oracle at the boundary."""
+    _check(inputs.make_kernelized(1, 2, N, 64, 64, dtype="f32", mode=mode, seed=150 + N))
+
+
 @pytest.mark.parametrize("d,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
 def test_decay_f32_heads(d, dv):
     _check(inputs.make_kernelized(1, 4, 150, d, dv, dtype="f32", mode="decay", seed=200 + d + dv))
