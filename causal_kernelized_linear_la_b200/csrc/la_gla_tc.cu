@@ -274,8 +274,9 @@ struct GlaChunkPlan {
     static constexpr int OFF_S = STAGES * STAGE;           // S bf16, DV / 64 blocks of D x 64
     static constexpr int OFF_P = OFF_S + (DV / 64) * SBLK; // P~ bf16 [C][C]
     static constexpr int OFF_O = OFF_P + TILE;             // output staging bf16 [C][DV]
-    static constexpr int OFF_VEC = OFF_O + C * DV * 2;     // tot[TPC][D], b0[D], bc[D], r[D], ebc[2][D]
-    static constexpr int OFF_BAR = OFF_VEC + (TPC + 5) * D * 4;
+    // tot[TPC][D], b0[D], bc[D], r[D], ebc[2][D], e^R[D], e^{B_C - R}[D], slow-path flag[2]
+    static constexpr int OFF_VEC = OFF_O + C * DV * 2;
+    static constexpr int OFF_BAR = OFF_VEC + (TPC + 7) * D * 4 + 16;
     static constexpr int NBAR = 2 * STAGES + 10;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
@@ -305,6 +306,9 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float* bcv = b0v + D;              // B_C per channel
     float* rv = bcv + D;               // midpoint R per channel
     float* ebc = rv + D;               // [2][D] e^{B_C} per chunk parity
+    float* erv = ebc + 2 * D;          // e^R per channel
+    float* ecr = erv + D;              // e^{B_C - R} per channel
+    int* slow = reinterpret_cast<int*>(ecr + D);   // [2] some channel has e^R below the normal range
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* empty = full + P::STAGES;
     uint64_t* phi_rdy = empty + P::STAGES;   // workers: Q~, K~, Q^, K^ of the chunk in place
@@ -456,6 +460,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             tot[part * D + i] = sum;
             if (part == 0) b0v[i] = la[0];
+            if (tid == 0) slow[c & 1] = 0;
             if (named_bar_or(1, NWT, bad)) return true;
             float acc = 0.f, bc = 0.f;
             for (int q2 = 0; q2 < P::TPC; ++q2) {
@@ -473,12 +478,18 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 bcv[i] = bc;
                 rv[i] = R;
                 ebc[(c & 1) * D + i] = __expf(bc);
+                erv[i] = __expf(R);
+                ecr[i] = __expf(bc - R);
+                if (R < -80.f) slow[c & 1] = 1;
                 if (bc - R < -kHalfRangeMax) atomicCAS(&g_device_error, 0u, (unsigned int)kErrRange);
             }
             if (named_bar_or(1, NWT, bad)) return true;
-            // Q^ = q e^{B}, Q~ = q e^{B - R}, K^ = k e^{B_C - B}, K~ = k e^{R - B}: each factor is
-            // its own exponential, so none passes through a value outside the fp32 range
+            // Q^ = q e^{B}, Q~ = q e^{B - R}, K^ = k e^{B_C - B}, K~ = k e^{R - B}.  In range,
+            // |B - R| <= 80, so e^{B - R} and e^{R - B} are finite and the other two follow
+            // with the per-channel constants e^R and e^{B_C - R}; when some channel's e^R is
+            // below the normal range (R < -80) each factor is its own exponential instead
             constexpr int PER = (D / 8) * C / NWT;
+            const bool fast = slow[c & 1] == 0;
             uint4 qh[PER], kh[PER];
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
@@ -498,13 +509,32 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 *reinterpret_cast<float4*>(bcv8 + 4) = *reinterpret_cast<const float4*>(bcv + f0 + 4);
                 *reinterpret_cast<float4*>(rv8) = *reinterpret_cast<const float4*>(rv + f0);
                 *reinterpret_cast<float4*>(rv8 + 4) = *reinterpret_cast<const float4*>(rv + f0 + 4);
+                if (fast) {
+                    // e^{B} = e^{B - R} e^R and e^{B_C - B} = e^{R - B} e^{B_C - R}: two exponentials a
+                    // (token, channel); every factor is within e^{+-80} and e^R is a normal float
+                    float er8[8], ecr8[8];
+                    *reinterpret_cast<float4*>(er8) = *reinterpret_cast<const float4*>(erv + f0);
+                    *reinterpret_cast<float4*>(er8 + 4) = *reinterpret_cast<const float4*>(erv + f0 + 4);
+                    *reinterpret_cast<float4*>(ecr8) = *reinterpret_cast<const float4*>(ecr + f0);
+                    *reinterpret_cast<float4*>(ecr8 + 4) = *reinterpret_cast<const float4*>(ecr + f0 + 4);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const float B = Bv[x], bcx = bcv8[x], R = rv8[x];
-                    fqt[x] = fq[x] * __expf(B - R);
-                    fkt[x] = valid ? fk[x] * __expf(R - B) : 0.f;
-                    fq[x] *= __expf(B);
-                    fk[x] = valid ? fk[x] * __expf(bcx - B) : 0.f;
+                    for (int x = 0; x < 8; ++x) {
+                        const float d = Bv[x] - rv8[x];
+                        const float E = __expf(d), Ei = __expf(-d);
+                        fqt[x] = fq[x] * E;
+                        fkt[x] = valid ? fk[x] * Ei : 0.f;
+                        fq[x] = (fq[x] * E) * er8[x];
+                        fk[x] = valid ? (fk[x] * Ei) * ecr8[x] : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) {
+                        const float B = Bv[x], bcx = bcv8[x], R = rv8[x];
+                        fqt[x] = fq[x] * __expf(B - R);
+                        fkt[x] = valid ? fk[x] * __expf(R - B) : 0.f;
+                        fq[x] *= __expf(B);
+                        fk[x] = valid ? fk[x] * __expf(bcx - B) : 0.f;
+                    }
                 }
                 *pq = pack8(fqt, 1.f);
                 *pk = pack8(fkt, 1.f);

@@ -53,6 +53,16 @@ def test_gla_closed_gates():
     assert_close(p, run_library(p), run_oracle(p), chains)
 
 
+def test_gla_closed_gates_at_chunk_start():
+    """A closed gate on a chunk's first token and a second one later in the
+    chunk: the chunk's midpoint log decay falls below -80, where e^R is no
+    longer a normal float and the gate factors take their own exponentials."""
+    p = inputs.make_gla(1, 2, 300, 128, 128, dtype="bf16", seed=47)
+    _closed_gates(p, [(0, 64, 9), (0, 90, 9), (1, 128, 2), (1, 129, 2), (1, 192, 100), (1, 250, 100)])
+    chains = [(0, h) for h in range(2)]
+    assert_close(p, run_library(p), run_oracle(p), chains)
+
+
 def test_gla_chunk_out_of_range_is_reported():
     """Three closed gates of one channel inside one 64-token chunk exceed the
     chunk form's factor range: reported as unsupported by la_prefill_check
