@@ -232,27 +232,49 @@ gla_summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 // ---------------------------------------------------------------------------
 // Kernel B: scan of segment summaries with a per-row (channel) decay.  In
 // place: slot s <- state at the start of segment s; writes the final state.
+// Grid (chains, kGlaScanSplit) of kGlaScanThreads threads; each thread takes
+// 16-byte pieces of state rows (four values of one row share its decay) with
+// eight segments' loads in flight, so the scan holds few SMs and the chunk
+// kernel, launched behind it, becomes resident on the others meanwhile.
+constexpr int kGlaScanThreads = 1024, kGlaScanSplit = 4;
+
 template <int D, int DV>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kGlaScanThreads, 1)
 gla_scan_kernel(float* __restrict__ ws, const float* __restrict__ S0, float* __restrict__ S_out, int G)
 {
-    constexpr int SLOT = D * DV + D;
+    constexpr int SLOT = D * DV + D, S4 = D * DV / 4, BATCH = 8;
     grid_launch_dependents();   // the chunk kernel may set up and load q, k, v meanwhile
     grid_dependency_wait();     // the segment summaries are complete
     const int chain = blockIdx.x;
-    const int e = blockIdx.y * 256 + threadIdx.x;
-    if (e >= D * DV) return;
-    const int row = e / DV;
-    float acc = S0 ? S0[(size_t)chain * D * DV + e] : 0.f;
     float* base = ws + (size_t)chain * G * SLOT;
-    for (int s = 0; s < G; ++s) {
-        float* slot = base + (size_t)s * SLOT;
-        const float delta = slot[e];
-        const float dec = slot[D * DV + row];   // the decays are never overwritten
-        slot[e] = acc;
-        acc = fmaf(dec, acc, delta);
+    const int per = (S4 + gridDim.y - 1) / gridDim.y;   // 16-byte pieces of this CTA
+    const int lo = blockIdx.y * per, hi = min(S4, lo + per);
+    for (int e = lo + (int)threadIdx.x; e < hi; e += kGlaScanThreads) {
+        const int row = (4 * e) / DV;
+        float4 acc = S0 ? reinterpret_cast<const float4*>(S0 + (size_t)chain * D * DV)[e]
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < G; s0 += BATCH) {
+            float4 delta[BATCH];
+            float dec[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                const float* slot = base + (size_t)(s0 + i) * SLOT;
+                delta[i] = s0 + i < G ? reinterpret_cast<const float4*>(slot)[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+                dec[i] = s0 + i < G ? slot[D * DV + row] : 0.f;   // the decays are never overwritten
+            }
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                if (s0 + i < G) {
+                    reinterpret_cast<float4*>(base + (size_t)(s0 + i) * SLOT)[e] = acc;
+                    acc.x = fmaf(dec[i], acc.x, delta[i].x);
+                    acc.y = fmaf(dec[i], acc.y, delta[i].y);
+                    acc.z = fmaf(dec[i], acc.z, delta[i].z);
+                    acc.w = fmaf(dec[i], acc.w, delta[i].w);
+                }
+            }
+        }
+        reinterpret_cast<float4*>(S_out + (size_t)chain * D * DV)[e] = acc;
     }
-    S_out[(size_t)chain * D * DV + e] = acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -716,8 +738,8 @@ cudaError_t launch_gla(const PrefillArgs& a, const TcSegments& sg)
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(0, a.stream);
 
-    lc.gridDim = dim3(chains, (D * DV + 255) / 256);
-    lc.blockDim = dim3(256);
+    lc.gridDim = dim3(chains, kGlaScanSplit);
+    lc.blockDim = dim3(kGlaScanThreads);
     lc.dynamicSmemBytes = 0;
     lc.numAttrs = 1;
     e = cudaLaunchKernelEx(&lc, gla_scan_kernel<D, DV>, ws, a.S0, a.S_out, sg.G);

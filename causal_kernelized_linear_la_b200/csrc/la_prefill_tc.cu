@@ -337,47 +337,58 @@ summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 
 // ---------------------------------------------------------------------------
 // Kernel B: scan of segment summaries.  In place: slot s <- state at the start
-// of segment s; writes the final state (S_N, z_N).
+// of segment s; writes the final state (S_N, z_N).  Every element is a short
+// serial sum over its chain's segments.  Grid (chains, kScanSplit) of
+// kScanThreads threads, each 16-byte column with eight segments' loads in
+// flight: the scan holds few SMs, so the chunk kernel (launched behind it with
+// programmatic serialization) becomes resident on the others and loads and
+// applies phi to its first chunks while the scan runs.
+constexpr int kScanThreads = 1024, kScanSplit = 4;
+
 template <int D, int DV, bool DECAY>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kScanThreads, 1)
 scan_kernel(float* __restrict__ ws, const float* __restrict__ gamma, const float* __restrict__ S0,
             const float* __restrict__ z0, float* __restrict__ S_out, float* __restrict__ z_out,
             const __grid_constant__ SegMap m)
 {
-    constexpr int SLOT = D * DV + D;
+    constexpr int SLOT4 = (D * DV + D) / 4, S4 = D * DV / 4, BATCH = 8;
     grid_launch_dependents();   // the chunk kernel may set up and load q, k, v meanwhile
     grid_dependency_wait();     // the segment summaries are complete
     const int chain = blockIdx.x;
-    const int e = blockIdx.y * 256 + threadIdx.x;
-    if (e >= SLOT) return;
     int slot0, G, N;
     chain_of(m, chain, slot0, G, N);
     const int L = m.L;
     const float lam = DECAY ? logf(gamma[chain % m.H]) : 0.f;
-    const bool isz = e >= D * DV;
-    float acc;
-    if (!isz) acc = S0 ? S0[(size_t)chain * D * DV + e] : 0.f;
-    else acc = z0 ? z0[(size_t)chain * D + (e - D * DV)] : 0.f;
-    float* base = ws + (size_t)slot0 * SLOT + e;
     const float full_dec = DECAY ? expf((float)L * lam) : 1.f;
-    constexpr int BATCH = 8;
-    for (int s0 = 0; s0 < G; s0 += BATCH) {
-        float delta[BATCH];
+    float4* base = reinterpret_cast<float4*>(ws + (size_t)slot0 * (D * DV + D));
+    const int per = (SLOT4 + gridDim.y - 1) / gridDim.y;   // columns of this CTA
+    const int lo = blockIdx.y * per, hi = min(SLOT4, lo + per);
+    for (int e = lo + (int)threadIdx.x; e < hi; e += kScanThreads) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e < S4) { if (S0) acc = reinterpret_cast<const float4*>(S0 + (size_t)chain * D * DV)[e]; }
+        else if (z0) acc = reinterpret_cast<const float4*>(z0 + (size_t)chain * D)[e - S4];
+        for (int s0 = 0; s0 < G; s0 += BATCH) {
+            float4 delta[BATCH];
 #pragma unroll
-        for (int i = 0; i < BATCH; ++i) delta[i] = (s0 + i < G) ? base[(size_t)(s0 + i) * SLOT] : 0.f;
+            for (int i = 0; i < BATCH; ++i)
+                delta[i] = (s0 + i < G) ? base[(size_t)(s0 + i) * SLOT4 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < BATCH; ++i) {
-            const int s = s0 + i;
-            if (s < G) {
-                base[(size_t)s * SLOT] = acc;
-                const int len = min(L, N - s * L);
-                const float dec = DECAY ? (len == L ? full_dec : expf((float)len * lam)) : 1.f;
-                acc = fmaf(dec, acc, delta[i]);
+            for (int i = 0; i < BATCH; ++i) {
+                const int sg = s0 + i;
+                if (sg < G) {
+                    base[(size_t)sg * SLOT4 + e] = acc;
+                    const int len = min(L, N - sg * L);
+                    const float dec = DECAY ? (len == L ? full_dec : expf((float)len * lam)) : 1.f;
+                    acc.x = fmaf(dec, acc.x, delta[i].x);
+                    acc.y = fmaf(dec, acc.y, delta[i].y);
+                    acc.z = fmaf(dec, acc.z, delta[i].z);
+                    acc.w = fmaf(dec, acc.w, delta[i].w);
+                }
             }
         }
+        if (e < S4) reinterpret_cast<float4*>(S_out + (size_t)chain * D * DV)[e] = acc;
+        else reinterpret_cast<float4*>(z_out + (size_t)chain * D)[e - S4] = acc;
     }
-    if (!isz) S_out[(size_t)chain * D * DV + e] = acc;
-    else z_out[(size_t)chain * D + (e - D * DV)] = acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -898,9 +909,8 @@ cudaError_t launch_tc_map(const PrefillArgs& a, const SegMap& m, int units)
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stage_mark(0, a.stream);
 
-    constexpr int SLOT = D * DV + D;
-    lc.gridDim = dim3(chains, (SLOT + 255) / 256);
-    lc.blockDim = dim3(256);
+    lc.gridDim = dim3(chains, kScanSplit);
+    lc.blockDim = dim3(kScanThreads);
     lc.dynamicSmemBytes = 0;
     lc.numAttrs = 1;
     e = cudaLaunchKernelEx(&lc, scan_kernel<D, DV, DECAY>, ws, a.gamma, a.S0, a.z0, a.S_out, a.z_out, m);
