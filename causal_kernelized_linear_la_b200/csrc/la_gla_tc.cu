@@ -58,24 +58,29 @@ __device__ __forceinline__ float log_gate(float a, bool valid)
 // a running per-channel suffix sum.
 template <int D, int DV>
 struct GlaSummaryPlan {
-    static constexpr int THREADS = 512;
+    static constexpr int WORKERS = 512;          // sixteen gate warps
+    static constexpr int THREADS = WORKERS + 32; // + the issuing warp
     static constexpr int STAGES = (D + DV > 128) ? 3 : 4;
     static constexpr int KB = C * D * 2, VB = C * DV * 2, AB = C * D * 4;
     static constexpr int LOAD_BYTES = KB + VB;   // + the alpha block of the chunk (bulk copy)
     static constexpr int STAGE = KB + VB + AB;
-    static constexpr int TPC = THREADS / D;      // threads per channel in the suffix scan
+    static constexpr int TPC = WORKERS / D;      // threads per channel in the suffix scan
     static constexpr int TOK = C / TPC;          // tokens per thread
     static constexpr int OFF_TOT = STAGES * STAGE;               // [TPC][D] part sums
     static constexpr int OFF_CARRY = OFF_TOT + TPC * D * 4;      // [D] log decay after the chunk
-    static constexpr int OFF_BAR = OFF_CARRY + D * 4;
-    static constexpr int OFF_TMEM = OFF_BAR + (2 * STAGES + 1) * 8;
+    static constexpr int OFF_BAR = OFF_CARRY + D * 4;            // full[S], empty[S], wrdy[S], done
+    static constexpr int OFF_TMEM = OFF_BAR + (3 * STAGES + 1) * 8;
     static constexpr int BYTES = OFF_TMEM + 16 + 1024;
     static_assert(BYTES <= 232448, "shared memory plan exceeds the per-block limit");
     static constexpr uint32_t T_S = 0, T_COLS = DV <= 64 ? 64 : 128;
 };
 
+// Roles: warps 0..15 (the gate warps) form each chunk's weights and scale its K
+// in place, then signal the chunk's stage barrier; lane 0 of warp 16 issues
+// the TMA loads and the MMAs, and refills a stage once its MMA is complete, so
+// the gate warps never wait for an issue or a refill.
 template <int D, int DV>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(GlaSummaryPlan<D, DV>::THREADS, 1)
 gla_summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const float* __restrict__ alpha, float* __restrict__ ws, int N, int G, int L, int ld)
 {
@@ -87,11 +92,13 @@ gla_summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     float* carry = reinterpret_cast<float*>(sm + P::OFF_CARRY);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + P::OFF_BAR);
     uint64_t* empty = full + P::STAGES;
-    uint64_t* done = empty + P::STAGES;
+    uint64_t* wrdy = empty + P::STAGES;   // gate warps: K^ of the stage's chunk in place
+    uint64_t* done = wrdy + P::STAGES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P::OFF_TMEM);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, wg = warp >> 2;
+    const bool issuer = tid == P::WORKERS;
     const int unit = blockIdx.x;
     const int chain = unit / G, seg = unit % G;
     const int t0 = seg * L, t1 = min(N, t0 + L);
@@ -100,7 +107,11 @@ gla_summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const float* achain = alpha + (size_t)chain * ld * D;
 
     if (tid == 0) {
-        for (int s = 0; s < P::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < P::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&wrdy[s], P::WORKERS / 32);
+        }
         mbar_init(done, 1);
         fence_mbar_init();
     }
@@ -111,79 +122,30 @@ gla_summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
-    // chunk slot r processes segment chunk nch - 1 - r
-    int loads_issued = 0, loads_waited = 0, commits = 0;
-    auto issue = [&](int r) {
-        const int c = nch - 1 - r;
-        const int s = r % P::STAGES;
-        unsigned char* st = sm + s * P::STAGE;
-        const int y = t0 + c * C;
-        const int n = min(C, t1 - y);
-        mbar_expect_tx(&full[s], P::LOAD_BYTES + n * D * 4);
-        for (int b = 0; b < D / 64; ++b) tma_load_3d(st + b * TILE, &tm_k, b * 64, y, chain, &full[s], pol);
-        for (int b = 0; b < DV / 64; ++b) tma_load_3d(st + P::KB + b * TILE, &tm_v, b * 64, y, chain, &full[s], pol);
-        bulk_load(st + P::KB + P::VB, achain + (size_t)y * D, n * D * 4, &full[s]);
-        loads_issued = r + 1;
-    };
-    if (tid == 0)
-        for (int r = 0; r < min(nch, P::STAGES); ++r) issue(r);
-
     bool bad = false;
-    for (int r = 0; r < nch; ++r) {
-        const int c = nch - 1 - r;
-        const int s = r % P::STAGES;
-        unsigned char* kt = sm + s * P::STAGE;
-        unsigned char* vt = kt + P::KB;
-        float* at = reinterpret_cast<float*>(vt + P::VB);
-        const int n = min(C, t1 - (t0 + c * C));
-        if (!mbar_wait(&full[s], (r / P::STAGES) & 1, kErrTmaLoad)) bad = true;
-        else loads_waited = r + 1;
-        // per channel i: weight of token t = e^{carry_i + sum_{t < u < chunk end} log alpha_u}
-        {
-            const int i = tid % D, part = tid / D;
-            float la[P::TOK];
-            float sum = 0.f;
-#pragma unroll
-            for (int x = P::TOK - 1; x >= 0; --x) {
-                const int t = part * P::TOK + x;
-                la[x] = log_gate(at[t * D + i], t < n);
-                sum += la[x];
-            }
-            tot[part * D + i] = sum;
-            named_bar(1, P::THREADS);
-            float after = carry[i];   // log decay of the tokens after this thread's part
-            for (int q2 = part + 1; q2 < P::TPC; ++q2) after += tot[q2 * D + i];
-#pragma unroll
-            for (int x = P::TOK - 1; x >= 0; --x) {
-                const int t = part * P::TOK + x;
-                at[t * D + i] = t < n ? __expf(after) : 0.f;
-                after += la[x];
-            }
-            named_bar(1, P::THREADS);
-            if (part == 0) carry[i] = after;   // now includes this whole chunk
-        }
-        // K^ = k . weight (zero past the end of the sequence), in place
-        for (int e = tid; e < (D / 8) * C; e += P::THREADS) {
-            const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
-            const int f0 = b * 64 + (((rem % 8) ^ (row & 7)) * 8);   // first channel of this 16-byte chunk
-            uint4* p = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
-            const float4 w0 = *reinterpret_cast<const float4*>(at + row * D + f0);
-            const float4 w1 = *reinterpret_cast<const float4*>(at + row * D + f0 + 4);
-            const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            float f[8];
-            unpack8(*p, f);
-#pragma unroll
-            for (int x = 0; x < 8; ++x) f[x] *= w[x];
-            *p = pack8(f, 1.f);
-        }
-        fence_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(bad)) { bad = true; break; }
-        if (tid == 0) {
-            // Delta S += K^^T V   (M = d, N = dv)
+    // chunk slot r processes segment chunk nch - 1 - r
+    if (issuer) {
+        int loads = 0, commits = 0;
+        auto issue = [&](int r) {
+            const int c = nch - 1 - r;
+            const int s = r % P::STAGES;
+            unsigned char* st = sm + s * P::STAGE;
+            const int y = t0 + c * C;
+            const int n = min(C, t1 - y);
+            mbar_expect_tx(&full[s], P::LOAD_BYTES + n * D * 4);
+            for (int b = 0; b < D / 64; ++b) tma_load_3d(st + b * TILE, &tm_k, b * 64, y, chain, &full[s], pol);
+            for (int b = 0; b < DV / 64; ++b) tma_load_3d(st + P::KB + b * TILE, &tm_v, b * 64, y, chain, &full[s], pol);
+            bulk_load(st + P::KB + P::VB, achain + (size_t)y * D, n * D * 4, &full[s]);
+            loads = r + 1;
+        };
+        for (int r = 0; r < min(nch, P::STAGES); ++r) issue(r);
+        const uint32_t id_s = idesc_bf16_f32(D, DV, 1, 1);
+        for (int r = 0; r < nch; ++r) {
+            const int s = r % P::STAGES;
+            if (!mbar_wait(&wrdy[s], (r / P::STAGES) & 1, kErrMma)) { bad = true; break; }
             tc_fence_after();
-            const uint32_t ka = smem_u32(kt), va = smem_u32(vt);
-            const uint32_t id_s = idesc_bf16_f32(D, DV, 1, 1);
+            // Delta S += K^^T V   (M = d, N = dv)
+            const uint32_t ka = smem_u32(sm + s * P::STAGE), va = ka + P::KB;
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks)
                 mma_bf16(tbase + P::T_S, sdesc_sw128(ka + ks * 2048, TILE, 1024),
@@ -191,18 +153,76 @@ gla_summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             mma_commit(&empty[s]);
             if (r == nch - 1) mma_commit(done);
             commits = r + 1;
+            // refill the stage chunk slot r - 1 used: its MMA was issued a chunk ago
+            if (r >= 1 && r - 1 + P::STAGES < nch) {
+                if (!mbar_wait(&empty[(r - 1) % P::STAGES], ((r - 1) / P::STAGES) & 1, kErrMma)) { bad = true; break; }
+                issue(r - 1 + P::STAGES);
+            }
         }
-        // refill the stage chunk slot r - 1 used: its MMA was issued a chunk ago
-        if (tid == 0 && r >= 1 && r - 1 + P::STAGES < nch) {
-            const int sp = (r - 1) % P::STAGES;
-            if (!mbar_wait(&empty[sp], ((r - 1) / P::STAGES) & 1, kErrMma)) bad = true;
-            else issue(r - 1 + P::STAGES);
+        if (bad) {
+            // leave no copy or MMA in flight before TMEM is released
+            for (int cc = max(0, loads - P::STAGES); cc < loads; ++cc)
+                mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
+            if (commits > 0)
+                mbar_wait(&empty[(commits - 1) % P::STAGES], ((commits - 1) / P::STAGES) & 1, kErrMma);
         }
+    } else if (tid < P::WORKERS) {
+        for (int r = 0; r < nch; ++r) {
+            const int c = nch - 1 - r;
+            const int s = r % P::STAGES;
+            unsigned char* kt = sm + s * P::STAGE;
+            float* at = reinterpret_cast<float*>(kt + P::KB + P::VB);
+            const int n = min(C, t1 - (t0 + c * C));
+            if (!mbar_wait(&full[s], (r / P::STAGES) & 1, kErrTmaLoad)) bad = true;
+            // per channel i: weight of token t = e^{carry_i + sum_{t < u < chunk end} log alpha_u}
+            // (log alpha replaces alpha in place, then the weight replaces log alpha)
+            const int i = tid % D, part = tid / D;
+            float sum = 0.f;
+#pragma unroll
+            for (int x = P::TOK - 1; x >= 0; --x) {
+                const int t = part * P::TOK + x;
+                const float la = log_gate(at[t * D + i], t < n);
+                at[t * D + i] = la;
+                sum += la;
+            }
+            tot[part * D + i] = sum;
+            if (named_bar_or(1, P::WORKERS, bad)) { bad = true; break; }
+            float after = carry[i];   // log decay of the tokens after this thread's part
+            for (int q2 = part + 1; q2 < P::TPC; ++q2) after += tot[q2 * D + i];
+#pragma unroll
+            for (int x = P::TOK - 1; x >= 0; --x) {
+                const int t = part * P::TOK + x;
+                const float la = at[t * D + i];
+                at[t * D + i] = t < n ? __expf(after) : 0.f;
+                after += la;
+            }
+            named_bar(1, P::WORKERS);
+            if (part == 0) carry[i] = after;   // now includes this whole chunk
+            // K^ = k . weight (zero past the end of the sequence), in place
+            for (int e = tid; e < (D / 8) * C; e += P::WORKERS) {
+                const int b = e / (8 * C), rem = e % (8 * C), row = rem / 8;
+                const int f0 = b * 64 + (((rem % 8) ^ (row & 7)) * 8);   // first channel of this 16-byte chunk
+                uint4* p = reinterpret_cast<uint4*>(kt + b * TILE) + rem;
+                const float4 w0 = *reinterpret_cast<const float4*>(at + row * D + f0);
+                const float4 w1 = *reinterpret_cast<const float4*>(at + row * D + f0 + 4);
+                const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                float f[8];
+                unpack8(*p, f);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) f[x] *= w[x];
+                *p = pack8(f, 1.f);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wrdy[s]);
+        }
+        if (!bad && !mbar_wait(done, 0, kErrMma)) bad = true;
     }
-    if (!bad && !mbar_wait(done, 0, kErrMma)) bad = true;
+    // every thread agrees whether the summary is complete before it is read out
+    const bool any_bad = __syncthreads_or(bad);
     tc_fence_after();
     float* slot = ws + (size_t)unit * (D * DV + D);
-    if (!bad) {
+    if (!any_bad && tid < P::WORKERS) {
         const int f = acc_row<D>(quad, lane);
         for (int g = wg; g < DV / 16; g += 4) {
             float v[16];
@@ -216,12 +236,6 @@ gla_summary_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             }
         }
         if (tid < D) slot[D * DV + tid] = __expf(carry[tid]);   // the segment's decay e^{B_L}
-    }
-    if (bad && tid == 0) {
-        for (int cc = loads_waited; cc < loads_issued; ++cc)
-            mbar_wait(&full[cc % P::STAGES], (cc / P::STAGES) & 1, kErrTmaLoad);
-        if (commits > 0)
-            mbar_wait(&empty[(commits - 1) % P::STAGES], ((commits - 1) / P::STAGES) & 1, kErrMma);
     }
     tc_fence_before();
     __syncthreads();
