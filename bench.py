@@ -601,14 +601,14 @@ TRAFFIC_CAPTURES = {
         "bytes": 2721053696 + 405298688, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
         "sha256": "6603babe911794e43ae63435e60faa7a51603d44a692bffe61c96349acd135fc"},
     ("plain_bf16", "chunk_kernel"): {
-        "bytes": 54633216 + 431104, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "1210dc256f4e02ac5d869765fc94411e086bcd0679139979b221db85bd2dce5f"},
+        "bytes": 54631424 + 760064, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "2d1423379900cb8bcbda6d09bcd00835f6410ba5de2a92d2bc6ad2add4531edd"},
     ("decay_bf16", "chunk_kernel"): {
-        "bytes": 824388608 + 209968896, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
-        "sha256": "1210dc256f4e02ac5d869765fc94411e086bcd0679139979b221db85bd2dce5f"},
+        "bytes": 824389888 + 209698560, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
+        "sha256": "2d1423379900cb8bcbda6d09bcd00835f6410ba5de2a92d2bc6ad2add4531edd"},
     ("gla_bf16", "gla_chunk_kernel"): {
-        "bytes": 343999488 + 34967808, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
-        "sha256": "fe9b2686838a7a2713b4a95fecbfe3a5888b77d963b639eaaf06c87e4ed8d9ea"},
+        "bytes": 344009216 + 34973440, "source": "causal_kernelized_linear_la_b200/csrc/la_gla_tc.cu",
+        "sha256": "635c8cade52f824b03c80c4f7dd276d836c8dc69d0eb41394c1641fffd759e46"},
 }
 
 
