@@ -37,6 +37,7 @@
 // The columns of S evolve independently under the delta rule, so value tiles
 // need no communication.
 #include <algorithm>
+#include <cmath>
 
 #include <cudaTypedefs.h>
 
@@ -951,14 +952,30 @@ GdParts gd_parts(int B, int H, int N, int d, int dv)
     (void)d;
     GdParts p;
     p.P = 1;
-    p.len = N;
+    p.start[0] = 0;
+    p.start[1] = N;
     const long long nch = (N + C - 1) / C;
     const long long ctas = (long long)B * H * (dv / DVT);
     if (N >= 8192 && ctas <= 96) {
-        const long long P = std::min<long long>(kMaxGdParts, nch / 32);
-        const long long per = (nch + P - 1) / P;   // chunks per part
-        p.len = (int)(per * C);
-        p.P = (int)((N + p.len - 1) / p.len);
+        // Part i holds about g^i times part 0's chunks.  Part 0's prep pass runs
+        // alone, so a short part 0 exposes little of it; the prep pass of part
+        // i + 1 runs on the SMs the chain pass leaves idle, at ~0.84 of the
+        // chain's speed per token, so it still ends within the chain pass of
+        // part i while parts grow by less than 1 / 0.84.  g = 1.16 measured
+        // fastest at 65536 tokens (1.08 to 1.20 tried).
+        constexpr double g = 1.16;
+        const int P = (int)std::min<long long>(kMaxGdParts, nch / 32);
+        double wsum = 0.0, w = 1.0;
+        for (int i = 0; i < P; ++i, w *= g) wsum += w;
+        long long done = 0;
+        w = 1.0;
+        for (int i = 0; i < P; ++i, w *= g) {
+            p.start[i] = (int)(done * C);
+            const long long cnt = i == P - 1 ? nch - done : std::max(1LL, std::llround((double)nch * w / wsum));
+            done += cnt;
+        }
+        p.start[P] = N;
+        p.P = P;
     }
     return p;
 }
@@ -982,7 +999,7 @@ size_t gd_workspace_bytes(int B, int H, int N, int d, int dv)
     const GdParts p = gd_parts(B, H, N, d, dv);
     const long long chains = (long long)B * H;
     size_t total = 0;
-    for (int i = 0; i < p.P; ++i) total += gd_part_bytes(chains, std::min(p.len, N - i * p.len), d);
+    for (int i = 0; i < p.P; ++i) total += gd_part_bytes(chains, p.start[i + 1] - p.start[i], d);
     // two fp32 states that carry the chain from one part to the next
     if (p.P > 1) total += 2 * (size_t)chains * d * dv * sizeof(float);
     return total;
@@ -1001,14 +1018,14 @@ cudaError_t launch_prefill_tc_gated_delta(const PrefillArgs& a)
     const int side_ctas = std::max(2, 2 * (sms - busy));
     unsigned char* ws = static_cast<unsigned char*>(a.workspace);
     size_t off = 0;
-    for (int i = 0; i < parts.P; ++i) off += gd_part_bytes(chains, std::min(parts.len, a.N - i * parts.len), a.d);
+    for (int i = 0; i < parts.P; ++i) off += gd_part_bytes(chains, parts.start[i + 1] - parts.start[i], a.d);
     float* carry[2] = {reinterpret_cast<float*>(ws + off),
                        reinterpret_cast<float*>(ws + off) + (size_t)chains * a.d * a.dv};
     const size_t es = 2;   // bf16 elements
     off = 0;
     for (int i = 0; i < parts.P; ++i) {
-        const int t0 = i * parts.len;
-        const int n = std::min(parts.len, a.N - t0);
+        const int t0 = parts.start[i];
+        const int n = parts.start[i + 1] - t0;
         PrefillArgs pa = a;
         pa.q = static_cast<const char*>(a.q) + (size_t)t0 * a.d * es;
         pa.k = static_cast<const char*>(a.k) + (size_t)t0 * a.d * es;

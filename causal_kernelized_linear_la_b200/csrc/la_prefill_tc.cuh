@@ -64,7 +64,7 @@ bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains, in
 constexpr int kMaxGdParts = 8;
 struct GdParts {
     int P = 1;
-    int len = 0;
+    int start[kMaxGdParts + 1] = {};   // part i is tokens start[i] .. start[i + 1] - 1
 };
 GdParts gd_parts(int B, int H, int N, int d, int dv);
 size_t gd_workspace_bytes(int B, int H, int N, int d, int dv);

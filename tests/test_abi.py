@@ -124,7 +124,8 @@ def test_gated_delta_workspace_size():
     n = la.la_prefill_workspace_bytes(1, 32, 1000, 128, 128, "bf16", "gated_delta")
     assert n == 32 * (1024 * (128 + 128) * 2 + 1024 * 2 * 4)
     assert la.la_prefill_workspace_bytes(1, 32, 1000, 128, 128, "f32", "gated_delta") == 0
-    # the long workload runs as eight parts of 8192 tokens, plus two carry states
+    # the long workload runs as eight parts (whole chunks of 64 tokens, 65536 in
+    # all), plus two carry states
     part = 32 * (8192 * (128 + 128) * 2 + 8192 * 2 * 4)
     n = la.la_prefill_workspace_bytes(1, 32, 65536, 128, 128, "bf16", "gated_delta")
     assert n == 8 * part + 2 * 32 * 128 * 128 * 4
@@ -135,7 +136,7 @@ def test_kernel_count():
     assert kc(4, 8, 4096, 64, 64, "bf16", "plain") == 3
     assert kc(2, 16, 32768, 128, 128, "bf16", "decay") == 3
     assert kc(1, 32, 65536, 128, 128, "bf16", "gated_delta") == 16    # eight overlapped parts
-    assert kc(1, 32, 8192, 128, 128, "bf16", "gated_delta") == 8      # four parts of 2048
+    assert kc(1, 32, 8192, 128, 128, "bf16", "gated_delta") == 8      # four parts
     assert kc(1, 3, 2100, 128, 128, "bf16", "gated_delta") == 2
     assert kc(64, 32, 65536, 128, 128, "bf16", "gated_delta") == 2    # enough chains to fill the GPU
     assert kc(1, 1, 256, 64, 64, "f32", "plain") == 2        # parallel form: outputs, final state
