@@ -596,10 +596,10 @@ def la_launches_per_step(p) -> int:
 # records the source file's sha256 at capture time, and the benchmark reports
 # null when the file differs now.
 TRAFFIC_CAPTURES = {
-    # one call's eight chain launches (8 parts of 8192 tokens)
+    # one call's eight chain launches (8 parts, 72 ... 204 chunks)
     ("gdelta_bf16", "gd_chain_kernel"): {
-        "bytes": 2721053696 + 405298688, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
-        "sha256": "6603babe911794e43ae63435e60faa7a51603d44a692bffe61c96349acd135fc"},
+        "bytes": 2721121024 + 408967168, "source": "causal_kernelized_linear_la_b200/csrc/la_gdelta_tc.cu",
+        "sha256": "16f1b3dfdea98f964829fc419b4ccc15394068910c17a373dc30ca1ff4b51191"},
     ("plain_bf16", "chunk_kernel"): {
         "bytes": 54631424 + 760064, "source": "causal_kernelized_linear_la_b200/csrc/la_prefill_tc.cu",
         "sha256": "2d1423379900cb8bcbda6d09bcd00835f6410ba5de2a92d2bc6ad2add4531edd"},
