@@ -59,8 +59,9 @@ bool make_map(CUtensorMap* m, const void* base, int inner, int N, int chains, in
 
 // Gated-delta prefill on the tensor cores (bf16 inputs).  The workspace holds
 // the per-chunk operands the parallel pass hands to the sequential pass.  A
-// long sequence runs as up to kMaxGdParts parts of len tokens (a multiple of
-// the 64-token chunk) whose passes overlap; a call launches 2 P kernels.
+// long sequence runs as up to kMaxGdParts parts (whole 64-token chunks, the
+// last part excepted; each part longer than the one before) whose passes
+// overlap; a call launches 2 P kernels.
 constexpr int kMaxGdParts = 8;
 struct GdParts {
     int P = 1;
