@@ -72,6 +72,14 @@ def test_gated_delta_bf16_small(N):
     _check(inputs.make_gated_delta(1, 3, N, 128, 128, dtype="bf16", seed=500 + N))
 
 
+@pytest.mark.parametrize("N,d", [(9000, 128), (12345, 64)])
+def test_gated_delta_bf16_parts(N, d):
+    """Long enough for the overlapped parts (four here, growing from part to
+    part, the last one ending in a ragged chunk): each part's chain pass
+    starts from the previous part's final state."""
+    _check(inputs.make_gated_delta(1, 2, N, d, d, dtype="bf16", seed=650 + N))
+
+
 @pytest.mark.parametrize("d,dv", [(64, 64), (64, 128), (128, 64)])
 def test_gated_delta_bf16_heads(d, dv):
     _check(inputs.make_gated_delta(2, 2, 333, d, dv, dtype="bf16", seed=600 + d + dv))
