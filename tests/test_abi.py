@@ -131,6 +131,22 @@ def test_gated_delta_workspace_size():
     assert n == 8 * part + 2 * 32 * 128 * 128 * 4
 
 
+def test_gated_delta_parts_are_whole_chunks():
+    """Long gated-delta sequences run as growing parts; every part but the last
+    is whole 64-token chunks, so the parts' workspace slices add up to the
+    workspace of the whole padded sequence (a ragged middle part would pad
+    itself), plus the two carry states (host-only query)."""
+    for B, H, N, d in ((1, 2, 9000, 128), (1, 2, 12345, 64), (1, 32, 65536, 128), (1, 4, 100000, 128),
+                       (2, 8, 8192, 64)):
+        chains, nch = B * H, -(-N // 64)
+        one = chains * (nch * 64 * (d + 128) * 2 + nch * 2 * 64 * 4)
+        parts = la.la_prefill_kernel_count(B, H, N, d, d, "bf16", "gated_delta") // 2
+        assert parts == min(8, nch // 32), (N, d, parts)
+        carries = 2 * chains * d * d * 4 if parts > 1 else 0
+        got = la.la_prefill_workspace_bytes(B, H, N, d, d, "bf16", "gated_delta")
+        assert got == one + carries, (B, H, N, d, got, one + carries)
+
+
 def test_kernel_count():
     kc = la.la_prefill_kernel_count
     assert kc(4, 8, 4096, 64, 64, "bf16", "plain") == 3
